@@ -1,0 +1,161 @@
+"""Seeded synthetic inputs shared by the fp64 oracle, the tests and bench.py.
+
+This module holds no attention arithmetic: it only draws random numbers,
+rounds them to bfloat16 bit patterns and describes the workloads.  Both the
+oracle (``oracle/``) and the CUDA path take their inputs from here, and
+neither imports the other.
+
+Recipe (stated once, used everywhere):
+  * workload ``k`` draws from ``numpy.random.default_rng(k)``;
+  * Q, K, V and dO are drawn in that order as float32 ``standard_normal`` of
+    shapes ``[B][Hq][Sq][D]``, ``[B][Hkv][Skv][D]`` (twice) and
+    ``[B][Hq][Sq][D]``, then rounded to bfloat16 (round-to-nearest-even);
+  * document lengths for the packed-document workload come from
+    ``default_rng(100 + k)``: uniform integers in [512, 4096] until the
+    sequence is filled, the last one truncated to fit.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+# Score-mod identifiers; the same numbering as ``attn_mod_kind`` in
+# include/attn25.h (a C enum cannot be shared with Python without a parser).
+MOD_NONE = 0
+MOD_CAUSAL = 1
+MOD_ALIBI = 2
+MOD_SOFTCAP = 3
+MOD_SLIDING_WINDOW = 4
+MOD_LOCAL_BOOST = 5
+MOD_DOCUMENT = 6
+
+MOD_NAMES = {
+    "none": MOD_NONE,
+    "causal": MOD_CAUSAL,
+    "alibi": MOD_ALIBI,
+    "softcap": MOD_SOFTCAP,
+    "sliding_window": MOD_SLIDING_WINDOW,
+    "local_boost": MOD_LOCAL_BOOST,
+    "document": MOD_DOCUMENT,
+}
+
+
+@dataclasses.dataclass
+class ModParams:
+    """Runtime scalars of the score mods (host-side description)."""
+
+    softcap: float = 50.0
+    window: int = 1024
+    boost: float = 1.1
+    boost_radius: int = 128
+    # per batch row, the ascending document start offsets plus the end (S)
+    doc_offsets: list | None = None
+
+
+@dataclasses.dataclass
+class Workload:
+    name: str
+    seed: int
+    B: int
+    Hq: int
+    Hkv: int
+    Sq: int
+    Skv: int
+    D: int
+    mods: tuple
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+
+# The five workloads the method is measured on (shapes and mods of the
+# FlexAttention / FlashAttention workloads described by the pages).
+WORKLOADS = {
+    "tiny": Workload("tiny", 1, 1, 2, 2, 256, 256, 64, ("none",)),
+    "dense": Workload("dense", 2, 4, 8, 8, 4096, 4096, 128, ("none", "causal")),
+    "gqa_long": Workload("gqa_long", 3, 1, 32, 8, 32768, 32768, 128, ("causal",)),
+    "score_mods": Workload("score_mods", 4, 2, 16, 16, 8192, 8192, 128,
+                           ("alibi", "softcap", "sliding_window", "local_boost")),
+    "documents": Workload("documents", 5, 1, 16, 16, 32768, 32768, 128, ("document",)),
+}
+
+
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bfloat16 (nearest-even); return the uint16 bit patterns."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return rounded.astype(np.uint16)
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of bfloat16 bit patterns to float64."""
+    u = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return u.view(np.float32).astype(np.float64)
+
+
+def draw_qkv(seed: int, B: int, Hq: int, Hkv: int, Sq: int, Skv: int, D: int,
+             with_dout: bool = True) -> dict:
+    """Q, K, V (and dO) as bfloat16 bit patterns, drawn in the order Q, K, V, dO."""
+    rng = np.random.default_rng(seed)
+    out = {}
+    out["q"] = bf16_bits(rng.standard_normal((B, Hq, Sq, D), dtype=np.float32))
+    out["k"] = bf16_bits(rng.standard_normal((B, Hkv, Skv, D), dtype=np.float32))
+    out["v"] = bf16_bits(rng.standard_normal((B, Hkv, Skv, D), dtype=np.float32))
+    if with_dout:
+        out["dout"] = bf16_bits(rng.standard_normal((B, Hq, Sq, D), dtype=np.float32))
+    return out
+
+
+def draw_workload(w: Workload, with_dout: bool = True) -> dict:
+    return draw_qkv(w.seed, w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D, with_dout)
+
+
+def doc_lengths(seed: int, S: int, lo: int = 512, hi: int = 4096) -> list:
+    """Document lengths drawn uniformly from [lo, hi] until S is filled; the last is truncated."""
+    rng = np.random.default_rng(seed)
+    lengths = []
+    total = 0
+    while total < S:
+        n = int(rng.integers(lo, hi, endpoint=True))
+        n = min(n, S - total)
+        lengths.append(n)
+        total += n
+    return lengths
+
+
+def offsets_from_lengths(lengths) -> list:
+    """Start offsets of consecutive documents plus the final end."""
+    offs = [0]
+    for n in lengths:
+        offs.append(offs[-1] + int(n))
+    return offs
+
+
+def doc_offsets_for(w: Workload) -> list:
+    """Per-batch-row document offsets of a workload (every row gets its own draw)."""
+    return [offsets_from_lengths(doc_lengths(100 + w.seed + 1000 * b, w.Skv)) for b in range(w.B)]
+
+
+def pad_offsets(offsets_per_b) -> tuple:
+    """Pack ragged per-row offset lists into an int32 [B][num_docs+1] array.
+
+    Rows with fewer documents repeat their final offset (empty documents).
+    Returns (array, num_docs).
+    """
+    num_docs = max(len(o) - 1 for o in offsets_per_b)
+    arr = np.empty((len(offsets_per_b), num_docs + 1), dtype=np.int32)
+    for b, o in enumerate(offsets_per_b):
+        arr[b, : len(o)] = o
+        arr[b, len(o):] = o[-1]
+    return arr, num_docs
+
+
+def mod_params_for(w: Workload, mod: str) -> ModParams:
+    p = ModParams()
+    if mod == "document":
+        p.doc_offsets = doc_offsets_for(w)
+    return p

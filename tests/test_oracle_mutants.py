@@ -1,0 +1,69 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check a pin catches each.
+
+Each mutant rewrites one expression of an oracle function from its source,
+installs it for the duration of one test, and runs a pin from test_oracle.py
+or test_oracle_block_mask.py that must then fail.
+"""
+import inspect
+import textwrap
+
+import pytest
+
+import oracle
+import oracle.attention as oa
+import oracle.block_sparsity as ob
+import test_oracle as pins
+import test_oracle_block_mask as bm_pins
+
+
+def _install(module, func_name, old, new, monkeypatch):
+    src = textwrap.dedent(inspect.getsource(getattr(module, func_name)))
+    assert old in src, (func_name, old)
+    src = src.replace(old, new, 1)
+    ns = dict(module.__dict__)
+    exec(compile(src, f"<mutant {func_name}>", "exec"), ns)
+    original = getattr(module, func_name)
+    monkeypatch.setattr(module, func_name, ns[func_name])
+    # the package re-exports some functions: patch those names too
+    if getattr(oracle, func_name, None) is original:
+        monkeypatch.setattr(oracle, func_name, ns[func_name])
+
+
+MUTANTS = [
+    # (module, function, original text, planted mistake, pin that must fail)
+    (oa, "attention_forward", "s = scale * (q[b, h, r] @ k[b, hk].T)", "s = (q[b, h, r] @ k[b, hk].T)",
+     lambda: pins.test_matches_torch_sdpa_float64(False)),
+    (oa, "score_mod", "s_mod = s - alibi_slope(h, Hq) * np.abs(qi - kj)", "s_mod = s + alibi_slope(h, Hq) * np.abs(qi - kj)",
+     pins.test_zero_queries_alibi_geometric_sums),
+    (oa, "alibi_slope", "(h + 1)", "h", pins.test_zero_queries_alibi_geometric_sums),
+    (oa, "score_mod", "keep = kj <= qi", "keep = kj < qi", pins.test_causal_first_query_attends_key0),
+    (oa, "score_mod", "keep = kj <= qi", "keep = kj >= qi", pins.test_causal_first_query_attends_key0),
+    (oa, "score_mod", "keep = (diff >= 0) & (diff < params.window)", "keep = (diff >= 0) & (diff <= params.window)",
+     pins.test_window_one_attends_only_self),
+    (oa, "score_mod", "inside = np.abs(qi - kj) < params.boost_radius", "inside = np.abs(qi - kj) <= params.boost_radius",
+     lambda: pins.test_single_key_gives_v0(oa.MOD_LOCAL_BOOST)),
+    (oa, "_kv_head", "return h // (Hq // Hkv)", "return h % Hkv", pins.test_gqa_equals_mha_with_repeated_kv),
+    (oa, "_row_softmax", "e = np.exp(x - m_safe[:, None])", "e = np.exp(x)",
+     lambda: pins.test_single_key_gives_v0(oa.MOD_NONE)),
+    (oa, "_row_softmax", "m_safe + np.log(", "m_safe + np.log2(", pins.test_zero_queries_mean_of_values),
+    (oa, "attention_backward", "dS = P * (dP - Di[:, None]) * dmod", "dS = P * dP * dmod",
+     lambda: pins.test_gradients_match_central_differences(oa.MOD_NONE)),
+    (oa, "score_mod", "dmod = 1.0 - t * t", "dmod = 1.0 - t",
+     lambda: pins.test_gradients_match_central_differences(oa.MOD_SOFTCAP)),
+    (oa, "attention_backward", "dv_acc += P[:, kv_sel].T @ dout[b, h, r]", "dv_acc += P[:, kv_sel].T @ dout[b, hk, r]",
+     pins.test_gqa_equals_mha_with_repeated_kv),
+    (oa, "attention_backward", "dq[b, h, r] = scale * (dS @ k[b, hk])", "dq[b, h, r] = (dS @ k[b, hk])",
+     lambda: pins.test_gradients_match_central_differences(oa.MOD_NONE)),
+    (oa, "online_forward", "l = l * alpha + p.sum(axis=1)", "l = l + p.sum(axis=1)",
+     lambda: pins.test_online_softmax_matches_two_pass(oa.MOD_NONE)),
+    (ob, "classify_tiles", "elif n_keep == blk.size:", "elif n_keep == tile * tile:", bm_pins.test_single_row_tail_tile_is_full),
+    (ob, "block_mask", "key=lambda u: (-pair_cost[u], u)", "key=lambda u: (pair_cost[u], u)", bm_pins.test_orders_are_lpt_permutations),
+]
+
+
+@pytest.mark.parametrize("i", range(len(MUTANTS)))
+def test_planted_mistake_is_caught(i, monkeypatch):
+    module, fn, old, new, pin = MUTANTS[i]
+    _install(module, fn, old, new, monkeypatch)
+    with pytest.raises(AssertionError):
+        pin()
