@@ -1,0 +1,378 @@
+"""Benchmark of the fused attention hot path on B200.
+
+One step = the whole path on one batch of synthetic input: build the block
+mask and work order, forward (O and LSE), backward (dQ, dK, dV).  The default
+workload is dense MHA B=4, Hq=Hkv=8, S=4096, D=128, non-causal, bf16 inputs
+drawn N(0,1) from a fixed seed.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME[:MOD]]
+    python bench.py --impl reference ...   # the fp64 CPU oracle, timed on the host
+    python bench.py --all                  # one line per workload/mod (not the default line)
+
+Prints one JSON line (rank 0).  Throughput counts only unmasked score
+elements: 4 D flop each forward, 10 D backward.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth_inputs import (MOD_NAMES, WORKLOADS, bf16_bits_to_f64, draw_workload,  # noqa: E402
+                          mod_params_for, pad_offsets)
+
+METRIC = "attention fwd/bwd useful TFLOPS on 1 B200 and % of BF16 tensor peak"
+UNIT = "TFLOP/s"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def parse_workload(spec):
+    name, _, mod = spec.partition(":")
+    w = WORKLOADS[name]
+    mod = mod or w.mods[0]
+    return w, mod
+
+
+def useful_counts(ta, w, mod_name, params):
+    mod = MOD_NAMES[mod_name]
+    n = ta.useful_elements(mod, w.B, w.Hq, w.Sq, w.Skv, window=params.window, doc_offsets=params.doc_offsets)
+    return n, ta.useful_flops(n, w.D), ta.useful_flops(n, w.D, backward=True)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import tiled_attention_25_b200 as ta
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w, mod_name = parse_workload(args.workload)
+    mod = MOD_NAMES[mod_name]
+    params = mod_params_for(w, mod_name)
+    bits = draw_workload(w)
+    to_dev = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
+    q, k, v, dout = (to_dev(bits[n]) for n in ("q", "k", "v", "dout"))
+    doc_t = None
+    if params.doc_offsets is not None:
+        doc_t = torch.from_numpy(pad_offsets(params.doc_offsets)[0]).to(dev)
+    dp = ta.ModParams(softcap=params.softcap, window=params.window, boost=params.boost,
+                      boost_radius=params.boost_radius, doc_offsets=doc_t)
+    B, Hq, Hkv, Sq, Skv, D = w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D
+    out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, Sq, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = ta.new_bwd_workspace(B, Hq, Sq, D, device=dev)
+    nbytes = ta.attn_block_mask_bytes(B, Sq, Skv)
+    mbuf = torch.empty(nbytes + 256, dtype=torch.uint8, device=dev)
+    off = (-mbuf.data_ptr()) % 256
+    mask = ta.attn_block_mask_bind(mbuf[off:off + nbytes], B, Sq, Skv)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 3 + 1 + 3  # block mask (3), forward (1), backward (3)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def step(times):
+        e0, e1, e2, e3 = ev(), ev(), ev(), ev()
+        e0.record(stream)
+        ta.build_block_mask(mod, dp, B, Sq, Skv, mask, stream)
+        e1.record(stream)
+        ta.attn_fwd(q, k, v, out, lse, scale=w.scale, mod_kind=mod, mod_params=dp, block_mask=mask, stream=stream)
+        e2.record(stream)
+        ta.attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, ws, scale=w.scale, mod_kind=mod, mod_params=dp,
+                    block_mask=mask, stream=stream)
+        e3.record(stream)
+        times.append((e0, e1, e2, e3))
+
+    warm = []
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step(warm)
+    torch.cuda.synchronize()
+    st = ta.attn_get_status(stream)
+    if st != 0:
+        raise RuntimeError(f"kernel status {st} during warm-up")
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.steps):
+        flush.fill_(1.0)  # L2 flush between steps (outside the timed events)
+        step(times)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    st = ta.attn_get_status(stream)
+    if st != 0:
+        raise RuntimeError(f"kernel status {st} in the timed region")
+    t_mask = [a.elapsed_time(b) for a, b, _, _ in times]
+    t_fwd = [b.elapsed_time(c) for _, b, c, _ in times]
+    t_bwd = [c.elapsed_time(d) for _, _, c, d in times]
+    t_step = [a.elapsed_time(d) for a, _, _, d in times]
+    ms_step = sum(t_step) / len(t_step)
+    ms_fwd = sum(t_fwd) / len(t_fwd)
+    ms_bwd = sum(t_bwd) / len(t_bwd)
+    ms_mask = sum(t_mask) / len(t_mask)
+    if world > 1:
+        tt = torch.tensor([ms_step, ms_fwd, ms_bwd, ms_mask], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms_step, ms_fwd, ms_bwd, ms_mask = tt.tolist()
+
+    # end-to-end through the same API with pinned host buffers: H2D of the
+    # step's inputs, the step, D2H of its results (O, dQ, dK, dV)
+    hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, dout))
+    ho, hdq, hdk, hdv = (torch.empty_like(t, device="cpu").pin_memory() for t in (out, dq, dk, dv))
+    e2e_times = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(1.0)
+        a0, a1 = ev(), ev()
+        a0.record(stream)
+        for d_, h_ in ((q, hq), (k, hk), (v, hv), (dout, hdo)):
+            d_.copy_(h_, non_blocking=True)
+        step([])
+        for h_, d_ in ((ho, out), (hdq, dq), (hdk, dk), (hdv, dv)):
+            h_.copy_(d_, non_blocking=True)
+        a1.record(stream)
+        if i >= args.warmup:
+            e2e_times.append((a0, a1))
+    torch.cuda.synchronize()
+    ms_e2e = sum(a.elapsed_time(b) for a, b in e2e_times) / len(e2e_times)
+    if world > 1:
+        tt = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms_e2e = tt.item()
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v, dout))
+    d2h = sum(t.numel() * t.element_size() for t in (out, dq, dk, dv))
+
+    n_u, f_fwd, f_bwd = useful_counts(ta, w, mod_name, params)
+    total = (f_fwd + f_bwd) * world
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    fwd_tf = f_fwd / (ms_fwd * 1e-3) / 1e12
+    bwd_tf = f_bwd / (ms_bwd * 1e-3) / 1e12
+
+    def roof(tf, traffic):
+        return {"bound": "tensor", "achieved": round(tf, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(tf / peak, 4), "traffic": traffic, "peak_source": f"{peak_kind} bf16_tflops (burst)"}
+
+    dominant = "backward" if ms_bwd >= ms_fwd else "forward"
+    line = {
+        "metric": METRIC,
+        "value": round(total / (ms_step * 1e-3) / 1e12, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 Q/K/V/dO, random-free mods)",
+        "config": {"workload": f"{w.name}:{mod_name}", "B": B, "Hq": Hq, "Hkv": Hkv, "Sq": Sq, "Skv": Skv,
+                   "D": D, "mod": mod_name, "seed": w.seed, "step": "block mask + forward(O, LSE) + backward",
+                   "l2": "flushed before every step (256 MiB write, outside the timed events)",
+                   "parallelism": f"independent replicas x{world} (no collective on the data path)"},
+        "fwd_tflops": round(fwd_tf, 1),
+        "bwd_tflops": round(bwd_tf, 1),
+        "fwd_frac_of_peak": round(fwd_tf / peak, 4),
+        "bwd_frac_of_peak": round(bwd_tf / peak, 4),
+        "ms_fwd": round(ms_fwd, 4),
+        "ms_bwd": round(ms_bwd, 4),
+        "ms_block_mask": round(ms_mask, 4),
+        "useful_elements": n_u,
+        "roofline": dict(roof(bwd_tf if dominant == "backward" else fwd_tf, None), kernel=f"attn_{dominant[:3]} call"),
+        "roofline_forward": roof(fwd_tf, None),
+        "roofline_backward": roof(bwd_tf, None),
+        "e2e": {"value": round(total / (ms_e2e * 1e-3) / 1e12, 2), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, mod_name, params, seconds=args.cpu_seconds)
+    return line
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) arm
+
+def cpu_baseline(w, mod_name, params, seconds=15.0, heads=None):
+    """Time the fp64 oracle (as it stands) on whole (b, head) problems of the workload."""
+    import oracle
+    mod = MOD_NAMES[mod_name]
+    bits = draw_workload(w)
+    qf, kf, vf, df = (bf16_bits_to_f64(bits[n]) for n in ("q", "k", "v", "dout"))
+    G = w.Hq // w.Hkv
+    done, flops, t_total = 0, 0.0, 0.0
+    n_per_head = oracle.useful_elements(mod, params, 1, 1, w.Sq, w.Skv)
+    for hk in range(w.Hkv):
+        if heads is not None and done >= heads:
+            break
+        t0 = time.perf_counter()
+        group = [(0, h) for h in range(hk * G, hk * G + G)]
+        oracle.attention_forward(qf, kf, vf, w.scale, mod, params, heads=group)
+        oracle.attention_backward(qf, kf, vf, df, w.scale, mod, params, groups=[(0, hk)])
+        t_total += time.perf_counter() - t0
+        done += G
+        flops += G * n_per_head * w.D * 14.0
+        if heads is None and t_total >= seconds:
+            break
+    cores = os.cpu_count()
+    return {"value": round(flops / t_total / 1e12, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"fp64 numpy oracle, fwd+bwd of {done} of {w.B * w.Hq} (b, head) problems "
+                      f"({w.Sq}x{w.Skv}, D={w.D}, {mod_name}), {t_total:.1f} s, BLAS threads = host cores"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w, mod_name = parse_workload(args.workload)
+    params = mod_params_for(w, mod_name)
+    per_step = []
+    cb = None
+    for _ in range(args.warmup + args.steps):
+        cb = cpu_baseline(w, mod_name, params, heads=1)
+        per_step.append(cb["value"])
+    vals = per_step[args.warmup:]
+    value = sum(vals) / len(vals)
+    cb["value"] = round(value, 6)
+    return {
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": f"{w.name}:{mod_name}", "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Sq": w.Sq,
+                   "Skv": w.Skv, "D": w.D, "mod": mod_name, "seed": w.seed,
+                   "step": "fp64 oracle fwd+bwd of one (b, head) problem of the workload"},
+        "cpu_baseline": cb,
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="dense:none")
+    ap.add_argument("--all", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        if args.all:
+            specs = [f"{n}:{m}" for n, w in WORKLOADS.items() for m in w.mods]
+            for s in specs:
+                args.workload = s
+                line = run_gpu(args, rank, world, local_rank)
+                if rank == 0:
+                    print(json.dumps(line), flush=True)
+        else:
+            line = run_gpu(args, rank, world, local_rank)
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,188 @@
+/*
+ * attn25 — exact fused scaled-dot-product attention for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libattn25.so.  Every pointer argument named "device" is a CUDA
+ * device pointer; every call is asynchronous on the given stream and returns
+ * before the GPU work ends.  The caller owns and allocates every buffer
+ * (inputs, outputs, the backward workspace, the block mask); the library
+ * keeps only one device status word per GPU.
+ *
+ * What is computed.  For each batch row b, query head h (KV head
+ * hk = h / (Hq / Hkv)), query i and key j:
+ *     s_ij  = scale * sum_d q_id k_jd
+ *     s'_ij = mod(s_ij; b, h, i, j), masked entries are -inf
+ *     O_i   = sum_j softmax_j(s'_i.) v_j,   LSE_i = ln sum_j exp(s'_ij)
+ * i.e. standard attention softmax(Q K^T * scale) V ("FlashAttention 설명",
+ * §1) with a FlexAttention-style score mod or mask ("PyTorch FlexAttention,
+ * FlashAttention-4 백엔드 도입으로 성능 최대 3.2배 향상", 섹션별 상세), computed
+ * tile by tile with an online softmax so that the score matrix never reaches
+ * global memory ("FlashAttention-2 — GPU attention의 사실상 표준", §3-§4;
+ * "FlashAttention 설명", §3-§6).  The backward pass recomputes the scores from
+ * the saved LSE ("FlashAttention-2 …", §3 Recomputation).
+ *
+ * Layouts.  Q, O, dQ, dO: bf16 [B][Hq][Sq][D]; K, V, dK, dV: bf16
+ * [B][Hkv][Skv][D]; LSE: fp32 [B][Hq][Sq] (natural log), contiguous, D
+ * innermost.  Supported: D in {64, 128}; Sq, Skv >= 1; Hq a multiple of Hkv.
+ * Every tensor base pointer must be 16-byte aligned.
+ *
+ * Errors.  Functions return ATTN_OK (0) or a negative attn_status; arguments
+ * are checked on the host before anything is launched.  A kernel that waits
+ * longer than the wait limit on one of its internal barriers stops, writes
+ * ATTN_ERR_TIMEOUT into the device status word and returns; the host reads
+ * (and clears) it with attn_get_status().
+ */
+#ifndef ATTN25_H
+#define ATTN25_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN25_API __attribute__((visibility("default")))
+#else
+#define ATTN25_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without including the CUDA headers (the same handle type). */
+typedef struct CUstream_st* attn_stream_t;
+
+/* A bfloat16 value as its 16-bit pattern. */
+typedef uint16_t attn_bf16;
+
+typedef enum attn_status {
+  ATTN_OK = 0,
+  ATTN_ERR_ARG = -1,          /* NULL pointer, bad size, Hq % Hkv != 0 */
+  ATTN_ERR_UNSUPPORTED = -2,  /* D not in {64,128}, or a mod/param combination not supported */
+  ATTN_ERR_ALIGN = -3,        /* a base pointer is not 16-byte aligned */
+  ATTN_ERR_WORKSPACE = -4,    /* workspace or block-mask buffer too small */
+  ATTN_ERR_LAUNCH = -5,       /* a CUDA call or kernel launch failed */
+  ATTN_ERR_TIMEOUT = -6,      /* a kernel gave up waiting on an internal barrier */
+  ATTN_ERR_DEVICE = -7        /* no usable sm_100 device, or the kernel image failed to load */
+} attn_status;
+
+/*
+ * Score mods and masks (the fixed set; each is applied to the scaled score
+ * s = scale * q.k of query i and key j, absolute indices, 0-based).
+ * The FlexAttention page shows score_mod(score, b, h, q_idx, kv_idx) with the
+ * local boost and tanh softcap examples ("PyTorch FlexAttention, …",
+ * 섹션별 상세) and names ALiBi, sliding window and document masking (핵심 요약).
+ */
+typedef enum attn_mod_kind {
+  ATTN_MOD_NONE = 0,            /* s' = s */
+  ATTN_MOD_CAUSAL = 1,          /* keep j <= i */
+  ATTN_MOD_ALIBI = 2,           /* s' = s - slope_h |i - j| */
+  ATTN_MOD_SOFTCAP = 3,         /* s' = c tanh(s / c) */
+  ATTN_MOD_SLIDING_WINDOW = 4,  /* keep 0 <= i - j < W */
+  ATTN_MOD_LOCAL_BOOST = 5,     /* s' = boost * s if |i - j| < radius, else s */
+  ATTN_MOD_DOCUMENT = 6         /* keep doc(i) == doc(j) and j <= i */
+} attn_mod_kind;
+
+/*
+ * Runtime scalars of the mods; a change needs no recompilation (the page
+ * notes that its JIT backend recompiles when such a scalar changes).
+ * Fields that the chosen mod does not use are ignored.
+ */
+typedef struct attn_mod_params {
+  float softcap;               /* ATTN_MOD_SOFTCAP: c > 0 (e.g. 50) */
+  int32_t window;              /* ATTN_MOD_SLIDING_WINDOW: W >= 1 (e.g. 1024) */
+  float boost;                 /* ATTN_MOD_LOCAL_BOOST: factor (e.g. 1.1) */
+  int32_t boost_radius;        /* ATTN_MOD_LOCAL_BOOST: radius >= 0 (e.g. 128) */
+  const float* alibi_slopes;   /* ATTN_MOD_ALIBI: device fp32 [Hq], or NULL for 2^(-8 (h+1) / Hq) */
+  const int32_t* doc_offsets;  /* ATTN_MOD_DOCUMENT: device int32 [B][num_docs+1]: ascending document
+                                  starts, offsets[b][0] = 0, offsets[b][num_docs] = Skv; repeat the last
+                                  value to pad rows with fewer documents.  Queries and keys share the
+                                  offsets (packed self-attention, Sq == Skv required). */
+  int32_t num_docs;            /* ATTN_MOD_DOCUMENT: 1 <= num_docs <= 4096 */
+} attn_mod_params;
+
+/*
+ * Block mask over 128x128 tiles ("PyTorch FlexAttention, …", 섹션별 상세:
+ * block-sparse iteration that skips fully masked blocks).  All arrays are
+ * device memory inside one caller-allocated buffer (attn_block_mask_bytes),
+ * laid out by attn_block_mask_bind and filled by build_block_mask:
+ *   tile_class [B][nq][nk] uint8: 0 EMPTY, 1 PARTIAL, 2 FULL over in-range elements
+ *   kv_count [B][nq], kv_index [B][nq][nk]: non-EMPTY KV tiles per query tile, ascending, -1 padded
+ *   q_count [B][nk], q_index [B][nk][nq]: non-EMPTY query tiles per KV tile, ascending, -1 padded
+ *   fwd_order [B * ceil(nq/2)]: forward work pairs (query tiles 2p, 2p+1 of row b, id b*np+p)
+ *       in longest-first order of their non-EMPTY KV tile count, ties by id
+ *   bwd_order [B * nk]: backward units (id b*nk+kv tile) longest-first by q_count, ties by id
+ */
+typedef struct attn_block_mask {
+  uint8_t* tile_class;
+  int32_t* kv_count;
+  int32_t* kv_index;
+  int32_t* q_count;
+  int32_t* q_index;
+  int32_t* fwd_order;
+  int32_t* bwd_order;
+  int32_t B, Sq, Skv, nq_tiles, nk_tiles;
+  int32_t mod_kind;            /* the mod it was built for; attn_fwd/attn_bwd check it */
+} attn_block_mask;
+
+/*
+ * Forward pass.  q, k, v: device bf16 inputs; out: device bf16 output;
+ * lse: device fp32 [B][Hq][Sq] or NULL (then a kernel specialisation that
+ * neither computes nor writes it runs, as the FlashInfer page's out-only
+ * path: "FlashInfer SM120 NVFP4 어텐션 최적화", 코드 분석 2-4).
+ * block_mask: NULL for dense iteration (causal and sliding-window tiles are
+ * then classified on the fly, document masks test every element), or a mask
+ * built by build_block_mask for the same mod and sizes.
+ * mod_params may be NULL only for ATTN_MOD_NONE / CAUSAL.
+ */
+ATTN25_API int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v,
+             attn_bf16* out, float* lse,
+             int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+             int mod_kind, const attn_mod_params* mod_params,
+             const attn_block_mask* block_mask, attn_stream_t stream);
+
+/* Bytes of device workspace attn_bwd needs (fp32 dQ accumulator and row statistics). */
+ATTN25_API size_t attn_bwd_workspace_size(int B, int Hq, int Sq, int D);
+
+/*
+ * Backward pass: dq, dk, dv (device bf16) from q, k, v, out, lse (as written
+ * by attn_fwd with the same arguments; required) and dout.  workspace:
+ * device memory of at least attn_bwd_workspace_size bytes, 256-byte aligned;
+ * its contents on entry do not matter.  dQ is accumulated in fp32 with
+ * atomic adds, so its last bits may differ from run to run.
+ */
+ATTN25_API int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v,
+             const attn_bf16* out, const float* lse, const attn_bf16* dout,
+             attn_bf16* dq, attn_bf16* dk, attn_bf16* dv,
+             void* workspace, size_t workspace_bytes,
+             int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+             int mod_kind, const attn_mod_params* mod_params,
+             const attn_block_mask* block_mask, attn_stream_t stream);
+
+/* Bytes of device memory one block mask for (B, Sq, Skv) occupies. */
+ATTN25_API size_t attn_block_mask_bytes(int B, int Sq, int Skv);
+
+/* Lay out a block mask inside a caller buffer (device, 256-byte aligned); no GPU work. */
+ATTN25_API int attn_block_mask_bind(void* buffer, size_t bytes, int B, int Sq, int Skv,
+                         attn_block_mask* out);
+
+/*
+ * Classify every 128x128 tile for the mod and fill all arrays of a bound
+ * block mask (bit-exact with a per-element classification).
+ */
+ATTN25_API int build_block_mask(int mod_kind, const attn_mod_params* mod_params,
+                     int B, int Sq, int Skv, attn_block_mask* mask,
+                     attn_stream_t stream);
+
+/* Synchronise the stream, then return and clear the device status word. */
+ATTN25_API int attn_get_status(attn_stream_t stream);
+
+/* Set the per-wait time limit of the kernels in milliseconds (default 4000). */
+ATTN25_API void attn_set_wait_limit_ms(uint32_t ms);
+
+/* A static description of an attn_status value. */
+ATTN25_API const char* attn_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN25_H */

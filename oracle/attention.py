@@ -166,7 +166,8 @@ def attention_probs(q, k, scale, mod=MOD_NONE, params=None, b=0, h=0):
 
 
 def attention_backward(q, k, v, dout, scale, mod=MOD_NONE, params=None,
-                       groups=None, q_rows=None, kv_rows=None, chunk=1024):
+                       groups=None, q_rows=None, kv_rows=None, chunk=1024,
+                       contrib_rows=None):
     """dQ, dK, dV of L = sum(dO * O) by the exact gradient formulas.
 
     With s = scale q.k, s' = mod(s), P = softmax_row(s' masked), O = P V:
@@ -179,6 +180,10 @@ def attention_backward(q, k, v, dout, scale, mod=MOD_NONE, params=None,
     groups: optional list of (b, hk) KV-head groups to compute (default all);
     q_rows / kv_rows: optional sorted index arrays restricting which rows of
     dQ and of dK/dV are returned (all query rows still enter dK/dV).
+    contrib_rows: optional sorted query rows whose terms are summed into
+    dK/dV (default: all rows).  Only for callers that know every other row's
+    P_ij is exactly zero for the requested keys (e.g. causal masks, keys past
+    the last excluded query), so that the sum is unchanged.
     Entries not computed are NaN.
     """
     B, Hq, Sq, D = q.shape
@@ -189,7 +194,7 @@ def attention_backward(q, k, v, dout, scale, mod=MOD_NONE, params=None,
     dv = np.full(v.shape, np.nan)
     if groups is None:
         groups = [(b, hk) for b in range(B) for hk in range(Hkv)]
-    all_rows = np.arange(Sq, dtype=np.int64)
+    all_rows = np.arange(Sq, dtype=np.int64) if contrib_rows is None else np.asarray(contrib_rows, dtype=np.int64)
     kv_sel = np.arange(Skv) if kv_rows is None else np.asarray(kv_rows, dtype=np.int64)
     q_sel = None if q_rows is None else set(int(x) for x in q_rows)
     kj = np.arange(Skv, dtype=np.int64)[None, :]

@@ -1,0 +1,95 @@
+"""The C ABI library loads and exports every entry point the header declares;
+host-side argument checks reject bad calls before any GPU work (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn25.h")
+
+
+def declared():
+    text = open(HEADER).read()
+    return re.findall(r"ATTN25_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from tiled_attention_25_b200.build import build
+    path = build()
+    return ctypes.CDLL(path)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared())
+    assert {"attn_fwd", "attn_bwd", "build_block_mask", "attn_bwd_workspace_size",
+            "attn_block_mask_bytes", "attn_block_mask_bind", "attn_get_status",
+            "attn_set_wait_limit_ms", "attn_strerror"} <= names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared():
+        assert hasattr(lib, name), name
+
+
+def test_binding_names_match_header(lib):
+    import tiled_attention_25_b200 as ta
+    for name in declared():
+        assert name in ta.EXPORTED and callable(getattr(ta, name)), name
+
+
+def test_sizes(lib):
+    lib.attn_block_mask_bytes.restype = ctypes.c_size_t
+    lib.attn_bwd_workspace_size.restype = ctypes.c_size_t
+    assert lib.attn_block_mask_bytes(0, 10, 10) == 0
+    n = lib.attn_block_mask_bytes(1, 32768, 32768)
+    assert n >= 256 * 256 * (1 + 4 + 4) + 256 * 4 * 2
+    ws = lib.attn_bwd_workspace_size(1, 32, 32768, 128)
+    assert ws >= 32 * 32768 * (128 * 4 + 8)
+    assert lib.attn_bwd_workspace_size(1, 1, 1, 96) == 0  # unsupported head dim
+
+
+def test_bind_lays_out_inside_the_buffer(lib):
+    import tiled_attention_25_b200.abi as abi
+    lib.attn_block_mask_bytes.restype = ctypes.c_size_t
+    B, Sq, Skv = 2, 1000, 300
+    n = lib.attn_block_mask_bytes(B, Sq, Skv)
+    fake = 1 << 40  # never dereferenced: bind only computes addresses
+    m = abi.CBlockMask()
+    rc = lib.attn_block_mask_bind(ctypes.c_void_p(fake), ctypes.c_size_t(n), B, Sq, Skv, ctypes.byref(m))
+    assert rc == 0
+    ptrs = [m.tile_class, m.kv_count, m.kv_index, m.q_count, m.q_index, m.fwd_order, m.bwd_order]
+    assert all(fake <= p < fake + n and p % 256 == 0 for p in ptrs)
+    assert (m.nq_tiles, m.nk_tiles) == (8, 3)
+    rc = lib.attn_block_mask_bind(ctypes.c_void_p(fake), ctypes.c_size_t(n - 1), B, Sq, Skv, ctypes.byref(m))
+    assert rc == -4
+    rc = lib.attn_block_mask_bind(ctypes.c_void_p(fake + 16), ctypes.c_size_t(n), B, Sq, Skv, ctypes.byref(m))
+    assert rc == -3
+
+
+def test_argument_errors_before_launch(lib):
+    P, I = ctypes.c_void_p, ctypes.c_int
+    lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, ctypes.c_float, I, P, P, P]
+    good = ctypes.c_void_p(1 << 32)
+    odd = ctypes.c_void_p((1 << 32) + 8)
+    args = lambda **kw: dict(dict(q=good, k=good, v=good, o=good, lse=None, B=1, Hq=4, Hkv=2, Sq=128,
+                                  Skv=128, D=128, scale=0.1, mod=0, mp=None, bm=None, s=None), **kw)
+    call = lambda a: lib.attn_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["Sq"],
+                                  a["Skv"], a["D"], a["scale"], a["mod"], a["mp"], a["bm"], a["s"])
+    assert call(args(q=None)) == -1
+    assert call(args(q=odd)) == -3
+    assert call(args(Hkv=3)) == -1
+    assert call(args(D=96)) == -2
+    assert call(args(Sq=0)) == -1
+    assert call(args(scale=0.0)) == -1
+    assert call(args(mod=9)) == -1
+    assert call(args(mod=3)) == -1   # softcap needs params
+    assert call(args(mod=6)) == -1   # document mask needs offsets
+
+
+def test_strerror(lib):
+    lib.attn_strerror.restype = ctypes.c_char_p
+    assert b"timed out" in lib.attn_strerror(-6)
+    assert lib.attn_strerror(0) == b"ok"

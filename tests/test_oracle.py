@@ -308,3 +308,17 @@ def test_printed_score_count():
         g = json.load(f)
     n = oracle.useful_elements(MOD_NONE, None, 1, 1, g["S"], g["S"])
     assert round(n / 1e6) == g["scores_millions_printed"]
+
+
+def test_backward_contributing_rows_under_causal_mask():
+    # keys j >= 200 are seen only by queries i >= j under the causal mask
+    B, Hq, Hkv, S, D = 1, 2, 1, 260, 4
+    q, k, v = rand((B, Hq, S, D), 54), rand((B, Hkv, S, D), 55), rand((B, Hkv, S, D), 56)
+    dout = rand((B, Hq, S, D), 57)
+    full = oracle.attention_backward(q, k, v, dout, 0.5, MOD_CAUSAL, chunk=64)
+    kv = np.arange(200, S)
+    part = oracle.attention_backward(q, k, v, dout, 0.5, MOD_CAUSAL, kv_rows=kv, q_rows=kv,
+                                     contrib_rows=np.arange(200, S))
+    assert np.allclose(part[1][0, 0, kv], full[1][0, 0, kv], atol=1e-13)
+    assert np.allclose(part[2][0, 0, kv], full[2][0, 0, kv], atol=1e-13)
+    assert np.allclose(part[0][0, :, kv], full[0][0, :, kv], atol=1e-13)

@@ -1,0 +1,55 @@
+"""attn25: exact fused attention for B200 (sm_100a) behind a small C ABI.
+
+The compute runs in libattn25.so (hand-written sm_100a kernels); this package
+is its ctypes binding plus helpers that allocate the caller-owned buffers
+with PyTorch.  Importing it fails if the library has not been built.
+"""
+from __future__ import annotations
+
+import torch
+
+from .abi import (  # noqa: F401
+    ATTN_ERR_TIMEOUT,
+    EXPORTED,
+    LIB,
+    LIB_PATH,
+    MOD_ALIBI,
+    MOD_CAUSAL,
+    MOD_DOCUMENT,
+    MOD_LOCAL_BOOST,
+    MOD_NONE,
+    MOD_SLIDING_WINDOW,
+    MOD_SOFTCAP,
+    AttnError,
+    BlockMask,
+    ModParams,
+    attn_block_mask_bind,
+    attn_block_mask_bytes,
+    attn_bwd,
+    attn_bwd_workspace_size,
+    attn_fwd,
+    attn_get_status,
+    attn_set_wait_limit_ms,
+    attn_strerror,
+    build_block_mask,
+)
+from .counts import useful_elements, useful_flops  # noqa: F401
+
+
+def new_block_mask(mod_kind, mod_params, B, Sq, Skv, device="cuda", stream=None) -> BlockMask:
+    """Allocate a block-mask buffer with torch, bind it and build it on the GPU."""
+    nbytes = attn_block_mask_bytes(B, Sq, Skv)
+    buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+    off = (-buf.data_ptr()) % 256
+    buf = buf[off:off + nbytes]
+    mask = attn_block_mask_bind(buf, B, Sq, Skv)
+    build_block_mask(mod_kind, mod_params, B, Sq, Skv, mask, stream)
+    return mask
+
+
+def new_bwd_workspace(B, Hq, Sq, D, device="cuda") -> torch.Tensor:
+    """A 256-byte-aligned workspace of attn_bwd_workspace_size bytes."""
+    nbytes = attn_bwd_workspace_size(B, Hq, Sq, D)
+    buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+    off = (-buf.data_ptr()) % 256
+    return buf[off:off + nbytes]

@@ -1,0 +1,244 @@
+"""ctypes binding of libattn25.so — argument marshalling only.
+
+Every function here has the name of the C entry point it calls (declared in
+include/attn25.h) and does no attention work of its own: it checks tensor
+metadata, turns torch tensors into device pointers and sizes, and raises
+AttnError on a non-zero status.  PyTorch provides device memory and streams.
+There is no fallback: if the shared library is missing or fails to load,
+importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn25.so")
+
+MOD_NONE = 0
+MOD_CAUSAL = 1
+MOD_ALIBI = 2
+MOD_SOFTCAP = 3
+MOD_SLIDING_WINDOW = 4
+MOD_LOCAL_BOOST = 5
+MOD_DOCUMENT = 6
+
+ATTN_ERR_TIMEOUT = -6
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {code} ({attn_strerror(code)})")
+        self.code = code
+
+
+class CModParams(ctypes.Structure):
+    _fields_ = [
+        ("softcap", ctypes.c_float),
+        ("window", ctypes.c_int32),
+        ("boost", ctypes.c_float),
+        ("boost_radius", ctypes.c_int32),
+        ("alibi_slopes", ctypes.c_void_p),
+        ("doc_offsets", ctypes.c_void_p),
+        ("num_docs", ctypes.c_int32),
+    ]
+
+
+class CBlockMask(ctypes.Structure):
+    _fields_ = [
+        ("tile_class", ctypes.c_void_p),
+        ("kv_count", ctypes.c_void_p),
+        ("kv_index", ctypes.c_void_p),
+        ("q_count", ctypes.c_void_p),
+        ("q_index", ctypes.c_void_p),
+        ("fwd_order", ctypes.c_void_p),
+        ("bwd_order", ctypes.c_void_p),
+        ("B", ctypes.c_int32),
+        ("Sq", ctypes.c_int32),
+        ("Skv", ctypes.c_int32),
+        ("nq_tiles", ctypes.c_int32),
+        ("nk_tiles", ctypes.c_int32),
+        ("mod_kind", ctypes.c_int32),
+    ]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m tiled_attention_25_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, P, P, P]
+    lib.attn_fwd.restype = I
+    lib.attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, S, I, I, I, I, I, I, F, I, P, P, P]
+    lib.attn_bwd.restype = I
+    lib.attn_bwd_workspace_size.argtypes = [I, I, I, I]
+    lib.attn_bwd_workspace_size.restype = S
+    lib.attn_block_mask_bytes.argtypes = [I, I, I]
+    lib.attn_block_mask_bytes.restype = S
+    lib.attn_block_mask_bind.argtypes = [P, S, I, I, I, ctypes.POINTER(CBlockMask)]
+    lib.attn_block_mask_bind.restype = I
+    lib.build_block_mask.argtypes = [I, P, I, I, I, ctypes.POINTER(CBlockMask), P]
+    lib.build_block_mask.restype = I
+    lib.attn_get_status.argtypes = [P]
+    lib.attn_get_status.restype = I
+    lib.attn_set_wait_limit_ms.argtypes = [ctypes.c_uint32]
+    lib.attn_set_wait_limit_ms.restype = None
+    lib.attn_strerror.argtypes = [I]
+    lib.attn_strerror.restype = ctypes.c_char_p
+    return lib
+
+
+LIB = _load()
+
+EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_block_mask_bytes",
+            "attn_block_mask_bind", "build_block_mask", "attn_get_status",
+            "attn_set_wait_limit_ms", "attn_strerror")
+
+
+def attn_strerror(code: int) -> str:
+    return LIB.attn_strerror(int(code)).decode()
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise AttnError(code, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+class ModParams:
+    """Mod scalars plus the device tensors they point at (kept alive here)."""
+
+    def __init__(self, softcap=50.0, window=1024, boost=1.1, boost_radius=128,
+                 alibi_slopes=None, doc_offsets=None):
+        self.softcap = float(softcap)
+        self.window = int(window)
+        self.boost = float(boost)
+        self.boost_radius = int(boost_radius)
+        self.alibi_slopes = alibi_slopes        # device fp32 [Hq] or None
+        self.doc_offsets = doc_offsets          # device int32 [B][num_docs+1] or None
+        if doc_offsets is not None:
+            assert doc_offsets.dtype == torch.int32 and doc_offsets.is_contiguous() and doc_offsets.dim() == 2
+        if alibi_slopes is not None:
+            assert alibi_slopes.dtype == torch.float32 and alibi_slopes.is_contiguous()
+
+    def c(self) -> CModParams:
+        return CModParams(self.softcap, self.window, self.boost, self.boost_radius,
+                          None if self.alibi_slopes is None else self.alibi_slopes.data_ptr(),
+                          None if self.doc_offsets is None else self.doc_offsets.data_ptr(),
+                          0 if self.doc_offsets is None else self.doc_offsets.shape[1] - 1)
+
+
+class BlockMask:
+    """A bound block mask: the C struct plus the device buffer that holds it."""
+
+    def __init__(self, buffer: torch.Tensor, c: CBlockMask):
+        self.buffer = buffer
+        self.c = c
+
+    def view(self, name):
+        """The named array as a torch view of the buffer (for inspection and tests)."""
+        c = self.c
+        B, nq, nk = c.B, c.nq_tiles, c.nk_tiles
+        npairs = (nq + 1) // 2
+        shapes = {"tile_class": (torch.uint8, (B, nq, nk)), "kv_count": (torch.int32, (B, nq)),
+                  "kv_index": (torch.int32, (B, nq, nk)), "q_count": (torch.int32, (B, nk)),
+                  "q_index": (torch.int32, (B, nk, nq)), "fwd_order": (torch.int32, (B * npairs,)),
+                  "bwd_order": (torch.int32, (B * nk,))}
+        dtype, shape = shapes[name]
+        off = getattr(c, name) - self.buffer.data_ptr()
+        n = 1
+        for s in shape:
+            n *= s
+        size = n * (1 if dtype == torch.uint8 else 4)
+        return self.buffer[off:off + size].view(dtype).view(shape)
+
+
+def _mp(mod_params):
+    if mod_params is None:
+        return None
+    cm = mod_params.c()
+    return ctypes.byref(cm), cm
+
+
+def _dims(q, k, v, out):
+    for t in (q, k, v, out):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("q, k, v, out must be contiguous CUDA bf16 [B][H][S][D] tensors")
+    B, Hq, Sq, D = q.shape
+    Bk, Hkv, Skv, Dk = k.shape
+    if tuple(v.shape) != (Bk, Hkv, Skv, Dk) or Bk != B or Dk != D or tuple(out.shape) != (B, Hq, Sq, D):
+        raise ValueError("inconsistent q/k/v/out shapes")
+    return B, Hq, Hkv, Sq, Skv, D
+
+
+def attn_fwd(q, k, v, out, lse=None, scale=None, mod_kind=MOD_NONE, mod_params=None,
+             block_mask=None, stream=None):
+    B, Hq, Hkv, Sq, Skv, D = _dims(q, k, v, out)
+    if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hq, Sq) or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous fp32 [B][Hq][Sq] tensor")
+    scale = D ** -0.5 if scale is None else float(scale)
+    mp = _mp(mod_params)
+    rc = LIB.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
+                      scale, int(mod_kind), None if mp is None else mp[0],
+                      None if block_mask is None else ctypes.byref(block_mask.c), _stream(stream))
+    _check(rc, "attn_fwd")
+
+
+def attn_bwd_workspace_size(B, Hq, Sq, D) -> int:
+    return int(LIB.attn_bwd_workspace_size(B, Hq, Sq, D))
+
+
+def attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, workspace, scale=None, mod_kind=MOD_NONE,
+             mod_params=None, block_mask=None, stream=None):
+    B, Hq, Hkv, Sq, Skv, D = _dims(q, k, v, out)
+    for t in (dout, dq):
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != (B, Hq, Sq, D) or not t.is_contiguous():
+            raise ValueError("dout/dq must be contiguous bf16 like q")
+    for t in (dk, dv):
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != (B, Hkv, Skv, D) or not t.is_contiguous():
+            raise ValueError("dk/dv must be contiguous bf16 like k")
+    scale = D ** -0.5 if scale is None else float(scale)
+    mp = _mp(mod_params)
+    rc = LIB.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+                      _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                      B, Hq, Hkv, Sq, Skv, D, scale, int(mod_kind), None if mp is None else mp[0],
+                      None if block_mask is None else ctypes.byref(block_mask.c), _stream(stream))
+    _check(rc, "attn_bwd")
+
+
+def attn_block_mask_bytes(B, Sq, Skv) -> int:
+    return int(LIB.attn_block_mask_bytes(B, Sq, Skv))
+
+
+def attn_block_mask_bind(buffer, B, Sq, Skv) -> BlockMask:
+    c = CBlockMask()
+    rc = LIB.attn_block_mask_bind(_ptr(buffer), buffer.numel() * buffer.element_size(), B, Sq, Skv,
+                                  ctypes.byref(c))
+    _check(rc, "attn_block_mask_bind")
+    return BlockMask(buffer, c)
+
+
+def build_block_mask(mod_kind, mod_params, B, Sq, Skv, mask: BlockMask, stream=None):
+    mp = _mp(mod_params)
+    rc = LIB.build_block_mask(int(mod_kind), None if mp is None else mp[0], B, Sq, Skv,
+                              ctypes.byref(mask.c), _stream(stream))
+    _check(rc, "build_block_mask")
+
+
+def attn_get_status(stream=None) -> int:
+    return int(LIB.attn_get_status(_stream(stream)))
+
+
+def attn_set_wait_limit_ms(ms: int):
+    LIB.attn_set_wait_limit_ms(int(ms))

@@ -1,0 +1,413 @@
+// The C ABI of libattn25.so: argument checks, TMA descriptor encoding and
+// kernel dispatch.  Every exported function is declared in include/attn25.h.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "attn25.h"
+#include "launch.h"
+
+namespace attn25 {
+
+// One status word per device that loads the library.
+__device__ int g_attn_status;
+
+namespace {
+
+std::atomic<uint32_t> g_wait_ms{4000};
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  bool usable = false;
+  int sms = 0;
+  int* status = nullptr;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int current_device(DeviceInfo** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    d.ready = true;
+    int major = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    void* p = nullptr;
+    const bool sym_ok = cudaGetSymbolAddress(&p, g_attn_status) == cudaSuccess;
+    d.status = static_cast<int*>(p);
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+              cudaSuccess &&
+          q == cudaDriverEntryPointSuccess)
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    d.usable = (major == 10) && sym_ok && d.sms > 0 && g_encode != nullptr;
+    cudaGetLastError();  // do not leak a sticky-free error from the probes
+  }
+  if (!d.usable) return ATTN_ERR_DEVICE;
+  *out = &d;
+  return ATTN_OK;
+}
+
+// bf16 tensor [outer][rows][inner] with rows x 64-column boxes, 128-byte swizzle.
+bool encode_bf16(CUtensorMap* m, const void* base, int inner, int rows, int outer, int box_rows) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * 2,
+                           static_cast<cuuint64_t>(inner) * rows * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp32 tensor [outer][rows][inner], boxes of box_inner x box_rows, no swizzle.
+bool encode_f32(CUtensorMap* m, const void* base, int inner, int rows, int outer, int box_inner,
+                int box_rows) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * 4,
+                           static_cast<cuuint64_t>(inner) * rows * 4};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+uint64_t wait_ns() { return static_cast<uint64_t>(g_wait_ms.load()) * 1000000ull; }
+
+// Shared validation of shapes, mod and mask.
+int check_common(int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale, int mod_kind,
+                 const attn_mod_params* mp, const attn_block_mask* bm) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Skv < 1) return ATTN_ERR_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  // coordinates and unit counts stay well inside int32
+  if (static_cast<long long>(B) * Hq * (cdiv(Sq, TILE) + 1) >= (1ll << 30)) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * Hq >= (1ll << 30) || Sq >= (1 << 30) || Skv >= (1 << 30))
+    return ATTN_ERR_UNSUPPORTED;
+  if (mod_kind < ATTN_MOD_NONE || mod_kind > ATTN_MOD_DOCUMENT) return ATTN_ERR_ARG;
+  switch (mod_kind) {
+    case ATTN_MOD_SOFTCAP:
+      if (mp == nullptr || !(mp->softcap > 0.f) || !std::isfinite(mp->softcap)) return ATTN_ERR_ARG;
+      break;
+    case ATTN_MOD_SLIDING_WINDOW:
+      if (mp == nullptr || mp->window < 1) return ATTN_ERR_ARG;
+      break;
+    case ATTN_MOD_LOCAL_BOOST:
+      if (mp == nullptr || !std::isfinite(mp->boost) || mp->boost_radius < 0) return ATTN_ERR_ARG;
+      break;
+    case ATTN_MOD_DOCUMENT:
+      if (mp == nullptr || mp->doc_offsets == nullptr || mp->num_docs < 1 || mp->num_docs > 4096)
+        return ATTN_ERR_ARG;
+      if (Sq != Skv) return ATTN_ERR_UNSUPPORTED;
+      if (!aligned16(mp->doc_offsets) && (reinterpret_cast<uintptr_t>(mp->doc_offsets) & 3u))
+        return ATTN_ERR_ALIGN;
+      break;
+    case ATTN_MOD_ALIBI:
+      if (mp != nullptr && mp->alibi_slopes != nullptr &&
+          (reinterpret_cast<uintptr_t>(mp->alibi_slopes) & 3u))
+        return ATTN_ERR_ALIGN;
+      break;
+    default:
+      break;
+  }
+  if (bm != nullptr) {
+    if (bm->tile_class == nullptr || bm->kv_count == nullptr || bm->kv_index == nullptr ||
+        bm->q_count == nullptr || bm->q_index == nullptr || bm->fwd_order == nullptr ||
+        bm->bwd_order == nullptr)
+      return ATTN_ERR_ARG;
+    if (bm->B != B || bm->Sq != Sq || bm->Skv != Skv || bm->nq_tiles != cdiv(Sq, TILE) ||
+        bm->nk_tiles != cdiv(Skv, TILE) || bm->mod_kind != mod_kind)
+      return ATTN_ERR_ARG;
+  }
+  return ATTN_OK;
+}
+
+ModDev make_mod(int mod_kind, const attn_mod_params* mp) {
+  ModDev m{};
+  m.kind = mod_kind;
+  if (mp != nullptr) {
+    m.softcap = mp->softcap;
+    m.window = mp->window;
+    m.boost = mp->boost;
+    m.boost_radius = mp->boost_radius;
+    m.alibi_slopes = mp->alibi_slopes;
+    m.doc_offsets = mp->doc_offsets;
+    m.num_docs = mp->num_docs;
+  }
+  if (mod_kind != ATTN_MOD_SLIDING_WINDOW) m.window = 1 << 30;
+  return m;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct MaskLayout {
+  size_t off[7];
+  size_t total;
+};
+
+MaskLayout mask_layout(int B, int Sq, int Skv) {
+  const size_t nQ = cdiv(Sq, TILE), nK = cdiv(Skv, TILE), nP = (nQ + 1) / 2;
+  const size_t sizes[7] = {B * nQ * nK,      B * nQ * 4, B * nQ * nK * 4, B * nK * 4,
+                           B * nK * nQ * 4, B * nP * 4, B * nK * 4};
+  MaskLayout L;
+  size_t o = 0;
+  for (int i = 0; i < 7; ++i) {
+    L.off[i] = o;
+    o += align256(sizes[i]);
+  }
+  L.total = o;
+  return L;
+}
+
+}  // namespace
+
+}  // namespace attn25
+
+using namespace attn25;
+
+extern "C" {
+
+const char* attn_strerror(int status) {
+  switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case ATTN_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case ATTN_ERR_WORKSPACE: return "workspace or mask buffer too small";
+    case ATTN_ERR_LAUNCH: return "CUDA launch failed";
+    case ATTN_ERR_TIMEOUT: return "kernel timed out waiting on an internal barrier";
+    case ATTN_ERR_DEVICE: return "no usable sm_100 device";
+    default: return "unknown status";
+  }
+}
+
+void attn_set_wait_limit_ms(uint32_t ms) { g_wait_ms.store(ms < 1 ? 1 : ms); }
+
+int attn_get_status(attn_stream_t stream) {
+  DeviceInfo* d = nullptr;
+  int rc = current_device(&d);
+  if (rc != ATTN_OK) return rc;
+  int value = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&value, d->status, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return ATTN_ERR_LAUNCH;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_LAUNCH;
+  if (value != 0) {
+    const int zero = 0;
+    cudaMemcpyAsync(d->status, &zero, sizeof(int), cudaMemcpyHostToDevice, s);
+    cudaStreamSynchronize(s);
+  }
+  return value;
+}
+
+size_t attn_block_mask_bytes(int B, int Sq, int Skv) {
+  if (B < 1 || Sq < 1 || Skv < 1) return 0;
+  return mask_layout(B, Sq, Skv).total;
+}
+
+int attn_block_mask_bind(void* buffer, size_t bytes, int B, int Sq, int Skv,
+                         attn_block_mask* out) {
+  if (buffer == nullptr || out == nullptr || B < 1 || Sq < 1 || Skv < 1) return ATTN_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(buffer) & 255u) return ATTN_ERR_ALIGN;
+  const MaskLayout L = mask_layout(B, Sq, Skv);
+  if (bytes < L.total) return ATTN_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(buffer);
+  out->tile_class = base + L.off[0];
+  out->kv_count = reinterpret_cast<int32_t*>(base + L.off[1]);
+  out->kv_index = reinterpret_cast<int32_t*>(base + L.off[2]);
+  out->q_count = reinterpret_cast<int32_t*>(base + L.off[3]);
+  out->q_index = reinterpret_cast<int32_t*>(base + L.off[4]);
+  out->fwd_order = reinterpret_cast<int32_t*>(base + L.off[5]);
+  out->bwd_order = reinterpret_cast<int32_t*>(base + L.off[6]);
+  out->B = B;
+  out->Sq = Sq;
+  out->Skv = Skv;
+  out->nq_tiles = cdiv(Sq, TILE);
+  out->nk_tiles = cdiv(Skv, TILE);
+  out->mod_kind = -1;
+  return ATTN_OK;
+}
+
+int build_block_mask(int mod_kind, const attn_mod_params* mod_params, int B, int Sq, int Skv,
+                     attn_block_mask* mask, attn_stream_t stream) {
+  if (mask == nullptr) return ATTN_ERR_ARG;
+  if (mask->tile_class == nullptr || mask->B != B || mask->Sq != Sq || mask->Skv != Skv)
+    return ATTN_ERR_ARG;
+  int rc = check_common(B, 1, 1, Sq, Skv, 64, 1.f, mod_kind, mod_params, nullptr);
+  if (rc != ATTN_OK) return rc;
+  DeviceInfo* d = nullptr;
+  rc = current_device(&d);
+  if (rc != ATTN_OK) return rc;
+  MaskArgs a{};
+  a.kind = mod_kind;
+  a.window = (mod_kind == ATTN_MOD_SLIDING_WINDOW) ? mod_params->window : (1 << 30);
+  a.doc_offsets = (mod_kind == ATTN_MOD_DOCUMENT) ? mod_params->doc_offsets : nullptr;
+  a.num_docs = (mod_kind == ATTN_MOD_DOCUMENT) ? mod_params->num_docs : 0;
+  a.B = B;
+  a.Sq = Sq;
+  a.Skv = Skv;
+  a.nQ = cdiv(Sq, TILE);
+  a.nK = cdiv(Skv, TILE);
+  a.nP = (a.nQ + 1) / 2;
+  a.tile_class = mask->tile_class;
+  a.kv_count = mask->kv_count;
+  a.kv_index = mask->kv_index;
+  a.q_count = mask->q_count;
+  a.q_index = mask->q_index;
+  a.fwd_order = mask->fwd_order;
+  a.bwd_order = mask->bwd_order;
+  if (launch_block_mask(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ATTN_ERR_LAUNCH;
+  mask->mod_kind = mod_kind;
+  return ATTN_OK;
+}
+
+int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* out,
+             float* lse, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+             int mod_kind, const attn_mod_params* mod_params, const attn_block_mask* block_mask,
+             attn_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ATTN_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return ATTN_ERR_ALIGN;
+  int rc = check_common(B, Hq, Hkv, Sq, Skv, D, scale, mod_kind, mod_params, block_mask);
+  if (rc != ATTN_OK) return rc;
+  DeviceInfo* d = nullptr;
+  rc = current_device(&d);
+  if (rc != ATTN_OK) return rc;
+
+  CUtensorMap tq, tk, tv;
+  if (!encode_bf16(&tq, q, D, Sq, B * Hq, TILE) || !encode_bf16(&tk, k, D, Skv, B * Hkv, TILE) ||
+      !encode_bf16(&tv, v, D, Skv, B * Hkv, TILE))
+    return ATTN_ERR_ARG;
+
+  FwdArgs a{};
+  a.out = reinterpret_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = Hq / Hkv;
+  a.Sq = Sq;
+  a.Skv = Skv;
+  a.nQ = cdiv(Sq, TILE);
+  a.nK = cdiv(Skv, TILE);
+  a.nP = (a.nQ + 1) / 2;
+  a.n_units = B * a.nP * Hq;
+  a.scale = scale;
+  a.sl2 = scale * LOG2E;
+  a.mod = make_mod(mod_kind, mod_params);
+  if (block_mask != nullptr) {
+    a.tile_class = block_mask->tile_class;
+    a.kv_count = block_mask->kv_count;
+    a.kv_index = block_mask->kv_index;
+    a.fwd_order = block_mask->fwd_order;
+  }
+  a.wait_ns = wait_ns();
+  a.status = d->status;
+  const int grid = a.n_units < d->sms ? a.n_units : d->sms;
+  if (launch_fwd(tq, tk, tv, a, D, mod_kind, lse != nullptr, grid,
+                 reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ATTN_ERR_LAUNCH;
+  return ATTN_OK;
+}
+
+size_t attn_bwd_workspace_size(int B, int Hq, int Sq, int D) {
+  if (B < 1 || Hq < 1 || Sq < 1 || (D != 64 && D != 128)) return 0;
+  const size_t rows = static_cast<size_t>(B) * Hq * (cdiv(Sq, TILE) * TILE);
+  return align256(rows * D * 4) + 2 * align256(rows * 4);
+}
+
+int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* out,
+             const float* lse, const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk, attn_bf16* dv,
+             void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int Sq, int Skv,
+             int D, float scale, int mod_kind, const attn_mod_params* mod_params,
+             const attn_block_mask* block_mask, attn_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr ||
+      dout == nullptr || dq == nullptr || dk == nullptr || dv == nullptr || workspace == nullptr)
+    return ATTN_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return ATTN_ERR_ALIGN;
+  int rc = check_common(B, Hq, Hkv, Sq, Skv, D, scale, mod_kind, mod_params, block_mask);
+  if (rc != ATTN_OK) return rc;
+  if (workspace_bytes < attn_bwd_workspace_size(B, Hq, Sq, D)) return ATTN_ERR_WORKSPACE;
+  DeviceInfo* d = nullptr;
+  rc = current_device(&d);
+  if (rc != ATTN_OK) return rc;
+
+  const int Sq_pad = cdiv(Sq, TILE) * TILE;
+  const size_t rows = static_cast<size_t>(B) * Hq * Sq_pad;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  BwdArgs a{};
+  a.out = reinterpret_cast<const __nv_bfloat16*>(out);
+  a.dout = reinterpret_cast<const __nv_bfloat16*>(dout);
+  a.lse = lse;
+  a.dq_acc = reinterpret_cast<float*>(ws);
+  a.lse2 = reinterpret_cast<float*>(ws + align256(rows * D * 4));
+  a.delta = reinterpret_cast<float*>(ws + align256(rows * D * 4) + align256(rows * 4));
+  a.dq = reinterpret_cast<__nv_bfloat16*>(dq);
+  a.dk = reinterpret_cast<__nv_bfloat16*>(dk);
+  a.dv = reinterpret_cast<__nv_bfloat16*>(dv);
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = Hq / Hkv;
+  a.Sq = Sq;
+  a.Skv = Skv;
+  a.Sq_pad = Sq_pad;
+  a.nQ = cdiv(Sq, TILE);
+  a.nK = cdiv(Skv, TILE);
+  a.n_units = B * Hkv * a.nK;
+  a.scale = scale;
+  a.sl2 = scale * LOG2E;
+  a.mod = make_mod(mod_kind, mod_params);
+  if (block_mask != nullptr) {
+    a.tile_class = block_mask->tile_class;
+    a.q_count = block_mask->q_count;
+    a.q_index = block_mask->q_index;
+    a.bwd_order = block_mask->bwd_order;
+  }
+  a.wait_ns = wait_ns();
+  a.status = d->status;
+
+  CUtensorMap tq, tk, tv, tdo, tdq;
+  if (!encode_bf16(&tq, q, D, Sq, B * Hq, 64) || !encode_bf16(&tk, k, D, Skv, B * Hkv, TILE) ||
+      !encode_bf16(&tv, v, D, Skv, B * Hkv, TILE) || !encode_bf16(&tdo, dout, D, Sq, B * Hq, 64) ||
+      !encode_f32(&tdq, a.dq_acc, D, Sq_pad, B * Hq, 32, 64))
+    return ATTN_ERR_ARG;
+  const int grid = a.n_units < d->sms ? a.n_units : d->sms;
+  if (launch_bwd(tq, tk, tv, tdo, tdq, a, D, mod_kind, grid,
+                 reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ATTN_ERR_LAUNCH;
+  return ATTN_OK;
+}
+
+}  // extern "C"

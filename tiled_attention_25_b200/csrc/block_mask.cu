@@ -1,0 +1,159 @@
+// Block-mask construction and work ordering (plain CUDA, integer only).
+//
+// Classifies every 128x128 (query tile, key tile) pair as EMPTY / PARTIAL /
+// FULL so that the attention kernels can skip empty KV tiles and run the
+// element predicate only on partial ones ("PyTorch FlexAttention,
+// FlashAttention-4 백엔드 …", 섹션별 상세: block-sparse iteration; "FlashInfer
+// SM120 NVFP4 어텐션 최적화", 코드 분석 4: masking only where the tile needs
+// it).  Every mask of the fixed set keeps an interval of keys [lo(i), hi(i)]
+// per query row, so the kept count of a tile row is a closed-form interval
+// length; summing it over the tile's rows counts kept elements exactly, which
+// is the same classification as testing every element.
+//
+// Then the work orders: query-tile pairs and key tiles sorted longest first
+// (stable counting sort), the longest-processing-time-first order that the
+// persistent kernels walk ("PyTorch FlexAttention, …", 실무 Takeaway: load
+// balance across SMs under data-dependent masks).
+#include <cuda_runtime.h>
+
+#include "launch.h"
+#include "mods.cuh"
+
+namespace attn25 {
+
+namespace {
+
+__device__ __forceinline__ void row_keep_interval(const MaskArgs& a, int b, int i, int& lo,
+                                                  int& hi) {
+  lo = 0;
+  hi = a.Skv - 1;
+  if (a.kind == MOD_CAUSAL) {
+    hi = min(hi, i);
+  } else if (a.kind == MOD_WINDOW) {
+    hi = min(hi, i);
+    lo = max(0, i - a.window + 1);
+  } else if (a.kind == MOD_DOCUMENT) {
+    hi = min(hi, i);
+    lo = doc_start(a.doc_offsets + static_cast<size_t>(b) * (a.num_docs + 1), a.num_docs, i);
+  }
+}
+
+// grid (nQ, B): classify one query-tile row of tiles and write its KV list.
+__global__ void __launch_bounds__(256) classify_kernel(const MaskArgs a) {
+  const int qt = blockIdx.x, b = blockIdx.y;
+  __shared__ int s_lo[TILE], s_hi[TILE];
+  __shared__ uint8_t s_cls[1024];
+  const int q0 = qt * TILE, q1 = min(a.Sq, q0 + TILE);
+  for (int r = threadIdx.x; r < TILE; r += blockDim.x) {
+    int lo = 0, hi = -1;
+    if (q0 + r < q1) row_keep_interval(a, b, q0 + r, lo, hi);
+    s_lo[r] = lo;
+    s_hi[r] = hi;
+  }
+  __syncthreads();
+  const size_t row = static_cast<size_t>(b) * a.nQ + qt;
+  for (int kt = threadIdx.x; kt < a.nK; kt += blockDim.x) {
+    const int k0 = kt * TILE, k1 = min(a.Skv, k0 + TILE);
+    long long kept = 0;
+    for (int r = 0; r < q1 - q0; ++r) {
+      const int lo = max(s_lo[r], k0), hi = min(s_hi[r], k1 - 1);
+      kept += max(0, hi - lo + 1);
+    }
+    const long long total = static_cast<long long>(q1 - q0) * (k1 - k0);
+    const uint8_t c = kept == 0 ? 0 : (kept == total ? 2 : 1);
+    a.tile_class[row * a.nK + kt] = c;
+    if (kt < 1024) s_cls[kt] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int n = 0;
+    int32_t* list = a.kv_index + row * a.nK;
+    for (int kt = 0; kt < a.nK; ++kt) {
+      const uint8_t c = (kt < 1024) ? s_cls[kt] : a.tile_class[row * a.nK + kt];
+      if (c != 0) list[n++] = kt;
+    }
+    a.kv_count[row] = n;
+    for (int kt = n; kt < a.nK; ++kt) list[kt] = -1;
+  }
+}
+
+// grid (nK, B): the transposed lists (query tiles per key tile).
+__global__ void __launch_bounds__(32) transpose_kernel(const MaskArgs a) {
+  const int kt = blockIdx.x, b = blockIdx.y;
+  if (threadIdx.x != 0) return;
+  const size_t col = static_cast<size_t>(b) * a.nK + kt;
+  int32_t* list = a.q_index + col * a.nQ;
+  int n = 0;
+  for (int qt = 0; qt < a.nQ; ++qt)
+    if (a.tile_class[(static_cast<size_t>(b) * a.nQ + qt) * a.nK + kt] != 0) list[n++] = qt;
+  a.q_count[col] = n;
+  for (int qt = n; qt < a.nQ; ++qt) list[qt] = -1;
+}
+
+// One block: costs of the forward pairs and backward units, then a stable
+// counting sort of each by descending cost.
+__global__ void __launch_bounds__(1024) order_kernel(const MaskArgs a) {
+  extern __shared__ int s_hist[];  // max(nQ, nK) + 2 counters
+  const int n_pairs = a.B * a.nP;
+  const int n_units = a.B * a.nK;
+  const int max_cost = a.nQ > a.nK ? a.nQ : a.nK;
+  for (int pass = 0; pass < 2; ++pass) {
+    const int n = pass == 0 ? n_pairs : n_units;
+    int32_t* out = pass == 0 ? a.fwd_order : a.bwd_order;
+    for (int c = threadIdx.x; c <= max_cost + 1; c += blockDim.x) s_hist[c] = 0;
+    __syncthreads();
+    for (int u = threadIdx.x; u < n; u += blockDim.x) {
+      int cost;
+      if (pass == 0) {
+        const int b = u / a.nP, p = u - b * a.nP;
+        const uint8_t* r0 = a.tile_class + (static_cast<size_t>(b) * a.nQ + 2 * p) * a.nK;
+        const bool has1 = 2 * p + 1 < a.nQ;
+        cost = 0;
+        for (int kt = 0; kt < a.nK; ++kt) cost += (r0[kt] != 0 || (has1 && r0[a.nK + kt] != 0));
+      } else {
+        cost = a.q_count[u];
+      }
+      atomicAdd(&s_hist[cost], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      // start position of each cost class, longest first
+      int start = 0;
+      for (int c = max_cost; c >= 0; --c) {
+        const int cnt = s_hist[c];
+        s_hist[c] = start;
+        start += cnt;
+      }
+      // stable placement in ascending unit id
+      for (int u = 0; u < n; ++u) {
+        int cost;
+        if (pass == 0) {
+          const int b = u / a.nP, p = u - b * a.nP;
+          const uint8_t* r0 = a.tile_class + (static_cast<size_t>(b) * a.nQ + 2 * p) * a.nK;
+          const bool has1 = 2 * p + 1 < a.nQ;
+          cost = 0;
+          for (int kt = 0; kt < a.nK; ++kt) cost += (r0[kt] != 0 || (has1 && r0[a.nK + kt] != 0));
+        } else {
+          cost = a.q_count[u];
+        }
+        out[s_hist[cost]++] = u;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_block_mask(const MaskArgs& a, cudaStream_t stream) {
+  classify_kernel<<<dim3(a.nQ, a.B), 256, 0, stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  transpose_kernel<<<dim3(a.nK, a.B), 32, 0, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  order_kernel<<<1, 1024, ((a.nQ > a.nK ? a.nQ : a.nK) + 2) * sizeof(int), stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace attn25

@@ -1,0 +1,767 @@
+// Backward attention kernels for sm_100a.
+//
+// The scores are recomputed from Q, K and the saved logsumexp instead of
+// being stored ("FlashAttention-2 — GPU attention의 사실상 표준", §3
+// Recomputation and §4 Backward).  With s' = mod(scale q.k) and
+// P = exp(s' - LSE), the exact gradient of O = P V is
+//     dV = P^T dO,  dP = dO V^T,  Delta_i = rowsum(dO_i * O_i),
+//     dS = P * (dP - Delta) * ds'/ds,  dQ = scale dS K,  dK = scale dS^T Q.
+//
+// Three kernels run on the stream:
+//   bwd_prep     Delta and LSE * log2(e) per row; zero the fp32 dQ accumulator
+//   bwd_main     persistent over (batch row, KV head, 128-key tile) units
+//   bwd_dq_cast  dQ accumulator * scale -> bf16
+// bwd_main keeps K and V of its key tile in shared memory and dK, dV in
+// tensor memory while it walks every query head of the KV head's group and
+// every non-empty 64-row query sub-tile.  Per step it computes, in the
+// transposed (key-major) orientation so that one thread owns one key row:
+//     S^T = K Q^T,  dP^T = V dO^T               (tcgen05, smem x smem)
+//     P^T, dS^T                                  (4 warps, thread = key row)
+//     dV += P^T dO  (P^T from tensor memory),  dK += dS^T Q,
+//     dQ^T = K^T dS^T                            (tcgen05)
+// and adds dQ into the fp32 accumulator with a TMA reduce-add (the add runs
+// in L2, so the order of the adds, and the last bits of dQ, vary run to run).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "kernel_common.cuh"
+#include "launch.h"
+
+namespace attn25 {
+
+namespace {
+
+constexpr int kBwdThreads = 320;
+constexpr int BM = 64;  // query rows per step
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kKVBytes = TILE * D * 2;           // one 128-key tile of K or V
+  static constexpr int kQBytes = BM * D * 2;              // one 64-row tile of Q or dO
+  static constexpr int kStageBytes = 2 * kQBytes + 1024;  // Q, dO, LSE2 and Delta rows
+  static constexpr int kStages = 2;
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = kKVBytes;
+  static constexpr int kStageOff = 2 * kKVBytes;
+  static constexpr int kDSOff = kStageOff + kStages * kStageBytes;  // two 128 x 64 bf16 buffers
+  static constexpr int kDSBytes = TILE * BM * 2;
+  static constexpr int kStgOff = kDSOff + 2 * kDSBytes;            // dQ staging [D/32][64][32] fp32
+  static constexpr int kStgBytes = BM * D * 4;
+  static constexpr int kBarOff = kStgOff + kStgBytes;
+  static constexpr int kSmemBytes = kBarOff + 1024;
+  static constexpr int kAllocBytes = kSmemBytes + 1024;
+  // TMEM columns
+  static constexpr int kColS = 0, kColDP = 64, kColDV = 128, kColDK = 128 + D, kColDQ = 128 + 2 * D;
+  static constexpr uint32_t kIdescST = idesc_bf16_f32(128, BM, false, false);   // K Q^T, V dO^T
+  static constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, false, true);    // P^T dO, dS^T Q
+  static constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, BM, true, true);     // K^T dS^T
+};
+
+struct BwdBarriers {
+  uint64_t kv_full, kv_empty;
+  uint64_t q_full[2], q_empty[2];
+  uint64_t s_full, dp_full, p_ready, ds_ready;
+  uint64_t ds_empty[2];
+  uint64_t dq_full, dq_empty;
+  uint64_t stg_written, stg_free;
+  uint64_t acc_full, acc_empty;
+  uint64_t drain;
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+struct BwdUnit {
+  int b, hk, kt;
+};
+
+__device__ __forceinline__ BwdUnit decode_bwd_unit(const BwdArgs& a, int u) {
+  const int pair_idx = u / a.Hkv;
+  const int hk = u - pair_idx * a.Hkv;
+  const int pair = (a.bwd_order != nullptr) ? __ldg(a.bwd_order + pair_idx) : pair_idx;
+  BwdUnit r;
+  r.b = pair / a.nK;
+  r.kt = pair - r.b * a.nK;
+  r.hk = hk;
+  return r;
+}
+
+// Walks the steps of one unit: for each query head of the group, each
+// non-EMPTY 128-row query tile (block-mask list or analytic range), and each
+// 64-row half of it that starts inside Sq.
+struct StepIter {
+  const int32_t* list;
+  const uint8_t* cls_col;  // tile_class + b*nQ*nK + kt, stride nK
+  int n_list, nK, nQ, Sq, Skv, kind, window, kt, G;
+  int g, li, half, qt_dense, qt_end;
+  int cur_qt, cur_cls;
+  bool list_mode, tail_kv;
+
+  __device__ void init(const BwdArgs& a, const BwdUnit& u) {
+    nK = a.nK;
+    nQ = a.nQ;
+    Sq = a.Sq;
+    Skv = a.Skv;
+    kind = a.mod.kind;
+    window = a.mod.window;
+    kt = u.kt;
+    G = a.G;
+    g = 0;
+    li = 0;
+    half = 2;  // forces fetching the first query tile
+    tail_kv = (Skv % TILE) != 0 && kt == nK - 1;
+    list_mode = a.tile_class != nullptr;
+    if (list_mode) {
+      const size_t col = static_cast<size_t>(u.b) * nK + kt;
+      list = a.q_index + col * nQ;
+      n_list = __ldg(a.q_count + col);
+      cls_col = a.tile_class + static_cast<size_t>(u.b) * nQ * nK + kt;
+    } else {
+      list = nullptr;
+      cls_col = nullptr;
+      n_list = 0;
+    }
+    qt_dense = 0;
+    qt_end = nQ;
+    if (!list_mode && is_interval_mask(kind)) qt_dense = (kt * TILE) / TILE;
+    li = qt_dense;
+  }
+
+  __device__ __forceinline__ int dense_class(int qt) const {
+    const int q0 = qt * TILE, q1 = min(Sq, q0 + TILE);
+    const int k0 = kt * TILE, k1 = min(Skv, k0 + TILE);
+    if (kind == MOD_CAUSAL || kind == MOD_WINDOW)
+      return interval_tile_class(kind, window, q0, q1, k0, k1);
+    if (kind == MOD_DOCUMENT) return 1;
+    return 2;
+  }
+
+  // Advance to the next query tile (any head); false when the unit is done.
+  __device__ bool next_tile() {
+    while (g < G) {
+      if (list_mode) {
+        if (li < n_list) {
+          cur_qt = __ldg(list + li);
+          cur_cls = __ldg(cls_col + static_cast<size_t>(cur_qt) * nK);
+          ++li;
+          return true;
+        }
+      } else {
+        while (li < qt_end) {
+          const int qt = li++;
+          const int c = dense_class(qt);
+          if (c != 0) {
+            cur_qt = qt;
+            cur_cls = c;
+            return true;
+          }
+        }
+      }
+      ++g;
+      li = list_mode ? 0 : qt_dense;
+    }
+    return false;
+  }
+
+  // Next step: head offset g_out in the group, first query row q0, and
+  // whether the element predicate is needed.
+  __device__ bool next(int& g_out, int& q0, bool& pred) {
+    while (true) {
+      if (half >= 2) {
+        if (!next_tile()) return false;
+        half = 0;
+      }
+      const int h = half++;
+      const int start = cur_qt * TILE + h * BM;
+      if (start >= Sq) continue;
+      g_out = g;
+      q0 = start;
+      pred = (cur_cls == 1) || tail_kv;
+      return true;
+    }
+  }
+};
+
+template <int D>
+__device__ __forceinline__ void load_kv_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                             int row0, int bh) {
+#pragma unroll
+  for (int c = 0; c < D / 64; ++c) tma_load_3d(dst + c * (TILE * 128), map, bar, c * 64, row0, bh);
+}
+
+template <int D>
+__device__ __forceinline__ void load_q_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int row0, int bh) {
+#pragma unroll
+  for (int c = 0; c < D / 64; ++c) tma_load_3d(dst + c * (BM * 128), map, bar, c * 64, row0, bh);
+}
+
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes,
+                                             uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// A (M=128 rows) x B^T with both operands K-major, 128-byte swizzle; the
+// M-side tile has 128 rows (chunk stride 16 KB), the N-side 64 rows (8 KB).
+template <int D>
+__device__ __forceinline__ void issue_st(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t ka = (kk >> 2) * (TILE * 128) + (kk & 3) * 32;
+    const uint32_t kb = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+    mma_ss(d_tmem, smem_desc_sw128(a_smem + ka, 16, 1024), smem_desc_sw128(b_smem + kb, 16, 1024),
+           BwdCfg<D>::kIdescST, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+struct BwdRow {
+  int kv;        // absolute key row of this thread
+  int qlo, qhi;  // kept query interval of this key (transposed mask)
+  float sl2, aux, aux2, dmod_in;
+};
+
+template <int D, int MOD>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_dq, const BwdArgs a) {
+  using Cfg = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  BwdBarriers* bars = reinterpret_cast<BwdBarriers*>(smem + Cfg::kBarOff);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t k_smem = sbase + Cfg::kKOff;
+  const uint32_t v_smem = sbase + Cfg::kVOff;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->kv_full), 1);
+    mbar_init(smem_u32(&bars->kv_empty), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&bars->q_full[s]), 1);
+      mbar_init(smem_u32(&bars->q_empty[s]), 1);
+      mbar_init(smem_u32(&bars->ds_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&bars->s_full), 1);
+    mbar_init(smem_u32(&bars->dp_full), 1);
+    mbar_init(smem_u32(&bars->p_ready), 128);
+    mbar_init(smem_u32(&bars->ds_ready), 128);
+    mbar_init(smem_u32(&bars->dq_full), 1);
+    mbar_init(smem_u32(&bars->dq_empty), 128);
+    mbar_init(smem_u32(&bars->stg_written), 128);
+    mbar_init(smem_u32(&bars->stg_free), 1);
+    mbar_init(smem_u32(&bars->acc_full), 1);
+    mbar_init(smem_u32(&bars->acc_empty), 128);
+    mbar_init(smem_u32(&bars->drain), 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_relinquish();
+  }
+  if (warp == 9 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_dq);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const WaitCtl wc{a.wait_ns, &bars->abort_flag, a.status};
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int unit_iter = 0, step = 0;
+      uint32_t kv_loads = 0, stage_uses[2] = {0, 0};
+      bool ok = true;
+      for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+        const BwdUnit un = decode_bwd_unit(a, u);
+        if (!mbar_wait_thread(smem_u32(&bars->kv_empty), (unit_iter & 1) ^ 1, wc)) { ok = false; break; }
+        mbar_arrive_expect_tx(smem_u32(&bars->kv_full), 2 * Cfg::kKVBytes);
+        ++kv_loads;
+        const int bh_kv = un.b * a.Hkv + un.hk;
+        load_kv_tile<D>(k_smem, &tm_k, smem_u32(&bars->kv_full), un.kt * TILE, bh_kv);
+        load_kv_tile<D>(v_smem, &tm_v, smem_u32(&bars->kv_full), un.kt * TILE, bh_kv);
+        StepIter it;
+        it.init(a, un);
+        int g, q0;
+        bool pred;
+        while (it.next(g, q0, pred)) {
+          const int s = step & 1;
+          if (!mbar_wait_thread(smem_u32(&bars->q_empty[s]), ((step >> 1) & 1) ^ 1, wc)) { ok = false; break; }
+          const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
+          const uint32_t bar = smem_u32(&bars->q_full[s]);
+          mbar_arrive_expect_tx(bar, 2 * Cfg::kQBytes + 2 * BM * 4);
+          ++stage_uses[s];
+          const int bh = un.b * a.Hq + un.hk * a.G + g;
+          load_q_tile<D>(st, &tm_q, bar, q0, bh);
+          load_q_tile<D>(st + Cfg::kQBytes, &tm_do, bar, q0, bh);
+          const size_t row = static_cast<size_t>(bh) * a.Sq_pad + q0;
+          bulk_load_1d(st + 2 * Cfg::kQBytes, a.lse2 + row, BM * 4, bar);
+          bulk_load_1d(st + 2 * Cfg::kQBytes + 512, a.delta + row, BM * 4, bar);
+          ++step;
+        }
+      }
+      if (!ok) {
+        uint32_t local_flag = 0;
+        const WaitCtl dwc{a.wait_ns, &local_flag, a.status};
+        if (kv_loads) mbar_wait_thread(smem_u32(&bars->kv_full), (kv_loads - 1) & 1, dwc);
+        for (int s = 0; s < 2; ++s)
+          if (stage_uses[s]) mbar_wait_thread(smem_u32(&bars->q_full[s]), (stage_uses[s] - 1) & 1, dwc);
+      }
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t t_s = tmem + Cfg::kColS, t_dp = tmem + Cfg::kColDP;
+    const uint32_t t_dv = tmem + Cfg::kColDV, t_dk = tmem + Cfg::kColDK, t_dq = tmem + Cfg::kColDQ;
+    int unit_iter = 0, step = 0;
+    uint32_t p_cnt = 0, ds_cnt = 0, dq_cnt = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+      const BwdUnit un = decode_bwd_unit(a, u);
+      if (!mbar_wait_warp(smem_u32(&bars->kv_full), unit_iter & 1, wc)) { ok = false; break; }
+      // dK, dV accumulators are free once the previous unit's epilogue read them
+      if (!mbar_wait_warp(smem_u32(&bars->acc_empty), (unit_iter & 1) ^ 1, wc)) { ok = false; break; }
+      tc_fence_after();
+      StepIter it;
+      it.init(a, un);
+      int g, q0;
+      bool pred;
+      bool has = it.next(g, q0, pred);
+      int n_steps = 0;
+      // prologue: S^T and dP^T of the first step
+      if (has) {
+        const int s = step & 1;
+        if (!mbar_wait_warp(smem_u32(&bars->q_full[s]), (step >> 1) & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
+        if (lane == 0) {
+          issue_st<D>(t_s, k_smem, st);
+          mma_commit(smem_u32(&bars->s_full));
+          issue_st<D>(t_dp, v_smem, st + Cfg::kQBytes);
+          mma_commit(smem_u32(&bars->dp_full));
+        }
+        __syncwarp();
+      }
+      while (has) {
+        const int s = step & 1;
+        const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
+        // dV += P^T dO once the probabilities are in tensor memory
+        if (!mbar_wait_warp(smem_u32(&bars->p_ready), p_cnt & 1, wc)) { ok = false; break; }
+        ++p_cnt;
+        tc_fence_after();
+        if (lane == 0) {
+#pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk)
+            mma_ts(t_dv, t_s + kk * 8, smem_desc_sw128(st + Cfg::kQBytes + kk * 2048, BM * 128, 1024),
+                   Cfg::kIdescAcc, (n_steps > 0 || kk > 0) ? 1u : 0u);
+        }
+        __syncwarp();
+        int g_n, q0_n;
+        bool pred_n;
+        const bool has_n = it.next(g_n, q0_n, pred_n);
+        const int s_n = (step + 1) & 1;
+        const uint32_t st_n = sbase + Cfg::kStageOff + s_n * Cfg::kStageBytes;
+        if (has_n) {  // S^T of the next step overlaps this step's dS work
+          if (!mbar_wait_warp(smem_u32(&bars->q_full[s_n]), ((step + 1) >> 1) & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+          if (lane == 0) {
+            issue_st<D>(t_s, k_smem, st_n);
+            mma_commit(smem_u32(&bars->s_full));
+          }
+          __syncwarp();
+        }
+        // dK += dS^T Q and dQ^T = K^T dS^T once dS^T is in shared memory
+        if (!mbar_wait_warp(smem_u32(&bars->ds_ready), ds_cnt & 1, wc)) { ok = false; break; }
+        const uint32_t ds_smem = sbase + Cfg::kDSOff + (ds_cnt & 1) * Cfg::kDSBytes;
+        ++ds_cnt;
+        // the dQ^T columns must have been drained by the previous step
+        if (!mbar_wait_warp(smem_u32(&bars->dq_empty), (dq_cnt & 1) ^ 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        if (lane == 0) {
+#pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk)
+            mma_ss(t_dk, smem_desc_sw128(ds_smem + kk * 32, 16, 1024),
+                   smem_desc_sw128(st + kk * 2048, BM * 128, 1024), Cfg::kIdescAcc,
+                   (n_steps > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < TILE / 16; ++kk)
+            mma_ss(t_dq, smem_desc_sw128(k_smem + kk * 2048, TILE * 128, 1024),
+                   smem_desc_sw128(ds_smem + kk * 2048, BM * 128, 1024), Cfg::kIdescDQ,
+                   kk > 0 ? 1u : 0u);
+          mma_commit(smem_u32(&bars->dq_full));
+          mma_commit(smem_u32(&bars->q_empty[s]));
+          mma_commit(smem_u32(&bars->ds_empty[(ds_cnt - 1) & 1]));
+          if (has_n) {
+            issue_st<D>(t_dp, v_smem, st_n + Cfg::kQBytes);
+            mma_commit(smem_u32(&bars->dp_full));
+          }
+        }
+        __syncwarp();
+        ++dq_cnt;
+        ++n_steps;
+        ++step;
+        has = has_n;
+        g = g_n;
+        q0 = q0_n;
+        pred = pred_n;
+      }
+      if (!ok) break;
+      if (lane == 0) {
+        mma_commit(smem_u32(&bars->kv_empty));
+        mma_commit(smem_u32(&bars->acc_full));
+      }
+      __syncwarp();
+    }
+    if (lane == 0) {
+      mma_commit(smem_u32(&bars->drain));
+      uint32_t local_flag = 0;
+      mbar_wait_thread(smem_u32(&bars->drain), 0, WaitCtl{a.wait_ns, &local_flag, a.status});
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ P^T / dS^T (thread = key row)
+    const int r = threadIdx.x;  // TMEM lane = key row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t t_s = tmem + Cfg::kColS + lane_off, t_dp = tmem + Cfg::kColDP + lane_off;
+    const uint32_t t_dv = tmem + Cfg::kColDV + lane_off, t_dk = tmem + Cfg::kColDK + lane_off;
+    int unit_iter = 0, step = 0;
+    uint32_t s_cnt = 0, dp_cnt = 0, ds_cnt = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+      const BwdUnit un = decode_bwd_unit(a, u);
+      const int kv = un.kt * TILE + r;
+      // kept query interval of this key: transposed form of the row intervals
+      int qlo = 0, qhi = a.Sq - 1;
+      if constexpr (MOD == MOD_CAUSAL) {
+        qlo = kv;
+      } else if constexpr (MOD == MOD_WINDOW) {
+        qlo = kv;
+        qhi = min(qhi, kv + a.mod.window - 1);
+      } else if constexpr (MOD == MOD_DOCUMENT) {
+        qlo = kv;
+        const int32_t* offs = a.mod.doc_offsets + static_cast<size_t>(un.b) * (a.mod.num_docs + 1);
+        const int kvc = min(kv, a.Skv - 1);
+        int lo = 0, hi = a.mod.num_docs;  // find the document end after kvc
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (__ldg(offs + mid) <= kvc) lo = mid; else hi = mid;
+        }
+        qhi = min(qhi, __ldg(offs + lo + 1) - 1);
+      }
+      if (kv >= a.Skv) qhi = qlo - 1;  // key rows past the end keep nothing
+      StepIter it;
+      it.init(a, un);
+      int g, q0;
+      bool pred;
+      int n_steps = 0;
+      while (it.next(g, q0, pred)) {
+        const int s = step & 1;
+        const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
+        const float* lse2_s = reinterpret_cast<const float*>(smem + Cfg::kStageOff + s * Cfg::kStageBytes + 2 * Cfg::kQBytes);
+        const float* delta_s = lse2_s + 128;
+        // stage contents (Q, dO, statistics) have landed
+        if (!mbar_wait_warp(smem_u32(&bars->q_full[s]), (step >> 1) & 1, wc)) { ok = false; break; }
+        if (!mbar_wait_warp(smem_u32(&bars->s_full), s_cnt & 1, wc)) { ok = false; break; }
+        ++s_cnt;
+        tc_fence_after();
+        const int h = un.hk * a.G + g;
+        float sl2 = a.sl2, aux = 0.f, aux2 = 0.f;
+        if constexpr (MOD == MOD_ALIBI) aux = alibi_slope(a.mod, h, a.Hq) * LOG2E;
+        if constexpr (MOD == MOD_SOFTCAP) {
+          aux = a.scale / a.mod.softcap;
+          aux2 = a.mod.softcap * LOG2E;
+        }
+        if constexpr (MOD == MOD_BOOST) aux = a.mod.boost * a.sl2;
+        float x[BM];
+        tmem_ld32(t_s, reinterpret_cast<uint32_t(&)[32]>(x[0]));
+        tmem_ld32(t_s + 32, reinterpret_cast<uint32_t(&)[32]>(x[32]));
+        tmem_wait_ld();
+        const float dq0 = static_cast<float>(q0 - kv);  // (query - key) of column 0
+        // softcap: d s'/d s = 1 - tanh^2, kept as fp16 pairs to save registers
+        __half2 dcap[MOD == MOD_SOFTCAP ? BM / 2 : 1];
+        (void)dcap;
+#pragma unroll
+        for (int c = 0; c < BM; ++c) {
+          float v = x[c];
+          if constexpr (MOD == MOD_ALIBI) {
+            v = fmaf(v, sl2, -aux * fabsf(dq0 + static_cast<float>(c)));
+          } else if constexpr (MOD == MOD_SOFTCAP) {
+            const float t = tanhf(v * aux);
+            if (c & 1) dcap[c >> 1].y = __float2half_rn(1.f - t * t);
+            else dcap[c >> 1].x = __float2half_rn(1.f - t * t);
+            v = aux2 * t;
+          } else if constexpr (MOD == MOD_BOOST) {
+            const bool inside = fabsf(dq0 + static_cast<float>(c)) < static_cast<float>(a.mod.boost_radius);
+            v = v * (inside ? aux : sl2);
+          } else {
+            v = v * sl2;
+          }
+          if (pred) {
+            const int qq = q0 + c;
+            v = (qq >= qlo && qq <= qhi) ? v : -INFINITY;
+          }
+          x[c] = ex2_approx(v - lse2_s[c]);  // P^T, 0 where masked
+        }
+        // P^T (bf16 pairs) over the first 32 columns of S^T
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+        tmem_st32(t_s, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&bars->p_ready));
+        // dS^T = P^T (dP^T - Delta) ds'/ds
+        if (!mbar_wait_warp(smem_u32(&bars->dp_full), dp_cnt & 1, wc)) { ok = false; break; }
+        ++dp_cnt;
+        tc_fence_after();
+        float dp[BM];
+        tmem_ld32(t_dp, reinterpret_cast<uint32_t(&)[32]>(dp[0]));
+        tmem_ld32(t_dp + 32, reinterpret_cast<uint32_t(&)[32]>(dp[32]));
+        tmem_wait_ld();
+        // the dS buffer is free once the MMAs of two steps ago completed
+        if (!mbar_wait_warp(smem_u32(&bars->ds_empty[ds_cnt & 1]), ((ds_cnt >> 1) & 1) ^ 1, wc)) { ok = false; break; }
+        uint8_t* ds_row = smem + Cfg::kDSOff + (ds_cnt & 1) * Cfg::kDSBytes + r * 128;
+        ++ds_cnt;
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16) {  // 8 columns (16 bytes) at a time
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = c16 * 8 + 2 * e;
+            float d0 = x[c] * (dp[c] - delta_s[c]);
+            float d1 = x[c + 1] * (dp[c + 1] - delta_s[c + 1]);
+            if constexpr (MOD == MOD_SOFTCAP) {
+              d0 *= __low2float(dcap[c >> 1]);
+              d1 *= __high2float(dcap[c >> 1]);
+            } else if constexpr (MOD == MOD_BOOST) {
+              const float rad = static_cast<float>(a.mod.boost_radius);
+              d0 *= fabsf(dq0 + static_cast<float>(c)) < rad ? a.mod.boost : 1.f;
+              d1 *= fabsf(dq0 + static_cast<float>(c + 1)) < rad ? a.mod.boost : 1.f;
+            }
+            w[e] = pack_bf16x2(d0, d1);
+          }
+          // 128-byte swizzle: 16-byte chunk c16 of row r lands at chunk c16 ^ (r % 8)
+          *reinterpret_cast<uint4*>(ds_row + ((c16 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&bars->ds_ready));
+        ++n_steps;
+        ++step;
+      }
+      if (!ok) break;
+      // ---- unit epilogue: dV, scale * dK -> bf16
+      if (!mbar_wait_warp(smem_u32(&bars->acc_full), unit_iter & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+      const bool row_ok = kv < a.Skv;
+      const size_t row = (static_cast<size_t>(un.b) * a.Hkv + un.hk) * a.Skv + kv;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        __nv_bfloat16* dst = (which == 0 ? a.dv : a.dk) + row * D;
+        const float mul = which == 0 ? 1.f : a.scale;
+        const uint32_t src = which == 0 ? t_dv : t_dk;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          if (n_steps > 0) {
+            tmem_ld32(src + c * 32, o);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = 0u;
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * mul, __uint_as_float(o[2 * e + 1]) * mul);
+          if (row_ok) {
+            uint4* p = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) p[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bars->acc_empty));
+    }
+  } else {
+    // ------------------------------------------------------------ dQ drain (thread = head-dim lane)
+    const int w = warp - 4;      // TMEM lane quarter = 32-column block of D
+    const uint32_t lane_off = static_cast<uint32_t>(w * 32) << 16;
+    const uint32_t t_dq = tmem + Cfg::kColDQ + lane_off;
+    const bool active = w * 32 < D;
+    float* stg = reinterpret_cast<float*>(smem + Cfg::kStgOff) + w * (BM * 32);
+    int unit_iter = 0;
+    uint32_t dq_cnt = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+      const BwdUnit un = decode_bwd_unit(a, u);
+      StepIter it;
+      it.init(a, un);
+      int g, q0;
+      bool pred;
+      while (it.next(g, q0, pred)) {
+        if (!mbar_wait_warp(smem_u32(&bars->dq_full), dq_cnt & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        float v[BM];
+        tmem_ld32(t_dq, reinterpret_cast<uint32_t(&)[32]>(v[0]));
+        tmem_ld32(t_dq + 32, reinterpret_cast<uint32_t(&)[32]>(v[32]));
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&bars->dq_empty));
+        // staging is free once the previous reduce has read it
+        if (!mbar_wait_warp(smem_u32(&bars->stg_free), (dq_cnt & 1) ^ 1, wc)) { ok = false; break; }
+        if (active) {
+#pragma unroll
+          for (int c = 0; c < BM; ++c) stg[c * 32 + lane] = v[c];
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(smem_u32(&bars->stg_written));
+        if (threadIdx.x == 128) {
+          if (!mbar_wait_thread(smem_u32(&bars->stg_written), dq_cnt & 1, wc)) {
+            ok = false;
+          } else {
+            const int bh = un.b * a.Hq + un.hk * a.G + g;
+            for (int c = 0; c < D / 32; ++c)
+              tma_reduce_add_3d(&tm_dq, sbase + Cfg::kStgOff + c * (BM * 32 * 4), c * 32, q0, bh);
+            bulk_commit();
+            bulk_wait_read_all();
+            mbar_arrive(smem_u32(&bars->stg_free));
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 && ok;
+        ++dq_cnt;
+        if (!ok) break;
+      }
+    }
+    if (threadIdx.x == 128) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 8) tmem_dealloc(tmem, 512);
+}
+
+// Delta_i = sum_d dO_id O_id, LSE2_i = LSE_i log2(e) (+inf where the row kept
+// nothing or lies past Sq), and zero the fp32 dQ accumulator.  One warp per row.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
+  const long long total_rows = static_cast<long long>(a.B) * a.Hq * a.Sq_pad;
+  const int lane = threadIdx.x & 31;
+  for (long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+       row < total_rows; row += (static_cast<long long>(gridDim.x) * blockDim.x) >> 5) {
+    const long long bh = row / a.Sq_pad;
+    const int q = static_cast<int>(row - bh * a.Sq_pad);
+    float acc = 0.f;
+    if (q < a.Sq) {
+      const size_t base = (static_cast<size_t>(bh) * a.Sq + q) * D;
+      for (int d = lane * 2; d < D; d += 64) {
+        const __nv_bfloat162 o2 = *reinterpret_cast<const __nv_bfloat162*>(a.out + base + d);
+        const __nv_bfloat162 g2 = *reinterpret_cast<const __nv_bfloat162*>(a.dout + base + d);
+        acc = fmaf(__bfloat162float(o2.x), __bfloat162float(g2.x), acc);
+        acc = fmaf(__bfloat162float(o2.y), __bfloat162float(g2.y), acc);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    float4* z = reinterpret_cast<float4*>(a.dq_acc + static_cast<size_t>(row) * D);
+    for (int i = lane; i < D / 4; i += 32) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (lane == 0) {
+      float l2 = INFINITY;
+      if (q < a.Sq) {
+        const float l = a.lse[static_cast<size_t>(bh) * a.Sq + q];
+        l2 = (l == -INFINITY) ? INFINITY : l * LOG2E;
+      }
+      a.lse2[row] = l2;
+      a.delta[row] = q < a.Sq ? acc : 0.f;
+    }
+  }
+}
+
+// dQ = scale * accumulator, rounded to bf16; 8 elements per thread.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dq_cast_kernel(const BwdArgs a) {
+  const long long n8 = static_cast<long long>(a.B) * a.Hq * a.Sq * (D / 8);
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long e = i * 8;
+    const long long row = e / D;
+    const int d = static_cast<int>(e - row * D);
+    const long long bh = row / a.Sq;
+    const int q = static_cast<int>(row - bh * a.Sq);
+    const float4* src = reinterpret_cast<const float4*>(a.dq_acc + (static_cast<size_t>(bh) * a.Sq_pad + q) * D + d);
+    const float4 x0 = src[0], x1 = src[1];
+    uint4 o;
+    o.x = pack_bf16x2(x0.x * a.scale, x0.y * a.scale);
+    o.y = pack_bf16x2(x0.z * a.scale, x0.w * a.scale);
+    o.z = pack_bf16x2(x1.x * a.scale, x1.y * a.scale);
+    o.w = pack_bf16x2(x1.z * a.scale, x1.w * a.scale);
+    *reinterpret_cast<uint4*>(a.dq + e) = o;
+  }
+}
+
+template <int D, int MOD>
+cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int grid,
+                         cudaStream_t stream) {
+  const long long rows = static_cast<long long>(a.B) * a.Hq * a.Sq_pad;
+  int prep_blocks = static_cast<int>((rows * 32 + 255) / 256);
+  if (prep_blocks > 148 * 16) prep_blocks = 148 * 16;
+  bwd_prep_kernel<D><<<prep_blocks, 256, 0, stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  auto kernel = attn_bwd_kernel<D, MOD>;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg<D>::kAllocBytes);
+  if (e != cudaSuccess) return e;
+  kernel<<<grid, kBwdThreads, BwdCfg<D>::kAllocBytes, stream>>>(tq, tk, tv, tdo, tdq, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long n8 = static_cast<long long>(a.B) * a.Hq * a.Sq * (D / 8);
+  int cast_blocks = static_cast<int>((n8 + 255) / 256);
+  if (cast_blocks > 148 * 16) cast_blocks = 148 * 16;
+  bwd_dq_cast_kernel<D><<<cast_blocks, 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_bwd_mod(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int mod,
+                           int grid, cudaStream_t s) {
+  switch (mod) {
+    case MOD_NONE: return launch_bwd_t<D, MOD_NONE>(tq, tk, tv, tdo, tdq, a, grid, s);
+    case MOD_CAUSAL: return launch_bwd_t<D, MOD_CAUSAL>(tq, tk, tv, tdo, tdq, a, grid, s);
+    case MOD_ALIBI: return launch_bwd_t<D, MOD_ALIBI>(tq, tk, tv, tdo, tdq, a, grid, s);
+    case MOD_SOFTCAP: return launch_bwd_t<D, MOD_SOFTCAP>(tq, tk, tv, tdo, tdq, a, grid, s);
+    case MOD_WINDOW: return launch_bwd_t<D, MOD_WINDOW>(tq, tk, tv, tdo, tdq, a, grid, s);
+    case MOD_BOOST: return launch_bwd_t<D, MOD_BOOST>(tq, tk, tv, tdo, tdq, a, grid, s);
+    case MOD_DOCUMENT: return launch_bwd_t<D, MOD_DOCUMENT>(tq, tk, tv, tdo, tdq, a, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int D,
+                       int mod, int grid, cudaStream_t stream) {
+  if (D == 128) return launch_bwd_mod<128>(tq, tk, tv, tdo, tdq, a, mod, grid, stream);
+  if (D == 64) return launch_bwd_mod<64>(tq, tk, tv, tdo, tdq, a, mod, grid, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace attn25

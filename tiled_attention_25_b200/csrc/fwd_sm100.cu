@@ -1,0 +1,540 @@
+// Forward attention kernel for sm_100a.
+//
+// One persistent CTA per SM walks work units (batch row, query head, pair of
+// 128-row query tiles).  Warp roles:
+//   warps 0-3  softmax for query tile 0 of the pair (thread = query row)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    MMA issuer (one thread issues tcgen05.mma)
+//   warp  9    TMA producer
+// Scores S_t = Q_t K^T accumulate in tensor memory (TMEM), the softmax warps
+// read them with tcgen05.ld, write the bf16 probabilities P_t back over S_t,
+// and O_t += P_t V runs with P_t taken straight from TMEM.  The two query
+// tiles ping-pong: while one tile's softmax runs, the tensor core works on the
+// other tile's products (the ping-pong pipeline of "PyTorch FlexAttention,
+// FlashAttention-4 백엔드 …", 섹션별 상세, and the warp-specialised
+// producer/consumer split of "FlashAttention-3 (KO)", 비동기 실행 및 워프 특화).
+//
+// Online softmax ("FlashAttention 설명", §5; "FlashAttention-2 …", §4): per
+// row a running maximum m, running sum l and the accumulator O in TMEM.  The
+// running maximum is only moved when a new score exceeds it by more than
+// 2^8 (in the base-2 domain), and only then is O rescaled; otherwise the
+// stale maximum stays the reference.  Every term keeps the same reference,
+// so O / l is unchanged while rescales become rare.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kernel_common.cuh"
+#include "launch.h"
+
+namespace attn25 {
+
+namespace {
+
+constexpr int kFwdThreads = 320;
+constexpr float kRescaleThreshold = 8.0f;
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kTileBytes = TILE * D * 2;           // one 128 x D bf16 tile
+  static constexpr int kStages = (D == 128) ? 4 : 6;        // K/V ring slots
+  static constexpr int kQOff = 0;                           // Q0, Q1
+  static constexpr int kRingOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
+  static constexpr int kSmemBytes = kBarOff + 1024;         // + barriers, flags
+  static constexpr int kAllocBytes = kSmemBytes + 1024;     // + alignment slack
+  static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
+  static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);
+};
+
+struct FwdBarriers {
+  uint64_t q_full, q_empty;
+  uint64_t s_full[2], p_full[2], o_full[2], o_final[2];
+  uint64_t drain;
+  uint64_t kv_full[8], kv_empty[8];
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+struct UnitCoord {
+  int b, h, p;
+};
+
+__device__ __forceinline__ UnitCoord decode_unit(const FwdArgs& a, int u) {
+  const int pair_idx = u / a.Hq;
+  const int h = u - pair_idx * a.Hq;
+  const int pair = (a.fwd_order != nullptr) ? __ldg(a.fwd_order + pair_idx) : pair_idx;
+  UnitCoord c;
+  c.b = pair / a.nP;
+  c.p = pair - c.b * a.nP;
+  c.h = h;
+  return c;
+}
+
+// Load the tile rows [row0, row0+128) of head `bh` (all D columns) as
+// D/64 boxes of 64 columns, each 128 rows x 128 bytes with 128-byte swizzle.
+template <int D>
+__device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                          int row0, int bh) {
+#pragma unroll
+  for (int c = 0; c < D / 64; ++c) tma_load_3d(dst + c * (TILE * 128), map, bar, c * 64, row0, bh);
+}
+
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * (TILE * 128) + (kk & 3) * 32;
+    mma_ss(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024), smem_desc_sw128(k_smem + off, 16, 1024),
+           FwdCfg<D>::kIdescQK, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem,
+                                         bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < TILE / 16; ++kk) {
+    mma_ts(d_tmem, p_tmem + kk * 8, smem_desc_sw128(v_smem + kk * 2048, TILE * 128, 1024),
+           FwdCfg<D>::kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// Per-row constants of one work unit.
+struct RowCtx {
+  int row;      // absolute query index
+  int lo, hi;   // kept key interval
+  float sl2;    // scale * log2(e)
+  float aux;    // ALiBi: slope * log2(e); softcap: scale / c; boost: boost * sl2
+  float aux2;   // softcap: c * log2(e)
+};
+
+// Raw scores of one row (32 columns starting at key k0 + c0) -> base-2 modded scores.
+template <int MOD>
+__device__ __forceinline__ void transform32(float (&x)[32], const RowCtx& r, const ModDev& md,
+                                            int k0, int c0, bool pred) {
+  const float di = static_cast<float>(r.row - k0 - c0);
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    float v = x[c];
+    if constexpr (MOD == MOD_ALIBI) {
+      v = fmaf(v, r.sl2, -r.aux * fabsf(di - static_cast<float>(c)));
+    } else if constexpr (MOD == MOD_SOFTCAP) {
+      v = r.aux2 * tanhf(v * r.aux);
+    } else if constexpr (MOD == MOD_BOOST) {
+      const bool inside = fabsf(di - static_cast<float>(c)) < static_cast<float>(md.boost_radius);
+      v = v * (inside ? r.aux : r.sl2);
+    } else {
+      v = v * r.sl2;
+    }
+    x[c] = v;
+  }
+  if (pred) {
+    const int jlo = r.lo - k0 - c0, jhi = r.hi - k0 - c0;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) x[c] = (c >= jlo && c <= jhi) ? x[c] : -INFINITY;
+  }
+}
+
+template <int D, int MOD, bool HAS_LSE>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
+  using Cfg = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the 128-byte-swizzled tiles
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  FwdBarriers* bars = reinterpret_cast<FwdBarriers*>(smem + Cfg::kBarOff);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t q_smem[2] = {sbase + Cfg::kQOff, sbase + Cfg::kQOff + Cfg::kTileBytes};
+  const uint32_t ring = sbase + Cfg::kRingOff;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->q_full), 1);
+    mbar_init(smem_u32(&bars->q_empty), 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(smem_u32(&bars->s_full[t]), 1);
+      mbar_init(smem_u32(&bars->p_full[t]), 128);
+      mbar_init(smem_u32(&bars->o_full[t]), 1);
+      mbar_init(smem_u32(&bars->o_final[t]), 1);
+    }
+    mbar_init(smem_u32(&bars->drain), 1);
+    for (int s = 0; s < Cfg::kStages; ++s) {
+      mbar_init(smem_u32(&bars->kv_full[s]), 1);
+      mbar_init(smem_u32(&bars->kv_empty[s]), 1);
+    }
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {  // allocate all 512 TMEM columns (one CTA per SM)
+    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_relinquish();
+  }
+  if (warp == 9 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const WaitCtl wc{a.wait_ns, &bars->abort_flag, a.status};
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t slot_uses[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      int ring_pos = 0;
+      int unit_iter = 0;
+      uint32_t q_loads = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+        const UnitCoord uc = decode_unit(a, u);
+        const int hk = uc.h / a.G;
+        // Q buffers are free once the previous unit's QK^T products finished
+        if (!mbar_wait_thread(smem_u32(&bars->q_empty), (unit_iter & 1) ^ 1, wc)) { ok = false; break; }
+        mbar_arrive_expect_tx(smem_u32(&bars->q_full), 2 * Cfg::kTileBytes);
+        ++q_loads;
+        const int bh_q = uc.b * a.Hq + uc.h;
+        load_tile<D>(q_smem[0], &tm_q, smem_u32(&bars->q_full), (2 * uc.p) * TILE, bh_q);
+        load_tile<D>(q_smem[1], &tm_q, smem_u32(&bars->q_full), (2 * uc.p + 1) * TILE, bh_q);
+        PairIter it;
+        it.init(a.tile_class, a.kv_count, a.kv_index, uc.b, uc.p, a.nQ, a.nK, a.Sq, a.Skv,
+                MOD, a.mod.window);
+        int kt;
+        bool a0, a1, p0, p1;
+        const int bh_kv = uc.b * a.Hkv + hk;
+        while (it.next(kt, a0, a1, p0, p1)) {
+#pragma unroll
+          for (int which = 0; which < 2; ++which) {  // K then V
+            const int slot = ring_pos % Cfg::kStages;
+            const uint32_t phase = (ring_pos / Cfg::kStages) & 1;
+            if (!mbar_wait_thread(smem_u32(&bars->kv_empty[slot]), phase ^ 1, wc)) { ok = false; break; }
+            const uint32_t bar = smem_u32(&bars->kv_full[slot]);
+            mbar_arrive_expect_tx(bar, Cfg::kTileBytes);
+            load_tile<D>(ring + slot * Cfg::kTileBytes, which == 0 ? &tm_k : &tm_v, bar, kt * TILE,
+                         bh_kv);
+            ++slot_uses[slot];
+            ++ring_pos;
+          }
+          if (!ok) break;
+        }
+      }
+      if (!ok) {
+        // let copies already in flight land before the CTA exits
+        uint32_t local_flag = 0;
+        const WaitCtl drain_wc{a.wait_ns, &local_flag, a.status};
+        for (int s = 0; s < Cfg::kStages; ++s) {
+          if (slot_uses[s] == 0) continue;
+          mbar_wait_thread(smem_u32(&bars->kv_full[s]), (slot_uses[s] - 1) & 1, drain_wc);
+        }
+        if (q_loads > 0)
+          mbar_wait_thread(smem_u32(&bars->q_full), (q_loads - 1) & 1, drain_wc);
+      }
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    // all lanes run the loop (waits are warp-collective); lane 0 issues
+    int ring_pos = 0;
+    int unit_iter = 0;
+    uint32_t p_cnt[2] = {0, 0};
+    bool ok = true;
+    const uint32_t s_tmem[2] = {tmem, tmem + 128};
+    const uint32_t o_tmem[2] = {tmem + 256, tmem + 256 + D};
+    for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+      const UnitCoord uc = decode_unit(a, u);
+      if (!mbar_wait_warp(smem_u32(&bars->q_full), unit_iter & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+      PairIter it;
+      it.init(a.tile_class, a.kv_count, a.kv_index, uc.b, uc.p, a.nQ, a.nK, a.Sq, a.Skv, MOD,
+              a.mod.window);
+      int kt;
+      bool act[2], prt[2];
+      bool has = it.next(kt, act[0], act[1], prt[0], prt[1]);
+      bool o_started[2] = {false, false};
+      if (has) {
+        const int slot_k = ring_pos % Cfg::kStages;
+        if (!mbar_wait_warp(smem_u32(&bars->kv_full[slot_k]), (ring_pos / Cfg::kStages) & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        if (lane == 0) {
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+            if (act[t]) {
+              issue_qk<D>(s_tmem[t], q_smem[t], ring + slot_k * Cfg::kTileBytes);
+              mma_commit(smem_u32(&bars->s_full[t]));
+            }
+          mma_commit(smem_u32(&bars->kv_empty[slot_k]));
+        }
+        __syncwarp();
+        ++ring_pos;
+      }
+      while (has && ok) {
+        const int slot_v = ring_pos % Cfg::kStages;
+        const uint32_t ph_v = (ring_pos / Cfg::kStages) & 1;
+        ++ring_pos;
+        int kt_n;
+        bool act_n[2], prt_n[2];
+        const bool has_n = it.next(kt_n, act_n[0], act_n[1], prt_n[0], prt_n[1]);
+        const int slot_kn = ring_pos % Cfg::kStages;
+        const uint32_t ph_kn = (ring_pos / Cfg::kStages) & 1;
+        if (!mbar_wait_warp(smem_u32(&bars->kv_full[slot_v]), ph_v, wc)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (act[t]) {
+            if (!mbar_wait_warp(smem_u32(&bars->p_full[t]), p_cnt[t] & 1, wc)) { ok = false; break; }
+            ++p_cnt[t];
+            tc_fence_after();
+            if (lane == 0) {
+              issue_pv<D>(o_tmem[t], s_tmem[t], ring + slot_v * Cfg::kTileBytes, o_started[t]);
+              mma_commit(smem_u32(&bars->o_full[t]));
+            }
+            __syncwarp();
+            o_started[t] = true;
+          }
+          if (has_n) {
+            if (t == 0) {
+              if (!mbar_wait_warp(smem_u32(&bars->kv_full[slot_kn]), ph_kn, wc)) { ok = false; break; }
+              tc_fence_after();
+            }
+            if (act_n[t] && lane == 0) {
+              issue_qk<D>(s_tmem[t], q_smem[t], ring + slot_kn * Cfg::kTileBytes);
+              mma_commit(smem_u32(&bars->s_full[t]));
+            }
+            __syncwarp();
+          }
+        }
+        if (!ok) break;
+        if (lane == 0) {
+          if (has_n) mma_commit(smem_u32(&bars->kv_empty[slot_kn]));
+          mma_commit(smem_u32(&bars->kv_empty[slot_v]));
+        }
+        __syncwarp();
+        if (has_n) ++ring_pos;
+        has = has_n;
+        kt = kt_n;
+        act[0] = act_n[0];
+        act[1] = act_n[1];
+      }
+      if (!ok) break;
+      if (lane == 0) {
+        mma_commit(smem_u32(&bars->q_empty));
+        mma_commit(smem_u32(&bars->o_final[0]));
+        mma_commit(smem_u32(&bars->o_final[1]));
+      }
+      __syncwarp();
+    }
+    // drain: wait until every MMA this thread issued has completed
+    if (lane == 0) {
+      mma_commit(smem_u32(&bars->drain));
+      uint32_t dummy_flag = 0;
+      mbar_wait_thread(smem_u32(&bars->drain), 0, WaitCtl{a.wait_ns, &dummy_flag, a.status});
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int t = warp >> 2;                  // query tile of the pair
+    const int r = threadIdx.x & 127;          // row within the tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_addr = tmem + t * 128 + lane_off;
+    const uint32_t o_addr = tmem + 256 + t * D + lane_off;
+    uint32_t s_cnt = 0, p_cnt = 0;
+    int unit_iter = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+      const UnitCoord uc = decode_unit(a, u);
+      RowCtx rc;
+      rc.row = (2 * uc.p + t) * TILE + r;
+      rc.sl2 = a.sl2;
+      rc.aux = 0.f;
+      rc.aux2 = 0.f;
+      if constexpr (MOD == MOD_ALIBI) rc.aux = alibi_slope(a.mod, uc.h, a.Hq) * LOG2E;
+      if constexpr (MOD == MOD_SOFTCAP) {
+        rc.aux = a.scale / a.mod.softcap;
+        rc.aux2 = a.mod.softcap * LOG2E;
+      }
+      if constexpr (MOD == MOD_BOOST) rc.aux = a.mod.boost * a.sl2;
+      row_interval(a.mod, uc.b, min(rc.row, a.Sq - 1), a.Skv, rc.lo, rc.hi);
+      if (rc.row >= a.Sq) rc.hi = rc.lo - 1;  // padding rows keep nothing
+      if constexpr (!is_interval_mask(MOD)) { rc.lo = 0; }
+
+      float m_run = -INFINITY, l_run = 0.f;
+      int n_act = 0;
+      PairIter it;
+      it.init(a.tile_class, a.kv_count, a.kv_index, uc.b, uc.p, a.nQ, a.nK, a.Sq, a.Skv, MOD,
+              a.mod.window);
+      int kt;
+      bool act[2], prt[2];
+      while (it.next(kt, act[0], act[1], prt[0], prt[1])) {
+        if (!act[t]) continue;
+        if (!mbar_wait_warp(smem_u32(&bars->s_full[t]), s_cnt & 1, wc)) { ok = false; break; }
+        ++s_cnt;
+        tc_fence_after();
+        const int k0 = kt * TILE;
+        float x[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          tmem_ld32(s_addr + c * 32, reinterpret_cast<uint32_t(&)[32]>(x[c]));
+        tmem_wait_ld();
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          transform32<MOD>(x[c], rc, a.mod, k0, c * 32, prt[t]);
+          float m0 = x[c][0], m1 = x[c][1], m2 = x[c][2], m3 = x[c][3];
+#pragma unroll
+          for (int e = 4; e < 32; e += 4) {
+            m0 = fmaxf(m0, x[c][e]);
+            m1 = fmaxf(m1, x[c][e + 1]);
+            m2 = fmaxf(m2, x[c][e + 2]);
+            m3 = fmaxf(m3, x[c][e + 3]);
+          }
+          mx = fmaxf(mx, fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)));
+        }
+        const float m_new = fmaxf(m_run, mx);
+        const bool need = m_new > m_run + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new);
+          if (n_act > 0) {
+            // O must be complete (previous P V finished) before it is rescaled
+            if (!mbar_wait_warp(smem_u32(&bars->o_full[t]), (p_cnt - 1) & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(o_addr + c * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(o_addr + c * 32, o);
+            }
+          }
+          l_run *= alpha;
+          m_run = m_new;
+        }
+        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+        float lsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+          float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float pa = ex2_approx(x[c][e] - m_use);
+            const float pb = ex2_approx(x[c][e + 1] - m_use);
+            s0 += pa;
+            s1 += pb;
+            pk[e >> 1] = pack_bf16x2(pa, pb);
+          }
+          lsum += s0 + s1;
+          // P (bf16 pairs) overwrites the first 64 columns of S
+          asm volatile(
+              "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+              "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(s_addr + c * 16),
+              "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]),
+              "r"(pk[7]), "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]), "r"(pk[12]),
+              "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
+              : "memory");
+        }
+        l_run += lsum;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&bars->p_full[t]));
+        ++p_cnt;
+        ++n_act;
+      }
+      if (!ok) break;
+      // ---- epilogue of this unit: O / l -> bf16, LSE
+      if (!mbar_wait_warp(smem_u32(&bars->o_final[t]), unit_iter & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+      const bool row_valid = rc.row < a.Sq;
+      const size_t row_idx = (static_cast<size_t>(uc.b) * a.Hq + uc.h) * a.Sq + rc.row;
+      __nv_bfloat16* orow = a.out + row_idx * D;
+      const float inv_l = (l_run > 0.f) ? 1.0f / l_run : 0.f;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (n_act > 0) {
+          tmem_ld32(o_addr + c * 32, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+        if (row_valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+      }
+      if constexpr (HAS_LSE) {
+        if (row_valid)
+          a.lse[row_idx] = (l_run > 0.f) ? (m_run + __log2f(l_run)) * LN2 : -INFINITY;
+      }
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 8) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+}  // namespace attn25
+
+namespace attn25 {
+
+namespace {
+
+template <int D, int MOD, bool LSE>
+cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const FwdArgs& a, int grid, cudaStream_t stream) {
+  auto kernel = attn_fwd_kernel<D, MOD, LSE>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       FwdCfg<D>::kAllocBytes);
+  if (e != cudaSuccess) return e;
+  kernel<<<grid, kFwdThreads, FwdCfg<D>::kAllocBytes, stream>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+template <int D, bool LSE>
+cudaError_t launch_fwd_mod(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const FwdArgs& a, int mod, int grid, cudaStream_t s) {
+  switch (mod) {
+    case MOD_NONE: return launch_fwd_t<D, MOD_NONE, LSE>(tq, tk, tv, a, grid, s);
+    case MOD_CAUSAL: return launch_fwd_t<D, MOD_CAUSAL, LSE>(tq, tk, tv, a, grid, s);
+    case MOD_ALIBI: return launch_fwd_t<D, MOD_ALIBI, LSE>(tq, tk, tv, a, grid, s);
+    case MOD_SOFTCAP: return launch_fwd_t<D, MOD_SOFTCAP, LSE>(tq, tk, tv, a, grid, s);
+    case MOD_WINDOW: return launch_fwd_t<D, MOD_WINDOW, LSE>(tq, tk, tv, a, grid, s);
+    case MOD_BOOST: return launch_fwd_t<D, MOD_BOOST, LSE>(tq, tk, tv, a, grid, s);
+    case MOD_DOCUMENT: return launch_fwd_t<D, MOD_DOCUMENT, LSE>(tq, tk, tv, a, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const FwdArgs& a, int D, int mod, bool has_lse, int grid,
+                       cudaStream_t stream) {
+  if (D == 128)
+    return has_lse ? launch_fwd_mod<128, true>(tq, tk, tv, a, mod, grid, stream)
+                   : launch_fwd_mod<128, false>(tq, tk, tv, a, mod, grid, stream);
+  if (D == 64)
+    return has_lse ? launch_fwd_mod<64, true>(tq, tk, tv, a, mod, grid, stream)
+                   : launch_fwd_mod<64, false>(tq, tk, tv, a, mod, grid, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace attn25

@@ -1,0 +1,78 @@
+// Kernel argument blocks and launchers shared between the kernels and the C ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "mods.cuh"
+
+namespace attn25 {
+
+struct FwdArgs {
+  __nv_bfloat16* out;
+  float* lse;
+  int B, Hq, Hkv, G, Sq, Skv;
+  int nQ, nK, nP, n_units;
+  float scale;  // softmax scale
+  float sl2;    // scale * log2(e)
+  ModDev mod;
+  const uint8_t* tile_class;  // block mask (all nullptr for dense iteration)
+  const int32_t* kv_count;
+  const int32_t* kv_index;
+  const int32_t* fwd_order;
+  uint64_t wait_ns;
+  int* status;
+};
+
+struct BwdArgs {
+  const __nv_bfloat16* out;   // forward output O
+  const __nv_bfloat16* dout;  // dO
+  const float* lse;           // forward LSE (natural log)
+  float* dq_acc;              // [B*Hq][Sq_pad][D] fp32
+  float* lse2;                // [B*Hq][Sq_pad]: LSE * log2(e), +inf where the row keeps nothing
+  float* delta;               // [B*Hq][Sq_pad]: rowsum(dO * O)
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  int B, Hq, Hkv, G, Sq, Skv, Sq_pad;
+  int nQ, nK, n_units;
+  float scale, sl2;
+  ModDev mod;
+  const uint8_t* tile_class;
+  const int32_t* q_count;
+  const int32_t* q_index;
+  const int32_t* bwd_order;
+  uint64_t wait_ns;
+  int* status;
+};
+
+struct MaskArgs {
+  int kind;
+  int window;
+  const int32_t* doc_offsets;
+  int num_docs;
+  int B, Sq, Skv, nQ, nK, nP;
+  uint8_t* tile_class;
+  int32_t* kv_count;
+  int32_t* kv_index;
+  int32_t* q_count;
+  int32_t* q_index;
+  int32_t* fwd_order;
+  int32_t* bwd_order;
+};
+
+// Each returns cudaSuccess or the launch error.
+cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const FwdArgs& a, int D, int mod, bool has_lse, int grid,
+                       cudaStream_t stream);
+cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int D,
+                       int mod, int grid, cudaStream_t stream);
+cudaError_t launch_block_mask(const MaskArgs& a, cudaStream_t stream);
+
+// Register count ptxas gave the forward kernel (for the host's sanity checks).
+int fwd_kernel_regs(int D, int mod, bool has_lse);
+
+}  // namespace attn25
