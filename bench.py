@@ -62,7 +62,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -199,10 +199,13 @@ def run_gpu(args, rank, world, local_rank):
 
     # end-to-end through the same API with pinned host buffers: H2D of the
     # step's inputs, the step, D2H of its results (O, dQ, dK, dV)
-    hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, dout))
+    if args.no_e2e:
+        hq = None
+    else:
+        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, dout))
     ho, hdq, hdk, hdv = (torch.empty_like(t, device="cpu").pin_memory() for t in (out, dq, dk, dv))
     e2e_times = []
-    for i in range(args.warmup + args.steps):
+    for i in range(0 if args.no_e2e else args.warmup + args.steps):
         flush.fill_(1.0)
         a0, a1 = ev(), ev()
         a0.record(stream)
@@ -215,7 +218,7 @@ def run_gpu(args, rank, world, local_rank):
         if i >= args.warmup:
             e2e_times.append((a0, a1))
     torch.cuda.synchronize()
-    ms_e2e = sum(a.elapsed_time(b) for a, b in e2e_times) / len(e2e_times)
+    ms_e2e = sum(a.elapsed_time(b) for a, b in e2e_times) / max(1, len(e2e_times))
     if world > 1:
         tt = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
         torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
@@ -263,7 +266,7 @@ def run_gpu(args, rank, world, local_rank):
         "roofline": dict(roof(bwd_tf if dominant == "backward" else fwd_tf, None), kernel=f"attn_{dominant[:3]} call"),
         "roofline_forward": roof(fwd_tf, None),
         "roofline_backward": roof(bwd_tf, None),
-        "e2e": {"value": round(total / (ms_e2e * 1e-3) / 1e12, 2), "unit": UNIT,
+        "e2e": None if args.no_e2e else {"value": round(total / (ms_e2e * 1e-3) / 1e12, 2), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4)},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
@@ -283,19 +286,19 @@ def cpu_baseline(w, mod_name, params, seconds=15.0, heads=None):
     qf, kf, vf, df = (bf16_bits_to_f64(bits[n]) for n in ("q", "k", "v", "dout"))
     G = w.Hq // w.Hkv
     done, flops, t_total = 0, 0.0, 0.0
-    n_per_head = oracle.useful_elements(mod, params, 1, 1, w.Sq, w.Skv)
-    for hk in range(w.Hkv):
-        if heads is not None and done >= heads:
-            break
-        t0 = time.perf_counter()
-        group = [(0, h) for h in range(hk * G, hk * G + G)]
-        oracle.attention_forward(qf, kf, vf, w.scale, mod, params, heads=group)
-        oracle.attention_backward(qf, kf, vf, df, w.scale, mod, params, groups=[(0, hk)])
-        t_total += time.perf_counter() - t0
-        done += G
-        flops += G * n_per_head * w.D * 14.0
-        if heads is None and t_total >= seconds:
-            break
+    for b in range(w.B):
+        n_per_head = oracle.useful_elements(mod, params, b + 1, 1, w.Sq, w.Skv) - \
+            oracle.useful_elements(mod, params, b, 1, w.Sq, w.Skv)
+        for hk in range(w.Hkv):
+            if (heads is not None and done >= heads) or (heads is None and t_total >= seconds):
+                break
+            t0 = time.perf_counter()
+            group = [(b, h) for h in range(hk * G, hk * G + G)]
+            oracle.attention_forward(qf, kf, vf, w.scale, mod, params, heads=group)
+            oracle.attention_backward(qf, kf, vf, df, w.scale, mod, params, groups=[(b, hk)])
+            t_total += time.perf_counter() - t0
+            done += G
+            flops += G * n_per_head * w.D * 14.0
     cores = os.cpu_count()
     return {"value": round(flops / t_total / 1e12, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"fp64 numpy oracle, fwd+bwd of {done} of {w.B * w.Hq} (b, head) problems "
@@ -330,12 +333,13 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="dense:none")
     ap.add_argument("--all", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     if args.warmup < 3:

@@ -45,9 +45,10 @@ class Case:
         return oracle.attention_forward(self.qf, self.kf, self.vf, self.scale, self.mod, self.p,
                                         heads=heads, rows=rows)
 
-    def oracle_bwd(self, groups=None, q_rows=None, kv_rows=None):
+    def oracle_bwd(self, groups=None, q_rows=None, kv_rows=None, contrib_rows=None):
         return oracle.attention_backward(self.qf, self.kf, self.vf, self.doutf, self.scale, self.mod,
-                                         self.p, groups=groups, q_rows=q_rows, kv_rows=kv_rows)
+                                         self.p, groups=groups, q_rows=q_rows, kv_rows=kv_rows,
+                                         contrib_rows=contrib_rows)
 
 
 def check_o(o_gpu, o_ref, what=""):

@@ -15,7 +15,8 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libattn25.so")
+# ATTN25_LIBRARY may name the profiling build (libattn25_trace.so) instead.
+LIB_PATH = os.environ.get("ATTN25_LIBRARY") or os.path.join(_HERE, "libattn25.so")
 
 MOD_NONE = 0
 MOD_CAUSAL = 1
@@ -87,6 +88,11 @@ def _load():
     lib.attn_set_wait_limit_ms.restype = None
     lib.attn_strerror.argtypes = [I]
     lib.attn_strerror.restype = ctypes.c_char_p
+    if hasattr(lib, "attn_trace_read"):  # profiling build only
+        lib.attn_trace_read.argtypes = [ctypes.POINTER(ctypes.c_ulonglong), I]
+        lib.attn_trace_read.restype = I
+        lib.attn_trace_reset.argtypes = []
+        lib.attn_trace_reset.restype = I
     return lib
 
 
@@ -242,3 +248,14 @@ def attn_get_status(stream=None) -> int:
 
 def attn_set_wait_limit_ms(ms: int):
     LIB.attn_set_wait_limit_ms(int(ms))
+
+
+def attn_trace_read(n: int = 128) -> list:
+    """Per-role cycle counters of the profiling build (libattn25_trace.so)."""
+    buf = (ctypes.c_ulonglong * n)()
+    _check(LIB.attn_trace_read(buf, n), "attn_trace_read")
+    return list(buf)
+
+
+def attn_trace_reset():
+    _check(LIB.attn_trace_reset(), "attn_trace_reset")

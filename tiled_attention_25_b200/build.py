@@ -18,6 +18,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libattn25.so")
+TRACE_LIB = os.path.join(HERE, "libattn25_trace.so")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
@@ -32,25 +33,25 @@ def _sources():
     return sorted(f for f in os.listdir(CSRC) if f.endswith(".cu"))
 
 
-def _headers_digest():
+def _headers_digest(flags):
     h = hashlib.sha256()
     for d in (CSRC, INCLUDE):
         for f in sorted(os.listdir(d)):
             if f.endswith((".h", ".cuh")):
                 with open(os.path.join(d, f), "rb") as fh:
                     h.update(f.encode() + fh.read())
-    h.update(" ".join(FLAGS).encode())
+    h.update(" ".join(flags).encode())
     return h.hexdigest()
 
 
-def _compile(src, digest, verbose):
+def _compile(src, digest, verbose, flags):
     path = os.path.join(CSRC, src)
     with open(path, "rb") as fh:
         key = hashlib.sha256(fh.read() + digest.encode()).hexdigest()[:16]
     obj = os.path.join(BUILD, f"{src[:-3]}.{key}.o")
     if os.path.exists(obj):
         return obj
-    cmd = [NVCC, *FLAGS, "-c", path, "-o", obj + ".tmp"]
+    cmd = [NVCC, *flags, "-c", path, "-o", obj + ".tmp"]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -62,25 +63,29 @@ def _compile(src, digest, verbose):
     return obj
 
 
-def build(verbose: bool = False) -> str:
+def build(verbose: bool = False, trace: bool = False) -> str:
+    """Build libattn25.so (or, with trace=True, the profiling variant
+    libattn25_trace.so whose kernels count cycles per warp role)."""
     os.makedirs(BUILD, exist_ok=True)
-    digest = _headers_digest()
+    flags = FLAGS + (["-DATTN25_TRACE"] if trace else [])
+    lib = TRACE_LIB if trace else LIB
+    digest = _headers_digest(flags)
     with concurrent.futures.ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
-        objs = list(ex.map(lambda s: _compile(s, digest, verbose), _sources()))
+        objs = list(ex.map(lambda s: _compile(s, digest, verbose, flags), _sources()))
     link_key = hashlib.sha256("".join(objs).encode()).hexdigest()[:16]
-    stamp = os.path.join(BUILD, "libattn25.stamp")
-    if os.path.exists(LIB) and os.path.exists(stamp) and open(stamp).read() == link_key:
-        return LIB
-    cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", LIB + ".tmp",
+    stamp = os.path.join(BUILD, os.path.basename(lib) + ".stamp")
+    if os.path.exists(lib) and os.path.exists(stamp) and open(stamp).read() == link_key:
+        return lib
+    cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", lib + ".tmp",
            *objs, "-cudart", "static", "-Xlinker", "--no-undefined"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stderr}")
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(lib + ".tmp", lib)
     with open(stamp, "w") as fh:
         fh.write(link_key)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(verbose="-v" in sys.argv))
+    print(build(verbose="-v" in sys.argv, trace="--trace" in sys.argv))

@@ -18,6 +18,11 @@ namespace attn25 {
 // One status word per device that loads the library.
 __device__ int g_attn_status;
 
+#if defined(ATTN25_TRACE)
+// Profiling builds: per-role cycle counters (forward at 0, backward at 64).
+__device__ unsigned long long g_attn_trace[128];
+#endif
+
 namespace {
 
 std::atomic<uint32_t> g_wait_ms{4000};
@@ -29,6 +34,7 @@ struct DeviceInfo {
   bool usable = false;
   int sms = 0;
   int* status = nullptr;
+  unsigned long long* trace = nullptr;
 };
 
 std::mutex g_mu;
@@ -48,6 +54,10 @@ int current_device(DeviceInfo** out) {
     void* p = nullptr;
     const bool sym_ok = cudaGetSymbolAddress(&p, g_attn_status) == cudaSuccess;
     d.status = static_cast<int*>(p);
+#if defined(ATTN25_TRACE)
+    void* tp = nullptr;
+    if (cudaGetSymbolAddress(&tp, g_attn_trace) == cudaSuccess) d.trace = static_cast<unsigned long long*>(tp);
+#endif
     if (g_encode == nullptr) {
       void* fn = nullptr;
       cudaDriverEntryPointQueryResult q;
@@ -331,6 +341,7 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
   }
   a.wait_ns = wait_ns();
   a.status = d->status;
+  a.trace = d->trace;
   const int grid = a.n_units < d->sms ? a.n_units : d->sms;
   if (launch_fwd(tq, tk, tv, a, D, mod_kind, lse != nullptr, grid,
                  reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
@@ -397,6 +408,7 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
   }
   a.wait_ns = wait_ns();
   a.status = d->status;
+  a.trace = d->trace == nullptr ? nullptr : d->trace + 64;
 
   CUtensorMap tq, tk, tv, tdo, tdq;
   if (!encode_bf16(&tq, q, D, Sq, B * Hq, 64) || !encode_bf16(&tk, k, D, Skv, B * Hkv, TILE) ||
@@ -409,5 +421,27 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
     return ATTN_ERR_LAUNCH;
   return ATTN_OK;
 }
+
+#if defined(ATTN25_TRACE)
+ATTN25_API int attn_trace_read(unsigned long long* host_out, int n) {
+  DeviceInfo* d = nullptr;
+  int rc = current_device(&d);
+  if (rc != ATTN_OK) return rc;
+  if (host_out == nullptr || n < 0 || n > 128 || d->trace == nullptr) return ATTN_ERR_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  if (cudaMemcpy(host_out, d->trace, n * sizeof(unsigned long long), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return ATTN_ERR_LAUNCH;
+  return ATTN_OK;
+}
+
+ATTN25_API int attn_trace_reset(void) {
+  DeviceInfo* d = nullptr;
+  int rc = current_device(&d);
+  if (rc != ATTN_OK) return rc;
+  if (d->trace == nullptr) return ATTN_ERR_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  return cudaMemset(d->trace, 0, 128 * sizeof(unsigned long long)) == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+#endif
 
 }  // extern "C"

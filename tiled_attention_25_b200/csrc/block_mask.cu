@@ -90,56 +90,60 @@ __global__ void __launch_bounds__(32) transpose_kernel(const MaskArgs a) {
   for (int qt = n; qt < a.nQ; ++qt) list[qt] = -1;
 }
 
-// One block: costs of the forward pairs and backward units, then a stable
-// counting sort of each by descending cost.
+__device__ __forceinline__ int pair_cost(const MaskArgs& a, int u) {
+  const int b = u / a.nP, p = u - b * a.nP;
+  const uint8_t* r0 = a.tile_class + (static_cast<size_t>(b) * a.nQ + 2 * p) * a.nK;
+  const bool has1 = 2 * p + 1 < a.nQ;
+  int cost = 0;
+  for (int kt = 0; kt < a.nK; ++kt) cost += (r0[kt] != 0 || (has1 && r0[a.nK + kt] != 0));
+  return cost;
+}
+
+// One block: the forward pairs and the backward units, each sorted by
+// descending cost with ties in ascending id.  Costs go to shared memory and
+// every thread places its units at their rank: the number of units that sort
+// before them.
+constexpr int kOrderSmemUnits = 16384;
+
 __global__ void __launch_bounds__(1024) order_kernel(const MaskArgs a) {
-  extern __shared__ int s_hist[];  // max(nQ, nK) + 2 counters
-  const int n_pairs = a.B * a.nP;
-  const int n_units = a.B * a.nK;
-  const int max_cost = a.nQ > a.nK ? a.nQ : a.nK;
+  extern __shared__ int s_cost[];  // kOrderSmemUnits entries
   for (int pass = 0; pass < 2; ++pass) {
-    const int n = pass == 0 ? n_pairs : n_units;
+    const int n = pass == 0 ? a.B * a.nP : a.B * a.nK;
     int32_t* out = pass == 0 ? a.fwd_order : a.bwd_order;
-    for (int c = threadIdx.x; c <= max_cost + 1; c += blockDim.x) s_hist[c] = 0;
+    for (int u = threadIdx.x; u < n; u += blockDim.x)
+      s_cost[u] = pass == 0 ? pair_cost(a, u) : a.q_count[u];
     __syncthreads();
     for (int u = threadIdx.x; u < n; u += blockDim.x) {
-      int cost;
-      if (pass == 0) {
-        const int b = u / a.nP, p = u - b * a.nP;
-        const uint8_t* r0 = a.tile_class + (static_cast<size_t>(b) * a.nQ + 2 * p) * a.nK;
-        const bool has1 = 2 * p + 1 < a.nQ;
-        cost = 0;
-        for (int kt = 0; kt < a.nK; ++kt) cost += (r0[kt] != 0 || (has1 && r0[a.nK + kt] != 0));
-      } else {
-        cost = a.q_count[u];
+      const int c = s_cost[u];
+      int rank = 0;
+      for (int v = 0; v < n; ++v) {
+        const int cv = s_cost[v];
+        rank += (cv > c) || (cv == c && v < u);
       }
-      atomicAdd(&s_hist[cost], 1);
+      out[rank] = u;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      // start position of each cost class, longest first
-      int start = 0;
-      for (int c = max_cost; c >= 0; --c) {
-        const int cnt = s_hist[c];
-        s_hist[c] = start;
-        start += cnt;
-      }
-      // stable placement in ascending unit id
-      for (int u = 0; u < n; ++u) {
-        int cost;
-        if (pass == 0) {
-          const int b = u / a.nP, p = u - b * a.nP;
-          const uint8_t* r0 = a.tile_class + (static_cast<size_t>(b) * a.nQ + 2 * p) * a.nK;
-          const bool has1 = 2 * p + 1 < a.nQ;
-          cost = 0;
-          for (int kt = 0; kt < a.nK; ++kt) cost += (r0[kt] != 0 || (has1 && r0[a.nK + kt] != 0));
-        } else {
-          cost = a.q_count[u];
-        }
-        out[s_hist[cost]++] = u;
-      }
+  }
+}
+
+// The same order for unit counts beyond the shared-memory table: a stable
+// counting sort by one thread over costs in [0, max(nQ, nK)].
+__global__ void __launch_bounds__(32) order_serial_kernel(const MaskArgs a) {
+  if (threadIdx.x != 0) return;
+  extern __shared__ int s_hist[];  // max(nQ, nK) + 2 counters
+  const int max_cost = a.nQ > a.nK ? a.nQ : a.nK;
+  for (int pass = 0; pass < 2; ++pass) {
+    const int n = pass == 0 ? a.B * a.nP : a.B * a.nK;
+    int32_t* out = pass == 0 ? a.fwd_order : a.bwd_order;
+    for (int c = 0; c <= max_cost + 1; ++c) s_hist[c] = 0;
+    for (int u = 0; u < n; ++u) ++s_hist[pass == 0 ? pair_cost(a, u) : a.q_count[u]];
+    int start = 0;
+    for (int c = max_cost; c >= 0; --c) {
+      const int cnt = s_hist[c];
+      s_hist[c] = start;
+      start += cnt;
     }
-    __syncthreads();
+    for (int u = 0; u < n; ++u) out[s_hist[pass == 0 ? pair_cost(a, u) : a.q_count[u]]++] = u;
   }
 }
 
@@ -152,7 +156,18 @@ cudaError_t launch_block_mask(const MaskArgs& a, cudaStream_t stream) {
   transpose_kernel<<<dim3(a.nK, a.B), 32, 0, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  order_kernel<<<1, 1024, ((a.nQ > a.nK ? a.nQ : a.nK) + 2) * sizeof(int), stream>>>(a);
+  const int n_max = a.B * (a.nP > a.nK ? a.nP : a.nK);
+  if (n_max <= kOrderSmemUnits) {
+    const int smem = n_max * static_cast<int>(sizeof(int));
+    if (smem > 48 * 1024) {
+      e = cudaFuncSetAttribute(order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kOrderSmemUnits * static_cast<int>(sizeof(int)));
+      if (e != cudaSuccess) return e;
+    }
+    order_kernel<<<1, 1024, smem, stream>>>(a);
+  } else {
+    order_serial_kernel<<<1, 32, ((a.nQ > a.nK ? a.nQ : a.nK) + 2) * sizeof(int), stream>>>(a);
+  }
   return cudaGetLastError();
 }
 

@@ -70,6 +70,7 @@ struct BwdBarriers {
   uint64_t drain;
   uint32_t tmem_base;
   uint32_t abort_flag;
+  uint32_t never_set;  // abort word for drain waits that must not stop early
 };
 
 struct BwdUnit {
@@ -262,6 +263,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(smem_u32(&bars->acc_empty), 128);
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort_flag = 0;
+    bars->never_set = 0;
     fence_mbar_init();
   }
   if (warp == 8) {
@@ -279,7 +281,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const WaitCtl wc{a.wait_ns, &bars->abort_flag, a.status};
+  const WaitCtl wc{a.wait_ns, smem_u32(&bars->abort_flag), a.status};
+  long long tr[12] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
+  (void)tr;
+  ATTN25_TRACE_ONLY(const long long t_start = clock64();)
 
   if (warp == 9) {
     // ------------------------------------------------------------ TMA producer
@@ -289,7 +294,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
         const BwdUnit un = decode_bwd_unit(a, u);
-        if (!mbar_wait_thread(smem_u32(&bars->kv_empty), (unit_iter & 1) ^ 1, wc)) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[1], mbar_wait_thread(smem_u32(&bars->kv_empty), (unit_iter & 1) ^ 1, wc))) { ok = false; break; }
         mbar_arrive_expect_tx(smem_u32(&bars->kv_full), 2 * Cfg::kKVBytes);
         ++kv_loads;
         const int bh_kv = un.b * a.Hkv + un.hk;
@@ -301,7 +306,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bool pred;
         while (it.next(g, q0, pred)) {
           const int s = step & 1;
-          if (!mbar_wait_thread(smem_u32(&bars->q_empty[s]), ((step >> 1) & 1) ^ 1, wc)) { ok = false; break; }
+          if (!ATTN25_TIMED(tr[2], mbar_wait_thread(smem_u32(&bars->q_empty[s]), ((step >> 1) & 1) ^ 1, wc))) { ok = false; break; }
           const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
           const uint32_t bar = smem_u32(&bars->q_full[s]);
           mbar_arrive_expect_tx(bar, 2 * Cfg::kQBytes + 2 * BM * 4);
@@ -316,12 +321,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
       if (!ok) {
-        uint32_t local_flag = 0;
-        const WaitCtl dwc{a.wait_ns, &local_flag, a.status};
+        const WaitCtl dwc{a.wait_ns, smem_u32(&bars->never_set), a.status};
         if (kv_loads) mbar_wait_thread(smem_u32(&bars->kv_full), (kv_loads - 1) & 1, dwc);
         for (int s = 0; s < 2; ++s)
           if (stage_uses[s]) mbar_wait_thread(smem_u32(&bars->q_full[s]), (stage_uses[s] - 1) & 1, dwc);
       }
+      ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
+      trace_flush(a.trace, 48, tr);
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
@@ -332,9 +338,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
     for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
       const BwdUnit un = decode_bwd_unit(a, u);
-      if (!mbar_wait_warp(smem_u32(&bars->kv_full), unit_iter & 1, wc)) { ok = false; break; }
+      if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->kv_full), unit_iter & 1, wc))) { ok = false; break; }
       // dK, dV accumulators are free once the previous unit's epilogue read them
-      if (!mbar_wait_warp(smem_u32(&bars->acc_empty), (unit_iter & 1) ^ 1, wc)) { ok = false; break; }
+      if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->acc_empty), (unit_iter & 1) ^ 1, wc))) { ok = false; break; }
       tc_fence_after();
       StepIter it;
       it.init(a, un);
@@ -345,7 +351,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // prologue: S^T and dP^T of the first step
       if (has) {
         const int s = step & 1;
-        if (!mbar_wait_warp(smem_u32(&bars->q_full[s]), (step >> 1) & 1, wc)) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step >> 1) & 1, wc))) { ok = false; break; }
         tc_fence_after();
         const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
         if (lane == 0) {
@@ -360,7 +366,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int s = step & 1;
         const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
         // dV += P^T dO once the probabilities are in tensor memory
-        if (!mbar_wait_warp(smem_u32(&bars->p_ready), p_cnt & 1, wc)) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->p_ready), p_cnt & 1, wc))) { ok = false; break; }
         ++p_cnt;
         tc_fence_after();
         if (lane == 0) {
@@ -376,7 +382,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int s_n = (step + 1) & 1;
         const uint32_t st_n = sbase + Cfg::kStageOff + s_n * Cfg::kStageBytes;
         if (has_n) {  // S^T of the next step overlaps this step's dS work
-          if (!mbar_wait_warp(smem_u32(&bars->q_full[s_n]), ((step + 1) >> 1) & 1, wc)) { ok = false; break; }
+          if (!ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s_n]), ((step + 1) >> 1) & 1, wc))) { ok = false; break; }
           tc_fence_after();
           if (lane == 0) {
             issue_st<D>(t_s, k_smem, st_n);
@@ -385,11 +391,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           __syncwarp();
         }
         // dK += dS^T Q and dQ^T = K^T dS^T once dS^T is in shared memory
-        if (!mbar_wait_warp(smem_u32(&bars->ds_ready), ds_cnt & 1, wc)) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[5], mbar_wait_warp(smem_u32(&bars->ds_ready), ds_cnt & 1, wc))) { ok = false; break; }
         const uint32_t ds_smem = sbase + Cfg::kDSOff + (ds_cnt & 1) * Cfg::kDSBytes;
         ++ds_cnt;
         // the dQ^T columns must have been drained by the previous step
-        if (!mbar_wait_warp(smem_u32(&bars->dq_empty), (dq_cnt & 1) ^ 1, wc)) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[6], mbar_wait_warp(smem_u32(&bars->dq_empty), (dq_cnt & 1) ^ 1, wc))) { ok = false; break; }
         tc_fence_after();
         if (lane == 0) {
 #pragma unroll
@@ -428,10 +434,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     if (lane == 0) {
       mma_commit(smem_u32(&bars->drain));
-      uint32_t local_flag = 0;
-      mbar_wait_thread(smem_u32(&bars->drain), 0, WaitCtl{a.wait_ns, &local_flag, a.status});
+      mbar_wait_thread(smem_u32(&bars->drain), 0, WaitCtl{a.wait_ns, smem_u32(&bars->never_set), a.status});
     }
     __syncwarp();
+    ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start; tr[7] = step;)
+    trace_flush(a.trace, 32, tr);
   } else if (warp < 4) {
     // ------------------------------------------------------------ P^T / dS^T (thread = key row)
     const int r = threadIdx.x;  // TMEM lane = key row within the tile
@@ -474,10 +481,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float* lse2_s = reinterpret_cast<const float*>(smem + Cfg::kStageOff + s * Cfg::kStageBytes + 2 * Cfg::kQBytes);
         const float* delta_s = lse2_s + 128;
         // stage contents (Q, dO, statistics) have landed
-        if (!mbar_wait_warp(smem_u32(&bars->q_full[s]), (step >> 1) & 1, wc)) { ok = false; break; }
-        if (!mbar_wait_warp(smem_u32(&bars->s_full), s_cnt & 1, wc)) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step >> 1) & 1, wc))) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->s_full), s_cnt & 1, wc))) { ok = false; break; }
         ++s_cnt;
         tc_fence_after();
+        ATTN25_TRACE_ONLY(const long long t_p = clock64();)
         const int h = un.hk * a.G + g;
         float sl2 = a.sl2, aux = 0.f, aux2 = 0.f;
         if constexpr (MOD == MOD_ALIBI) aux = alibi_slope(a.mod, h, a.Hq) * LOG2E;
@@ -524,8 +532,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(smem_u32(&bars->p_ready));
+        ATTN25_TRACE_ONLY(tr[3] += clock64() - t_p;)
         // dS^T = P^T (dP^T - Delta) ds'/ds
-        if (!mbar_wait_warp(smem_u32(&bars->dp_full), dp_cnt & 1, wc)) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->dp_full), dp_cnt & 1, wc))) { ok = false; break; }
+        ATTN25_TRACE_ONLY(const long long t_ds = clock64();)
         ++dp_cnt;
         tc_fence_after();
         float dp[BM];
@@ -533,7 +543,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(t_dp + 32, reinterpret_cast<uint32_t(&)[32]>(dp[32]));
         tmem_wait_ld();
         // the dS buffer is free once the MMAs of two steps ago completed
-        if (!mbar_wait_warp(smem_u32(&bars->ds_empty[ds_cnt & 1]), ((ds_cnt >> 1) & 1) ^ 1, wc)) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[5], mbar_wait_warp(smem_u32(&bars->ds_empty[ds_cnt & 1]), ((ds_cnt >> 1) & 1) ^ 1, wc))) { ok = false; break; }
         uint8_t* ds_row = smem + Cfg::kDSOff + (ds_cnt & 1) * Cfg::kDSBytes + r * 128;
         ++ds_cnt;
 #pragma unroll
@@ -560,12 +570,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(smem_u32(&bars->ds_ready));
+        ATTN25_TRACE_ONLY(tr[6] += clock64() - t_ds;)
         ++n_steps;
         ++step;
       }
       if (!ok) break;
       // ---- unit epilogue: dV, scale * dK -> bf16
-      if (!mbar_wait_warp(smem_u32(&bars->acc_full), unit_iter & 1, wc)) { ok = false; break; }
+      if (!ATTN25_TIMED(tr[7], mbar_wait_warp(smem_u32(&bars->acc_full), unit_iter & 1, wc))) { ok = false; break; }
+      ATTN25_TRACE_ONLY(const long long t_e = clock64();)
       tc_fence_after();
       const bool row_ok = kv < a.Skv;
       const size_t row = (static_cast<size_t>(un.b) * a.Hkv + un.hk) * a.Skv + kv;
@@ -597,7 +609,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(smem_u32(&bars->acc_empty));
+      ATTN25_TRACE_ONLY(tr[8] += clock64() - t_e;)
     }
+    ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
+    trace_flush(a.trace, 0, tr);
   } else {
     // ------------------------------------------------------------ dQ drain (thread = head-dim lane)
     const int w = warp - 4;      // TMEM lane quarter = 32-column block of D
@@ -615,7 +630,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int g, q0;
       bool pred;
       while (it.next(g, q0, pred)) {
-        if (!mbar_wait_warp(smem_u32(&bars->dq_full), dq_cnt & 1, wc)) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->dq_full), dq_cnt & 1, wc))) { ok = false; break; }
         tc_fence_after();
         float v[BM];
         tmem_ld32(t_dq, reinterpret_cast<uint32_t(&)[32]>(v[0]));
@@ -624,7 +639,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_before();
         mbar_arrive(smem_u32(&bars->dq_empty));
         // staging is free once the previous reduce has read it
-        if (!mbar_wait_warp(smem_u32(&bars->stg_free), (dq_cnt & 1) ^ 1, wc)) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->stg_free), (dq_cnt & 1) ^ 1, wc))) { ok = false; break; }
         if (active) {
 #pragma unroll
           for (int c = 0; c < BM; ++c) stg[c * 32 + lane] = v[c];
@@ -632,14 +647,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         fence_proxy_async_smem();
         mbar_arrive(smem_u32(&bars->stg_written));
         if (threadIdx.x == 128) {
-          if (!mbar_wait_thread(smem_u32(&bars->stg_written), dq_cnt & 1, wc)) {
+          if (!ATTN25_TIMED(tr[3], mbar_wait_thread(smem_u32(&bars->stg_written), dq_cnt & 1, wc))) {
             ok = false;
           } else {
             const int bh = un.b * a.Hq + un.hk * a.G + g;
             for (int c = 0; c < D / 32; ++c)
               tma_reduce_add_3d(&tm_dq, sbase + Cfg::kStgOff + c * (BM * 32 * 4), c * 32, q0, bh);
             bulk_commit();
-            bulk_wait_read_all();
+            ATTN25_TIMED(tr[4], (bulk_wait_read_all(), 0));
             mbar_arrive(smem_u32(&bars->stg_free));
           }
         }
@@ -649,6 +664,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
     if (threadIdx.x == 128) bulk_wait_all();
+    ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
+    trace_flush(a.trace, 16, tr);
   }
 
   tc_fence_before();

@@ -24,6 +24,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "exp2_poly.h"
 #include "kernel_common.cuh"
 #include "launch.h"
 
@@ -31,7 +32,14 @@ namespace attn25 {
 
 namespace {
 
-constexpr int kFwdThreads = 320;
+constexpr int kFwdThreads = 384;  // 2 softmax warpgroups + 1 control warpgroup
+// Register split (setmaxnreg): the launch gives 168 per thread (384 x 168 =
+// 64512 in the CTA pool); the control warpgroup drops to 104 so that the two
+// softmax warpgroups can rise to 200: 2 x 128 x 200 + 128 x 104 = 64512.
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 200;
+constexpr int kControlRegs = 104;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kFwdThreads * kLaunchRegs, "register split");
 constexpr float kRescaleThreshold = 8.0f;
 
 template <int D>
@@ -54,6 +62,7 @@ struct FwdBarriers {
   uint64_t kv_full[8], kv_empty[8];
   uint32_t tmem_base;
   uint32_t abort_flag;
+  uint32_t never_set;  // abort word for drain waits that must not stop early
 };
 
 struct UnitCoord {
@@ -136,6 +145,84 @@ __device__ __forceinline__ void transform32(float (&x)[32], const RowCtx& r, con
   }
 }
 
+// Scores whose mod is the plain scale (none and the interval masks) stay raw
+// until the exponent: the row maximum is taken on raw scores and the scale is
+// folded into the exponent's FFMA.
+__host__ __device__ constexpr bool pure_scale(int mod) {
+  return mod == MOD_NONE || mod == MOD_CAUSAL || mod == MOD_WINDOW || mod == MOD_DOCUMENT;
+}
+
+// Apply mask (and, for the other mods, the mod itself) to one row of raw
+// scores; return the row maximum in the base-2 domain.
+template <int MOD, bool PRED>
+__device__ __forceinline__ float row_scores(float (&x)[4][32], const RowCtx& rc, const ModDev& md,
+                                            int k0) {
+  float mx = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    if constexpr (pure_scale(MOD)) {
+      if constexpr (PRED) {
+        const int jlo = rc.lo - k0 - c * 32, jhi = rc.hi - k0 - c * 32;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[c][e] = (e >= jlo && e <= jhi) ? x[c][e] : -INFINITY;
+      }
+    } else {
+      transform32<MOD>(x[c], rc, md, k0, c * 32, PRED);
+    }
+    float m0 = x[c][0], m1 = x[c][1], m2 = x[c][2], m3 = x[c][3];
+#pragma unroll
+    for (int e = 4; e < 32; e += 4) {
+      m0 = fmaxf(m0, x[c][e]);
+      m1 = fmaxf(m1, x[c][e + 1]);
+      m2 = fmaxf(m2, x[c][e + 2]);
+      m3 = fmaxf(m3, x[c][e + 3]);
+    }
+    mx = fmaxf(mx, fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)));
+  }
+  if constexpr (pure_scale(MOD)) mx *= rc.sl2;  // -inf stays -inf
+  return mx;
+}
+
+// P = 2^(x - m) for one row, written as bf16 pairs over the first 64 TMEM
+// columns of the row's S tile; returns the fp32 row sum.  With EMUL, every
+// fourth column uses the FMA-pipe polynomial instead of the MUFU ex2.
+template <int MOD, bool EMUL>
+__device__ __forceinline__ float row_probs(float (&x)[4][32], const RowCtx& rc, float m_use,
+                                           uint32_t s_addr) {
+  float lsum = 0.f;
+  const float neg_m = -m_use;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t pk[16];
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      float arg0, arg1;
+      if constexpr (pure_scale(MOD)) {
+        arg0 = fmaf(x[c][e], rc.sl2, neg_m);
+        arg1 = fmaf(x[c][e + 1], rc.sl2, neg_m);
+      } else {
+        arg0 = x[c][e] + neg_m;
+        arg1 = x[c][e + 1] + neg_m;
+      }
+      const float pa = ex2_approx(arg0);
+      const float pb = (EMUL && (e & 3) == 2) ? exp2_poly(arg1) : ex2_approx(arg1);
+      s0 += pa;
+      s1 += pb;
+      pk[e >> 1] = pack_bf16x2(pa, pb);
+    }
+    lsum += s0 + s1;
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(s_addr + c * 16),
+        "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]),
+        "r"(pk[7]), "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]), "r"(pk[12]),
+        "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
+        : "memory");
+  }
+  return lsum;
+}
+
 template <int D, int MOD, bool HAS_LSE>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -168,6 +255,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(smem_u32(&bars->kv_empty[s]), 1);
     }
     bars->abort_flag = 0;
+    bars->never_set = 0;
     fence_mbar_init();
   }
   if (warp == 8) {  // allocate all 512 TMEM columns (one CTA per SM)
@@ -183,8 +271,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const WaitCtl wc{a.wait_ns, &bars->abort_flag, a.status};
+  const WaitCtl wc{a.wait_ns, smem_u32(&bars->abort_flag), a.status};
+  long long tr[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  (void)tr;
+  ATTN25_TRACE_ONLY(const long long t_start = clock64();)
 
+  // softcap and local boost keep the even split: their per-element mods need
+  // more registers than any split can give, so they spill either way
+  constexpr bool kSplitRegs = MOD != MOD_SOFTCAP && MOD != MOD_BOOST;
+  if (warp >= 8) {
+  if constexpr (kSplitRegs) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
   if (warp == 9) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -197,7 +293,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const UnitCoord uc = decode_unit(a, u);
         const int hk = uc.h / a.G;
         // Q buffers are free once the previous unit's QK^T products finished
-        if (!mbar_wait_thread(smem_u32(&bars->q_empty), (unit_iter & 1) ^ 1, wc)) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[1], mbar_wait_thread(smem_u32(&bars->q_empty), (unit_iter & 1) ^ 1, wc))) { ok = false; break; }
         mbar_arrive_expect_tx(smem_u32(&bars->q_full), 2 * Cfg::kTileBytes);
         ++q_loads;
         const int bh_q = uc.b * a.Hq + uc.h;
@@ -214,7 +310,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int which = 0; which < 2; ++which) {  // K then V
             const int slot = ring_pos % Cfg::kStages;
             const uint32_t phase = (ring_pos / Cfg::kStages) & 1;
-            if (!mbar_wait_thread(smem_u32(&bars->kv_empty[slot]), phase ^ 1, wc)) { ok = false; break; }
+            if (!ATTN25_TIMED(tr[2], mbar_wait_thread(smem_u32(&bars->kv_empty[slot]), phase ^ 1, wc))) { ok = false; break; }
             const uint32_t bar = smem_u32(&bars->kv_full[slot]);
             mbar_arrive_expect_tx(bar, Cfg::kTileBytes);
             load_tile<D>(ring + slot * Cfg::kTileBytes, which == 0 ? &tm_k : &tm_v, bar, kt * TILE,
@@ -227,8 +323,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (!ok) {
         // let copies already in flight land before the CTA exits
-        uint32_t local_flag = 0;
-        const WaitCtl drain_wc{a.wait_ns, &local_flag, a.status};
+        const WaitCtl drain_wc{a.wait_ns, smem_u32(&bars->never_set), a.status};
         for (int s = 0; s < Cfg::kStages; ++s) {
           if (slot_uses[s] == 0) continue;
           mbar_wait_thread(smem_u32(&bars->kv_full[s]), (slot_uses[s] - 1) & 1, drain_wc);
@@ -236,6 +331,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (q_loads > 0)
           mbar_wait_thread(smem_u32(&bars->q_full), (q_loads - 1) & 1, drain_wc);
       }
+      ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
+      trace_flush(a.trace, 48, tr);
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
@@ -248,7 +345,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t o_tmem[2] = {tmem + 256, tmem + 256 + D};
     for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
       const UnitCoord uc = decode_unit(a, u);
-      if (!mbar_wait_warp(smem_u32(&bars->q_full), unit_iter & 1, wc)) { ok = false; break; }
+      if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->q_full), unit_iter & 1, wc))) { ok = false; break; }
       tc_fence_after();
       PairIter it;
       it.init(a.tile_class, a.kv_count, a.kv_index, uc.b, uc.p, a.nQ, a.nK, a.Sq, a.Skv, MOD,
@@ -259,7 +356,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       bool o_started[2] = {false, false};
       if (has) {
         const int slot_k = ring_pos % Cfg::kStages;
-        if (!mbar_wait_warp(smem_u32(&bars->kv_full[slot_k]), (ring_pos / Cfg::kStages) & 1, wc)) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->kv_full[slot_k]), (ring_pos / Cfg::kStages) & 1, wc))) { ok = false; break; }
         tc_fence_after();
         if (lane == 0) {
 #pragma unroll
@@ -282,12 +379,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const bool has_n = it.next(kt_n, act_n[0], act_n[1], prt_n[0], prt_n[1]);
         const int slot_kn = ring_pos % Cfg::kStages;
         const uint32_t ph_kn = (ring_pos / Cfg::kStages) & 1;
-        if (!mbar_wait_warp(smem_u32(&bars->kv_full[slot_v]), ph_v, wc)) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->kv_full[slot_v]), ph_v, wc))) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           if (act[t]) {
-            if (!mbar_wait_warp(smem_u32(&bars->p_full[t]), p_cnt[t] & 1, wc)) { ok = false; break; }
+            if (!ATTN25_TIMED(tr[4 + t], mbar_wait_warp(smem_u32(&bars->p_full[t]), p_cnt[t] & 1, wc))) { ok = false; break; }
             ++p_cnt[t];
             tc_fence_after();
             if (lane == 0) {
@@ -299,7 +396,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
           if (has_n) {
             if (t == 0) {
-              if (!mbar_wait_warp(smem_u32(&bars->kv_full[slot_kn]), ph_kn, wc)) { ok = false; break; }
+              if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->kv_full[slot_kn]), ph_kn, wc))) { ok = false; break; }
               tc_fence_after();
             }
             if (act_n[t] && lane == 0) {
@@ -332,11 +429,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // drain: wait until every MMA this thread issued has completed
     if (lane == 0) {
       mma_commit(smem_u32(&bars->drain));
-      uint32_t dummy_flag = 0;
-      mbar_wait_thread(smem_u32(&bars->drain), 0, WaitCtl{a.wait_ns, &dummy_flag, a.status});
+      mbar_wait_thread(smem_u32(&bars->drain), 0, WaitCtl{a.wait_ns, smem_u32(&bars->never_set), a.status});
     }
     __syncwarp();
+    ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
+    trace_flush(a.trace, 32, tr);
+  }
   } else {
+    if constexpr (kSplitRegs) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     // ------------------------------------------------------------ softmax warpgroups
     const int t = warp >> 2;                  // query tile of the pair
     const int r = threadIdx.x & 127;          // row within the tile = TMEM lane
@@ -372,8 +472,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       bool act[2], prt[2];
       while (it.next(kt, act[0], act[1], prt[0], prt[1])) {
         if (!act[t]) continue;
-        if (!mbar_wait_warp(smem_u32(&bars->s_full[t]), s_cnt & 1, wc)) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->s_full[t]), s_cnt & 1, wc))) { ok = false; break; }
         ++s_cnt;
+        ATTN25_TRACE_ONLY(const long long t_tile = clock64(); tr[7] += 1;)
         tc_fence_after();
         const int k0 = kt * TILE;
         float x[4][32];
@@ -381,20 +482,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int c = 0; c < 4; ++c)
           tmem_ld32(s_addr + c * 32, reinterpret_cast<uint32_t(&)[32]>(x[c]));
         tmem_wait_ld();
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          transform32<MOD>(x[c], rc, a.mod, k0, c * 32, prt[t]);
-          float m0 = x[c][0], m1 = x[c][1], m2 = x[c][2], m3 = x[c][3];
-#pragma unroll
-          for (int e = 4; e < 32; e += 4) {
-            m0 = fmaxf(m0, x[c][e]);
-            m1 = fmaxf(m1, x[c][e + 1]);
-            m2 = fmaxf(m2, x[c][e + 2]);
-            m3 = fmaxf(m3, x[c][e + 3]);
-          }
-          mx = fmaxf(mx, fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)));
-        }
+        const float mx = prt[t] ? row_scores<MOD, true>(x, rc, a.mod, k0)
+                                : row_scores<MOD, false>(x, rc, a.mod, k0);
         const float m_new = fmaxf(m_run, mx);
         const bool need = m_new > m_run + kRescaleThreshold;
         if (__any_sync(0xffffffffu, need)) {
@@ -403,44 +492,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             // O must be complete (previous P V finished) before it is rescaled
             if (!mbar_wait_warp(smem_u32(&bars->o_full[t]), (p_cnt - 1) & 1, wc)) { ok = false; break; }
             tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t o[32];
-              tmem_ld32(o_addr + c * 32, o);
+#pragma unroll 1
+            for (int c = 0; c < D / 16; ++c) {
+              uint32_t o[16];
+              tmem_ld16(o_addr + c * 16, o);
               tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st32(o_addr + c * 32, o);
+              for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st16(o_addr + c * 16, o);
             }
           }
           l_run *= alpha;
           m_run = m_new;
+          ATTN25_TRACE_ONLY(tr[6] += 1;)
         }
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        float lsum = 0.f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-          float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float pa = ex2_approx(x[c][e] - m_use);
-            const float pb = ex2_approx(x[c][e + 1] - m_use);
-            s0 += pa;
-            s1 += pb;
-            pk[e >> 1] = pack_bf16x2(pa, pb);
-          }
-          lsum += s0 + s1;
-          // P (bf16 pairs) overwrites the first 64 columns of S
-          asm volatile(
-              "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-              "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(s_addr + c * 16),
-              "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]),
-              "r"(pk[7]), "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]), "r"(pk[12]),
-              "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
-              : "memory");
-        }
+        ATTN25_TRACE_ONLY(const long long t_mid = clock64(); tr[2] += t_mid - t_tile;)
+        // full tiles hold no -inf, so part of their exponentials can run on the FMA pipe
+        const float lsum = prt[t] ? row_probs<MOD, false>(x, rc, m_use, s_addr)
+                                  : row_probs<MOD, true>(x, rc, m_use, s_addr);
         l_run += lsum;
+        ATTN25_TRACE_ONLY(tr[3] += clock64() - t_mid;)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(smem_u32(&bars->p_full[t]));
@@ -449,7 +521,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (!ok) break;
       // ---- epilogue of this unit: O / l -> bf16, LSE
-      if (!mbar_wait_warp(smem_u32(&bars->o_final[t]), unit_iter & 1, wc)) { ok = false; break; }
+      if (!ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->o_final[t]), unit_iter & 1, wc))) { ok = false; break; }
+      ATTN25_TRACE_ONLY(const long long t_epi = clock64();)
       tc_fence_after();
       const bool row_valid = rc.row < a.Sq;
       const size_t row_idx = (static_cast<size_t>(uc.b) * a.Hq + uc.h) * a.Sq + rc.row;
@@ -480,7 +553,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           a.lse[row_idx] = (l_run > 0.f) ? (m_run + __log2f(l_run)) * LN2 : -INFINITY;
       }
       tc_fence_before();
+      ATTN25_TRACE_ONLY(tr[5] += clock64() - t_epi;)
     }
+    ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
+    trace_flush(a.trace, 16 * t, tr);
   }
 
   tc_fence_before();
@@ -501,6 +577,16 @@ template <int D, int MOD, bool LSE>
 cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const FwdArgs& a, int grid, cudaStream_t stream) {
   auto kernel = attn_fwd_kernel<D, MOD, LSE>;
+  // The register split assumes the kernel launches with kLaunchRegs per
+  // thread; with fewer, setmaxnreg.inc could wait forever, so refuse.
+  static int launch_regs = -1;
+  if (launch_regs < 0) {
+    cudaFuncAttributes attr;
+    cudaError_t e0 = cudaFuncGetAttributes(&attr, kernel);
+    if (e0 != cudaSuccess) return e0;
+    launch_regs = attr.numRegs;
+  }
+  if (launch_regs < kLaunchRegs) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        FwdCfg<D>::kAllocBytes);
   if (e != cudaSuccess) return e;

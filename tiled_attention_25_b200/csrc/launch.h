@@ -24,6 +24,7 @@ struct FwdArgs {
   const int32_t* fwd_order;
   uint64_t wait_ns;
   int* status;
+  unsigned long long* trace;  // profiling builds only (else nullptr)
 };
 
 struct BwdArgs {
@@ -46,6 +47,7 @@ struct BwdArgs {
   const int32_t* bwd_order;
   uint64_t wait_ns;
   int* status;
+  unsigned long long* trace;  // profiling builds only (else nullptr)
 };
 
 struct MaskArgs {

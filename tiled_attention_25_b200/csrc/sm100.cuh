@@ -6,15 +6,49 @@
 #include <cstdint>
 #include <cuda.h>
 
+#include "exp2_poly.h"
+
 namespace attn25 {
 
 // ------------------------------------------------------------------ status
 
 constexpr int kErrTimeout = -6;
 
+// Profiling builds (-DATTN25_TRACE) time selected waits and phases per warp
+// role with clock64 and add the totals into a device trace buffer; in normal
+// builds the macro is the bare expression and the counters compile away.
+#if defined(ATTN25_TRACE)
+#define ATTN25_TIMED(acc, expr)            \
+  ({                                       \
+    const long long _t0 = clock64();       \
+    auto _r = (expr);                      \
+    (acc) += clock64() - _t0;              \
+    _r;                                    \
+  })
+#define ATTN25_TRACE_ONLY(x) x
+#else
+#define ATTN25_TIMED(acc, expr) (expr)
+#define ATTN25_TRACE_ONLY(x)
+#endif
+
+// Add one warp's counters into the trace buffer (lane 0 only).
+template <int N>
+__device__ __forceinline__ void trace_flush(unsigned long long* trace, int base, const long long (&tr)[N]) {
+#if defined(ATTN25_TRACE)
+  if (trace != nullptr && (threadIdx.x & 31) == 0) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) atomicAdd(trace + base + i, static_cast<unsigned long long>(tr[i]));
+  }
+#else
+  (void)trace;
+  (void)base;
+  (void)tr;
+#endif
+}
+
 struct WaitCtl {
   uint64_t limit_ns;     // per-wait time limit
-  uint32_t* abort_flag;  // shared-memory flag: set once any role gave up
+  uint32_t abort_addr;   // shared-memory word: non-zero once any role gave up
   int* status;           // device status word (0, or the first error recorded)
 };
 
@@ -24,14 +58,22 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 
-__device__ __forceinline__ void record_error(int code, const WaitCtl& w) {
-  if (w.status != nullptr) atomicCAS(w.status, 0, code);
-  *reinterpret_cast<volatile uint32_t*>(w.abort_flag) = 1u;
+__device__ __forceinline__ uint32_t ld_shared_volatile(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
 }
 
-__device__ __forceinline__ bool aborted(const WaitCtl& w) {
-  return *reinterpret_cast<volatile uint32_t*>(w.abort_flag) != 0u;
+__device__ __forceinline__ void st_shared_volatile(uint32_t addr, uint32_t v) {
+  asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
+
+__device__ __forceinline__ void record_error(int code, WaitCtl w) {
+  if (w.status != nullptr) atomicCAS(w.status, 0, code);
+  st_shared_volatile(w.abort_addr, 1u);
+}
+
+__device__ __forceinline__ bool aborted(WaitCtl w) { return ld_shared_volatile(w.abort_addr) != 0u; }
 
 // ------------------------------------------------------------------ smem / mbarrier
 
@@ -71,7 +113,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait for the phase with the given parity, executed by ONE thread.  Returns
 // false (after recording a timeout) if the limit passes or another role
 // already gave up.
-static __device__ __noinline__ bool mbar_wait_thread(uint32_t bar, uint32_t parity, const WaitCtl& w) {
+static __device__ __forceinline__ bool mbar_wait_thread(uint32_t bar, uint32_t parity, WaitCtl w) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
@@ -87,7 +129,7 @@ static __device__ __noinline__ bool mbar_wait_thread(uint32_t bar, uint32_t pari
 // Warp-collective wait: every lane of the (converged) warp calls it and all
 // lanes get the same answer, so warp-collective instructions that follow stay
 // aligned even when the wait gives up.
-static __device__ __noinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtl& w) {
+static __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, WaitCtl w) {
   const uint64_t t0 = globaltimer();
   while (true) {
     const bool ok = mbar_try_wait(bar, parity);
@@ -241,6 +283,26 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
 // ------------------------------------------------------------------ descriptors
 
 // Shared-memory matrix descriptor, 128-byte swizzle, Blackwell version field.
@@ -275,6 +337,23 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe (finite x only): x = n + f with n = round(x) taken from
+// the low mantissa bits of x + 1.5 * 2^23 (round-to-nearest, Cody-Waite
+// style), 2^f from the minimax polynomial of exp2_poly.h, and 2^n added into
+// the exponent field.  x is clamped to -126 first, so tiny results become the
+// smallest normal number instead of garbage.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;
+  const float n = t - 12582912.0f;
+  const float f = x - n;
+  float p = fmaf(kExp2C4, f, kExp2C3);
+  p = fmaf(p, f, kExp2C2);
+  p = fmaf(p, f, kExp2C1);
+  p = fmaf(p, f, kExp2C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
