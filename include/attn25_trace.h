@@ -2,7 +2,7 @@
  * Profiling entry points of libattn25_trace.so, the build of attn25 compiled
  * with -DATTN25_TRACE.  Its kernels time selected barrier waits and phases
  * per warp role with clock64 and add them into a device counter buffer
- * (128 x uint64: forward roles at 0..63, backward roles at 64..127, 16 per
+ * (256 x uint64: forward roles at 0..63, backward roles at 128..255, 16 per
  * role).  The normal library (libattn25.so) does not export these.
  */
 #ifndef ATTN25_TRACE_H
@@ -14,7 +14,7 @@
 extern "C" {
 #endif
 
-/* Synchronise the device, then copy the first n (<= 128) counters to host memory. */
+/* Synchronise the device, then copy the first n (<= 256) counters to host memory. */
 ATTN25_API int attn_trace_read(unsigned long long* host_out, int n);
 
 /* Synchronise the device, then zero all counters. */

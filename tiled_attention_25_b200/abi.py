@@ -250,7 +250,7 @@ def attn_set_wait_limit_ms(ms: int):
     LIB.attn_set_wait_limit_ms(int(ms))
 
 
-def attn_trace_read(n: int = 128) -> list:
+def attn_trace_read(n: int = 256) -> list:
     """Per-role cycle counters of the profiling build (libattn25_trace.so)."""
     buf = (ctypes.c_ulonglong * n)()
     _check(LIB.attn_trace_read(buf, n), "attn_trace_read")

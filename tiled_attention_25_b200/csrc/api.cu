@@ -19,8 +19,8 @@ namespace attn25 {
 __device__ int g_attn_status;
 
 #if defined(ATTN25_TRACE)
-// Profiling builds: per-role cycle counters (forward at 0, backward at 64).
-__device__ unsigned long long g_attn_trace[128];
+// Profiling builds: per-role cycle counters (forward at 0, backward at 128).
+__device__ unsigned long long g_attn_trace[256];
 #endif
 
 namespace {
@@ -408,7 +408,7 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
   }
   a.wait_ns = wait_ns();
   a.status = d->status;
-  a.trace = d->trace == nullptr ? nullptr : d->trace + 64;
+  a.trace = d->trace == nullptr ? nullptr : d->trace + 128;
 
   CUtensorMap tq, tk, tv, tdo, tdq;
   if (!encode_bf16(&tq, q, D, Sq, B * Hq, 64) || !encode_bf16(&tk, k, D, Skv, B * Hkv, TILE) ||
@@ -427,7 +427,7 @@ ATTN25_API int attn_trace_read(unsigned long long* host_out, int n) {
   DeviceInfo* d = nullptr;
   int rc = current_device(&d);
   if (rc != ATTN_OK) return rc;
-  if (host_out == nullptr || n < 0 || n > 128 || d->trace == nullptr) return ATTN_ERR_ARG;
+  if (host_out == nullptr || n < 0 || n > 256 || d->trace == nullptr) return ATTN_ERR_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_LAUNCH;
   if (cudaMemcpy(host_out, d->trace, n * sizeof(unsigned long long), cudaMemcpyDeviceToHost) != cudaSuccess)
     return ATTN_ERR_LAUNCH;
@@ -440,7 +440,7 @@ ATTN25_API int attn_trace_reset(void) {
   if (rc != ATTN_OK) return rc;
   if (d->trace == nullptr) return ATTN_ERR_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_LAUNCH;
-  return cudaMemset(d->trace, 0, 128 * sizeof(unsigned long long)) == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+  return cudaMemset(d->trace, 0, 256 * sizeof(unsigned long long)) == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 #endif
 

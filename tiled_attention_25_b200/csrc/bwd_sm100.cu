@@ -33,8 +33,17 @@ namespace attn25 {
 
 namespace {
 
-constexpr int kBwdThreads = 320;
+constexpr int kBwdThreads = 512;
 constexpr int BM = 64;  // query rows per step
+// Warpgroups: 0 = P^T, 1 = dS^T, 2 = dQ drain, 3 = MMA (warp 12), TMA (warp 13).
+// Register split (setmaxnreg) of the 512 x 128 launch pool, per warpgroup.
+constexpr int kBwdLaunchRegs = 128;
+constexpr int kRegsP = 160;
+constexpr int kRegsDS = 152;
+constexpr int kRegsDrain = 96;
+constexpr int kRegsCtl = 104;
+static_assert(128 * (kRegsP + kRegsDS + kRegsDrain + kRegsCtl) <= kBwdThreads * kBwdLaunchRegs,
+              "register split");
 
 template <int D>
 struct BwdCfg {
@@ -52,8 +61,10 @@ struct BwdCfg {
   static constexpr int kBarOff = kStgOff + kStgBytes;
   static constexpr int kSmemBytes = kBarOff + 1024;
   static constexpr int kAllocBytes = kSmemBytes + 1024;
-  // TMEM columns
-  static constexpr int kColS = 0, kColDP = 64, kColDV = 128, kColDK = 128 + D, kColDQ = 128 + 2 * D;
+  // TMEM columns: two S^T buffers (P^T overwrites their first 32 columns), dP^T,
+  // the dV and dK accumulators, dQ^T
+  static constexpr int kColS = 0, kColDP = 128, kColDV = 192, kColDK = 192 + D, kColDQ = 192 + 2 * D;
+  static_assert(kColDQ + BM <= 512, "TMEM columns");
   static constexpr uint32_t kIdescST = idesc_bf16_f32(128, BM, false, false);   // K Q^T, V dO^T
   static constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, false, true);    // P^T dO, dS^T Q
   static constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, BM, true, true);     // K^T dS^T
@@ -62,7 +73,8 @@ struct BwdCfg {
 struct BwdBarriers {
   uint64_t kv_full, kv_empty;
   uint64_t q_full[2], q_empty[2];
-  uint64_t s_full, dp_full, p_ready, ds_ready;
+  uint64_t s_full[2], s_free[2], p_ready[2];
+  uint64_t dp_full, ds_ready;
   uint64_t ds_empty[2];
   uint64_t dq_full, dq_empty;
   uint64_t stg_written, stg_free;
@@ -220,12 +232,90 @@ __device__ __forceinline__ void issue_st(uint32_t d_tmem, uint32_t a_smem, uint3
   }
 }
 
+
+// Kept query interval of key row kv (the transposed form of the row
+// intervals): causal [kv, Sq), window [kv, kv + W), document [kv, end of kv's
+// document); key rows past Skv keep nothing.
+template <int MOD>
+__device__ __forceinline__ void key_interval(const BwdArgs& a, int b, int kv, int& qlo, int& qhi) {
+  qlo = 0;
+  qhi = a.Sq - 1;
+  if constexpr (MOD == MOD_CAUSAL) {
+    qlo = kv;
+  } else if constexpr (MOD == MOD_WINDOW) {
+    qlo = kv;
+    qhi = min(qhi, kv + a.mod.window - 1);
+  } else if constexpr (MOD == MOD_DOCUMENT) {
+    qlo = kv;
+    const int32_t* offs = a.mod.doc_offsets + static_cast<size_t>(b) * (a.mod.num_docs + 1);
+    const int kvc = min(kv, a.Skv - 1);
+    int lo = 0, hi = a.mod.num_docs;  // the document holding kvc, then its end
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(offs + mid) <= kvc) lo = mid; else hi = mid;
+    }
+    qhi = min(qhi, __ldg(offs + lo + 1) - 1);
+  }
+  if (kv >= a.Skv) qhi = qlo - 1;
+}
+
+// One key row of S^T (raw q.k for 64 queries) -> P^T = 2^(x - LSE2) in place.
+template <int MOD>
+__device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h, float dq0, int q0,
+                                        int qlo, int qhi, bool pred, const float* lse2_s) {
+  float aux = 0.f, aux2 = 0.f;
+  if constexpr (MOD == MOD_ALIBI) aux = alibi_slope(a.mod, h, a.Hq) * LOG2E;
+  if constexpr (MOD == MOD_SOFTCAP) {
+    aux = a.scale / a.mod.softcap;
+    aux2 = a.mod.softcap * LOG2E;
+  }
+  if constexpr (MOD == MOD_BOOST) aux = a.mod.boost * a.sl2;
+#pragma unroll
+  for (int c = 0; c < BM; ++c) {
+    float v = x[c];
+    if constexpr (MOD == MOD_ALIBI) {
+      v = fmaf(v, a.sl2, -aux * fabsf(dq0 + static_cast<float>(c)));
+    } else if constexpr (MOD == MOD_SOFTCAP) {
+      v = aux2 * tanhf(v * aux);
+    } else if constexpr (MOD == MOD_BOOST) {
+      const bool inside = fabsf(dq0 + static_cast<float>(c)) < static_cast<float>(a.mod.boost_radius);
+      v = v * (inside ? aux : a.sl2);
+    } else {
+      v = v * a.sl2;
+    }
+    if (pred) {
+      const int qq = q0 + c;
+      v = (qq >= qlo && qq <= qhi) ? v : -INFINITY;
+    }
+    x[c] = ex2_approx(v - lse2_s[c]);  // 0 where masked or on padding rows (LSE2 = +inf)
+  }
+}
+
+// One accumulator row (dV or dK) of this thread's key: TMEM fp32 -> mul -> bf16 -> global.
 template <int D>
-struct BwdRow {
-  int kv;        // absolute key row of this thread
-  int qlo, qhi;  // kept query interval of this key (transposed mask)
-  float sl2, aux, aux2, dmod_in;
-};
+__device__ __forceinline__ void store_acc_rows(__nv_bfloat16* dst, uint32_t src, float mul, bool have,
+                                               bool row_ok) {
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    if (have) {
+      tmem_ld32(src + c * 32, o);
+      tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = 0u;
+    }
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * mul, __uint_as_float(o[2 * e + 1]) * mul);
+    if (row_ok) {
+      uint4* p = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) p[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+    }
+  }
+}
 
 template <int D, int MOD>
 __global__ void __launch_bounds__(kBwdThreads, 1)
@@ -242,35 +332,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t v_smem = sbase + Cfg::kVOff;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  constexpr bool kSplitRegs = MOD != MOD_SOFTCAP && MOD != MOD_BOOST;
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bars->kv_full), 1);
     mbar_init(smem_u32(&bars->kv_empty), 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(smem_u32(&bars->q_full[s]), 1);
-      mbar_init(smem_u32(&bars->q_empty[s]), 1);
-      mbar_init(smem_u32(&bars->ds_empty[s]), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&bars->q_full[b]), 1);
+      mbar_init(smem_u32(&bars->q_empty[b]), 1);
+      mbar_init(smem_u32(&bars->ds_empty[b]), 1);
+      mbar_init(smem_u32(&bars->s_full[b]), 1);
+      mbar_init(smem_u32(&bars->s_free[b]), 128);
+      mbar_init(smem_u32(&bars->p_ready[b]), 128);
     }
-    mbar_init(smem_u32(&bars->s_full), 1);
     mbar_init(smem_u32(&bars->dp_full), 1);
-    mbar_init(smem_u32(&bars->p_ready), 128);
     mbar_init(smem_u32(&bars->ds_ready), 128);
     mbar_init(smem_u32(&bars->dq_full), 1);
     mbar_init(smem_u32(&bars->dq_empty), 128);
     mbar_init(smem_u32(&bars->stg_written), 128);
     mbar_init(smem_u32(&bars->stg_free), 1);
     mbar_init(smem_u32(&bars->acc_full), 1);
-    mbar_init(smem_u32(&bars->acc_empty), 128);
+    mbar_init(smem_u32(&bars->acc_empty), 256);
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort_flag = 0;
     bars->never_set = 0;
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(smem_u32(&bars->tmem_base), 512);
     tmem_relinquish();
   }
-  if (warp == 9 && lane == 0) {
+  if (warp == 13 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
@@ -286,190 +378,176 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   (void)tr;
   ATTN25_TRACE_ONLY(const long long t_start = clock64();)
 
-  if (warp == 9) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+  if (warp >= 12) {
+    if constexpr (kSplitRegs) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
+    if (warp == 13) {
+      // ---------------------------------------------------------- TMA producer
+      if (lane == 0) {
+        int unit_iter = 0, step = 0;
+        uint32_t kv_loads = 0, stage_uses[2] = {0, 0};
+        bool ok = true;
+        for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+          const BwdUnit un = decode_bwd_unit(a, u);
+          if (!ATTN25_TIMED(tr[1], mbar_wait_thread(smem_u32(&bars->kv_empty), (unit_iter & 1) ^ 1, wc))) { ok = false; break; }
+          mbar_arrive_expect_tx(smem_u32(&bars->kv_full), 2 * Cfg::kKVBytes);
+          ++kv_loads;
+          const int bh_kv = un.b * a.Hkv + un.hk;
+          load_kv_tile<D>(k_smem, &tm_k, smem_u32(&bars->kv_full), un.kt * TILE, bh_kv);
+          load_kv_tile<D>(v_smem, &tm_v, smem_u32(&bars->kv_full), un.kt * TILE, bh_kv);
+          StepIter it;
+          it.init(a, un);
+          int g, q0;
+          bool pred;
+          while (it.next(g, q0, pred)) {
+            const int s = step & 1;
+            if (!ATTN25_TIMED(tr[2], mbar_wait_thread(smem_u32(&bars->q_empty[s]), ((step >> 1) & 1) ^ 1, wc))) { ok = false; break; }
+            const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
+            const uint32_t bar = smem_u32(&bars->q_full[s]);
+            mbar_arrive_expect_tx(bar, 2 * Cfg::kQBytes + 2 * BM * 4);
+            ++stage_uses[s];
+            const int bh = un.b * a.Hq + un.hk * a.G + g;
+            load_q_tile<D>(st, &tm_q, bar, q0, bh);
+            load_q_tile<D>(st + Cfg::kQBytes, &tm_do, bar, q0, bh);
+            const size_t row = static_cast<size_t>(bh) * a.Sq_pad + q0;
+            bulk_load_1d(st + 2 * Cfg::kQBytes, a.lse2 + row, BM * 4, bar);
+            bulk_load_1d(st + 2 * Cfg::kQBytes + 512, a.delta + row, BM * 4, bar);
+            ++step;
+          }
+        }
+        if (!ok) {
+          const WaitCtl dwc{a.wait_ns, smem_u32(&bars->never_set), a.status};
+          if (kv_loads) mbar_wait_thread(smem_u32(&bars->kv_full), (kv_loads - 1) & 1, dwc);
+          for (int s = 0; s < 2; ++s)
+            if (stage_uses[s]) mbar_wait_thread(smem_u32(&bars->q_full[s]), (stage_uses[s] - 1) & 1, dwc);
+        }
+        ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
+        trace_flush(a.trace, 48, tr);
+      }
+    } else if (warp == 12) {
+      // ---------------------------------------------------------- MMA issuer
+      const uint32_t t_dp = tmem + Cfg::kColDP;
+      const uint32_t t_dv = tmem + Cfg::kColDV, t_dk = tmem + Cfg::kColDK, t_dq = tmem + Cfg::kColDQ;
       int unit_iter = 0, step = 0;
-      uint32_t kv_loads = 0, stage_uses[2] = {0, 0};
+      uint32_t ds_cnt = 0, dq_cnt = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
         const BwdUnit un = decode_bwd_unit(a, u);
-        if (!ATTN25_TIMED(tr[1], mbar_wait_thread(smem_u32(&bars->kv_empty), (unit_iter & 1) ^ 1, wc))) { ok = false; break; }
-        mbar_arrive_expect_tx(smem_u32(&bars->kv_full), 2 * Cfg::kKVBytes);
-        ++kv_loads;
-        const int bh_kv = un.b * a.Hkv + un.hk;
-        load_kv_tile<D>(k_smem, &tm_k, smem_u32(&bars->kv_full), un.kt * TILE, bh_kv);
-        load_kv_tile<D>(v_smem, &tm_v, smem_u32(&bars->kv_full), un.kt * TILE, bh_kv);
+        if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->kv_full), unit_iter & 1, wc))) { ok = false; break; }
+        // dK, dV accumulators are free once the previous unit's epilogue read them
+        if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->acc_empty), (unit_iter & 1) ^ 1, wc))) { ok = false; break; }
+        tc_fence_after();
         StepIter it;
         it.init(a, un);
         int g, q0;
         bool pred;
-        while (it.next(g, q0, pred)) {
+        bool has = it.next(g, q0, pred);
+        int n_steps = 0;
+        if (has) {  // S^T and dP^T of the first step
           const int s = step & 1;
-          if (!ATTN25_TIMED(tr[2], mbar_wait_thread(smem_u32(&bars->q_empty[s]), ((step >> 1) & 1) ^ 1, wc))) { ok = false; break; }
-          const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
-          const uint32_t bar = smem_u32(&bars->q_full[s]);
-          mbar_arrive_expect_tx(bar, 2 * Cfg::kQBytes + 2 * BM * 4);
-          ++stage_uses[s];
-          const int bh = un.b * a.Hq + un.hk * a.G + g;
-          load_q_tile<D>(st, &tm_q, bar, q0, bh);
-          load_q_tile<D>(st + Cfg::kQBytes, &tm_do, bar, q0, bh);
-          const size_t row = static_cast<size_t>(bh) * a.Sq_pad + q0;
-          bulk_load_1d(st + 2 * Cfg::kQBytes, a.lse2 + row, BM * 4, bar);
-          bulk_load_1d(st + 2 * Cfg::kQBytes + 512, a.delta + row, BM * 4, bar);
-          ++step;
-        }
-      }
-      if (!ok) {
-        const WaitCtl dwc{a.wait_ns, smem_u32(&bars->never_set), a.status};
-        if (kv_loads) mbar_wait_thread(smem_u32(&bars->kv_full), (kv_loads - 1) & 1, dwc);
-        for (int s = 0; s < 2; ++s)
-          if (stage_uses[s]) mbar_wait_thread(smem_u32(&bars->q_full[s]), (stage_uses[s] - 1) & 1, dwc);
-      }
-      ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
-      trace_flush(a.trace, 48, tr);
-    }
-  } else if (warp == 8) {
-    // ------------------------------------------------------------ MMA issuer
-    const uint32_t t_s = tmem + Cfg::kColS, t_dp = tmem + Cfg::kColDP;
-    const uint32_t t_dv = tmem + Cfg::kColDV, t_dk = tmem + Cfg::kColDK, t_dq = tmem + Cfg::kColDQ;
-    int unit_iter = 0, step = 0;
-    uint32_t p_cnt = 0, ds_cnt = 0, dq_cnt = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
-      const BwdUnit un = decode_bwd_unit(a, u);
-      if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->kv_full), unit_iter & 1, wc))) { ok = false; break; }
-      // dK, dV accumulators are free once the previous unit's epilogue read them
-      if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->acc_empty), (unit_iter & 1) ^ 1, wc))) { ok = false; break; }
-      tc_fence_after();
-      StepIter it;
-      it.init(a, un);
-      int g, q0;
-      bool pred;
-      bool has = it.next(g, q0, pred);
-      int n_steps = 0;
-      // prologue: S^T and dP^T of the first step
-      if (has) {
-        const int s = step & 1;
-        if (!ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step >> 1) & 1, wc))) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
-        if (lane == 0) {
-          issue_st<D>(t_s, k_smem, st);
-          mma_commit(smem_u32(&bars->s_full));
-          issue_st<D>(t_dp, v_smem, st + Cfg::kQBytes);
-          mma_commit(smem_u32(&bars->dp_full));
-        }
-        __syncwarp();
-      }
-      while (has) {
-        const int s = step & 1;
-        const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
-        // dV += P^T dO once the probabilities are in tensor memory
-        if (!ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->p_ready), p_cnt & 1, wc))) { ok = false; break; }
-        ++p_cnt;
-        tc_fence_after();
-        if (lane == 0) {
-#pragma unroll
-          for (int kk = 0; kk < BM / 16; ++kk)
-            mma_ts(t_dv, t_s + kk * 8, smem_desc_sw128(st + Cfg::kQBytes + kk * 2048, BM * 128, 1024),
-                   Cfg::kIdescAcc, (n_steps > 0 || kk > 0) ? 1u : 0u);
-        }
-        __syncwarp();
-        int g_n, q0_n;
-        bool pred_n;
-        const bool has_n = it.next(g_n, q0_n, pred_n);
-        const int s_n = (step + 1) & 1;
-        const uint32_t st_n = sbase + Cfg::kStageOff + s_n * Cfg::kStageBytes;
-        if (has_n) {  // S^T of the next step overlaps this step's dS work
-          if (!ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s_n]), ((step + 1) >> 1) & 1, wc))) { ok = false; break; }
+          if (!ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step >> 1) & 1, wc))) { ok = false; break; }
+          if (!ATTN25_TIMED(tr[8], mbar_wait_warp(smem_u32(&bars->s_free[s]), ((step >> 1) & 1) ^ 1, wc))) { ok = false; break; }
           tc_fence_after();
+          const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
           if (lane == 0) {
-            issue_st<D>(t_s, k_smem, st_n);
-            mma_commit(smem_u32(&bars->s_full));
+            issue_st<D>(tmem + Cfg::kColS + s * BM, k_smem, st);
+            mma_commit(smem_u32(&bars->s_full[s]));
+            issue_st<D>(t_dp, v_smem, st + Cfg::kQBytes);
+            mma_commit(smem_u32(&bars->dp_full));
           }
           __syncwarp();
         }
-        // dK += dS^T Q and dQ^T = K^T dS^T once dS^T is in shared memory
-        if (!ATTN25_TIMED(tr[5], mbar_wait_warp(smem_u32(&bars->ds_ready), ds_cnt & 1, wc))) { ok = false; break; }
-        const uint32_t ds_smem = sbase + Cfg::kDSOff + (ds_cnt & 1) * Cfg::kDSBytes;
-        ++ds_cnt;
-        // the dQ^T columns must have been drained by the previous step
-        if (!ATTN25_TIMED(tr[6], mbar_wait_warp(smem_u32(&bars->dq_empty), (dq_cnt & 1) ^ 1, wc))) { ok = false; break; }
-        tc_fence_after();
-        if (lane == 0) {
-#pragma unroll
-          for (int kk = 0; kk < BM / 16; ++kk)
-            mma_ss(t_dk, smem_desc_sw128(ds_smem + kk * 32, 16, 1024),
-                   smem_desc_sw128(st + kk * 2048, BM * 128, 1024), Cfg::kIdescAcc,
-                   (n_steps > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < TILE / 16; ++kk)
-            mma_ss(t_dq, smem_desc_sw128(k_smem + kk * 2048, TILE * 128, 1024),
-                   smem_desc_sw128(ds_smem + kk * 2048, BM * 128, 1024), Cfg::kIdescDQ,
-                   kk > 0 ? 1u : 0u);
-          mma_commit(smem_u32(&bars->dq_full));
-          mma_commit(smem_u32(&bars->q_empty[s]));
-          mma_commit(smem_u32(&bars->ds_empty[(ds_cnt - 1) & 1]));
-          if (has_n) {
-            issue_st<D>(t_dp, v_smem, st_n + Cfg::kQBytes);
-            mma_commit(smem_u32(&bars->dp_full));
+        while (has) {
+          const int s = step & 1;  // stage and S^T buffer of this step
+          const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
+          int g_n, q0_n;
+          bool pred_n;
+          const bool has_n = it.next(g_n, q0_n, pred_n);
+          const int s_n = (step + 1) & 1;
+          const uint32_t st_n = sbase + Cfg::kStageOff + s_n * Cfg::kStageBytes;
+          if (has_n) {  // S^T of the next step into the other buffer, ahead of this step's dS
+            if (!ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s_n]), ((step + 1) >> 1) & 1, wc))) { ok = false; break; }
+            if (!ATTN25_TIMED(tr[8], mbar_wait_warp(smem_u32(&bars->s_free[s_n]), (((step + 1) >> 1) & 1) ^ 1, wc))) { ok = false; break; }
+            tc_fence_after();
+            if (lane == 0) {
+              issue_st<D>(tmem + Cfg::kColS + s_n * BM, k_smem, st_n);
+              mma_commit(smem_u32(&bars->s_full[s_n]));
+            }
+            __syncwarp();
           }
+          // dV += P^T dO once P^T is in tensor memory
+          if (!ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->p_ready[s]), (step >> 1) & 1, wc))) { ok = false; break; }
+          tc_fence_after();
+          if (lane == 0) {
+#pragma unroll
+            for (int kk = 0; kk < BM / 16; ++kk)
+              mma_ts(t_dv, tmem + Cfg::kColS + s * BM + kk * 8,
+                     smem_desc_sw128(st + Cfg::kQBytes + kk * 2048, BM * 128, 1024), Cfg::kIdescAcc,
+                     (n_steps > 0 || kk > 0) ? 1u : 0u);
+          }
+          __syncwarp();
+          // dK += dS^T Q and dQ^T = K^T dS^T once dS^T is in shared memory
+          if (!ATTN25_TIMED(tr[5], mbar_wait_warp(smem_u32(&bars->ds_ready), ds_cnt & 1, wc))) { ok = false; break; }
+          const uint32_t ds_smem = sbase + Cfg::kDSOff + (ds_cnt & 1) * Cfg::kDSBytes;
+          ++ds_cnt;
+          // the dQ^T columns must have been drained by the previous step
+          if (!ATTN25_TIMED(tr[6], mbar_wait_warp(smem_u32(&bars->dq_empty), (dq_cnt & 1) ^ 1, wc))) { ok = false; break; }
+          tc_fence_after();
+          if (lane == 0) {
+#pragma unroll
+            for (int kk = 0; kk < BM / 16; ++kk)
+              mma_ss(t_dk, smem_desc_sw128(ds_smem + kk * 32, 16, 1024),
+                     smem_desc_sw128(st + kk * 2048, BM * 128, 1024), Cfg::kIdescAcc,
+                     (n_steps > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+            for (int kk = 0; kk < TILE / 16; ++kk)
+              mma_ss(t_dq, smem_desc_sw128(k_smem + kk * 2048, TILE * 128, 1024),
+                     smem_desc_sw128(ds_smem + kk * 2048, BM * 128, 1024), Cfg::kIdescDQ,
+                     kk > 0 ? 1u : 0u);
+            mma_commit(smem_u32(&bars->dq_full));
+            mma_commit(smem_u32(&bars->q_empty[s]));
+            mma_commit(smem_u32(&bars->ds_empty[(ds_cnt - 1) & 1]));
+            if (has_n) {
+              issue_st<D>(t_dp, v_smem, st_n + Cfg::kQBytes);
+              mma_commit(smem_u32(&bars->dp_full));
+            }
+          }
+          __syncwarp();
+          ++dq_cnt;
+          ++n_steps;
+          ++step;
+          has = has_n;
+          g = g_n;
+          q0 = q0_n;
+          pred = pred_n;
+        }
+        if (!ok) break;
+        if (lane == 0) {
+          mma_commit(smem_u32(&bars->kv_empty));
+          mma_commit(smem_u32(&bars->acc_full));
         }
         __syncwarp();
-        ++dq_cnt;
-        ++n_steps;
-        ++step;
-        has = has_n;
-        g = g_n;
-        q0 = q0_n;
-        pred = pred_n;
       }
-      if (!ok) break;
       if (lane == 0) {
-        mma_commit(smem_u32(&bars->kv_empty));
-        mma_commit(smem_u32(&bars->acc_full));
+        mma_commit(smem_u32(&bars->drain));
+        mbar_wait_thread(smem_u32(&bars->drain), 0, WaitCtl{a.wait_ns, smem_u32(&bars->never_set), a.status});
       }
       __syncwarp();
+      ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start; tr[7] = step;)
+      trace_flush(a.trace, 32, tr);
     }
-    if (lane == 0) {
-      mma_commit(smem_u32(&bars->drain));
-      mbar_wait_thread(smem_u32(&bars->drain), 0, WaitCtl{a.wait_ns, smem_u32(&bars->never_set), a.status});
-    }
-    __syncwarp();
-    ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start; tr[7] = step;)
-    trace_flush(a.trace, 32, tr);
   } else if (warp < 4) {
-    // ------------------------------------------------------------ P^T / dS^T (thread = key row)
+    if constexpr (kSplitRegs) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsP));
+    // ------------------------------------------------------------ P^T (thread = key row)
     const int r = threadIdx.x;  // TMEM lane = key row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t t_s = tmem + Cfg::kColS + lane_off, t_dp = tmem + Cfg::kColDP + lane_off;
-    const uint32_t t_dv = tmem + Cfg::kColDV + lane_off, t_dk = tmem + Cfg::kColDK + lane_off;
+    const uint32_t t_dv = tmem + Cfg::kColDV + lane_off;
     int unit_iter = 0, step = 0;
-    uint32_t s_cnt = 0, dp_cnt = 0, ds_cnt = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
       const BwdUnit un = decode_bwd_unit(a, u);
       const int kv = un.kt * TILE + r;
-      // kept query interval of this key: transposed form of the row intervals
-      int qlo = 0, qhi = a.Sq - 1;
-      if constexpr (MOD == MOD_CAUSAL) {
-        qlo = kv;
-      } else if constexpr (MOD == MOD_WINDOW) {
-        qlo = kv;
-        qhi = min(qhi, kv + a.mod.window - 1);
-      } else if constexpr (MOD == MOD_DOCUMENT) {
-        qlo = kv;
-        const int32_t* offs = a.mod.doc_offsets + static_cast<size_t>(un.b) * (a.mod.num_docs + 1);
-        const int kvc = min(kv, a.Skv - 1);
-        int lo = 0, hi = a.mod.num_docs;  // find the document end after kvc
-        while (hi - lo > 1) {
-          const int mid = (lo + hi) >> 1;
-          if (__ldg(offs + mid) <= kvc) lo = mid; else hi = mid;
-        }
-        qhi = min(qhi, __ldg(offs + lo + 1) - 1);
-      }
-      if (kv >= a.Skv) qhi = qlo - 1;  // key rows past the end keep nothing
+      int qlo, qhi;
+      key_interval<MOD>(a, un.b, kv, qlo, qhi);
       StepIter it;
       it.init(a, un);
       int g, q0;
@@ -477,86 +555,103 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int n_steps = 0;
       while (it.next(g, q0, pred)) {
         const int s = step & 1;
-        const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
         const float* lse2_s = reinterpret_cast<const float*>(smem + Cfg::kStageOff + s * Cfg::kStageBytes + 2 * Cfg::kQBytes);
-        const float* delta_s = lse2_s + 128;
-        // stage contents (Q, dO, statistics) have landed
+        const uint32_t t_s = tmem + Cfg::kColS + s * BM + lane_off;
         if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step >> 1) & 1, wc))) { ok = false; break; }
-        if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->s_full), s_cnt & 1, wc))) { ok = false; break; }
-        ++s_cnt;
+        if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->s_full[s]), (step >> 1) & 1, wc))) { ok = false; break; }
         tc_fence_after();
         ATTN25_TRACE_ONLY(const long long t_p = clock64();)
         const int h = un.hk * a.G + g;
-        float sl2 = a.sl2, aux = 0.f, aux2 = 0.f;
-        if constexpr (MOD == MOD_ALIBI) aux = alibi_slope(a.mod, h, a.Hq) * LOG2E;
-        if constexpr (MOD == MOD_SOFTCAP) {
-          aux = a.scale / a.mod.softcap;
-          aux2 = a.mod.softcap * LOG2E;
-        }
-        if constexpr (MOD == MOD_BOOST) aux = a.mod.boost * a.sl2;
         float x[BM];
         tmem_ld32(t_s, reinterpret_cast<uint32_t(&)[32]>(x[0]));
         tmem_ld32(t_s + 32, reinterpret_cast<uint32_t(&)[32]>(x[32]));
         tmem_wait_ld();
-        const float dq0 = static_cast<float>(q0 - kv);  // (query - key) of column 0
-        // softcap: d s'/d s = 1 - tanh^2, kept as fp16 pairs to save registers
-        __half2 dcap[MOD == MOD_SOFTCAP ? BM / 2 : 1];
-        (void)dcap;
-#pragma unroll
-        for (int c = 0; c < BM; ++c) {
-          float v = x[c];
-          if constexpr (MOD == MOD_ALIBI) {
-            v = fmaf(v, sl2, -aux * fabsf(dq0 + static_cast<float>(c)));
-          } else if constexpr (MOD == MOD_SOFTCAP) {
-            const float t = tanhf(v * aux);
-            if (c & 1) dcap[c >> 1].y = __float2half_rn(1.f - t * t);
-            else dcap[c >> 1].x = __float2half_rn(1.f - t * t);
-            v = aux2 * t;
-          } else if constexpr (MOD == MOD_BOOST) {
-            const bool inside = fabsf(dq0 + static_cast<float>(c)) < static_cast<float>(a.mod.boost_radius);
-            v = v * (inside ? aux : sl2);
-          } else {
-            v = v * sl2;
-          }
-          if (pred) {
-            const int qq = q0 + c;
-            v = (qq >= qlo && qq <= qhi) ? v : -INFINITY;
-          }
-          x[c] = ex2_approx(v - lse2_s[c]);  // P^T, 0 where masked
-        }
-        // P^T (bf16 pairs) over the first 32 columns of S^T
+        probs_t<MOD>(x, a, h, static_cast<float>(q0 - kv), q0, qlo, qhi, pred, lse2_s);
+        // P^T (bf16 pairs) over the first 32 columns of this S^T buffer
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
         tmem_st32(t_s, pk);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(smem_u32(&bars->p_ready));
+        mbar_arrive(smem_u32(&bars->p_ready[s]));
         ATTN25_TRACE_ONLY(tr[3] += clock64() - t_p;)
-        // dS^T = P^T (dP^T - Delta) ds'/ds
+        ++n_steps;
+        ++step;
+      }
+      if (!ok) break;
+      // ---- unit epilogue: dV -> bf16
+      if (!ATTN25_TIMED(tr[7], mbar_wait_warp(smem_u32(&bars->acc_full), unit_iter & 1, wc))) { ok = false; break; }
+      tc_fence_after();
+      ATTN25_TRACE_ONLY(const long long t_e = clock64();)
+      store_acc_rows<D>(a.dv + ((static_cast<size_t>(un.b) * a.Hkv + un.hk) * a.Skv + kv) * D, t_dv, 1.f,
+                        n_steps > 0, kv < a.Skv);
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bars->acc_empty));
+      ATTN25_TRACE_ONLY(tr[8] += clock64() - t_e;)
+    }
+    ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
+    trace_flush(a.trace, 0, tr);
+  } else if (warp < 8) {
+    if constexpr (kSplitRegs) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsDS));
+    // ------------------------------------------------------------ dS^T (thread = key row)
+    const int r = threadIdx.x - 128;
+    const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
+    const uint32_t t_dp = tmem + Cfg::kColDP + lane_off, t_dk = tmem + Cfg::kColDK + lane_off;
+    int unit_iter = 0, step = 0;
+    uint32_t dp_cnt = 0, ds_cnt = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+      const BwdUnit un = decode_bwd_unit(a, u);
+      const int kv = un.kt * TILE + r;
+      StepIter it;
+      it.init(a, un);
+      int g, q0;
+      bool pred;
+      int n_steps = 0;
+      while (it.next(g, q0, pred)) {
+        const int s = step & 1;
+        const float* stats = reinterpret_cast<const float*>(smem + Cfg::kStageOff + s * Cfg::kStageBytes + 2 * Cfg::kQBytes);
+        const float* delta_s = stats + 128;
+        const uint32_t t_p = tmem + Cfg::kColS + s * BM + lane_off;
+        if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step >> 1) & 1, wc))) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->p_ready[s]), (step >> 1) & 1, wc))) { ok = false; break; }
         if (!ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->dp_full), dp_cnt & 1, wc))) { ok = false; break; }
-        ATTN25_TRACE_ONLY(const long long t_ds = clock64();)
         ++dp_cnt;
         tc_fence_after();
+        ATTN25_TRACE_ONLY(const long long t_ds = clock64();)
         float dp[BM];
+        uint32_t pb[32];
         tmem_ld32(t_dp, reinterpret_cast<uint32_t(&)[32]>(dp[0]));
         tmem_ld32(t_dp + 32, reinterpret_cast<uint32_t(&)[32]>(dp[32]));
+        tmem_ld32(t_p, pb);
         tmem_wait_ld();
+        // P^T of this buffer has been read: the next-but-one S^T may overwrite it
+        tc_fence_before();
+        mbar_arrive(smem_u32(&bars->s_free[s]));
         // the dS buffer is free once the MMAs of two steps ago completed
         if (!ATTN25_TIMED(tr[5], mbar_wait_warp(smem_u32(&bars->ds_empty[ds_cnt & 1]), ((ds_cnt >> 1) & 1) ^ 1, wc))) { ok = false; break; }
         uint8_t* ds_row = smem + Cfg::kDSOff + (ds_cnt & 1) * Cfg::kDSBytes + r * 128;
         ++ds_cnt;
+        const float dq0 = static_cast<float>(q0 - kv);
+        float cl2_inv = 0.f;
+        if constexpr (MOD == MOD_SOFTCAP) cl2_inv = 1.f / (a.mod.softcap * LOG2E);
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16) {  // 8 columns (16 bytes) at a time
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = c16 * 8 + 2 * e;
-            float d0 = x[c] * (dp[c] - delta_s[c]);
-            float d1 = x[c + 1] * (dp[c + 1] - delta_s[c + 1]);
+            const uint32_t pp = pb[c >> 1];
+            const float p0 = __uint_as_float(pp << 16), p1 = __uint_as_float(pp & 0xffff0000u);
+            float d0 = p0 * (dp[c] - delta_s[c]);
+            float d1 = p1 * (dp[c + 1] - delta_s[c + 1]);
             if constexpr (MOD == MOD_SOFTCAP) {
-              d0 *= __low2float(dcap[c >> 1]);
-              d1 *= __high2float(dcap[c >> 1]);
+              // d s'/d s = 1 - tanh^2 with tanh = (log2 P + LSE2) / (c log2 e)
+              const float t0 = (__log2f(p0) + stats[c]) * cl2_inv;
+              const float t1 = (__log2f(p1) + stats[c + 1]) * cl2_inv;
+              d0 = p0 > 0.f ? d0 * (1.f - t0 * t0) : 0.f;
+              d1 = p1 > 0.f ? d1 * (1.f - t1 * t1) : 0.f;
             } else if constexpr (MOD == MOD_BOOST) {
               const float rad = static_cast<float>(a.mod.boost_radius);
               d0 *= fabsf(dq0 + static_cast<float>(c)) < rad ? a.mod.boost : 1.f;
@@ -568,54 +663,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           *reinterpret_cast<uint4*>(ds_row + ((c16 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async_smem();
-        tc_fence_before();
         mbar_arrive(smem_u32(&bars->ds_ready));
         ATTN25_TRACE_ONLY(tr[6] += clock64() - t_ds;)
         ++n_steps;
         ++step;
       }
       if (!ok) break;
-      // ---- unit epilogue: dV, scale * dK -> bf16
+      // ---- unit epilogue: scale * dK -> bf16
       if (!ATTN25_TIMED(tr[7], mbar_wait_warp(smem_u32(&bars->acc_full), unit_iter & 1, wc))) { ok = false; break; }
-      ATTN25_TRACE_ONLY(const long long t_e = clock64();)
       tc_fence_after();
-      const bool row_ok = kv < a.Skv;
-      const size_t row = (static_cast<size_t>(un.b) * a.Hkv + un.hk) * a.Skv + kv;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        __nv_bfloat16* dst = (which == 0 ? a.dv : a.dk) + row * D;
-        const float mul = which == 0 ? 1.f : a.scale;
-        const uint32_t src = which == 0 ? t_dv : t_dk;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          if (n_steps > 0) {
-            tmem_ld32(src + c * 32, o);
-            tmem_wait_ld();
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = 0u;
-          }
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * mul, __uint_as_float(o[2 * e + 1]) * mul);
-          if (row_ok) {
-            uint4* p = reinterpret_cast<uint4*>(dst + c * 32);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) p[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-          }
-        }
-      }
+      ATTN25_TRACE_ONLY(const long long t_e = clock64();)
+      store_acc_rows<D>(a.dk + ((static_cast<size_t>(un.b) * a.Hkv + un.hk) * a.Skv + kv) * D, t_dk, a.scale,
+                        n_steps > 0, kv < a.Skv);
       tc_fence_before();
       mbar_arrive(smem_u32(&bars->acc_empty));
       ATTN25_TRACE_ONLY(tr[8] += clock64() - t_e;)
     }
     ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
-    trace_flush(a.trace, 0, tr);
+    trace_flush(a.trace, 64, tr);
   } else {
+    if constexpr (kSplitRegs) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsDrain));
     // ------------------------------------------------------------ dQ drain (thread = head-dim lane)
-    const int w = warp - 4;      // TMEM lane quarter = 32-column block of D
+    const int w = warp - 8;      // TMEM lane quarter = 32-column block of D
     const uint32_t lane_off = static_cast<uint32_t>(w * 32) << 16;
     const uint32_t t_dq = tmem + Cfg::kColDQ + lane_off;
     const bool active = w * 32 < D;
@@ -646,7 +715,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         fence_proxy_async_smem();
         mbar_arrive(smem_u32(&bars->stg_written));
-        if (threadIdx.x == 128) {
+        if (threadIdx.x == 256) {
           if (!ATTN25_TIMED(tr[3], mbar_wait_thread(smem_u32(&bars->stg_written), dq_cnt & 1, wc))) {
             ok = false;
           } else {
@@ -663,7 +732,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!ok) break;
       }
     }
-    if (threadIdx.x == 128) bulk_wait_all();
+    if (threadIdx.x == 256) bulk_wait_all();
     ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
     trace_flush(a.trace, 16, tr);
   }
@@ -671,7 +740,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 8) tmem_dealloc(tmem, 512);
+  if (warp == 12) tmem_dealloc(tmem, 512);
 }
 
 // Delta_i = sum_d dO_id O_id, LSE2_i = LSE_i log2(e) (+inf where the row kept
@@ -743,6 +812,16 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   auto kernel = attn_bwd_kernel<D, MOD>;
+  // The register split assumes the kernel launches with kBwdLaunchRegs per
+  // thread; with fewer, setmaxnreg.inc could wait forever, so refuse.
+  static int launch_regs = -1;
+  if (launch_regs < 0) {
+    cudaFuncAttributes attr;
+    e = cudaFuncGetAttributes(&attr, kernel);
+    if (e != cudaSuccess) return e;
+    launch_regs = attr.numRegs;
+  }
+  if (launch_regs < kBwdLaunchRegs) return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg<D>::kAllocBytes);
   if (e != cudaSuccess) return e;
   kernel<<<grid, kBwdThreads, BwdCfg<D>::kAllocBytes, stream>>>(tq, tk, tv, tdo, tdq, a);
