@@ -22,8 +22,8 @@
  *
  * Layouts.  Q, O, dQ, dO: bf16 [B][Hq][Sq][D]; K, V, dK, dV: bf16
  * [B][Hkv][Skv][D]; LSE: fp32 [B][Hq][Sq] (natural log), contiguous, D
- * innermost.  Supported: D in {64, 128}; Sq, Skv >= 1; Hq a multiple of Hkv.
- * Every tensor base pointer must be 16-byte aligned.
+ * innermost.  Supported: D in {64, 128}; 1 <= Sq, Skv <= 262144; Hq a
+ * multiple of Hkv.  Every tensor base pointer must be 16-byte aligned.
  *
  * Errors.  Functions return ATTN_OK (0) or a negative attn_status; arguments
  * are checked on the host before anything is launched.  A kernel that waits

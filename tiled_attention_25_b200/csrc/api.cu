@@ -11,6 +11,7 @@
 #include <cudaTypedefs.h>
 
 #include "attn25.h"
+#include "kernel_common.cuh"
 #include "launch.h"
 
 namespace attn25 {
@@ -88,21 +89,6 @@ bool encode_bf16(CUtensorMap* m, const void* base, int inner, int rows, int oute
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// fp32 tensor [outer][rows][inner], boxes of box_inner x box_rows, no swizzle.
-bool encode_f32(CUtensorMap* m, const void* base, int inner, int rows, int outer, int box_inner,
-                int box_rows) {
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
-                        static_cast<cuuint64_t>(outer)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * 4,
-                           static_cast<cuuint64_t>(inner) * rows * 4};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows), 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -118,8 +104,9 @@ int check_common(int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale, in
   if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
   // coordinates and unit counts stay well inside int32
   if (static_cast<long long>(B) * Hq * (cdiv(Sq, TILE) + 1) >= (1ll << 30)) return ATTN_ERR_UNSUPPORTED;
-  if (static_cast<long long>(B) * Hq >= (1ll << 30) || Sq >= (1 << 30) || Skv >= (1 << 30))
-    return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * Hq >= (1ll << 30)) return ATTN_ERR_UNSUPPORTED;
+  // per-unit step lists live in shared memory: at most kMaxSteps tiles each way
+  if (cdiv(Sq, TILE) > kMaxSteps || cdiv(Skv, TILE) > kMaxSteps) return ATTN_ERR_UNSUPPORTED;
   if (mod_kind < ATTN_MOD_NONE || mod_kind > ATTN_MOD_DOCUMENT) return ATTN_ERR_ARG;
   switch (mod_kind) {
     case ATTN_MOD_SOFTCAP:
@@ -410,13 +397,12 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
   a.status = d->status;
   a.trace = d->trace == nullptr ? nullptr : d->trace + 128;
 
-  CUtensorMap tq, tk, tv, tdo, tdq;
+  CUtensorMap tq, tk, tv, tdo;
   if (!encode_bf16(&tq, q, D, Sq, B * Hq, 64) || !encode_bf16(&tk, k, D, Skv, B * Hkv, TILE) ||
-      !encode_bf16(&tv, v, D, Skv, B * Hkv, TILE) || !encode_bf16(&tdo, dout, D, Sq, B * Hq, 64) ||
-      !encode_f32(&tdq, a.dq_acc, D, Sq_pad, B * Hq, 32, 64))
+      !encode_bf16(&tv, v, D, Skv, B * Hkv, TILE) || !encode_bf16(&tdo, dout, D, Sq, B * Hq, 64))
     return ATTN_ERR_ARG;
   const int grid = a.n_units < d->sms ? a.n_units : d->sms;
-  if (launch_bwd(tq, tk, tv, tdo, tdq, a, D, mod_kind, grid,
+  if (launch_bwd(tq, tk, tv, tdo, a, D, mod_kind, grid,
                  reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_LAUNCH;
   return ATTN_OK;

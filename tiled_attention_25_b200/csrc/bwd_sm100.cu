@@ -19,8 +19,8 @@
 //     P^T, dS^T                                  (4 warps, thread = key row)
 //     dV += P^T dO  (P^T from tensor memory),  dK += dS^T Q,
 //     dQ^T = K^T dS^T                            (tcgen05)
-// and adds dQ into the fp32 accumulator with a TMA reduce-add (the add runs
-// in L2, so the order of the adds, and the last bits of dQ, vary run to run).
+// and adds dQ into the fp32 accumulator with coalesced reductions performed
+// in L2 (the order of the adds, and the last bits of dQ, vary run to run).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -56,10 +56,9 @@ struct BwdCfg {
   static constexpr int kStageOff = 2 * kKVBytes;
   static constexpr int kDSOff = kStageOff + kStages * kStageBytes;  // two 128 x 64 bf16 buffers
   static constexpr int kDSBytes = TILE * BM * 2;
-  static constexpr int kStgOff = kDSOff + 2 * kDSBytes;            // dQ staging [D/32][64][32] fp32
-  static constexpr int kStgBytes = BM * D * 4;
-  static constexpr int kBarOff = kStgOff + kStgBytes;
-  static constexpr int kSmemBytes = kBarOff + 1024;
+  static constexpr int kBarOff = kDSOff + 2 * kDSBytes;
+  static constexpr int kListOff = kBarOff + 1024;  // two query-tile lists
+  static constexpr int kSmemBytes = kListOff + 2 * kMaxSteps * 4;
   static constexpr int kAllocBytes = kSmemBytes + 1024;
   // TMEM columns: two S^T buffers (P^T overwrites their first 32 columns), dP^T,
   // the dV and dK accumulators, dQ^T
@@ -71,19 +70,23 @@ struct BwdCfg {
 };
 
 struct BwdBarriers {
+  uint64_t list_full[2], list_empty[2];
   uint64_t kv_full, kv_empty;
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full[2], s_free[2], p_ready[2];
   uint64_t dp_full, ds_ready;
   uint64_t ds_empty[2];
   uint64_t dq_full, dq_empty;
-  uint64_t stg_written, stg_free;
   uint64_t acc_full, acc_empty;
   uint64_t drain;
   uint32_t tmem_base;
   uint32_t abort_flag;
   uint32_t never_set;  // abort word for drain waits that must not stop early
+  int32_t list_n[2];   // lengths of the two query-tile lists
 };
+
+// Consumers of a query-tile list: the MMA warp and the P, dS and drain warps (lane 0 each).
+constexpr int kBwdListConsumers = 13;
 
 struct BwdUnit {
   int b, hk, kt;
@@ -100,97 +103,44 @@ __device__ __forceinline__ BwdUnit decode_bwd_unit(const BwdArgs& a, int u) {
   return r;
 }
 
-// Walks the steps of one unit: for each query head of the group, each
-// non-EMPTY 128-row query tile (block-mask list or analytic range), and each
+// Walks the steps of one unit from its query-tile list in shared memory: for
+// each query head of the group, each listed 128-row query tile, and each
 // 64-row half of it that starts inside Sq.
 struct StepIter {
-  const int32_t* list;
-  const uint8_t* cls_col;  // tile_class + b*nQ*nK + kt, stride nK
-  int n_list, nK, nQ, Sq, Skv, kind, window, kt, G;
-  int g, li, half, qt_dense, qt_end;
-  int cur_qt, cur_cls;
-  bool list_mode, tail_kv;
+  const uint32_t* list;
+  int n, G, Sq;
+  int g, j, half;
+  uint32_t cur;
 
-  __device__ void init(const BwdArgs& a, const BwdUnit& u) {
-    nK = a.nK;
-    nQ = a.nQ;
-    Sq = a.Sq;
-    Skv = a.Skv;
-    kind = a.mod.kind;
-    window = a.mod.window;
-    kt = u.kt;
-    G = a.G;
+  __device__ __forceinline__ void init(const uint32_t* list_, int n_, int G_, int Sq_) {
+    list = list_;
+    n = n_;
+    G = G_;
+    Sq = Sq_;
     g = 0;
-    li = 0;
-    half = 2;  // forces fetching the first query tile
-    tail_kv = (Skv % TILE) != 0 && kt == nK - 1;
-    list_mode = a.tile_class != nullptr;
-    if (list_mode) {
-      const size_t col = static_cast<size_t>(u.b) * nK + kt;
-      list = a.q_index + col * nQ;
-      n_list = __ldg(a.q_count + col);
-      cls_col = a.tile_class + static_cast<size_t>(u.b) * nQ * nK + kt;
-    } else {
-      list = nullptr;
-      cls_col = nullptr;
-      n_list = 0;
-    }
-    qt_dense = 0;
-    qt_end = nQ;
-    if (!list_mode && is_interval_mask(kind)) qt_dense = (kt * TILE) / TILE;
-    li = qt_dense;
-  }
-
-  __device__ __forceinline__ int dense_class(int qt) const {
-    const int q0 = qt * TILE, q1 = min(Sq, q0 + TILE);
-    const int k0 = kt * TILE, k1 = min(Skv, k0 + TILE);
-    if (kind == MOD_CAUSAL || kind == MOD_WINDOW)
-      return interval_tile_class(kind, window, q0, q1, k0, k1);
-    if (kind == MOD_DOCUMENT) return 1;
-    return 2;
-  }
-
-  // Advance to the next query tile (any head); false when the unit is done.
-  __device__ bool next_tile() {
-    while (g < G) {
-      if (list_mode) {
-        if (li < n_list) {
-          cur_qt = __ldg(list + li);
-          cur_cls = __ldg(cls_col + static_cast<size_t>(cur_qt) * nK);
-          ++li;
-          return true;
-        }
-      } else {
-        while (li < qt_end) {
-          const int qt = li++;
-          const int c = dense_class(qt);
-          if (c != 0) {
-            cur_qt = qt;
-            cur_cls = c;
-            return true;
-          }
-        }
-      }
-      ++g;
-      li = list_mode ? 0 : qt_dense;
-    }
-    return false;
+    j = 0;
+    half = 2;
+    cur = 0;
   }
 
   // Next step: head offset g_out in the group, first query row q0, and
   // whether the element predicate is needed.
-  __device__ bool next(int& g_out, int& q0, bool& pred) {
+  __device__ __forceinline__ bool next(int& g_out, int& q0, bool& pred) {
     while (true) {
       if (half >= 2) {
-        if (!next_tile()) return false;
+        if (j >= n) {
+          j = 0;
+          if (++g >= G) return false;
+          if (n == 0) return false;
+        }
+        cur = list[j++];
         half = 0;
       }
-      const int h = half++;
-      const int start = cur_qt * TILE + h * BM;
+      const int start = static_cast<int>(cur & 0xFFFFFu) * TILE + (half++) * BM;
       if (start >= Sq) continue;
       g_out = g;
       q0 = start;
-      pred = (cur_cls == 1) || tail_kv;
+      pred = (cur & kQtPred) != 0;
       return true;
     }
   }
@@ -259,10 +209,17 @@ __device__ __forceinline__ void key_interval(const BwdArgs& a, int b, int kv, in
   if (kv >= a.Skv) qhi = qlo - 1;
 }
 
-// One key row of S^T (raw q.k for 64 queries) -> P^T = 2^(x - LSE2) in place.
+__device__ __forceinline__ float4 lds128(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
+
+// One key row of S^T (raw q.k for 64 queries) -> P^T = 2^(x - LSE2) in place;
+// nl2 is the shared address of the 64 negated base-2 LSEs.
 template <int MOD>
 __device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h, float dq0, int q0,
-                                        int qlo, int qhi, bool pred, const float* lse2_s) {
+                                        int qlo, int qhi, bool pred, uint32_t nl2) {
   float aux = 0.f, aux2 = 0.f;
   if constexpr (MOD == MOD_ALIBI) aux = alibi_slope(a.mod, h, a.Hq) * LOG2E;
   if constexpr (MOD == MOD_SOFTCAP) {
@@ -270,24 +227,36 @@ __device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h,
     aux2 = a.mod.softcap * LOG2E;
   }
   if constexpr (MOD == MOD_BOOST) aux = a.mod.boost * a.sl2;
+  const float2 sl2 = make_float2(a.sl2, a.sl2);
 #pragma unroll
-  for (int c = 0; c < BM; ++c) {
-    float v = x[c];
-    if constexpr (MOD == MOD_ALIBI) {
-      v = fmaf(v, a.sl2, -aux * fabsf(dq0 + static_cast<float>(c)));
-    } else if constexpr (MOD == MOD_SOFTCAP) {
-      v = aux2 * tanhf(v * aux);
-    } else if constexpr (MOD == MOD_BOOST) {
-      const bool inside = fabsf(dq0 + static_cast<float>(c)) < static_cast<float>(a.mod.boost_radius);
-      v = v * (inside ? aux : a.sl2);
-    } else {
-      v = v * a.sl2;
+  for (int c4 = 0; c4 < BM / 4; ++c4) {
+    const float4 l = lds128(nl2 + c4 * 16);
+#pragma unroll
+    for (int hp = 0; hp < 2; ++hp) {
+      const int c = c4 * 4 + hp * 2;
+      const float2 nl = hp == 0 ? make_float2(l.x, l.y) : make_float2(l.z, l.w);
+      float2 v;
+      if constexpr (MOD == MOD_ALIBI) {
+        v.x = fmaf(x[c], a.sl2, -aux * fabsf(dq0 + static_cast<float>(c))) + nl.x;
+        v.y = fmaf(x[c + 1], a.sl2, -aux * fabsf(dq0 + static_cast<float>(c + 1))) + nl.y;
+      } else if constexpr (MOD == MOD_SOFTCAP) {
+        v.x = fmaf(aux2, tanhf(x[c] * aux), nl.x);
+        v.y = fmaf(aux2, tanhf(x[c + 1] * aux), nl.y);
+      } else if constexpr (MOD == MOD_BOOST) {
+        const float r = static_cast<float>(a.mod.boost_radius);
+        v.x = fmaf(x[c], fabsf(dq0 + static_cast<float>(c)) < r ? aux : a.sl2, nl.x);
+        v.y = fmaf(x[c + 1], fabsf(dq0 + static_cast<float>(c + 1)) < r ? aux : a.sl2, nl.y);
+      } else {
+        v = __ffma2_rn(make_float2(x[c], x[c + 1]), sl2, nl);
+      }
+      if (pred) {
+        const int qq = q0 + c;
+        v.x = (qq >= qlo && qq <= qhi) ? v.x : -INFINITY;
+        v.y = (qq + 1 >= qlo && qq + 1 <= qhi) ? v.y : -INFINITY;
+      }
+      x[c] = ex2_approx(v.x);  // 0 where masked or on padding rows (-LSE2 = -inf)
+      x[c + 1] = ex2_approx(v.y);
     }
-    if (pred) {
-      const int qq = q0 + c;
-      v = (qq >= qlo && qq <= qhi) ? v : -INFINITY;
-    }
-    x[c] = ex2_approx(v - lse2_s[c]);  // 0 where masked or on padding rows (LSE2 = +inf)
   }
 }
 
@@ -321,7 +290,7 @@ template <int D, int MOD>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const __grid_constant__ CUtensorMap tm_dq, const BwdArgs a) {
+                    const BwdArgs a) {
   using Cfg = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -330,11 +299,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t k_smem = sbase + Cfg::kKOff;
   const uint32_t v_smem = sbase + Cfg::kVOff;
+  uint32_t* lists = reinterpret_cast<uint32_t*>(smem + Cfg::kListOff);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   constexpr bool kSplitRegs = MOD != MOD_SOFTCAP && MOD != MOD_BOOST;
 
   if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars->list_full[i]), 32);
+      mbar_init(smem_u32(&bars->list_empty[i]), kBwdListConsumers);
+    }
     mbar_init(smem_u32(&bars->kv_full), 1);
     mbar_init(smem_u32(&bars->kv_empty), 1);
     for (int b = 0; b < 2; ++b) {
@@ -349,8 +323,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(smem_u32(&bars->ds_ready), 128);
     mbar_init(smem_u32(&bars->dq_full), 1);
     mbar_init(smem_u32(&bars->dq_empty), 128);
-    mbar_init(smem_u32(&bars->stg_written), 128);
-    mbar_init(smem_u32(&bars->stg_free), 1);
     mbar_init(smem_u32(&bars->acc_full), 1);
     mbar_init(smem_u32(&bars->acc_empty), 256);
     mbar_init(smem_u32(&bars->drain), 1);
@@ -367,7 +339,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
-    tma_prefetch_desc(&tm_dq);
   }
   tc_fence_before();
   __syncthreads();
@@ -382,47 +353,59 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if constexpr (kSplitRegs) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
     if (warp == 13) {
       // ---------------------------------------------------------- TMA producer
-      if (lane == 0) {
-        int unit_iter = 0, step = 0;
-        uint32_t kv_loads = 0, stage_uses[2] = {0, 0};
-        bool ok = true;
-        for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
-          const BwdUnit un = decode_bwd_unit(a, u);
-          if (!ATTN25_TIMED(tr[1], mbar_wait_thread(smem_u32(&bars->kv_empty), (unit_iter & 1) ^ 1, wc))) { ok = false; break; }
-          mbar_arrive_expect_tx(smem_u32(&bars->kv_full), 2 * Cfg::kKVBytes);
-          ++kv_loads;
-          const int bh_kv = un.b * a.Hkv + un.hk;
-          load_kv_tile<D>(k_smem, &tm_k, smem_u32(&bars->kv_full), un.kt * TILE, bh_kv);
-          load_kv_tile<D>(v_smem, &tm_v, smem_u32(&bars->kv_full), un.kt * TILE, bh_kv);
-          StepIter it;
-          it.init(a, un);
-          int g, q0;
-          bool pred;
-          while (it.next(g, q0, pred)) {
-            const int s = step & 1;
-            if (!ATTN25_TIMED(tr[2], mbar_wait_thread(smem_u32(&bars->q_empty[s]), ((step >> 1) & 1) ^ 1, wc))) { ok = false; break; }
-            const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
-            const uint32_t bar = smem_u32(&bars->q_full[s]);
-            mbar_arrive_expect_tx(bar, 2 * Cfg::kQBytes + 2 * BM * 4);
-            ++stage_uses[s];
-            const int bh = un.b * a.Hq + un.hk * a.G + g;
-            load_q_tile<D>(st, &tm_q, bar, q0, bh);
-            load_q_tile<D>(st + Cfg::kQBytes, &tm_do, bar, q0, bh);
-            const size_t row = static_cast<size_t>(bh) * a.Sq_pad + q0;
-            bulk_load_1d(st + 2 * Cfg::kQBytes, a.lse2 + row, BM * 4, bar);
-            bulk_load_1d(st + 2 * Cfg::kQBytes + 512, a.delta + row, BM * 4, bar);
-            ++step;
+      // all lanes build the query-tile lists; lane 0 issues the copies
+      int unit_iter = 0, step = 0;
+      uint32_t kv_loads = 0, stage_uses[2] = {0, 0};
+      bool ok = true;
+      for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+        const BwdUnit un = decode_bwd_unit(a, u);
+        const int buf = unit_iter & 1;
+        uint32_t* lst = lists + buf * kMaxSteps;
+        if (!mbar_wait_warp(smem_u32(&bars->list_empty[buf]), ((unit_iter >> 1) & 1) ^ 1, wc)) { ok = false; break; }
+        const int n = build_kv_qtiles(a.tile_class, un.b, un.kt, a.nQ, a.nK, a.Sq, a.Skv, MOD,
+                                      a.mod.window, lst);
+        if (lane == 0) bars->list_n[buf] = n;
+        mbar_arrive(smem_u32(&bars->list_full[buf]));
+        if (lane == 0) {
+          if (!ATTN25_TIMED(tr[1], mbar_wait_thread(smem_u32(&bars->kv_empty), (unit_iter & 1) ^ 1, wc))) {
+            ok = false;
+          } else {
+            mbar_arrive_expect_tx(smem_u32(&bars->kv_full), 2 * Cfg::kKVBytes);
+            ++kv_loads;
+            const int bh_kv = un.b * a.Hkv + un.hk;
+            load_kv_tile<D>(k_smem, &tm_k, smem_u32(&bars->kv_full), un.kt * TILE, bh_kv);
+            load_kv_tile<D>(v_smem, &tm_v, smem_u32(&bars->kv_full), un.kt * TILE, bh_kv);
+            StepIter it;
+            it.init(lst, n, a.G, a.Sq);
+            int g, q0;
+            bool pred;
+            while (it.next(g, q0, pred)) {
+              const int s = step & 1;
+              if (!ATTN25_TIMED(tr[2], mbar_wait_thread(smem_u32(&bars->q_empty[s]), ((step >> 1) & 1) ^ 1, wc))) { ok = false; break; }
+              const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
+              const uint32_t bar = smem_u32(&bars->q_full[s]);
+              mbar_arrive_expect_tx(bar, 2 * Cfg::kQBytes + 2 * BM * 4);
+              ++stage_uses[s];
+              const int bh = un.b * a.Hq + un.hk * a.G + g;
+              load_q_tile<D>(st, &tm_q, bar, q0, bh);
+              load_q_tile<D>(st + Cfg::kQBytes, &tm_do, bar, q0, bh);
+              const size_t row = static_cast<size_t>(bh) * a.Sq_pad + q0;
+              bulk_load_1d(st + 2 * Cfg::kQBytes, a.lse2 + row, BM * 4, bar);
+              bulk_load_1d(st + 2 * Cfg::kQBytes + 512, a.delta + row, BM * 4, bar);
+              ++step;
+            }
           }
         }
-        if (!ok) {
-          const WaitCtl dwc{a.wait_ns, smem_u32(&bars->never_set), a.status};
-          if (kv_loads) mbar_wait_thread(smem_u32(&bars->kv_full), (kv_loads - 1) & 1, dwc);
-          for (int s = 0; s < 2; ++s)
-            if (stage_uses[s]) mbar_wait_thread(smem_u32(&bars->q_full[s]), (stage_uses[s] - 1) & 1, dwc);
-        }
-        ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
-        trace_flush(a.trace, 48, tr);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       }
+      if (!ok && lane == 0) {
+        const WaitCtl dwc{a.wait_ns, smem_u32(&bars->never_set), a.status};
+        if (kv_loads) mbar_wait_thread(smem_u32(&bars->kv_full), (kv_loads - 1) & 1, dwc);
+        for (int s = 0; s < 2; ++s)
+          if (stage_uses[s]) mbar_wait_thread(smem_u32(&bars->q_full[s]), (stage_uses[s] - 1) & 1, dwc);
+      }
+      ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
+      trace_flush(a.trace, 48, tr);
     } else if (warp == 12) {
       // ---------------------------------------------------------- MMA issuer
       const uint32_t t_dp = tmem + Cfg::kColDP;
@@ -436,8 +419,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // dK, dV accumulators are free once the previous unit's epilogue read them
         if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->acc_empty), (unit_iter & 1) ^ 1, wc))) { ok = false; break; }
         tc_fence_after();
+        const int buf = unit_iter & 1;
+        if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
         StepIter it;
-        it.init(a, un);
+        it.init(lists + buf * kMaxSteps, bars->list_n[buf], a.G, a.Sq);
         int g, q0;
         bool pred;
         bool has = it.next(g, q0, pred);
@@ -524,6 +509,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (lane == 0) {
           mma_commit(smem_u32(&bars->kv_empty));
           mma_commit(smem_u32(&bars->acc_full));
+          mbar_arrive(smem_u32(&bars->list_empty[buf]));
         }
         __syncwarp();
       }
@@ -548,14 +534,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int kv = un.kt * TILE + r;
       int qlo, qhi;
       key_interval<MOD>(a, un.b, kv, qlo, qhi);
+      const int buf = unit_iter & 1;
+      if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
       StepIter it;
-      it.init(a, un);
+      it.init(lists + buf * kMaxSteps, bars->list_n[buf], a.G, a.Sq);
       int g, q0;
       bool pred;
       int n_steps = 0;
       while (it.next(g, q0, pred)) {
         const int s = step & 1;
-        const float* lse2_s = reinterpret_cast<const float*>(smem + Cfg::kStageOff + s * Cfg::kStageBytes + 2 * Cfg::kQBytes);
+        const uint32_t nl2_s = sbase + Cfg::kStageOff + s * Cfg::kStageBytes + 2 * Cfg::kQBytes;
         const uint32_t t_s = tmem + Cfg::kColS + s * BM + lane_off;
         if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step >> 1) & 1, wc))) { ok = false; break; }
         if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->s_full[s]), (step >> 1) & 1, wc))) { ok = false; break; }
@@ -566,7 +554,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(t_s, reinterpret_cast<uint32_t(&)[32]>(x[0]));
         tmem_ld32(t_s + 32, reinterpret_cast<uint32_t(&)[32]>(x[32]));
         tmem_wait_ld();
-        probs_t<MOD>(x, a, h, static_cast<float>(q0 - kv), q0, qlo, qhi, pred, lse2_s);
+        probs_t<MOD>(x, a, h, static_cast<float>(q0 - kv), q0, qlo, qhi, pred, nl2_s);
         // P^T (bf16 pairs) over the first 32 columns of this S^T buffer
         uint32_t pk[32];
 #pragma unroll
@@ -588,6 +576,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         n_steps > 0, kv < a.Skv);
       tc_fence_before();
       mbar_arrive(smem_u32(&bars->acc_empty));
+      if (lane == 0) mbar_arrive(smem_u32(&bars->list_empty[buf]));
       ATTN25_TRACE_ONLY(tr[8] += clock64() - t_e;)
     }
     ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
@@ -604,15 +593,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
       const BwdUnit un = decode_bwd_unit(a, u);
       const int kv = un.kt * TILE + r;
+      const int buf = unit_iter & 1;
+      if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
       StepIter it;
-      it.init(a, un);
+      it.init(lists + buf * kMaxSteps, bars->list_n[buf], a.G, a.Sq);
       int g, q0;
       bool pred;
       int n_steps = 0;
       while (it.next(g, q0, pred)) {
         const int s = step & 1;
-        const float* stats = reinterpret_cast<const float*>(smem + Cfg::kStageOff + s * Cfg::kStageBytes + 2 * Cfg::kQBytes);
-        const float* delta_s = stats + 128;
+        const uint32_t stats = sbase + Cfg::kStageOff + s * Cfg::kStageBytes + 2 * Cfg::kQBytes;
         const uint32_t t_p = tmem + Cfg::kColS + s * BM + lane_off;
         if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step >> 1) & 1, wc))) { ok = false; break; }
         if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->p_ready[s]), (step >> 1) & 1, wc))) { ok = false; break; }
@@ -638,26 +628,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if constexpr (MOD == MOD_SOFTCAP) cl2_inv = 1.f / (a.mod.softcap * LOG2E);
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16) {  // 8 columns (16 bytes) at a time
+          const float4 nd0 = lds128(stats + 512 + c16 * 32), nd1 = lds128(stats + 512 + c16 * 32 + 16);
+          const float nd[8] = {nd0.x, nd0.y, nd0.z, nd0.w, nd1.x, nd1.y, nd1.z, nd1.w};
+          float4 nl0, nl1;
+          if constexpr (MOD == MOD_SOFTCAP) {
+            nl0 = lds128(stats + c16 * 32);
+            nl1 = lds128(stats + c16 * 32 + 16);
+          }
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = c16 * 8 + 2 * e;
             const uint32_t pp = pb[c >> 1];
-            const float p0 = __uint_as_float(pp << 16), p1 = __uint_as_float(pp & 0xffff0000u);
-            float d0 = p0 * (dp[c] - delta_s[c]);
-            float d1 = p1 * (dp[c + 1] - delta_s[c + 1]);
+            const float2 pr = make_float2(__uint_as_float(pp << 16), __uint_as_float(pp & 0xffff0000u));
+            // dS = P (dP - Delta)
+            float2 d = __fmul2_rn(pr, __fadd2_rn(make_float2(dp[c], dp[c + 1]), make_float2(nd[2 * e], nd[2 * e + 1])));
             if constexpr (MOD == MOD_SOFTCAP) {
               // d s'/d s = 1 - tanh^2 with tanh = (log2 P + LSE2) / (c log2 e)
-              const float t0 = (__log2f(p0) + stats[c]) * cl2_inv;
-              const float t1 = (__log2f(p1) + stats[c + 1]) * cl2_inv;
-              d0 = p0 > 0.f ? d0 * (1.f - t0 * t0) : 0.f;
-              d1 = p1 > 0.f ? d1 * (1.f - t1 * t1) : 0.f;
+              const float nlx = (e < 2) ? (e == 0 ? nl0.x : nl0.z) : (e == 2 ? nl1.x : nl1.z);
+              const float nly = (e < 2) ? (e == 0 ? nl0.y : nl0.w) : (e == 2 ? nl1.y : nl1.w);
+              const float t0 = (__log2f(pr.x) - nlx) * cl2_inv;
+              const float t1 = (__log2f(pr.y) - nly) * cl2_inv;
+              d.x = pr.x > 0.f ? d.x * (1.f - t0 * t0) : 0.f;
+              d.y = pr.y > 0.f ? d.y * (1.f - t1 * t1) : 0.f;
             } else if constexpr (MOD == MOD_BOOST) {
               const float rad = static_cast<float>(a.mod.boost_radius);
-              d0 *= fabsf(dq0 + static_cast<float>(c)) < rad ? a.mod.boost : 1.f;
-              d1 *= fabsf(dq0 + static_cast<float>(c + 1)) < rad ? a.mod.boost : 1.f;
+              d.x *= fabsf(dq0 + static_cast<float>(c)) < rad ? a.mod.boost : 1.f;
+              d.y *= fabsf(dq0 + static_cast<float>(c + 1)) < rad ? a.mod.boost : 1.f;
             }
-            w[e] = pack_bf16x2(d0, d1);
+            w[e] = pack_bf16x2(d.x, d.y);
           }
           // 128-byte swizzle: 16-byte chunk c16 of row r lands at chunk c16 ^ (r % 8)
           *reinterpret_cast<uint4*>(ds_row + ((c16 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -677,6 +676,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         n_steps > 0, kv < a.Skv);
       tc_fence_before();
       mbar_arrive(smem_u32(&bars->acc_empty));
+      if (lane == 0) mbar_arrive(smem_u32(&bars->list_empty[buf]));
       ATTN25_TRACE_ONLY(tr[8] += clock64() - t_e;)
     }
     ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
@@ -684,18 +684,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else {
     if constexpr (kSplitRegs) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsDrain));
     // ------------------------------------------------------------ dQ drain (thread = head-dim lane)
+    // dQ^T leaves TMEM row by row (lane = head dim) and is added into the
+    // fp32 accumulator with coalesced reductions in L2 (32 lanes = 128 bytes).
     const int w = warp - 8;      // TMEM lane quarter = 32-column block of D
     const uint32_t lane_off = static_cast<uint32_t>(w * 32) << 16;
     const uint32_t t_dq = tmem + Cfg::kColDQ + lane_off;
     const bool active = w * 32 < D;
-    float* stg = reinterpret_cast<float*>(smem + Cfg::kStgOff) + w * (BM * 32);
     int unit_iter = 0;
     uint32_t dq_cnt = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
       const BwdUnit un = decode_bwd_unit(a, u);
+      const int buf = unit_iter & 1;
+      if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
       StepIter it;
-      it.init(a, un);
+      it.init(lists + buf * kMaxSteps, bars->list_n[buf], a.G, a.Sq);
       int g, q0;
       bool pred;
       while (it.next(g, q0, pred)) {
@@ -707,32 +710,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(smem_u32(&bars->dq_empty));
-        // staging is free once the previous reduce has read it
-        if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->stg_free), (dq_cnt & 1) ^ 1, wc))) { ok = false; break; }
+        ATTN25_TRACE_ONLY(const long long t_r = clock64();)
         if (active) {
+          const int bh = un.b * a.Hq + un.hk * a.G + g;
+          float* dst = a.dq_acc + (static_cast<size_t>(bh) * a.Sq_pad + q0) * D + w * 32 + lane;
 #pragma unroll
-          for (int c = 0; c < BM; ++c) stg[c * 32 + lane] = v[c];
+          for (int c = 0; c < BM; ++c) atomicAdd(dst + static_cast<size_t>(c) * D, v[c]);
         }
-        fence_proxy_async_smem();
-        mbar_arrive(smem_u32(&bars->stg_written));
-        if (threadIdx.x == 256) {
-          if (!ATTN25_TIMED(tr[3], mbar_wait_thread(smem_u32(&bars->stg_written), dq_cnt & 1, wc))) {
-            ok = false;
-          } else {
-            const int bh = un.b * a.Hq + un.hk * a.G + g;
-            for (int c = 0; c < D / 32; ++c)
-              tma_reduce_add_3d(&tm_dq, sbase + Cfg::kStgOff + c * (BM * 32 * 4), c * 32, q0, bh);
-            bulk_commit();
-            ATTN25_TIMED(tr[4], (bulk_wait_read_all(), 0));
-            mbar_arrive(smem_u32(&bars->stg_free));
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 && ok;
+        ATTN25_TRACE_ONLY(tr[2] += clock64() - t_r;)
         ++dq_cnt;
-        if (!ok) break;
       }
+      if (!ok) break;
+      if (lane == 0) mbar_arrive(smem_u32(&bars->list_empty[buf]));
     }
-    if (threadIdx.x == 256) bulk_wait_all();
     ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
     trace_flush(a.trace, 16, tr);
   }
@@ -743,7 +733,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == 12) tmem_dealloc(tmem, 512);
 }
 
-// Delta_i = sum_d dO_id O_id, LSE2_i = LSE_i log2(e) (+inf where the row kept
+// -Delta_i = -sum_d dO_id O_id and -LSE_i log2(e) (-inf where the row kept
 // nothing or lies past Sq), and zero the fp32 dQ accumulator.  One warp per row.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
@@ -768,13 +758,15 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
     float4* z = reinterpret_cast<float4*>(a.dq_acc + static_cast<size_t>(row) * D);
     for (int i = lane; i < D / 4; i += 32) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (lane == 0) {
-      float l2 = INFINITY;
+      // stored negated, so that the main kernel's exponent is one FFMA:
+      // -LSE log2(e), or -inf where the row keeps nothing or lies past Sq (P = 0)
+      float nl2 = -INFINITY;
       if (q < a.Sq) {
         const float l = a.lse[static_cast<size_t>(bh) * a.Sq + q];
-        l2 = (l == -INFINITY) ? INFINITY : l * LOG2E;
+        nl2 = (l == -INFINITY) ? -INFINITY : -l * LOG2E;
       }
-      a.lse2[row] = l2;
-      a.delta[row] = q < a.Sq ? acc : 0.f;
+      a.lse2[row] = nl2;
+      a.delta[row] = q < a.Sq ? -acc : 0.f;
     }
   }
 }
@@ -803,8 +795,7 @@ __global__ void __launch_bounds__(256) bwd_dq_cast_kernel(const BwdArgs a) {
 
 template <int D, int MOD>
 cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int grid,
-                         cudaStream_t stream) {
+                         const CUtensorMap& tdo, const BwdArgs& a, int grid, cudaStream_t stream) {
   const long long rows = static_cast<long long>(a.B) * a.Hq * a.Sq_pad;
   int prep_blocks = static_cast<int>((rows * 32 + 255) / 256);
   if (prep_blocks > 148 * 16) prep_blocks = 148 * 16;
@@ -824,7 +815,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   if (launch_regs < kBwdLaunchRegs) return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg<D>::kAllocBytes);
   if (e != cudaSuccess) return e;
-  kernel<<<grid, kBwdThreads, BwdCfg<D>::kAllocBytes, stream>>>(tq, tk, tv, tdo, tdq, a);
+  kernel<<<grid, kBwdThreads, BwdCfg<D>::kAllocBytes, stream>>>(tq, tk, tv, tdo, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const long long n8 = static_cast<long long>(a.B) * a.Hq * a.Sq * (D / 8);
@@ -836,16 +827,16 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 
 template <int D>
 cudaError_t launch_bwd_mod(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                           const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int mod,
-                           int grid, cudaStream_t s) {
+                           const CUtensorMap& tdo, const BwdArgs& a, int mod, int grid,
+                           cudaStream_t s) {
   switch (mod) {
-    case MOD_NONE: return launch_bwd_t<D, MOD_NONE>(tq, tk, tv, tdo, tdq, a, grid, s);
-    case MOD_CAUSAL: return launch_bwd_t<D, MOD_CAUSAL>(tq, tk, tv, tdo, tdq, a, grid, s);
-    case MOD_ALIBI: return launch_bwd_t<D, MOD_ALIBI>(tq, tk, tv, tdo, tdq, a, grid, s);
-    case MOD_SOFTCAP: return launch_bwd_t<D, MOD_SOFTCAP>(tq, tk, tv, tdo, tdq, a, grid, s);
-    case MOD_WINDOW: return launch_bwd_t<D, MOD_WINDOW>(tq, tk, tv, tdo, tdq, a, grid, s);
-    case MOD_BOOST: return launch_bwd_t<D, MOD_BOOST>(tq, tk, tv, tdo, tdq, a, grid, s);
-    case MOD_DOCUMENT: return launch_bwd_t<D, MOD_DOCUMENT>(tq, tk, tv, tdo, tdq, a, grid, s);
+    case MOD_NONE: return launch_bwd_t<D, MOD_NONE>(tq, tk, tv, tdo, a, grid, s);
+    case MOD_CAUSAL: return launch_bwd_t<D, MOD_CAUSAL>(tq, tk, tv, tdo, a, grid, s);
+    case MOD_ALIBI: return launch_bwd_t<D, MOD_ALIBI>(tq, tk, tv, tdo, a, grid, s);
+    case MOD_SOFTCAP: return launch_bwd_t<D, MOD_SOFTCAP>(tq, tk, tv, tdo, a, grid, s);
+    case MOD_WINDOW: return launch_bwd_t<D, MOD_WINDOW>(tq, tk, tv, tdo, a, grid, s);
+    case MOD_BOOST: return launch_bwd_t<D, MOD_BOOST>(tq, tk, tv, tdo, a, grid, s);
+    case MOD_DOCUMENT: return launch_bwd_t<D, MOD_DOCUMENT>(tq, tk, tv, tdo, a, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -853,10 +844,10 @@ cudaError_t launch_bwd_mod(const CUtensorMap& tq, const CUtensorMap& tk, const C
 }  // namespace
 
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int D,
-                       int mod, int grid, cudaStream_t stream) {
-  if (D == 128) return launch_bwd_mod<128>(tq, tk, tv, tdo, tdq, a, mod, grid, stream);
-  if (D == 64) return launch_bwd_mod<64>(tq, tk, tv, tdo, tdq, a, mod, grid, stream);
+                       const CUtensorMap& tdo, const BwdArgs& a, int D, int mod, int grid,
+                       cudaStream_t stream) {
+  if (D == 128) return launch_bwd_mod<128>(tq, tk, tv, tdo, a, mod, grid, stream);
+  if (D == 64) return launch_bwd_mod<64>(tq, tk, tv, tdo, a, mod, grid, stream);
   return cudaErrorInvalidValue;
 }
 

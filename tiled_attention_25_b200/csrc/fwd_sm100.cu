@@ -49,13 +49,15 @@ struct FwdCfg {
   static constexpr int kQOff = 0;                           // Q0, Q1
   static constexpr int kRingOff = 2 * kTileBytes;
   static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
-  static constexpr int kSmemBytes = kBarOff + 1024;         // + barriers, flags
+  static constexpr int kListOff = kBarOff + 1024;           // two step lists
+  static constexpr int kSmemBytes = kListOff + 2 * kMaxSteps * 4;
   static constexpr int kAllocBytes = kSmemBytes + 1024;     // + alignment slack
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);
 };
 
 struct FwdBarriers {
+  uint64_t list_full[2], list_empty[2];
   uint64_t q_full, q_empty;
   uint64_t s_full[2], p_full[2], o_full[2], o_final[2];
   uint64_t drain;
@@ -63,7 +65,11 @@ struct FwdBarriers {
   uint32_t tmem_base;
   uint32_t abort_flag;
   uint32_t never_set;  // abort word for drain waits that must not stop early
+  int32_t list_n[2];   // step counts of the two step lists
 };
+
+// Consumers of a step list: the MMA warp and the 8 softmax warps (lane 0 each).
+constexpr int kListConsumers = 9;
 
 struct UnitCoord {
   int b, h, p;
@@ -152,6 +158,12 @@ __host__ __device__ constexpr bool pure_scale(int mod) {
   return mod == MOD_NONE || mod == MOD_CAUSAL || mod == MOD_WINDOW || mod == MOD_DOCUMENT;
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Apply mask (and, for the other mods, the mod itself) to one row of raw
 // scores; return the row maximum in the base-2 domain.
 template <int MOD, bool PRED>
@@ -169,49 +181,73 @@ __device__ __forceinline__ float row_scores(float (&x)[4][32], const RowCtx& rc,
     } else {
       transform32<MOD>(x[c], rc, md, k0, c * 32, PRED);
     }
-    float m0 = x[c][0], m1 = x[c][1], m2 = x[c][2], m3 = x[c][3];
+    // three-input max: 16 instructions per 32 columns, 4 independent chains
+    float m0 = max3(x[c][0], x[c][1], x[c][2]), m1 = max3(x[c][3], x[c][4], x[c][5]);
+    float m2 = max3(x[c][6], x[c][7], x[c][8]), m3 = max3(x[c][9], x[c][10], x[c][11]);
 #pragma unroll
-    for (int e = 4; e < 32; e += 4) {
-      m0 = fmaxf(m0, x[c][e]);
-      m1 = fmaxf(m1, x[c][e + 1]);
-      m2 = fmaxf(m2, x[c][e + 2]);
-      m3 = fmaxf(m3, x[c][e + 3]);
+    for (int e = 12; e < 28; e += 8) {
+      m0 = max3(m0, x[c][e], x[c][e + 1]);
+      m1 = max3(m1, x[c][e + 2], x[c][e + 3]);
+      m2 = max3(m2, x[c][e + 4], x[c][e + 5]);
+      m3 = max3(m3, x[c][e + 6], x[c][e + 7]);
     }
-    mx = fmaxf(mx, fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)));
+    m0 = max3(m0, x[c][28], x[c][29]);
+    m1 = max3(m1, x[c][30], x[c][31]);
+    mx = max3(mx, max3(m0, m1, m2), m3);
   }
   if constexpr (pure_scale(MOD)) mx *= rc.sl2;  // -inf stays -inf
   return mx;
 }
 
+// 2^(x0, x1) on the FMA pipe with packed fp32 pairs (finite inputs only),
+// the same range reduction and polynomial as exp2_poly.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 magic = make_float2(12582912.0f, 12582912.0f);
+  const float2 t = __fadd2_rn(x, magic);
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
+  float2 p = __ffma2_rn(make_float2(kExp2C4, kExp2C4), f, make_float2(kExp2C3, kExp2C3));
+  p = __ffma2_rn(p, f, make_float2(kExp2C2, kExp2C2));
+  p = __ffma2_rn(p, f, make_float2(kExp2C1, kExp2C1));
+  p = __ffma2_rn(p, f, make_float2(kExp2C0, kExp2C0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 // P = 2^(x - m) for one row, written as bf16 pairs over the first 64 TMEM
-// columns of the row's S tile; returns the fp32 row sum.  With EMUL, every
-// fourth column uses the FMA-pipe polynomial instead of the MUFU ex2.
+// columns of the row's S tile; returns the fp32 row sum.  Scale, shift and
+// the row sum use packed fp32 pairs.  With EMUL, 5 of every 16 pairs take the
+// FMA-pipe polynomial instead of the MUFU ex2, balancing the two pipes.
 template <int MOD, bool EMUL>
 __device__ __forceinline__ float row_probs(float (&x)[4][32], const RowCtx& rc, float m_use,
                                            uint32_t s_addr) {
-  float lsum = 0.f;
-  const float neg_m = -m_use;
+  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+  const float2 neg_m = make_float2(-m_use, -m_use);
+  const float2 sl2 = make_float2(rc.sl2, rc.sl2);
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     uint32_t pk[16];
-    float s0 = 0.f, s1 = 0.f;
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
-      float arg0, arg1;
+      const float2 xs = make_float2(x[c][e], x[c][e + 1]);
+      float2 arg;
       if constexpr (pure_scale(MOD)) {
-        arg0 = fmaf(x[c][e], rc.sl2, neg_m);
-        arg1 = fmaf(x[c][e + 1], rc.sl2, neg_m);
+        arg = __ffma2_rn(xs, sl2, neg_m);
       } else {
-        arg0 = x[c][e] + neg_m;
-        arg1 = x[c][e + 1] + neg_m;
+        arg = __fadd2_rn(xs, neg_m);
       }
-      const float pa = ex2_approx(arg0);
-      const float pb = (EMUL && (e & 3) == 2) ? exp2_poly(arg1) : ex2_approx(arg1);
-      s0 += pa;
-      s1 += pb;
-      pk[e >> 1] = pack_bf16x2(pa, pb);
+      float2 pr;
+      if (EMUL && ((e >> 1) % 3) == 2) {
+        pr = exp2_poly2(arg);
+      } else {
+        pr = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+      }
+      if ((e >> 1) & 1) acc1 = __fadd2_rn(acc1, pr);
+      else acc0 = __fadd2_rn(acc0, pr);
+      pk[e >> 1] = pack_bf16x2(pr.x, pr.y);
     }
-    lsum += s0 + s1;
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
         "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(s_addr + c * 16),
@@ -220,7 +256,8 @@ __device__ __forceinline__ float row_probs(float (&x)[4][32], const RowCtx& rc, 
         "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
         : "memory");
   }
-  return lsum;
+  const float2 acc = __fadd2_rn(acc0, acc1);
+  return acc.x + acc.y;
 }
 
 template <int D, int MOD, bool HAS_LSE>
@@ -236,11 +273,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t q_smem[2] = {sbase + Cfg::kQOff, sbase + Cfg::kQOff + Cfg::kTileBytes};
   const uint32_t ring = sbase + Cfg::kRingOff;
+  uint32_t* lists = reinterpret_cast<uint32_t*>(smem + Cfg::kListOff);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars->list_full[i]), 32);
+      mbar_init(smem_u32(&bars->list_empty[i]), kListConsumers);
+    }
     mbar_init(smem_u32(&bars->q_full), 1);
     mbar_init(smem_u32(&bars->q_empty), 1);
     for (int t = 0; t < 2; ++t) {
@@ -283,57 +325,64 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   if constexpr (kSplitRegs) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
   if (warp == 9) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      uint32_t slot_uses[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      int ring_pos = 0;
-      int unit_iter = 0;
-      uint32_t q_loads = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
-        const UnitCoord uc = decode_unit(a, u);
-        const int hk = uc.h / a.G;
+    // all lanes build the step lists; lane 0 issues the copies
+    uint32_t slot_uses[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    int ring_pos = 0;
+    int unit_iter = 0;
+    uint32_t q_loads = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+      const UnitCoord uc = decode_unit(a, u);
+      const int hk = uc.h / a.G;
+      const int buf = unit_iter & 1;
+      uint32_t* lst = lists + buf * kMaxSteps;
+      if (!mbar_wait_warp(smem_u32(&bars->list_empty[buf]), ((unit_iter >> 1) & 1) ^ 1, wc)) { ok = false; break; }
+      const int n = build_pair_steps(a.tile_class, uc.b, uc.p, a.nQ, a.nK, a.Sq, a.Skv, MOD,
+                                     a.mod.window, lst);
+      if (lane == 0) bars->list_n[buf] = n;
+      mbar_arrive(smem_u32(&bars->list_full[buf]));
+      if (lane == 0) {
         // Q buffers are free once the previous unit's QK^T products finished
-        if (!ATTN25_TIMED(tr[1], mbar_wait_thread(smem_u32(&bars->q_empty), (unit_iter & 1) ^ 1, wc))) { ok = false; break; }
-        mbar_arrive_expect_tx(smem_u32(&bars->q_full), 2 * Cfg::kTileBytes);
-        ++q_loads;
-        const int bh_q = uc.b * a.Hq + uc.h;
-        load_tile<D>(q_smem[0], &tm_q, smem_u32(&bars->q_full), (2 * uc.p) * TILE, bh_q);
-        load_tile<D>(q_smem[1], &tm_q, smem_u32(&bars->q_full), (2 * uc.p + 1) * TILE, bh_q);
-        PairIter it;
-        it.init(a.tile_class, a.kv_count, a.kv_index, uc.b, uc.p, a.nQ, a.nK, a.Sq, a.Skv,
-                MOD, a.mod.window);
-        int kt;
-        bool a0, a1, p0, p1;
-        const int bh_kv = uc.b * a.Hkv + hk;
-        while (it.next(kt, a0, a1, p0, p1)) {
+        if (!ATTN25_TIMED(tr[1], mbar_wait_thread(smem_u32(&bars->q_empty), (unit_iter & 1) ^ 1, wc))) {
+          ok = false;
+        } else {
+          mbar_arrive_expect_tx(smem_u32(&bars->q_full), 2 * Cfg::kTileBytes);
+          ++q_loads;
+          const int bh_q = uc.b * a.Hq + uc.h;
+          load_tile<D>(q_smem[0], &tm_q, smem_u32(&bars->q_full), (2 * uc.p) * TILE, bh_q);
+          load_tile<D>(q_smem[1], &tm_q, smem_u32(&bars->q_full), (2 * uc.p + 1) * TILE, bh_q);
+          const int bh_kv = uc.b * a.Hkv + hk;
+          for (int j2 = 0; j2 < n && ok; ++j2) {
+            const int kt = static_cast<int>(lst[j2] & 0xFFFFFu);
 #pragma unroll
-          for (int which = 0; which < 2; ++which) {  // K then V
-            const int slot = ring_pos % Cfg::kStages;
-            const uint32_t phase = (ring_pos / Cfg::kStages) & 1;
-            if (!ATTN25_TIMED(tr[2], mbar_wait_thread(smem_u32(&bars->kv_empty[slot]), phase ^ 1, wc))) { ok = false; break; }
-            const uint32_t bar = smem_u32(&bars->kv_full[slot]);
-            mbar_arrive_expect_tx(bar, Cfg::kTileBytes);
-            load_tile<D>(ring + slot * Cfg::kTileBytes, which == 0 ? &tm_k : &tm_v, bar, kt * TILE,
-                         bh_kv);
-            ++slot_uses[slot];
-            ++ring_pos;
+            for (int which = 0; which < 2; ++which) {  // K then V
+              const int slot = ring_pos % Cfg::kStages;
+              const uint32_t phase = (ring_pos / Cfg::kStages) & 1;
+              if (!ATTN25_TIMED(tr[2], mbar_wait_thread(smem_u32(&bars->kv_empty[slot]), phase ^ 1, wc))) { ok = false; break; }
+              const uint32_t bar = smem_u32(&bars->kv_full[slot]);
+              mbar_arrive_expect_tx(bar, Cfg::kTileBytes);
+              load_tile<D>(ring + slot * Cfg::kTileBytes, which == 0 ? &tm_k : &tm_v, bar, kt * TILE,
+                           bh_kv);
+              ++slot_uses[slot];
+              ++ring_pos;
+            }
           }
-          if (!ok) break;
         }
       }
-      if (!ok) {
-        // let copies already in flight land before the CTA exits
-        const WaitCtl drain_wc{a.wait_ns, smem_u32(&bars->never_set), a.status};
-        for (int s = 0; s < Cfg::kStages; ++s) {
-          if (slot_uses[s] == 0) continue;
-          mbar_wait_thread(smem_u32(&bars->kv_full[s]), (slot_uses[s] - 1) & 1, drain_wc);
-        }
-        if (q_loads > 0)
-          mbar_wait_thread(smem_u32(&bars->q_full), (q_loads - 1) & 1, drain_wc);
-      }
-      ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
-      trace_flush(a.trace, 48, tr);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     }
+    if (!ok && lane == 0) {
+      // let copies already in flight land before the CTA exits
+      const WaitCtl drain_wc{a.wait_ns, smem_u32(&bars->never_set), a.status};
+      for (int s2 = 0; s2 < Cfg::kStages; ++s2) {
+        if (slot_uses[s2] == 0) continue;
+        mbar_wait_thread(smem_u32(&bars->kv_full[s2]), (slot_uses[s2] - 1) & 1, drain_wc);
+      }
+      if (q_loads > 0)
+        mbar_wait_thread(smem_u32(&bars->q_full), (q_loads - 1) & 1, drain_wc);
+    }
+    ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
+    trace_flush(a.trace, 48, tr);
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
     // all lanes run the loop (waits are warp-collective); lane 0 issues
@@ -344,15 +393,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t s_tmem[2] = {tmem, tmem + 128};
     const uint32_t o_tmem[2] = {tmem + 256, tmem + 256 + D};
     for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
-      const UnitCoord uc = decode_unit(a, u);
+      const int buf = unit_iter & 1;
+      const uint32_t* lst = lists + buf * kMaxSteps;
+      if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+      const int n_steps = bars->list_n[buf];
       if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->q_full), unit_iter & 1, wc))) { ok = false; break; }
       tc_fence_after();
-      PairIter it;
-      it.init(a.tile_class, a.kv_count, a.kv_index, uc.b, uc.p, a.nQ, a.nK, a.Sq, a.Skv, MOD,
-              a.mod.window);
-      int kt;
-      bool act[2], prt[2];
-      bool has = it.next(kt, act[0], act[1], prt[0], prt[1]);
+      int j = 0;
+      bool act[2];
+      bool has = n_steps > 0;
+      if (has) {
+        const uint32_t e = lst[0];
+        act[0] = (e & kStepAct0) != 0;
+        act[1] = (e & kStepAct1) != 0;
+      }
       bool o_started[2] = {false, false};
       if (has) {
         const int slot_k = ring_pos % Cfg::kStages;
@@ -374,9 +428,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int slot_v = ring_pos % Cfg::kStages;
         const uint32_t ph_v = (ring_pos / Cfg::kStages) & 1;
         ++ring_pos;
-        int kt_n;
-        bool act_n[2], prt_n[2];
-        const bool has_n = it.next(kt_n, act_n[0], act_n[1], prt_n[0], prt_n[1]);
+        bool act_n[2] = {false, false};
+        const bool has_n = j + 1 < n_steps;
+        if (has_n) {
+          const uint32_t e = lst[j + 1];
+          act_n[0] = (e & kStepAct0) != 0;
+          act_n[1] = (e & kStepAct1) != 0;
+        }
         const int slot_kn = ring_pos % Cfg::kStages;
         const uint32_t ph_kn = (ring_pos / Cfg::kStages) & 1;
         if (!ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->kv_full[slot_v]), ph_v, wc))) { ok = false; break; }
@@ -414,7 +472,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         __syncwarp();
         if (has_n) ++ring_pos;
         has = has_n;
-        kt = kt_n;
+        ++j;
         act[0] = act_n[0];
         act[1] = act_n[1];
       }
@@ -423,6 +481,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mma_commit(smem_u32(&bars->q_empty));
         mma_commit(smem_u32(&bars->o_final[0]));
         mma_commit(smem_u32(&bars->o_final[1]));
+        mbar_arrive(smem_u32(&bars->list_empty[buf]));
       }
       __syncwarp();
     }
@@ -465,13 +524,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
       float m_run = -INFINITY, l_run = 0.f;
       int n_act = 0;
-      PairIter it;
-      it.init(a.tile_class, a.kv_count, a.kv_index, uc.b, uc.p, a.nQ, a.nK, a.Sq, a.Skv, MOD,
-              a.mod.window);
-      int kt;
-      bool act[2], prt[2];
-      while (it.next(kt, act[0], act[1], prt[0], prt[1])) {
-        if (!act[t]) continue;
+      const int buf = unit_iter & 1;
+      const uint32_t* lst = lists + buf * kMaxSteps;
+      if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+      const int n_steps = bars->list_n[buf];
+      const uint32_t act_bit = t == 0 ? kStepAct0 : kStepAct1;
+      const uint32_t prt_bit = t == 0 ? kStepPrt0 : kStepPrt1;
+      for (int j = 0; j < n_steps; ++j) {
+        const uint32_t e = lst[j];
+        if (!(e & act_bit)) continue;
+        const int kt = static_cast<int>(e & 0xFFFFFu);
+        const bool prt_t = (e & prt_bit) != 0;
         if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->s_full[t]), s_cnt & 1, wc))) { ok = false; break; }
         ++s_cnt;
         ATTN25_TRACE_ONLY(const long long t_tile = clock64(); tr[7] += 1;)
@@ -482,8 +545,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int c = 0; c < 4; ++c)
           tmem_ld32(s_addr + c * 32, reinterpret_cast<uint32_t(&)[32]>(x[c]));
         tmem_wait_ld();
-        const float mx = prt[t] ? row_scores<MOD, true>(x, rc, a.mod, k0)
-                                : row_scores<MOD, false>(x, rc, a.mod, k0);
+        const float mx = prt_t ? row_scores<MOD, true>(x, rc, a.mod, k0)
+                               : row_scores<MOD, false>(x, rc, a.mod, k0);
         const float m_new = fmaxf(m_run, mx);
         const bool need = m_new > m_run + kRescaleThreshold;
         if (__any_sync(0xffffffffu, need)) {
@@ -509,8 +572,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
         ATTN25_TRACE_ONLY(const long long t_mid = clock64(); tr[2] += t_mid - t_tile;)
         // full tiles hold no -inf, so part of their exponentials can run on the FMA pipe
-        const float lsum = prt[t] ? row_probs<MOD, false>(x, rc, m_use, s_addr)
-                                  : row_probs<MOD, true>(x, rc, m_use, s_addr);
+        const float lsum = prt_t ? row_probs<MOD, false>(x, rc, m_use, s_addr)
+                                 : row_probs<MOD, true>(x, rc, m_use, s_addr);
         l_run += lsum;
         ATTN25_TRACE_ONLY(tr[3] += clock64() - t_mid;)
         tmem_wait_st();
@@ -553,6 +616,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           a.lse[row_idx] = (l_run > 0.f) ? (m_run + __log2f(l_run)) * LN2 : -INFINITY;
       }
       tc_fence_before();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->list_empty[buf]));
       ATTN25_TRACE_ONLY(tr[5] += clock64() - t_epi;)
     }
     ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)

@@ -115,4 +115,109 @@ struct PairIter {
   }
 };
 
+// ------------------------------------------------------------------ step lists
+//
+// The TMA warp writes each work unit's list of steps into shared memory once
+// (all 32 lanes, coalesced reads of the block mask), and every other role
+// reads its steps from there: no role walks global memory per step.
+constexpr int kMaxSteps = 2048;  // list capacity: key tiles (forward) / query tiles (backward)
+
+// Forward step entry: key tile in bits 0-19; bit 20/21: query tile 0/1 has
+// work there; bit 22/23: query tile 0/1 needs the element predicate.
+constexpr uint32_t kStepAct0 = 1u << 20, kStepAct1 = 1u << 21;
+constexpr uint32_t kStepPrt0 = 1u << 22, kStepPrt1 = 1u << 23;
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Executed by a whole warp; returns the number of steps (all lanes).
+// tile_class == nullptr: dense iteration with closed-form classes.
+__device__ __forceinline__ int build_pair_steps(const uint8_t* tile_class, int b, int p, int nQ,
+                                                int nK, int Sq, int Skv, int kind, int window,
+                                                uint32_t* list) {
+  const int lane = threadIdx.x & 31;
+  const int qt0 = 2 * p, qt1 = 2 * p + 1;
+  const bool has1 = qt1 < nQ;
+  const int q0a = qt0 * TILE, q1a = min(Sq, q0a + TILE);
+  const int q0b = qt1 * TILE, q1b = has1 ? min(Sq, q0b + TILE) : q0b;
+  int k_begin = 0, k_end = nK;
+  if (tile_class == nullptr && is_interval_mask(kind)) {
+    k_end = min(nK, (max(q1a, q1b) - 1) / TILE + 1);
+    if (kind == MOD_WINDOW) k_begin = max(0, (q0a - window + 1) / TILE);
+  }
+  const bool tail = (Skv % TILE) != 0;
+  const uint8_t* r0 = tile_class == nullptr ? nullptr
+                                            : tile_class + (static_cast<size_t>(b) * nQ + qt0) * nK;
+  int n = 0;
+  for (int base = k_begin; base < k_end; base += 32) {
+    const int kt = base + lane;
+    int c0 = 0, c1 = 0;
+    if (kt < k_end) {
+      if (r0 != nullptr) {
+        c0 = __ldg(r0 + kt);
+        c1 = has1 ? __ldg(r0 + nK + kt) : 0;
+      } else {
+        const int k0 = kt * TILE, k1 = min(Skv, k0 + TILE);
+        if (kind == MOD_CAUSAL || kind == MOD_WINDOW) {
+          c0 = interval_tile_class(kind, window, q0a, q1a, k0, k1);
+          c1 = has1 ? interval_tile_class(kind, window, q0b, q1b, k0, k1) : 0;
+        } else {
+          c0 = kind == MOD_DOCUMENT ? 1 : 2;
+          c1 = has1 ? c0 : 0;
+        }
+      }
+    }
+    const bool active = (c0 | c1) != 0;
+    const uint32_t ballot = __ballot_sync(0xffffffffu, active);
+    if (active) {
+      const int pos = n + __popc(ballot & lanemask_lt());
+      const bool t = tail && kt == nK - 1;
+      uint32_t e = static_cast<uint32_t>(kt);
+      if (c0) e |= kStepAct0 | ((c0 == 1 || t) ? kStepPrt0 : 0u);
+      if (c1) e |= kStepAct1 | ((c1 == 1 || t) ? kStepPrt1 : 0u);
+      if (pos < kMaxSteps) list[pos] = e;
+    }
+    n += __popc(ballot);
+  }
+  return min(n, kMaxSteps);
+}
+
+// Backward step source: the query tiles (and their class) a key tile meets.
+// Entry: query tile in bits 0-19, bit 20: the element predicate is needed.
+constexpr uint32_t kQtPred = 1u << 20;
+
+__device__ __forceinline__ int build_kv_qtiles(const uint8_t* tile_class, int b, int kt, int nQ,
+                                               int nK, int Sq, int Skv, int kind, int window,
+                                               uint32_t* list) {
+  const int lane = threadIdx.x & 31;
+  int q_begin = 0;
+  if (tile_class == nullptr && is_interval_mask(kind)) q_begin = kt;  // every mask keeps q >= kv
+  const bool tail_kv = (Skv % TILE) != 0 && kt == nK - 1;
+  const int k0 = kt * TILE, k1 = min(Skv, k0 + TILE);
+  int n = 0;
+  for (int base = q_begin; base < nQ; base += 32) {
+    const int qt = base + lane;
+    int c = 0;
+    if (qt < nQ) {
+      if (tile_class != nullptr) {
+        c = __ldg(tile_class + (static_cast<size_t>(b) * nQ + qt) * nK + kt);
+      } else if (kind == MOD_CAUSAL || kind == MOD_WINDOW) {
+        c = interval_tile_class(kind, window, qt * TILE, min(Sq, qt * TILE + TILE), k0, k1);
+      } else {
+        c = kind == MOD_DOCUMENT ? 1 : 2;
+      }
+    }
+    const uint32_t ballot = __ballot_sync(0xffffffffu, c != 0);
+    if (c != 0) {
+      const int pos = n + __popc(ballot & lanemask_lt());
+      if (pos < kMaxSteps) list[pos] = static_cast<uint32_t>(qt) | ((c == 1 || tail_kv) ? kQtPred : 0u);
+    }
+    n += __popc(ballot);
+  }
+  return min(n, kMaxSteps);
+}
+
 }  // namespace attn25
