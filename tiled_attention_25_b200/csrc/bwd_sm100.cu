@@ -50,7 +50,7 @@ struct BwdCfg {
   static constexpr int kKVBytes = TILE * D * 2;           // one 128-key tile of K or V
   static constexpr int kQBytes = BM * D * 2;              // one 64-row tile of Q or dO
   static constexpr int kStageBytes = 2 * kQBytes + 1024;  // Q, dO, LSE2 and Delta rows
-  static constexpr int kStages = 2;
+  static constexpr int kStages = 3;  // Q / dO / statistics stages
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kKVBytes;
   static constexpr int kStageOff = 2 * kKVBytes;
@@ -72,7 +72,7 @@ struct BwdCfg {
 struct BwdBarriers {
   uint64_t list_full[2], list_empty[2];
   uint64_t kv_full, kv_empty;
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full[4], q_empty[4];
   uint64_t s_full[2], s_free[2], p_ready[2];
   uint64_t dp_full, ds_ready;
   uint64_t ds_empty[2];
@@ -311,9 +311,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(smem_u32(&bars->kv_full), 1);
     mbar_init(smem_u32(&bars->kv_empty), 1);
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < Cfg::kStages; ++b) {
       mbar_init(smem_u32(&bars->q_full[b]), 1);
       mbar_init(smem_u32(&bars->q_empty[b]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&bars->ds_empty[b]), 1);
       mbar_init(smem_u32(&bars->s_full[b]), 1);
       mbar_init(smem_u32(&bars->s_free[b]), 128);
@@ -355,7 +357,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // ---------------------------------------------------------- TMA producer
       // all lanes build the query-tile lists; lane 0 issues the copies
       int unit_iter = 0, step = 0;
-      uint32_t kv_loads = 0, stage_uses[2] = {0, 0};
+      uint32_t kv_loads = 0, stage_uses[4] = {0, 0, 0, 0};
       bool ok = true;
       for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
         const BwdUnit un = decode_bwd_unit(a, u);
@@ -380,8 +382,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             int g, q0;
             bool pred;
             while (it.next(g, q0, pred)) {
-              const int s = step & 1;
-              if (!ATTN25_TIMED(tr[2], mbar_wait_thread(smem_u32(&bars->q_empty[s]), ((step >> 1) & 1) ^ 1, wc))) { ok = false; break; }
+              const int s = step % Cfg::kStages;
+              if (!ATTN25_TIMED(tr[2], mbar_wait_thread(smem_u32(&bars->q_empty[s]), ((step / Cfg::kStages) & 1) ^ 1, wc))) { ok = false; break; }
               const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
               const uint32_t bar = smem_u32(&bars->q_full[s]);
               mbar_arrive_expect_tx(bar, 2 * Cfg::kQBytes + 2 * BM * 4);
@@ -401,7 +403,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ok && lane == 0) {
         const WaitCtl dwc{a.wait_ns, smem_u32(&bars->never_set), a.status};
         if (kv_loads) mbar_wait_thread(smem_u32(&bars->kv_full), (kv_loads - 1) & 1, dwc);
-        for (int s = 0; s < 2; ++s)
+        for (int s = 0; s < Cfg::kStages; ++s)
           if (stage_uses[s]) mbar_wait_thread(smem_u32(&bars->q_full[s]), (stage_uses[s] - 1) & 1, dwc);
       }
       ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
@@ -428,44 +430,44 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bool has = it.next(g, q0, pred);
         int n_steps = 0;
         if (has) {  // S^T and dP^T of the first step
-          const int s = step & 1;
-          if (!ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step >> 1) & 1, wc))) { ok = false; break; }
-          if (!ATTN25_TIMED(tr[8], mbar_wait_warp(smem_u32(&bars->s_free[s]), ((step >> 1) & 1) ^ 1, wc))) { ok = false; break; }
+          const int s = step % Cfg::kStages, sb = step & 1;
+          if (!ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step / Cfg::kStages) & 1, wc))) { ok = false; break; }
+          if (!ATTN25_TIMED(tr[8], mbar_wait_warp(smem_u32(&bars->s_free[sb]), ((step >> 1) & 1) ^ 1, wc))) { ok = false; break; }
           tc_fence_after();
           const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
           if (lane == 0) {
-            issue_st<D>(tmem + Cfg::kColS + s * BM, k_smem, st);
-            mma_commit(smem_u32(&bars->s_full[s]));
+            issue_st<D>(tmem + Cfg::kColS + sb * BM, k_smem, st);
+            mma_commit(smem_u32(&bars->s_full[sb]));
             issue_st<D>(t_dp, v_smem, st + Cfg::kQBytes);
             mma_commit(smem_u32(&bars->dp_full));
           }
           __syncwarp();
         }
         while (has) {
-          const int s = step & 1;  // stage and S^T buffer of this step
+          const int s = step % Cfg::kStages, sb = step & 1;  // stage and S^T buffer of this step
           const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
           int g_n, q0_n;
           bool pred_n;
           const bool has_n = it.next(g_n, q0_n, pred_n);
-          const int s_n = (step + 1) & 1;
+          const int s_n = (step + 1) % Cfg::kStages, sb_n = (step + 1) & 1;
           const uint32_t st_n = sbase + Cfg::kStageOff + s_n * Cfg::kStageBytes;
           if (has_n) {  // S^T of the next step into the other buffer, ahead of this step's dS
-            if (!ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s_n]), ((step + 1) >> 1) & 1, wc))) { ok = false; break; }
-            if (!ATTN25_TIMED(tr[8], mbar_wait_warp(smem_u32(&bars->s_free[s_n]), (((step + 1) >> 1) & 1) ^ 1, wc))) { ok = false; break; }
+            if (!ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s_n]), ((step + 1) / Cfg::kStages) & 1, wc))) { ok = false; break; }
+            if (!ATTN25_TIMED(tr[8], mbar_wait_warp(smem_u32(&bars->s_free[sb_n]), (((step + 1) >> 1) & 1) ^ 1, wc))) { ok = false; break; }
             tc_fence_after();
             if (lane == 0) {
-              issue_st<D>(tmem + Cfg::kColS + s_n * BM, k_smem, st_n);
-              mma_commit(smem_u32(&bars->s_full[s_n]));
+              issue_st<D>(tmem + Cfg::kColS + sb_n * BM, k_smem, st_n);
+              mma_commit(smem_u32(&bars->s_full[sb_n]));
             }
             __syncwarp();
           }
           // dV += P^T dO once P^T is in tensor memory
-          if (!ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->p_ready[s]), (step >> 1) & 1, wc))) { ok = false; break; }
+          if (!ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->p_ready[sb]), (step >> 1) & 1, wc))) { ok = false; break; }
           tc_fence_after();
           if (lane == 0) {
 #pragma unroll
             for (int kk = 0; kk < BM / 16; ++kk)
-              mma_ts(t_dv, tmem + Cfg::kColS + s * BM + kk * 8,
+              mma_ts(t_dv, tmem + Cfg::kColS + sb * BM + kk * 8,
                      smem_desc_sw128(st + Cfg::kQBytes + kk * 2048, BM * 128, 1024), Cfg::kIdescAcc,
                      (n_steps > 0 || kk > 0) ? 1u : 0u);
           }
@@ -542,11 +544,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       bool pred;
       int n_steps = 0;
       while (it.next(g, q0, pred)) {
-        const int s = step & 1;
+        const int s = step % Cfg::kStages, sb = step & 1;
         const uint32_t nl2_s = sbase + Cfg::kStageOff + s * Cfg::kStageBytes + 2 * Cfg::kQBytes;
-        const uint32_t t_s = tmem + Cfg::kColS + s * BM + lane_off;
-        if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step >> 1) & 1, wc))) { ok = false; break; }
-        if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->s_full[s]), (step >> 1) & 1, wc))) { ok = false; break; }
+        const uint32_t t_s = tmem + Cfg::kColS + sb * BM + lane_off;
+        if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step / Cfg::kStages) & 1, wc))) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->s_full[sb]), (step >> 1) & 1, wc))) { ok = false; break; }
         tc_fence_after();
         ATTN25_TRACE_ONLY(const long long t_p = clock64();)
         const int h = un.hk * a.G + g;
@@ -562,7 +564,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_st32(t_s, pk);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(smem_u32(&bars->p_ready[s]));
+        mbar_arrive(smem_u32(&bars->p_ready[sb]));
         ATTN25_TRACE_ONLY(tr[3] += clock64() - t_p;)
         ++n_steps;
         ++step;
@@ -601,11 +603,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       bool pred;
       int n_steps = 0;
       while (it.next(g, q0, pred)) {
-        const int s = step & 1;
+        const int s = step % Cfg::kStages, sb = step & 1;
         const uint32_t stats = sbase + Cfg::kStageOff + s * Cfg::kStageBytes + 2 * Cfg::kQBytes;
-        const uint32_t t_p = tmem + Cfg::kColS + s * BM + lane_off;
-        if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step >> 1) & 1, wc))) { ok = false; break; }
-        if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->p_ready[s]), (step >> 1) & 1, wc))) { ok = false; break; }
+        const uint32_t t_p = tmem + Cfg::kColS + sb * BM + lane_off;
+        if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step / Cfg::kStages) & 1, wc))) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->p_ready[sb]), (step >> 1) & 1, wc))) { ok = false; break; }
         if (!ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->dp_full), dp_cnt & 1, wc))) { ok = false; break; }
         ++dp_cnt;
         tc_fence_after();
@@ -618,7 +620,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_wait_ld();
         // P^T of this buffer has been read: the next-but-one S^T may overwrite it
         tc_fence_before();
-        mbar_arrive(smem_u32(&bars->s_free[s]));
+        mbar_arrive(smem_u32(&bars->s_free[sb]));
         // the dS buffer is free once the MMAs of two steps ago completed
         if (!ATTN25_TIMED(tr[5], mbar_wait_warp(smem_u32(&bars->ds_empty[ds_cnt & 1]), ((ds_cnt >> 1) & 1) ^ 1, wc))) { ok = false; break; }
         uint8_t* ds_row = smem + Cfg::kDSOff + (ds_cnt & 1) * Cfg::kDSBytes + r * 128;
