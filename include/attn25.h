@@ -157,6 +157,36 @@ ATTN25_API int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16*
              int mod_kind, const attn_mod_params* mod_params,
              const attn_block_mask* block_mask, attn_stream_t stream);
 
+/*
+ * attn_bwd without a workspace argument, for callers that cannot allocate
+ * device memory when they call it: for example a plugin host that hands its
+ * kernels no workspace, or an application whose device memory is carved up
+ * in advance by its own pool and must not grow.  The library itself holds a
+ * fixed 32 MiB block of device memory for this (reserved on every GPU that
+ * loads the library, until the process exits) and runs the same kernels as
+ * attn_bwd on it; this function allocates nothing.  The paper has no
+ * counterpart; it exists for this deployment constraint only.
+ *
+ * - Problems whose attn_bwd_workspace_size exceeds
+ *   attn_bwd_noalloc_max_workspace() are rejected with ATTN_ERR_WORKSPACE.
+ * - The first call of the library on a device (this one included) looks up
+ *   the block's device address; make that first call before any stream
+ *   capture.
+ * - All calls share the one block.  Calls whose GPU work overlaps in time
+ *   (two streams, or two host threads) race and corrupt each other's
+ *   results; serialise them on one stream.  Contents left by an earlier call
+ *   are rewritten before use, so back-to-back calls are fine.
+ */
+ATTN25_API int attn_bwd_noalloc(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v,
+             const attn_bf16* out, const float* lse, const attn_bf16* dout,
+             attn_bf16* dq, attn_bf16* dk, attn_bf16* dv,
+             int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+             int mod_kind, const attn_mod_params* mod_params,
+             const attn_block_mask* block_mask, attn_stream_t stream);
+
+/* Largest workspace attn_bwd_noalloc can use (bytes). */
+ATTN25_API size_t attn_bwd_noalloc_max_workspace(void);
+
 /* Bytes of device memory one block mask for (B, Sq, Skv) occupies. */
 ATTN25_API size_t attn_block_mask_bytes(int B, int Sq, int Skv);
 

@@ -17,9 +17,12 @@ def declared():
 
 @pytest.fixture(scope="module")
 def lib():
-    from tiled_attention_25_b200.build import build
-    path = build()
-    return ctypes.CDLL(path)
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "attn25_build", os.path.join(ROOT, "tiled_attention_25_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return ctypes.CDLL(mod.build())
 
 
 def test_header_declares_the_boundary():

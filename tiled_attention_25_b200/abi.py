@@ -67,13 +67,17 @@ class CBlockMask(ctypes.Structure):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m tiled_attention_25_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python tiled_attention_25_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, P, P, P]
     lib.attn_fwd.restype = I
     lib.attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, S, I, I, I, I, I, I, F, I, P, P, P]
     lib.attn_bwd.restype = I
+    lib.attn_bwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P, P, P]
+    lib.attn_bwd_noalloc.restype = I
+    lib.attn_bwd_noalloc_max_workspace.argtypes = []
+    lib.attn_bwd_noalloc_max_workspace.restype = S
     lib.attn_bwd_workspace_size.argtypes = [I, I, I, I]
     lib.attn_bwd_workspace_size.restype = S
     lib.attn_block_mask_bytes.argtypes = [I, I, I]
@@ -98,7 +102,8 @@ def _load():
 
 LIB = _load()
 
-EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_block_mask_bytes",
+EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_bwd_noalloc",
+            "attn_bwd_noalloc_max_workspace", "attn_block_mask_bytes",
             "attn_block_mask_bind", "build_block_mask", "attn_get_status",
             "attn_set_wait_limit_ms", "attn_strerror")
 
@@ -221,6 +226,29 @@ def attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, workspace, scale=None, mod_kin
                       B, Hq, Hkv, Sq, Skv, D, scale, int(mod_kind), None if mp is None else mp[0],
                       None if block_mask is None else ctypes.byref(block_mask.c), _stream(stream))
     _check(rc, "attn_bwd")
+
+
+def attn_bwd_noalloc(q, k, v, out, lse, dout, dq, dk, dv, scale=None, mod_kind=MOD_NONE,
+                     mod_params=None, block_mask=None, stream=None):
+    """attn_bwd on the library's own fixed workspace (see include/attn25.h)."""
+    B, Hq, Hkv, Sq, Skv, D = _dims(q, k, v, out)
+    for t in (dout, dq):
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != (B, Hq, Sq, D) or not t.is_contiguous():
+            raise ValueError("dout/dq must be contiguous bf16 like q")
+    for t in (dk, dv):
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != (B, Hkv, Skv, D) or not t.is_contiguous():
+            raise ValueError("dk/dv must be contiguous bf16 like k")
+    scale = D ** -0.5 if scale is None else float(scale)
+    mp = _mp(mod_params)
+    rc = LIB.attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+                              _ptr(dk), _ptr(dv), B, Hq, Hkv, Sq, Skv, D, scale, int(mod_kind),
+                              None if mp is None else mp[0],
+                              None if block_mask is None else ctypes.byref(block_mask.c), _stream(stream))
+    _check(rc, "attn_bwd_noalloc")
+
+
+def attn_bwd_noalloc_max_workspace() -> int:
+    return int(LIB.attn_bwd_noalloc_max_workspace())
 
 
 def attn_block_mask_bytes(B, Sq, Skv) -> int:

@@ -1,6 +1,7 @@
 """Build libattn25.so in-tree with nvcc for sm_100a.
 
-Usage: python -m tiled_attention_25_b200.build  (or call build()).
+Usage: python tiled_attention_25_b200/build.py [--trace]  (or call build()).
+Run it as a script: importing the package would first load the library.
 Each .cu file compiles to an object under _build/ in parallel; objects are
 reused while their sources and headers are unchanged.
 """

@@ -24,6 +24,12 @@ __device__ int g_attn_status;
 __device__ unsigned long long g_attn_trace[256];
 #endif
 
+// Backward workspace for attn_bwd_noalloc: a fixed block of device memory
+// that every GPU loading this library holds until the process exits, so
+// that callers without an allocator can still run the backward pass.
+constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(32) << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_bwd_scratch[kNoAllocScratchBytes];
+
 namespace {
 
 std::atomic<uint32_t> g_wait_ms{4000};
@@ -36,6 +42,7 @@ struct DeviceInfo {
   int sms = 0;
   int* status = nullptr;
   unsigned long long* trace = nullptr;
+  void* scratch = nullptr;  // device address of g_bwd_scratch (nullptr if unavailable)
 };
 
 std::mutex g_mu;
@@ -55,6 +62,10 @@ int current_device(DeviceInfo** out) {
     void* p = nullptr;
     const bool sym_ok = cudaGetSymbolAddress(&p, g_attn_status) == cudaSuccess;
     d.status = static_cast<int*>(p);
+    // Host code must not use g_bwd_scratch's name as a device address: look
+    // up the real address once, with this device current.
+    void* sp = nullptr;
+    if (cudaGetSymbolAddress(&sp, g_bwd_scratch) == cudaSuccess) d.scratch = sp;
 #if defined(ATTN25_TRACE)
     void* tp = nullptr;
     if (cudaGetSymbolAddress(&tp, g_attn_trace) == cudaSuccess) d.trace = static_cast<unsigned long long*>(tp);
@@ -406,6 +417,26 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
                  reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_LAUNCH;
   return ATTN_OK;
+}
+
+size_t attn_bwd_noalloc_max_workspace(void) { return kNoAllocScratchBytes; }
+
+int attn_bwd_noalloc(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v,
+                     const attn_bf16* out, const float* lse, const attn_bf16* dout, attn_bf16* dq,
+                     attn_bf16* dk, attn_bf16* dv, int B, int Hq, int Hkv, int Sq, int Skv, int D,
+                     float scale, int mod_kind, const attn_mod_params* mod_params,
+                     const attn_block_mask* block_mask, attn_stream_t stream) {
+  const size_t need = attn_bwd_workspace_size(B, Hq, Sq, D);
+  if (need == 0) return (D != 64 && D != 128) ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_ARG;
+  if (need > kNoAllocScratchBytes) return ATTN_ERR_WORKSPACE;
+  DeviceInfo* d = nullptr;
+  const int rc = current_device(&d);
+  if (rc != ATTN_OK) return rc;
+  if (d->scratch == nullptr) return ATTN_ERR_DEVICE;
+  // the backward's first kernel rewrites every word of the workspace it reads
+  // later (it zeroes the dQ accumulator), so stale contents do not matter
+  return attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, d->scratch, kNoAllocScratchBytes, B, Hq, Hkv,
+                  Sq, Skv, D, scale, mod_kind, mod_params, block_mask, stream);
 }
 
 #if defined(ATTN25_TRACE)
