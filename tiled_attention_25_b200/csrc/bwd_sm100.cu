@@ -464,6 +464,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           // dV += P^T dO once P^T is in tensor memory
           if (!ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->p_ready[sb]), (step >> 1) & 1, wc))) { ok = false; break; }
           tc_fence_after();
+          ATTN25_TRACE_ONLY(const long long t_i0 = clock64();)
           if (lane == 0) {
 #pragma unroll
             for (int kk = 0; kk < BM / 16; ++kk)
@@ -472,6 +473,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                      (n_steps > 0 || kk > 0) ? 1u : 0u);
           }
           __syncwarp();
+          ATTN25_TRACE_ONLY(tr[9] += clock64() - t_i0;)
           // dK += dS^T Q and dQ^T = K^T dS^T once dS^T is in shared memory
           if (!ATTN25_TIMED(tr[5], mbar_wait_warp(smem_u32(&bars->ds_ready), ds_cnt & 1, wc))) { ok = false; break; }
           const uint32_t ds_smem = sbase + Cfg::kDSOff + (ds_cnt & 1) * Cfg::kDSBytes;
@@ -479,6 +481,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           // the dQ^T columns must have been drained by the previous step
           if (!ATTN25_TIMED(tr[6], mbar_wait_warp(smem_u32(&bars->dq_empty), (dq_cnt & 1) ^ 1, wc))) { ok = false; break; }
           tc_fence_after();
+          ATTN25_TRACE_ONLY(const long long t_i1 = clock64();)
           if (lane == 0) {
 #pragma unroll
             for (int kk = 0; kk < BM / 16; ++kk)
@@ -499,6 +502,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
           }
           __syncwarp();
+          ATTN25_TRACE_ONLY(tr[10] += clock64() - t_i1;)
           ++dq_cnt;
           ++n_steps;
           ++step;
@@ -556,13 +560,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(t_s, reinterpret_cast<uint32_t(&)[32]>(x[0]));
         tmem_ld32(t_s + 32, reinterpret_cast<uint32_t(&)[32]>(x[32]));
         tmem_wait_ld();
+        ATTN25_TRACE_ONLY(const long long t_p1 = clock64(); tr[4] += t_p1 - t_p;)
         probs_t<MOD>(x, a, h, static_cast<float>(q0 - kv), q0, qlo, qhi, pred, nl2_s);
         // P^T (bf16 pairs) over the first 32 columns of this S^T buffer
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+        ATTN25_TRACE_ONLY(const long long t_p2 = clock64(); tr[5] += t_p2 - t_p1;)
         tmem_st32(t_s, pk);
         tmem_wait_st();
+        ATTN25_TRACE_ONLY(tr[6] += clock64() - t_p2;)
         tc_fence_before();
         mbar_arrive(smem_u32(&bars->p_ready[sb]));
         ATTN25_TRACE_ONLY(tr[3] += clock64() - t_p;)
@@ -618,6 +625,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(t_dp + 32, reinterpret_cast<uint32_t(&)[32]>(dp[32]));
         tmem_ld32(t_p, pb);
         tmem_wait_ld();
+        ATTN25_TRACE_ONLY(tr[3] += clock64() - t_ds;)
         // P^T of this buffer has been read: the next-but-one S^T may overwrite it
         tc_fence_before();
         mbar_arrive(smem_u32(&bars->s_free[sb]));
