@@ -3,7 +3,9 @@
  * with -DATTN25_TRACE.  Its kernels time selected barrier waits and phases
  * per warp role with clock64 and add them into a device counter buffer
  * (256 x uint64: forward roles at 0..63, backward roles at 128..255, 16 per
- * role).  The normal library (libattn25.so) does not export these.
+ * role).  After the counters, 512 words hold the clock64 of 16 events in
+ * each of 32 consecutive backward steps (steps 96..127 of CTA 0).  The normal
+ * library (libattn25.so) does not export these.
  */
 #ifndef ATTN25_TRACE_H
 #define ATTN25_TRACE_H
@@ -14,7 +16,7 @@
 extern "C" {
 #endif
 
-/* Synchronise the device, then copy the first n (<= 256) counters to host memory. */
+/* Synchronise the device, then copy the first n (<= 768) words to host memory. */
 ATTN25_API int attn_trace_read(unsigned long long* host_out, int n);
 
 /* Synchronise the device, then zero all counters. */

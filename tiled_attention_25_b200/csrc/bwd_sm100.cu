@@ -29,6 +29,25 @@
 #include "kernel_common.cuh"
 #include "launch.h"
 
+#ifndef ATTN25_DQ_RED
+#define ATTN25_DQ_RED 1
+#endif
+
+// Profiling builds: clock64 of event `id` of step `st` on CTA 0, written by
+// lane 0 of the first warp of each role, for a window of steps.
+#if defined(ATTN25_TRACE)
+#define BWD_EV(st, id)                                                                           \
+  do {                                                                                           \
+    if (blockIdx.x == 0 && lane == 0 && ((warp & 3) == 0 || warp >= 12) && (st) >= kEvStep0 &&  \
+        (st) < kEvStep0 + kEvSteps && a.trace != nullptr)                                        \
+      a.trace[kTraceCounters - 128 + ((st) - kEvStep0) * kEvPerStep + (id)] = clock64();          \
+  } while (0)
+#else
+#define BWD_EV(st, id) \
+  do {                 \
+  } while (0)
+#endif
+
 namespace attn25 {
 
 namespace {
@@ -56,10 +75,17 @@ struct BwdCfg {
   static constexpr int kStageOff = 2 * kKVBytes;
   static constexpr int kDSOff = kStageOff + kStages * kStageBytes;  // two 128 x 64 bf16 buffers
   static constexpr int kDSBytes = TILE * BM * 2;
-  static constexpr int kBarOff = kDSOff + 2 * kDSBytes;
-  static constexpr int kListOff = kBarOff + 1024;  // two query-tile lists
-  static constexpr int kSmemBytes = kListOff + 2 * kMaxSteps * 4;
+  // staging of dQ^T queries 32-63 ([d][32 q] fp32, 128-byte swizzle); queries
+  // 0-31 are staged in the step's dS buffer
+  static constexpr int kDQStageOff = kDSOff + 2 * kDSBytes;
+  static constexpr int kDQStageBytes = D * 32 * 4;
+  static_assert(kDQStageBytes <= kDSBytes, "dQ staging half must fit a dS buffer");
+  static_assert(kDSOff % 1024 == 0 && kDQStageOff % 1024 == 0, "swizzled staging alignment");
+  static constexpr int kBarOff = kDQStageOff + kDQStageBytes;
+  static constexpr int kListOff = kBarOff + 1024;  // two query-tile lists (16-bit entries)
+  static constexpr int kSmemBytes = kListOff + 2 * kMaxSteps * 2;
   static constexpr int kAllocBytes = kSmemBytes + 1024;
+  static_assert(kAllocBytes <= 232448, "shared memory");
   // TMEM columns: two S^T buffers (P^T overwrites their first 32 columns), dP^T,
   // the dV and dK accumulators, dQ^T
   static constexpr int kColS = 0, kColDP = 128, kColDV = 192, kColDK = 192 + D, kColDQ = 192 + 2 * D;
@@ -73,8 +99,8 @@ struct BwdBarriers {
   uint64_t list_full[2], list_empty[2];
   uint64_t kv_full, kv_empty;
   uint64_t q_full[4], q_empty[4];
-  uint64_t s_full[2], s_free[2], p_ready[2];
-  uint64_t dp_full, ds_ready;
+  uint64_t s_full[2], p_ready[2];
+  uint64_t dp_full, dp_empty, ds_ready;
   uint64_t ds_empty[2];
   uint64_t dq_full, dq_empty;
   uint64_t acc_full, acc_empty;
@@ -87,6 +113,7 @@ struct BwdBarriers {
 
 // Consumers of a query-tile list: the MMA warp and the P, dS and drain warps (lane 0 each).
 constexpr int kBwdListConsumers = 13;
+constexpr int kDrainWarps = 4;
 
 struct BwdUnit {
   int b, hk, kt;
@@ -107,12 +134,12 @@ __device__ __forceinline__ BwdUnit decode_bwd_unit(const BwdArgs& a, int u) {
 // each query head of the group, each listed 128-row query tile, and each
 // 64-row half of it that starts inside Sq.
 struct StepIter {
-  const uint32_t* list;
+  const uint16_t* list;
   int n, G, Sq;
   int g, j, half;
   uint32_t cur;
 
-  __device__ __forceinline__ void init(const uint32_t* list_, int n_, int G_, int Sq_) {
+  __device__ __forceinline__ void init(const uint16_t* list_, int n_, int G_, int Sq_) {
     list = list_;
     n = n_;
     G = G_;
@@ -136,11 +163,11 @@ struct StepIter {
         cur = list[j++];
         half = 0;
       }
-      const int start = static_cast<int>(cur & 0xFFFFFu) * TILE + (half++) * BM;
+      const int start = static_cast<int>(cur & kQtIndexMask) * TILE + (half++) * BM;
       if (start >= Sq) continue;
       g_out = g;
       q0 = start;
-      pred = (cur & kQtPred) != 0;
+      pred = (cur & kQtPred16) != 0;
       return true;
     }
   }
@@ -177,8 +204,8 @@ __device__ __forceinline__ void issue_st(uint32_t d_tmem, uint32_t a_smem, uint3
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t ka = (kk >> 2) * (TILE * 128) + (kk & 3) * 32;
     const uint32_t kb = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-    mma_ss(d_tmem, smem_desc_sw128(a_smem + ka, 16, 1024), smem_desc_sw128(b_smem + kb, 16, 1024),
-           BwdCfg<D>::kIdescST, kk > 0 ? 1u : 0u);
+    mma_ss_w(d_tmem, smem_desc_sw128(a_smem + ka, 16, 1024), smem_desc_sw128(b_smem + kb, 16, 1024),
+             BwdCfg<D>::kIdescST, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -215,11 +242,17 @@ __device__ __forceinline__ float4 lds128(uint32_t addr) {
   return v;
 }
 
-// One key row of S^T (raw q.k for 64 queries) -> P^T = 2^(x - LSE2) in place;
-// nl2 is the shared address of the 64 negated base-2 LSEs.
-template <int MOD>
+__device__ __forceinline__ void sts128(uint32_t addr, float x, float y, float z, float w) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(x), "f"(y), "f"(z), "f"(w) : "memory");
+}
+
+// One key row of S^T (raw q.k for 64 queries) -> P^T = 2^(x - LSE2) in place.
+// The 64 negated base-2 LSEs come from registers (nl2v, PREFETCHED) or from
+// shared memory at nl2_addr.
+template <int MOD, bool PREFETCHED>
 __device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h, float dq0, int q0,
-                                        int qlo, int qhi, bool pred, uint32_t nl2) {
+                                        int qlo, int qhi, bool pred, const float4 (&nl2v)[BM / 4],
+                                        uint32_t nl2_addr) {
   float aux = 0.f, aux2 = 0.f;
   if constexpr (MOD == MOD_ALIBI) aux = alibi_slope(a.mod, h, a.Hq) * LOG2E;
   if constexpr (MOD == MOD_SOFTCAP) {
@@ -230,7 +263,9 @@ __device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h,
   const float2 sl2 = make_float2(a.sl2, a.sl2);
 #pragma unroll
   for (int c4 = 0; c4 < BM / 4; ++c4) {
-    const float4 l = lds128(nl2 + c4 * 16);
+    float4 l;
+    if constexpr (PREFETCHED) l = nl2v[c4];
+    else l = lds128(nl2_addr + c4 * 16);
 #pragma unroll
     for (int hp = 0; hp < 2; ++hp) {
       const int c = c4 * 4 + hp * 2;
@@ -290,7 +325,7 @@ template <int D, int MOD>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const BwdArgs a) {
+                    const __grid_constant__ CUtensorMap tm_dq, const BwdArgs a) {
   using Cfg = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -299,7 +334,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t k_smem = sbase + Cfg::kKOff;
   const uint32_t v_smem = sbase + Cfg::kVOff;
-  uint32_t* lists = reinterpret_cast<uint32_t*>(smem + Cfg::kListOff);
+  uint16_t* lists = reinterpret_cast<uint16_t*>(smem + Cfg::kListOff);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   constexpr bool kSplitRegs = MOD != MOD_SOFTCAP && MOD != MOD_BOOST;
@@ -316,12 +351,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(smem_u32(&bars->q_empty[b]), 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&bars->ds_empty[b]), 1);
+      mbar_init(smem_u32(&bars->ds_empty[b]), kDrainWarps);
       mbar_init(smem_u32(&bars->s_full[b]), 1);
-      mbar_init(smem_u32(&bars->s_free[b]), 128);
       mbar_init(smem_u32(&bars->p_ready[b]), 128);
     }
     mbar_init(smem_u32(&bars->dp_full), 1);
+    mbar_init(smem_u32(&bars->dp_empty), 128);
     mbar_init(smem_u32(&bars->ds_ready), 128);
     mbar_init(smem_u32(&bars->dq_full), 1);
     mbar_init(smem_u32(&bars->dq_empty), 128);
@@ -342,6 +377,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
   }
+  if (warp == 8 && lane == 0) tma_prefetch_desc(&tm_dq);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -362,7 +398,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
         const BwdUnit un = decode_bwd_unit(a, u);
         const int buf = unit_iter & 1;
-        uint32_t* lst = lists + buf * kMaxSteps;
+        uint16_t* lst = lists + buf * kMaxSteps;
         if (!mbar_wait_warp(smem_u32(&bars->list_empty[buf]), ((unit_iter >> 1) & 1) ^ 1, wc)) { ok = false; break; }
         const int n = build_kv_qtiles(a.tile_class, un.b, un.kt, a.nQ, a.nK, a.Sq, a.Skv, MOD,
                                       a.mod.window, lst);
@@ -389,6 +425,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               mbar_arrive_expect_tx(bar, 2 * Cfg::kQBytes + 2 * BM * 4);
               ++stage_uses[s];
               const int bh = un.b * a.Hq + un.hk * a.G + g;
+              BWD_EV(step, 0);
               load_q_tile<D>(st, &tm_q, bar, q0, bh);
               load_q_tile<D>(st + Cfg::kQBytes, &tm_do, bar, q0, bh);
               const size_t row = static_cast<size_t>(bh) * a.Sq_pad + q0;
@@ -410,17 +447,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       trace_flush(a.trace, 48, tr);
     } else if (warp == 12) {
       // ---------------------------------------------------------- MMA issuer
+      // Per step j (global step counter; S^T buffer j & 1, stage j % 3):
+      //   S^T(j+1)           once Q(j+1) has landed
+      //   dV  += P^T(j) dO   once P^T(j) is in TMEM
+      //   dP^T(j+1)          once the dS warps have read dP^T(j)
+      //   dK  += dS^T(j) Q   once dS^T(j) is in shared memory
+      //   dQ^T(j) = K^T dS^T once the drain warps have read dQ^T(j-1)
+      // so that dP^T(j+1) runs while the dS warps still work on step j.
+      // S^T(j+1) overwrites the buffer of step j-1, whose P^T the dV MMA of
+      // step j-1 (issued earlier by this thread) and the dS warps (before
+      // their arrival on ds_ready(j-1)) have read.
       const uint32_t t_dp = tmem + Cfg::kColDP;
       const uint32_t t_dv = tmem + Cfg::kColDV, t_dk = tmem + Cfg::kColDK, t_dq = tmem + Cfg::kColDQ;
       int unit_iter = 0, step = 0;
-      uint32_t ds_cnt = 0, dq_cnt = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
-        const BwdUnit un = decode_bwd_unit(a, u);
-        if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->kv_full), unit_iter & 1, wc))) { ok = false; break; }
-        // dK, dV accumulators are free once the previous unit's epilogue read them
-        if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->acc_empty), (unit_iter & 1) ^ 1, wc))) { ok = false; break; }
-        tc_fence_after();
         const int buf = unit_iter & 1;
         if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
         StepIter it;
@@ -428,20 +469,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         int g, q0;
         bool pred;
         bool has = it.next(g, q0, pred);
+        if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->kv_full), unit_iter & 1, wc))) { ok = false; break; }
         int n_steps = 0;
-        if (has) {  // S^T and dP^T of the first step
+        if (has) {  // S^T and dP^T of the unit's first step
           const int s = step % Cfg::kStages, sb = step & 1;
           if (!ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step / Cfg::kStages) & 1, wc))) { ok = false; break; }
-          if (!ATTN25_TIMED(tr[8], mbar_wait_warp(smem_u32(&bars->s_free[sb]), ((step >> 1) & 1) ^ 1, wc))) { ok = false; break; }
           tc_fence_after();
           const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
-          if (lane == 0) {
-            issue_st<D>(tmem + Cfg::kColS + sb * BM, k_smem, st);
-            mma_commit(smem_u32(&bars->s_full[sb]));
-            issue_st<D>(t_dp, v_smem, st + Cfg::kQBytes);
-            mma_commit(smem_u32(&bars->dp_full));
-          }
-          __syncwarp();
+          issue_st<D>(tmem + Cfg::kColS + sb * BM, k_smem, st);
+          mma_commit_w(smem_u32(&bars->s_full[sb]));
+          issue_st<D>(t_dp, v_smem, st + Cfg::kQBytes);
+          mma_commit_w(smem_u32(&bars->dp_full));
         }
         while (has) {
           const int s = step % Cfg::kStages, sb = step & 1;  // stage and S^T buffer of this step
@@ -451,59 +489,60 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const bool has_n = it.next(g_n, q0_n, pred_n);
           const int s_n = (step + 1) % Cfg::kStages, sb_n = (step + 1) & 1;
           const uint32_t st_n = sbase + Cfg::kStageOff + s_n * Cfg::kStageBytes;
-          if (has_n) {  // S^T of the next step into the other buffer, ahead of this step's dS
+          if (has_n) {  // S^T of the next step into the other buffer
             if (!ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s_n]), ((step + 1) / Cfg::kStages) & 1, wc))) { ok = false; break; }
-            if (!ATTN25_TIMED(tr[8], mbar_wait_warp(smem_u32(&bars->s_free[sb_n]), (((step + 1) >> 1) & 1) ^ 1, wc))) { ok = false; break; }
             tc_fence_after();
-            if (lane == 0) {
-              issue_st<D>(tmem + Cfg::kColS + sb_n * BM, k_smem, st_n);
-              mma_commit(smem_u32(&bars->s_full[sb_n]));
-            }
-            __syncwarp();
+            BWD_EV(step + 1, 1);
+            issue_st<D>(tmem + Cfg::kColS + sb_n * BM, k_smem, st_n);
+            mma_commit_w(smem_u32(&bars->s_full[sb_n]));
           }
-          // dV += P^T dO once P^T is in tensor memory
+          // dV += P^T dO once P^T is in tensor memory (and, on the unit's first
+          // step, once the previous unit's epilogue has read the accumulators)
           if (!ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->p_ready[sb]), (step >> 1) & 1, wc))) { ok = false; break; }
+          if (n_steps == 0 &&
+              !ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->acc_empty), (unit_iter & 1) ^ 1, wc))) { ok = false; break; }
           tc_fence_after();
+          BWD_EV(step, 2);
           ATTN25_TRACE_ONLY(const long long t_i0 = clock64();)
-          if (lane == 0) {
 #pragma unroll
-            for (int kk = 0; kk < BM / 16; ++kk)
-              mma_ts(t_dv, tmem + Cfg::kColS + sb * BM + kk * 8,
+          for (int kk = 0; kk < BM / 16; ++kk)
+            mma_ts_w(t_dv, tmem + Cfg::kColS + sb * BM + kk * 8,
                      smem_desc_sw128(st + Cfg::kQBytes + kk * 2048, BM * 128, 1024), Cfg::kIdescAcc,
                      (n_steps > 0 || kk > 0) ? 1u : 0u);
-          }
-          __syncwarp();
           ATTN25_TRACE_ONLY(tr[9] += clock64() - t_i0;)
-          // dK += dS^T Q and dQ^T = K^T dS^T once dS^T is in shared memory
-          if (!ATTN25_TIMED(tr[5], mbar_wait_warp(smem_u32(&bars->ds_ready), ds_cnt & 1, wc))) { ok = false; break; }
-          const uint32_t ds_smem = sbase + Cfg::kDSOff + (ds_cnt & 1) * Cfg::kDSBytes;
-          ++ds_cnt;
-          // the dQ^T columns must have been drained by the previous step
-          if (!ATTN25_TIMED(tr[6], mbar_wait_warp(smem_u32(&bars->dq_empty), (dq_cnt & 1) ^ 1, wc))) { ok = false; break; }
+          BWD_EV(step, 3);
+          // dP^T of the next step once the dS warps have read this step's
+          if (has_n) {
+            if (!ATTN25_TIMED(tr[8], mbar_wait_warp(smem_u32(&bars->dp_empty), step & 1, wc))) { ok = false; break; }
+            tc_fence_after();
+            BWD_EV(step, 4);
+            issue_st<D>(t_dp, v_smem, st_n + Cfg::kQBytes);
+            mma_commit_w(smem_u32(&bars->dp_full));
+          }
+          // dK += dS^T Q once dS^T is in shared memory
+          if (!ATTN25_TIMED(tr[5], mbar_wait_warp(smem_u32(&bars->ds_ready), step & 1, wc))) { ok = false; break; }
+          const uint32_t ds_smem = sbase + Cfg::kDSOff + sb * Cfg::kDSBytes;
           tc_fence_after();
+          BWD_EV(step, 5);
           ATTN25_TRACE_ONLY(const long long t_i1 = clock64();)
-          if (lane == 0) {
 #pragma unroll
-            for (int kk = 0; kk < BM / 16; ++kk)
-              mma_ss(t_dk, smem_desc_sw128(ds_smem + kk * 32, 16, 1024),
+          for (int kk = 0; kk < BM / 16; ++kk)
+            mma_ss_w(t_dk, smem_desc_sw128(ds_smem + kk * 32, 16, 1024),
                      smem_desc_sw128(st + kk * 2048, BM * 128, 1024), Cfg::kIdescAcc,
                      (n_steps > 0 || kk > 0) ? 1u : 0u);
+          // dQ^T = K^T dS^T once the drain warps have read the previous dQ^T
+          if (!ATTN25_TIMED(tr[6], mbar_wait_warp(smem_u32(&bars->dq_empty), (step & 1) ^ 1, wc))) { ok = false; break; }
+          tc_fence_after();
+          BWD_EV(step, 6);
 #pragma unroll
-            for (int kk = 0; kk < TILE / 16; ++kk)
-              mma_ss(t_dq, smem_desc_sw128(k_smem + kk * 2048, TILE * 128, 1024),
+          for (int kk = 0; kk < TILE / 16; ++kk)
+            mma_ss_w(t_dq, smem_desc_sw128(k_smem + kk * 2048, TILE * 128, 1024),
                      smem_desc_sw128(ds_smem + kk * 2048, BM * 128, 1024), Cfg::kIdescDQ,
                      kk > 0 ? 1u : 0u);
-            mma_commit(smem_u32(&bars->dq_full));
-            mma_commit(smem_u32(&bars->q_empty[s]));
-            mma_commit(smem_u32(&bars->ds_empty[(ds_cnt - 1) & 1]));
-            if (has_n) {
-              issue_st<D>(t_dp, v_smem, st_n + Cfg::kQBytes);
-              mma_commit(smem_u32(&bars->dp_full));
-            }
-          }
-          __syncwarp();
+          mma_commit_w(smem_u32(&bars->dq_full));
+          mma_commit_w(smem_u32(&bars->q_empty[s]));
           ATTN25_TRACE_ONLY(tr[10] += clock64() - t_i1;)
-          ++dq_cnt;
+          BWD_EV(step, 7);
           ++n_steps;
           ++step;
           has = has_n;
@@ -512,18 +551,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           pred = pred_n;
         }
         if (!ok) break;
-        if (lane == 0) {
-          mma_commit(smem_u32(&bars->kv_empty));
-          mma_commit(smem_u32(&bars->acc_full));
-          mbar_arrive(smem_u32(&bars->list_empty[buf]));
-        }
+        mma_commit_w(smem_u32(&bars->kv_empty));
+        mma_commit_w(smem_u32(&bars->acc_full));
+        if (lane == 0) mbar_arrive(smem_u32(&bars->list_empty[buf]));
         __syncwarp();
       }
-      if (lane == 0) {
-        mma_commit(smem_u32(&bars->drain));
-        mbar_wait_thread(smem_u32(&bars->drain), 0, WaitCtl{a.wait_ns, smem_u32(&bars->never_set), a.status});
-      }
-      __syncwarp();
+      mma_commit_w(smem_u32(&bars->drain));
+      mbar_wait_warp(smem_u32(&bars->drain), 0, WaitCtl{a.wait_ns, smem_u32(&bars->never_set), a.status});
       ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start; tr[7] = step;)
       trace_flush(a.trace, 32, tr);
     }
@@ -552,8 +586,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t nl2_s = sbase + Cfg::kStageOff + s * Cfg::kStageBytes + 2 * Cfg::kQBytes;
         const uint32_t t_s = tmem + Cfg::kColS + sb * BM + lane_off;
         if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step / Cfg::kStages) & 1, wc))) { ok = false; break; }
+        // the statistics are read before S^T is ready, off the critical path
+        // (without the register split, the mods that need more registers read
+        // them where they are used)
+        float4 nl2v[BM / 4];
+        if constexpr (kSplitRegs) {
+#pragma unroll
+          for (int c4 = 0; c4 < BM / 4; ++c4) nl2v[c4] = lds128(nl2_s + c4 * 16);
+        }
         if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->s_full[sb]), (step >> 1) & 1, wc))) { ok = false; break; }
         tc_fence_after();
+        BWD_EV(step, 8);
         ATTN25_TRACE_ONLY(const long long t_p = clock64();)
         const int h = un.hk * a.G + g;
         float x[BM];
@@ -561,7 +604,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(t_s + 32, reinterpret_cast<uint32_t(&)[32]>(x[32]));
         tmem_wait_ld();
         ATTN25_TRACE_ONLY(const long long t_p1 = clock64(); tr[4] += t_p1 - t_p;)
-        probs_t<MOD>(x, a, h, static_cast<float>(q0 - kv), q0, qlo, qhi, pred, nl2_s);
+        probs_t<MOD, kSplitRegs>(x, a, h, static_cast<float>(q0 - kv), q0, qlo, qhi, pred, nl2v, nl2_s);
         // P^T (bf16 pairs) over the first 32 columns of this S^T buffer
         uint32_t pk[32];
 #pragma unroll
@@ -572,6 +615,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ATTN25_TRACE_ONLY(tr[6] += clock64() - t_p2;)
         tc_fence_before();
         mbar_arrive(smem_u32(&bars->p_ready[sb]));
+        BWD_EV(step, 9);
         ATTN25_TRACE_ONLY(tr[3] += clock64() - t_p;)
         ++n_steps;
         ++step;
@@ -597,7 +641,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
     const uint32_t t_dp = tmem + Cfg::kColDP + lane_off, t_dk = tmem + Cfg::kColDK + lane_off;
     int unit_iter = 0, step = 0;
-    uint32_t dp_cnt = 0, ds_cnt = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
       const BwdUnit un = decode_bwd_unit(a, u);
@@ -615,9 +658,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t t_p = tmem + Cfg::kColS + sb * BM + lane_off;
         if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step / Cfg::kStages) & 1, wc))) { ok = false; break; }
         if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->p_ready[sb]), (step >> 1) & 1, wc))) { ok = false; break; }
-        if (!ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->dp_full), dp_cnt & 1, wc))) { ok = false; break; }
-        ++dp_cnt;
+        if (!ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->dp_full), step & 1, wc))) { ok = false; break; }
         tc_fence_after();
+        BWD_EV(step, 10);
         ATTN25_TRACE_ONLY(const long long t_ds = clock64();)
         float dp[BM];
         uint32_t pb[32];
@@ -626,13 +669,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(t_p, pb);
         tmem_wait_ld();
         ATTN25_TRACE_ONLY(tr[3] += clock64() - t_ds;)
-        // P^T of this buffer has been read: the next-but-one S^T may overwrite it
+        // dP^T has been read: the next step's dP^T may overwrite it.  (P^T of
+        // this buffer is released through ds_ready below.)
         tc_fence_before();
-        mbar_arrive(smem_u32(&bars->s_free[sb]));
-        // the dS buffer is free once the MMAs of two steps ago completed
-        if (!ATTN25_TIMED(tr[5], mbar_wait_warp(smem_u32(&bars->ds_empty[ds_cnt & 1]), ((ds_cnt >> 1) & 1) ^ 1, wc))) { ok = false; break; }
-        uint8_t* ds_row = smem + Cfg::kDSOff + (ds_cnt & 1) * Cfg::kDSBytes + r * 128;
-        ++ds_cnt;
+        mbar_arrive(smem_u32(&bars->dp_empty));
+        BWD_EV(step, 11);
+        // the dS buffer is free once the drain warps have staged dQ of two steps ago through it
+        if (!ATTN25_TIMED(tr[5], mbar_wait_warp(smem_u32(&bars->ds_empty[sb]), ((step >> 1) & 1) ^ 1, wc))) { ok = false; break; }
+        uint8_t* ds_row = smem + Cfg::kDSOff + sb * Cfg::kDSBytes + r * 128;
         const float dq0 = static_cast<float>(q0 - kv);
         float cl2_inv = 0.f;
         if constexpr (MOD == MOD_SOFTCAP) cl2_inv = 1.f / (a.mod.softcap * LOG2E);
@@ -673,6 +717,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         fence_proxy_async_smem();
         mbar_arrive(smem_u32(&bars->ds_ready));
+        BWD_EV(step, 12);
         ATTN25_TRACE_ONLY(tr[6] += clock64() - t_ds;)
         ++n_steps;
         ++step;
@@ -694,14 +739,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else {
     if constexpr (kSplitRegs) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsDrain));
     // ------------------------------------------------------------ dQ drain (thread = head-dim lane)
-    // dQ^T leaves TMEM row by row (lane = head dim) and is added into the
-    // fp32 accumulator with coalesced reductions in L2 (32 lanes = 128 bytes).
-    const int w = warp - 8;      // TMEM lane quarter = 32-column block of D
+    // dQ^T leaves TMEM row by row (lane = head dim d), is staged in shared
+    // memory as [d][q] rows of 32 queries (128-byte swizzle), and is added
+    // into the fp32 accumulator [B*Hq][D][Sq_pad] by TMA bulk reductions
+    // performed in L2.  Queries 0-31 are staged in the step's dS buffer
+    // (free once dK and dQ^T of the step completed, i.e. at dq_full),
+    // queries 32-63 in a buffer of their own.
+    const int w = warp - 8;      // TMEM lane quarter = 32-row block of D
     const uint32_t lane_off = static_cast<uint32_t>(w * 32) << 16;
     const uint32_t t_dq = tmem + Cfg::kColDQ + lane_off;
     const bool active = w * 32 < D;
-    int unit_iter = 0;
-    uint32_t dq_cnt = 0;
+    int unit_iter = 0, step = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
       const BwdUnit un = decode_bwd_unit(a, u);
@@ -712,27 +760,62 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int g, q0;
       bool pred;
       while (it.next(g, q0, pred)) {
-        if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->dq_full), dq_cnt & 1, wc))) { ok = false; break; }
+        const int sb = step & 1;
+        if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->dq_full), step & 1, wc))) { ok = false; break; }
         tc_fence_after();
+        BWD_EV(step, 13);
         float v[BM];
         tmem_ld32(t_dq, reinterpret_cast<uint32_t(&)[32]>(v[0]));
         tmem_ld32(t_dq + 32, reinterpret_cast<uint32_t(&)[32]>(v[32]));
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(smem_u32(&bars->dq_empty));
+        BWD_EV(step, 14);
         ATTN25_TRACE_ONLY(const long long t_r = clock64();)
+#if ATTN25_DQ_RED
+        // dS buffer free already (dK and dQ^T of this step completed)
+        if (lane == 0) mbar_arrive(smem_u32(&bars->ds_empty[sb]));
         if (active) {
           const int bh = un.b * a.Hq + un.hk * a.G + g;
-          float* dst = a.dq_acc + (static_cast<size_t>(bh) * a.Sq_pad + q0) * D + w * 32 + lane;
+          float4* dst = reinterpret_cast<float4*>(a.dq_acc + (static_cast<size_t>(bh) * D + w * 32 + lane) * a.Sq_pad + q0);
 #pragma unroll
-          for (int c = 0; c < BM; ++c) atomicAdd(dst + static_cast<size_t>(c) * D, v[c]);
+          for (int k = 0; k < BM / 4; ++k) atomicAdd(dst + k, make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]));
         }
+#else
+        if (active) {
+          const uint32_t half0 = sbase + Cfg::kDSOff + sb * Cfg::kDSBytes + w * 4096;
+          const uint32_t half1 = sbase + Cfg::kDQStageOff + w * 4096;
+          const uint32_t row = static_cast<uint32_t>(lane) * 128;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t off = row + ((static_cast<uint32_t>(k) ^ (lane & 7)) << 4);
+            sts128(half0 + off, v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+            sts128(half1 + off, v[32 + 4 * k], v[32 + 4 * k + 1], v[32 + 4 * k + 2], v[32 + 4 * k + 3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int bh = un.b * a.Hq + un.hk * a.G + g;
+            tma_reduce_add_3d(&tm_dq, half0, q0, w * 32, bh);
+            tma_reduce_add_3d(&tm_dq, half1, q0 + 32, w * 32, bh);
+            bulk_commit();
+            // both staging buffers are read before the dS buffer is handed back
+            // and before the next step writes the second one
+            bulk_wait_read_all();
+          }
+          __syncwarp();
+        }
+        if (lane == 0) mbar_arrive(smem_u32(&bars->ds_empty[sb]));
+#endif
         ATTN25_TRACE_ONLY(tr[2] += clock64() - t_r;)
-        ++dq_cnt;
+        BWD_EV(step, 15);
+        ++step;
       }
       if (!ok) break;
       if (lane == 0) mbar_arrive(smem_u32(&bars->list_empty[buf]));
     }
+    // the reductions must have landed in global memory before the cast kernel runs
+    if (lane == 0) bulk_wait_all();
     ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
     trace_flush(a.trace, 16, tr);
   }
@@ -781,31 +864,37 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
   }
 }
 
-// dQ = scale * accumulator, rounded to bf16; 8 elements per thread.
+// dQ = scale * accumulator, rounded to bf16.  The accumulator is stored
+// [B*Hq][D][Sq_pad]; each block transposes 32 query rows x D through shared
+// memory and writes them [B*Hq][Sq][D].
 template <int D>
 __global__ void __launch_bounds__(256) bwd_dq_cast_kernel(const BwdArgs a) {
-  const long long n8 = static_cast<long long>(a.B) * a.Hq * a.Sq * (D / 8);
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long e = i * 8;
-    const long long row = e / D;
-    const int d = static_cast<int>(e - row * D);
-    const long long bh = row / a.Sq;
-    const int q = static_cast<int>(row - bh * a.Sq);
-    const float4* src = reinterpret_cast<const float4*>(a.dq_acc + (static_cast<size_t>(bh) * a.Sq_pad + q) * D + d);
-    const float4 x0 = src[0], x1 = src[1];
-    uint4 o;
-    o.x = pack_bf16x2(x0.x * a.scale, x0.y * a.scale);
-    o.y = pack_bf16x2(x0.z * a.scale, x0.w * a.scale);
-    o.z = pack_bf16x2(x1.x * a.scale, x1.y * a.scale);
-    o.w = pack_bf16x2(x1.z * a.scale, x1.w * a.scale);
-    *reinterpret_cast<uint4*>(a.dq + e) = o;
+  __shared__ float tile[D][33];
+  const int tiles_per_bh = a.Sq_pad / 32;
+  const long long n_tiles = static_cast<long long>(a.B) * a.Hq * tiles_per_bh;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (long long t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+    const long long bh = t / tiles_per_bh;
+    const int q0 = static_cast<int>(t - bh * tiles_per_bh) * 32;
+    const float* src = a.dq_acc + static_cast<size_t>(bh) * D * a.Sq_pad + q0 + tx;
+    for (int d = ty; d < D; d += 8) tile[d][tx] = src[static_cast<size_t>(d) * a.Sq_pad];
+    __syncthreads();
+    for (int qq = ty; qq < 32; qq += 8) {
+      const int q = q0 + qq;
+      if (q < a.Sq) {
+        __nv_bfloat16* dst = a.dq + (static_cast<size_t>(bh) * a.Sq + q) * D;
+        for (int d = 2 * tx; d < D; d += 64)
+          *reinterpret_cast<uint32_t*>(dst + d) = pack_bf16x2(tile[d][qq] * a.scale, tile[d + 1][qq] * a.scale);
+      }
+    }
+    __syncthreads();
   }
 }
 
 template <int D, int MOD>
 cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         const CUtensorMap& tdo, const BwdArgs& a, int grid, cudaStream_t stream) {
+                         const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int grid,
+                         cudaStream_t stream) {
   const long long rows = static_cast<long long>(a.B) * a.Hq * a.Sq_pad;
   int prep_blocks = static_cast<int>((rows * 32 + 255) / 256);
   if (prep_blocks > 148 * 16) prep_blocks = 148 * 16;
@@ -825,11 +914,11 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   if (launch_regs < kBwdLaunchRegs) return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg<D>::kAllocBytes);
   if (e != cudaSuccess) return e;
-  kernel<<<grid, kBwdThreads, BwdCfg<D>::kAllocBytes, stream>>>(tq, tk, tv, tdo, a);
+  kernel<<<grid, kBwdThreads, BwdCfg<D>::kAllocBytes, stream>>>(tq, tk, tv, tdo, tdq, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const long long n8 = static_cast<long long>(a.B) * a.Hq * a.Sq * (D / 8);
-  int cast_blocks = static_cast<int>((n8 + 255) / 256);
+  const long long cast_tiles = static_cast<long long>(a.B) * a.Hq * (a.Sq_pad / 32);
+  int cast_blocks = static_cast<int>(cast_tiles);
   if (cast_blocks > 148 * 16) cast_blocks = 148 * 16;
   bwd_dq_cast_kernel<D><<<cast_blocks, 256, 0, stream>>>(a);
   return cudaGetLastError();
@@ -837,16 +926,16 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 
 template <int D>
 cudaError_t launch_bwd_mod(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                           const CUtensorMap& tdo, const BwdArgs& a, int mod, int grid,
-                           cudaStream_t s) {
+                           const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int mod,
+                           int grid, cudaStream_t s) {
   switch (mod) {
-    case MOD_NONE: return launch_bwd_t<D, MOD_NONE>(tq, tk, tv, tdo, a, grid, s);
-    case MOD_CAUSAL: return launch_bwd_t<D, MOD_CAUSAL>(tq, tk, tv, tdo, a, grid, s);
-    case MOD_ALIBI: return launch_bwd_t<D, MOD_ALIBI>(tq, tk, tv, tdo, a, grid, s);
-    case MOD_SOFTCAP: return launch_bwd_t<D, MOD_SOFTCAP>(tq, tk, tv, tdo, a, grid, s);
-    case MOD_WINDOW: return launch_bwd_t<D, MOD_WINDOW>(tq, tk, tv, tdo, a, grid, s);
-    case MOD_BOOST: return launch_bwd_t<D, MOD_BOOST>(tq, tk, tv, tdo, a, grid, s);
-    case MOD_DOCUMENT: return launch_bwd_t<D, MOD_DOCUMENT>(tq, tk, tv, tdo, a, grid, s);
+    case MOD_NONE: return launch_bwd_t<D, MOD_NONE>(tq, tk, tv, tdo, tdq, a, grid, s);
+    case MOD_CAUSAL: return launch_bwd_t<D, MOD_CAUSAL>(tq, tk, tv, tdo, tdq, a, grid, s);
+    case MOD_ALIBI: return launch_bwd_t<D, MOD_ALIBI>(tq, tk, tv, tdo, tdq, a, grid, s);
+    case MOD_SOFTCAP: return launch_bwd_t<D, MOD_SOFTCAP>(tq, tk, tv, tdo, tdq, a, grid, s);
+    case MOD_WINDOW: return launch_bwd_t<D, MOD_WINDOW>(tq, tk, tv, tdo, tdq, a, grid, s);
+    case MOD_BOOST: return launch_bwd_t<D, MOD_BOOST>(tq, tk, tv, tdo, tdq, a, grid, s);
+    case MOD_DOCUMENT: return launch_bwd_t<D, MOD_DOCUMENT>(tq, tk, tv, tdo, tdq, a, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -854,10 +943,10 @@ cudaError_t launch_bwd_mod(const CUtensorMap& tq, const CUtensorMap& tk, const C
 }  // namespace
 
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const BwdArgs& a, int D, int mod, int grid,
-                       cudaStream_t stream) {
-  if (D == 128) return launch_bwd_mod<128>(tq, tk, tv, tdo, a, mod, grid, stream);
-  if (D == 64) return launch_bwd_mod<64>(tq, tk, tv, tdo, a, mod, grid, stream);
+                       const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int D, int mod,
+                       int grid, cudaStream_t stream) {
+  if (D == 128) return launch_bwd_mod<128>(tq, tk, tv, tdo, tdq, a, mod, grid, stream);
+  if (D == 64) return launch_bwd_mod<64>(tq, tk, tv, tdo, tdq, a, mod, grid, stream);
   return cudaErrorInvalidValue;
 }
 

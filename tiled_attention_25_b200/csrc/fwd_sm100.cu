@@ -4,7 +4,8 @@
 // 128-row query tiles).  Warp roles:
 //   warps 0-3  softmax for query tile 0 of the pair (thread = query row)
 //   warps 4-7  softmax for query tile 1
-//   warp  8    MMA issuer (one thread issues tcgen05.mma)
+//   warp  8    MMA issuer (the whole warp runs the issue code; one lane,
+//              chosen by elect.sync, issues each tcgen05.mma)
 //   warp  9    TMA producer
 // Scores S_t = Q_t K^T accumulate in tensor memory (TMEM), the softmax warps
 // read them with tcgen05.ld, write the bf16 probabilities P_t back over S_t,
@@ -100,8 +101,8 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint3
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t off = (kk >> 2) * (TILE * 128) + (kk & 3) * 32;
-    mma_ss(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024), smem_desc_sw128(k_smem + off, 16, 1024),
-           FwdCfg<D>::kIdescQK, kk > 0 ? 1u : 0u);
+    mma_ss_w(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024), smem_desc_sw128(k_smem + off, 16, 1024),
+             FwdCfg<D>::kIdescQK, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -110,8 +111,8 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
                                          bool accumulate) {
 #pragma unroll
   for (int kk = 0; kk < TILE / 16; ++kk) {
-    mma_ts(d_tmem, p_tmem + kk * 8, smem_desc_sw128(v_smem + kk * 2048, TILE * 128, 1024),
-           FwdCfg<D>::kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
+    mma_ts_w(d_tmem, p_tmem + kk * 8, smem_desc_sw128(v_smem + kk * 2048, TILE * 128, 1024),
+             FwdCfg<D>::kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -412,16 +413,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int slot_k = ring_pos % Cfg::kStages;
         if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->kv_full[slot_k]), (ring_pos / Cfg::kStages) & 1, wc))) { ok = false; break; }
         tc_fence_after();
-        if (lane == 0) {
 #pragma unroll
-          for (int t = 0; t < 2; ++t)
-            if (act[t]) {
-              issue_qk<D>(s_tmem[t], q_smem[t], ring + slot_k * Cfg::kTileBytes);
-              mma_commit(smem_u32(&bars->s_full[t]));
-            }
-          mma_commit(smem_u32(&bars->kv_empty[slot_k]));
-        }
-        __syncwarp();
+        for (int t = 0; t < 2; ++t)
+          if (act[t]) {
+            issue_qk<D>(s_tmem[t], q_smem[t], ring + slot_k * Cfg::kTileBytes);
+            mma_commit_w(smem_u32(&bars->s_full[t]));
+          }
+        mma_commit_w(smem_u32(&bars->kv_empty[slot_k]));
         ++ring_pos;
       }
       while (has && ok) {
@@ -445,11 +443,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (!ATTN25_TIMED(tr[4 + t], mbar_wait_warp(smem_u32(&bars->p_full[t]), p_cnt[t] & 1, wc))) { ok = false; break; }
             ++p_cnt[t];
             tc_fence_after();
-            if (lane == 0) {
-              issue_pv<D>(o_tmem[t], s_tmem[t], ring + slot_v * Cfg::kTileBytes, o_started[t]);
-              mma_commit(smem_u32(&bars->o_full[t]));
-            }
-            __syncwarp();
+            issue_pv<D>(o_tmem[t], s_tmem[t], ring + slot_v * Cfg::kTileBytes, o_started[t]);
+            mma_commit_w(smem_u32(&bars->o_full[t]));
             o_started[t] = true;
           }
           if (has_n) {
@@ -457,19 +452,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->kv_full[slot_kn]), ph_kn, wc))) { ok = false; break; }
               tc_fence_after();
             }
-            if (act_n[t] && lane == 0) {
+            if (act_n[t]) {
               issue_qk<D>(s_tmem[t], q_smem[t], ring + slot_kn * Cfg::kTileBytes);
-              mma_commit(smem_u32(&bars->s_full[t]));
+              mma_commit_w(smem_u32(&bars->s_full[t]));
             }
-            __syncwarp();
           }
         }
         if (!ok) break;
-        if (lane == 0) {
-          if (has_n) mma_commit(smem_u32(&bars->kv_empty[slot_kn]));
-          mma_commit(smem_u32(&bars->kv_empty[slot_v]));
-        }
-        __syncwarp();
+        if (has_n) mma_commit_w(smem_u32(&bars->kv_empty[slot_kn]));
+        mma_commit_w(smem_u32(&bars->kv_empty[slot_v]));
         if (has_n) ++ring_pos;
         has = has_n;
         ++j;
@@ -477,20 +468,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         act[1] = act_n[1];
       }
       if (!ok) break;
-      if (lane == 0) {
-        mma_commit(smem_u32(&bars->q_empty));
-        mma_commit(smem_u32(&bars->o_final[0]));
-        mma_commit(smem_u32(&bars->o_final[1]));
-        mbar_arrive(smem_u32(&bars->list_empty[buf]));
-      }
+      mma_commit_w(smem_u32(&bars->q_empty));
+      mma_commit_w(smem_u32(&bars->o_final[0]));
+      mma_commit_w(smem_u32(&bars->o_final[1]));
+      if (lane == 0) mbar_arrive(smem_u32(&bars->list_empty[buf]));
       __syncwarp();
     }
-    // drain: wait until every MMA this thread issued has completed
-    if (lane == 0) {
-      mma_commit(smem_u32(&bars->drain));
-      mbar_wait_thread(smem_u32(&bars->drain), 0, WaitCtl{a.wait_ns, smem_u32(&bars->never_set), a.status});
-    }
-    __syncwarp();
+    // drain: wait until every MMA this warp issued has completed
+    mma_commit_w(smem_u32(&bars->drain));
+    mbar_wait_warp(smem_u32(&bars->drain), 0, WaitCtl{a.wait_ns, smem_u32(&bars->never_set), a.status});
     ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
     trace_flush(a.trace, 32, tr);
   }

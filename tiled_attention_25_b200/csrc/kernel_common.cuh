@@ -186,12 +186,15 @@ __device__ __forceinline__ int build_pair_steps(const uint8_t* tile_class, int b
 }
 
 // Backward step source: the query tiles (and their class) a key tile meets.
-// Entry: query tile in bits 0-19, bit 20: the element predicate is needed.
-constexpr uint32_t kQtPred = 1u << 20;
+// Entries are 16 bits: the query-tile index, and bit 15 when the tile needs
+// the element predicate.
+constexpr uint32_t kQtPred16 = 1u << 15;
+constexpr uint32_t kQtIndexMask = kQtPred16 - 1;
+static_assert(kMaxSteps <= static_cast<int>(kQtIndexMask) + 1, "query-tile index width");
 
 __device__ __forceinline__ int build_kv_qtiles(const uint8_t* tile_class, int b, int kt, int nQ,
                                                int nK, int Sq, int Skv, int kind, int window,
-                                               uint32_t* list) {
+                                               uint16_t* list) {
   const int lane = threadIdx.x & 31;
   int q_begin = 0;
   if (tile_class == nullptr && is_interval_mask(kind)) q_begin = kt;  // every mask keeps q >= kv
@@ -213,7 +216,7 @@ __device__ __forceinline__ int build_kv_qtiles(const uint8_t* tile_class, int b,
     const uint32_t ballot = __ballot_sync(0xffffffffu, c != 0);
     if (c != 0) {
       const int pos = n + __popc(ballot & lanemask_lt());
-      if (pos < kMaxSteps) list[pos] = static_cast<uint32_t>(qt) | ((c == 1 || tail_kv) ? kQtPred : 0u);
+      if (pos < kMaxSteps) list[pos] = static_cast<uint16_t>(static_cast<uint32_t>(qt) | ((c == 1 || tail_kv) ? kQtPred16 : 0u));
     }
     n += __popc(ballot);
   }
