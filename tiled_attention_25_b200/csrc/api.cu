@@ -101,20 +101,6 @@ bool encode_bf16(CUtensorMap* m, const void* base, int inner, int rows, int oute
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// fp32 dQ accumulator [outer][rows][inner] (inner = padded query index) with
-// 32 x 32 boxes and 128-byte swizzle, the target of the backward's bulk reductions.
-bool encode_dq_acc(CUtensorMap* m, void* base, int inner, int rows, int outer) {
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
-                        static_cast<cuuint64_t>(outer)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * 4,
-                           static_cast<cuuint64_t>(inner) * rows * 4};
-  cuuint32_t box[3] = {32, 32, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -423,13 +409,12 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
   a.status = d->status;
   a.trace = d->trace == nullptr ? nullptr : d->trace + 128;
 
-  CUtensorMap tq, tk, tv, tdo, tdq;
+  CUtensorMap tq, tk, tv, tdo;
   if (!encode_bf16(&tq, q, D, Sq, B * Hq, 64) || !encode_bf16(&tk, k, D, Skv, B * Hkv, TILE) ||
-      !encode_bf16(&tv, v, D, Skv, B * Hkv, TILE) || !encode_bf16(&tdo, dout, D, Sq, B * Hq, 64) ||
-      !encode_dq_acc(&tdq, a.dq_acc, Sq_pad, D, B * Hq))
+      !encode_bf16(&tv, v, D, Skv, B * Hkv, TILE) || !encode_bf16(&tdo, dout, D, Sq, B * Hq, 64))
     return ATTN_ERR_ARG;
   const int grid = a.n_units < d->sms ? a.n_units : d->sms;
-  if (launch_bwd(tq, tk, tv, tdo, tdq, a, D, mod_kind, grid,
+  if (launch_bwd(tq, tk, tv, tdo, a, D, mod_kind, grid,
                  reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_LAUNCH;
   return ATTN_OK;

@@ -29,9 +29,6 @@
 #include "kernel_common.cuh"
 #include "launch.h"
 
-#ifndef ATTN25_DQ_RED
-#define ATTN25_DQ_RED 1
-#endif
 
 // Profiling builds: clock64 of event `id` of step `st` on CTA 0, written by
 // lane 0 of the first warp of each role, for a window of steps.
@@ -75,13 +72,7 @@ struct BwdCfg {
   static constexpr int kStageOff = 2 * kKVBytes;
   static constexpr int kDSOff = kStageOff + kStages * kStageBytes;  // two 128 x 64 bf16 buffers
   static constexpr int kDSBytes = TILE * BM * 2;
-  // staging of dQ^T queries 32-63 ([d][32 q] fp32, 128-byte swizzle); queries
-  // 0-31 are staged in the step's dS buffer
-  static constexpr int kDQStageOff = kDSOff + 2 * kDSBytes;
-  static constexpr int kDQStageBytes = D * 32 * 4;
-  static_assert(kDQStageBytes <= kDSBytes, "dQ staging half must fit a dS buffer");
-  static_assert(kDSOff % 1024 == 0 && kDQStageOff % 1024 == 0, "swizzled staging alignment");
-  static constexpr int kBarOff = kDQStageOff + kDQStageBytes;
+  static constexpr int kBarOff = kDSOff + 2 * kDSBytes;
   static constexpr int kListOff = kBarOff + 1024;  // two query-tile lists (16-bit entries)
   static constexpr int kSmemBytes = kListOff + 2 * kMaxSteps * 2;
   static constexpr int kAllocBytes = kSmemBytes + 1024;
@@ -111,7 +102,8 @@ struct BwdBarriers {
   int32_t list_n[2];   // lengths of the two query-tile lists
 };
 
-// Consumers of a query-tile list: the MMA warp and the P, dS and drain warps (lane 0 each).
+// Consumers of a query-tile list: the MMA warp and the P, dS and drain warps
+// (lane 0 each).
 constexpr int kBwdListConsumers = 13;
 constexpr int kDrainWarps = 4;
 
@@ -242,10 +234,6 @@ __device__ __forceinline__ float4 lds128(uint32_t addr) {
   return v;
 }
 
-__device__ __forceinline__ void sts128(uint32_t addr, float x, float y, float z, float w) {
-  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(x), "f"(y), "f"(z), "f"(w) : "memory");
-}
-
 // One key row of S^T (raw q.k for 64 queries) -> P^T = 2^(x - LSE2) in place.
 // The 64 negated base-2 LSEs come from registers (nl2v, PREFETCHED) or from
 // shared memory at nl2_addr.
@@ -325,7 +313,7 @@ template <int D, int MOD>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const __grid_constant__ CUtensorMap tm_dq, const BwdArgs a) {
+                    const BwdArgs a) {
   using Cfg = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -377,7 +365,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
   }
-  if (warp == 8 && lane == 0) tma_prefetch_desc(&tm_dq);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -455,25 +442,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       //   dQ^T(j) = K^T dS^T once the drain warps have read dQ^T(j-1)
       // so that dP^T(j+1) runs while the dS warps still work on step j.
       // S^T(j+1) overwrites the buffer of step j-1, whose P^T the dV MMA of
-      // step j-1 (issued earlier by this thread) and the dS warps (before
-      // their arrival on ds_ready(j-1)) have read.
+      // step j-1 (issued earlier by this warp) and the dS warps (before
+      // their arrival on ds_ready(j-1)) have read.  The whole warp runs the
+      // loop; one elected lane issues.
       const uint32_t t_dp = tmem + Cfg::kColDP;
       const uint32_t t_dv = tmem + Cfg::kColDV, t_dk = tmem + Cfg::kColDK, t_dq = tmem + Cfg::kColDQ;
       int unit_iter = 0, step = 0;
       bool ok = true;
+#define MMA_WAIT(wait_expr) \
+  {                         \
+    if (!(wait_expr)) {     \
+      ok = false;           \
+      break;                \
+    }                       \
+  }
       for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
         const int buf = unit_iter & 1;
-        if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+        MMA_WAIT(mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc) &&
+                 ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->kv_full), unit_iter & 1, wc)));
         StepIter it;
         it.init(lists + buf * kMaxSteps, bars->list_n[buf], a.G, a.Sq);
         int g, q0;
         bool pred;
         bool has = it.next(g, q0, pred);
-        if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->kv_full), unit_iter & 1, wc))) { ok = false; break; }
         int n_steps = 0;
         if (has) {  // S^T and dP^T of the unit's first step
           const int s = step % Cfg::kStages, sb = step & 1;
-          if (!ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step / Cfg::kStages) & 1, wc))) { ok = false; break; }
+          MMA_WAIT(ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step / Cfg::kStages) & 1, wc)));
           tc_fence_after();
           const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
           issue_st<D>(tmem + Cfg::kColS + sb * BM, k_smem, st);
@@ -490,7 +485,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const int s_n = (step + 1) % Cfg::kStages, sb_n = (step + 1) & 1;
           const uint32_t st_n = sbase + Cfg::kStageOff + s_n * Cfg::kStageBytes;
           if (has_n) {  // S^T of the next step into the other buffer
-            if (!ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s_n]), ((step + 1) / Cfg::kStages) & 1, wc))) { ok = false; break; }
+            MMA_WAIT(ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s_n]), ((step + 1) / Cfg::kStages) & 1, wc)));
             tc_fence_after();
             BWD_EV(step + 1, 1);
             issue_st<D>(tmem + Cfg::kColS + sb_n * BM, k_smem, st_n);
@@ -498,40 +493,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           // dV += P^T dO once P^T is in tensor memory (and, on the unit's first
           // step, once the previous unit's epilogue has read the accumulators)
-          if (!ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->p_ready[sb]), (step >> 1) & 1, wc))) { ok = false; break; }
-          if (n_steps == 0 &&
-              !ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->acc_empty), (unit_iter & 1) ^ 1, wc))) { ok = false; break; }
+          MMA_WAIT(ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->p_ready[sb]), (step >> 1) & 1, wc)) &&
+                   (n_steps > 0 ||
+                    ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->acc_empty), (unit_iter & 1) ^ 1, wc))));
           tc_fence_after();
           BWD_EV(step, 2);
-          ATTN25_TRACE_ONLY(const long long t_i0 = clock64();)
 #pragma unroll
           for (int kk = 0; kk < BM / 16; ++kk)
             mma_ts_w(t_dv, tmem + Cfg::kColS + sb * BM + kk * 8,
                      smem_desc_sw128(st + Cfg::kQBytes + kk * 2048, BM * 128, 1024), Cfg::kIdescAcc,
                      (n_steps > 0 || kk > 0) ? 1u : 0u);
-          ATTN25_TRACE_ONLY(tr[9] += clock64() - t_i0;)
           BWD_EV(step, 3);
           // dP^T of the next step once the dS warps have read this step's
           if (has_n) {
-            if (!ATTN25_TIMED(tr[8], mbar_wait_warp(smem_u32(&bars->dp_empty), step & 1, wc))) { ok = false; break; }
+            MMA_WAIT(ATTN25_TIMED(tr[8], mbar_wait_warp(smem_u32(&bars->dp_empty), step & 1, wc)));
             tc_fence_after();
             BWD_EV(step, 4);
             issue_st<D>(t_dp, v_smem, st_n + Cfg::kQBytes);
             mma_commit_w(smem_u32(&bars->dp_full));
           }
           // dK += dS^T Q once dS^T is in shared memory
-          if (!ATTN25_TIMED(tr[5], mbar_wait_warp(smem_u32(&bars->ds_ready), step & 1, wc))) { ok = false; break; }
           const uint32_t ds_smem = sbase + Cfg::kDSOff + sb * Cfg::kDSBytes;
+          MMA_WAIT(ATTN25_TIMED(tr[5], mbar_wait_warp(smem_u32(&bars->ds_ready), step & 1, wc)));
           tc_fence_after();
           BWD_EV(step, 5);
-          ATTN25_TRACE_ONLY(const long long t_i1 = clock64();)
 #pragma unroll
           for (int kk = 0; kk < BM / 16; ++kk)
             mma_ss_w(t_dk, smem_desc_sw128(ds_smem + kk * 32, 16, 1024),
                      smem_desc_sw128(st + kk * 2048, BM * 128, 1024), Cfg::kIdescAcc,
                      (n_steps > 0 || kk > 0) ? 1u : 0u);
           // dQ^T = K^T dS^T once the drain warps have read the previous dQ^T
-          if (!ATTN25_TIMED(tr[6], mbar_wait_warp(smem_u32(&bars->dq_empty), (step & 1) ^ 1, wc))) { ok = false; break; }
+          MMA_WAIT(ATTN25_TIMED(tr[6], mbar_wait_warp(smem_u32(&bars->dq_empty), (step & 1) ^ 1, wc)));
           tc_fence_after();
           BWD_EV(step, 6);
 #pragma unroll
@@ -541,7 +533,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                      kk > 0 ? 1u : 0u);
           mma_commit_w(smem_u32(&bars->dq_full));
           mma_commit_w(smem_u32(&bars->q_empty[s]));
-          ATTN25_TRACE_ONLY(tr[10] += clock64() - t_i1;)
           BWD_EV(step, 7);
           ++n_steps;
           ++step;
@@ -556,6 +547,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (lane == 0) mbar_arrive(smem_u32(&bars->list_empty[buf]));
         __syncwarp();
       }
+#undef MMA_WAIT
       mma_commit_w(smem_u32(&bars->drain));
       mbar_wait_warp(smem_u32(&bars->drain), 0, WaitCtl{a.wait_ns, smem_u32(&bars->never_set), a.status});
       ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start; tr[7] = step;)
@@ -739,12 +731,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else {
     if constexpr (kSplitRegs) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsDrain));
     // ------------------------------------------------------------ dQ drain (thread = head-dim lane)
-    // dQ^T leaves TMEM row by row (lane = head dim d), is staged in shared
-    // memory as [d][q] rows of 32 queries (128-byte swizzle), and is added
-    // into the fp32 accumulator [B*Hq][D][Sq_pad] by TMA bulk reductions
-    // performed in L2.  Queries 0-31 are staged in the step's dS buffer
-    // (free once dK and dQ^T of the step completed, i.e. at dq_full),
-    // queries 32-63 in a buffer of their own.
+    // dQ^T leaves TMEM row by row (lane = head dim d) and is added into the
+    // fp32 accumulator [B*Hq][Sq_pad][D] with reductions performed in L2: one
+    // instruction covers 32 consecutive d of one query row (128 bytes, one
+    // L1 wavefront).  (Four-wide reductions into a transposed accumulator
+    // need 32 wavefronts per instruction and starve the tensor core of
+    // shared-memory bandwidth; staging through shared memory for bulk
+    // reductions costs twice the wavefronts.)
     const int w = warp - 8;      // TMEM lane quarter = 32-row block of D
     const uint32_t lane_off = static_cast<uint32_t>(w * 32) << 16;
     const uint32_t t_dq = tmem + Cfg::kColDQ + lane_off;
@@ -772,41 +765,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_arrive(smem_u32(&bars->dq_empty));
         BWD_EV(step, 14);
         ATTN25_TRACE_ONLY(const long long t_r = clock64();)
-#if ATTN25_DQ_RED
-        // dS buffer free already (dK and dQ^T of this step completed)
+        // the dS buffer is free already (dK and dQ^T of this step completed)
         if (lane == 0) mbar_arrive(smem_u32(&bars->ds_empty[sb]));
         if (active) {
           const int bh = un.b * a.Hq + un.hk * a.G + g;
-          float4* dst = reinterpret_cast<float4*>(a.dq_acc + (static_cast<size_t>(bh) * D + w * 32 + lane) * a.Sq_pad + q0);
+          float* dst = a.dq_acc + (static_cast<size_t>(bh) * a.Sq_pad + q0) * D + w * 32 + lane;
 #pragma unroll
-          for (int k = 0; k < BM / 4; ++k) atomicAdd(dst + k, make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]));
+          for (int c = 0; c < BM; ++c) atomicAdd(dst + static_cast<size_t>(c) * D, v[c]);
         }
-#else
-        if (active) {
-          const uint32_t half0 = sbase + Cfg::kDSOff + sb * Cfg::kDSBytes + w * 4096;
-          const uint32_t half1 = sbase + Cfg::kDQStageOff + w * 4096;
-          const uint32_t row = static_cast<uint32_t>(lane) * 128;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint32_t off = row + ((static_cast<uint32_t>(k) ^ (lane & 7)) << 4);
-            sts128(half0 + off, v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-            sts128(half1 + off, v[32 + 4 * k], v[32 + 4 * k + 1], v[32 + 4 * k + 2], v[32 + 4 * k + 3]);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            const int bh = un.b * a.Hq + un.hk * a.G + g;
-            tma_reduce_add_3d(&tm_dq, half0, q0, w * 32, bh);
-            tma_reduce_add_3d(&tm_dq, half1, q0 + 32, w * 32, bh);
-            bulk_commit();
-            // both staging buffers are read before the dS buffer is handed back
-            // and before the next step writes the second one
-            bulk_wait_read_all();
-          }
-          __syncwarp();
-        }
-        if (lane == 0) mbar_arrive(smem_u32(&bars->ds_empty[sb]));
-#endif
         ATTN25_TRACE_ONLY(tr[2] += clock64() - t_r;)
         BWD_EV(step, 15);
         ++step;
@@ -814,8 +780,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ok) break;
       if (lane == 0) mbar_arrive(smem_u32(&bars->list_empty[buf]));
     }
-    // the reductions must have landed in global memory before the cast kernel runs
-    if (lane == 0) bulk_wait_all();
     ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
     trace_flush(a.trace, 16, tr);
   }
@@ -864,37 +828,31 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
   }
 }
 
-// dQ = scale * accumulator, rounded to bf16.  The accumulator is stored
-// [B*Hq][D][Sq_pad]; each block transposes 32 query rows x D through shared
-// memory and writes them [B*Hq][Sq][D].
+// dQ = scale * accumulator, rounded to bf16; 8 elements per thread.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_dq_cast_kernel(const BwdArgs a) {
-  __shared__ float tile[D][33];
-  const int tiles_per_bh = a.Sq_pad / 32;
-  const long long n_tiles = static_cast<long long>(a.B) * a.Hq * tiles_per_bh;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  for (long long t = blockIdx.x; t < n_tiles; t += gridDim.x) {
-    const long long bh = t / tiles_per_bh;
-    const int q0 = static_cast<int>(t - bh * tiles_per_bh) * 32;
-    const float* src = a.dq_acc + static_cast<size_t>(bh) * D * a.Sq_pad + q0 + tx;
-    for (int d = ty; d < D; d += 8) tile[d][tx] = src[static_cast<size_t>(d) * a.Sq_pad];
-    __syncthreads();
-    for (int qq = ty; qq < 32; qq += 8) {
-      const int q = q0 + qq;
-      if (q < a.Sq) {
-        __nv_bfloat16* dst = a.dq + (static_cast<size_t>(bh) * a.Sq + q) * D;
-        for (int d = 2 * tx; d < D; d += 64)
-          *reinterpret_cast<uint32_t*>(dst + d) = pack_bf16x2(tile[d][qq] * a.scale, tile[d + 1][qq] * a.scale);
-      }
-    }
-    __syncthreads();
+  const long long n8 = static_cast<long long>(a.B) * a.Hq * a.Sq * (D / 8);
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long e = i * 8;
+    const long long row = e / D;
+    const int d = static_cast<int>(e - row * D);
+    const long long bh = row / a.Sq;
+    const int q = static_cast<int>(row - bh * a.Sq);
+    const float4* src = reinterpret_cast<const float4*>(a.dq_acc + (static_cast<size_t>(bh) * a.Sq_pad + q) * D + d);
+    const float4 x0 = src[0], x1 = src[1];
+    uint4 o;
+    o.x = pack_bf16x2(x0.x * a.scale, x0.y * a.scale);
+    o.y = pack_bf16x2(x0.z * a.scale, x0.w * a.scale);
+    o.z = pack_bf16x2(x1.x * a.scale, x1.y * a.scale);
+    o.w = pack_bf16x2(x1.z * a.scale, x1.w * a.scale);
+    *reinterpret_cast<uint4*>(a.dq + e) = o;
   }
 }
 
 template <int D, int MOD>
 cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int grid,
-                         cudaStream_t stream) {
+                         const CUtensorMap& tdo, const BwdArgs& a, int grid, cudaStream_t stream) {
   const long long rows = static_cast<long long>(a.B) * a.Hq * a.Sq_pad;
   int prep_blocks = static_cast<int>((rows * 32 + 255) / 256);
   if (prep_blocks > 148 * 16) prep_blocks = 148 * 16;
@@ -914,11 +872,11 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   if (launch_regs < kBwdLaunchRegs) return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg<D>::kAllocBytes);
   if (e != cudaSuccess) return e;
-  kernel<<<grid, kBwdThreads, BwdCfg<D>::kAllocBytes, stream>>>(tq, tk, tv, tdo, tdq, a);
+  kernel<<<grid, kBwdThreads, BwdCfg<D>::kAllocBytes, stream>>>(tq, tk, tv, tdo, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const long long cast_tiles = static_cast<long long>(a.B) * a.Hq * (a.Sq_pad / 32);
-  int cast_blocks = static_cast<int>(cast_tiles);
+  const long long n8 = static_cast<long long>(a.B) * a.Hq * a.Sq * (D / 8);
+  int cast_blocks = static_cast<int>((n8 + 255) / 256);
   if (cast_blocks > 148 * 16) cast_blocks = 148 * 16;
   bwd_dq_cast_kernel<D><<<cast_blocks, 256, 0, stream>>>(a);
   return cudaGetLastError();
@@ -926,16 +884,15 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 
 template <int D>
 cudaError_t launch_bwd_mod(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                           const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int mod,
-                           int grid, cudaStream_t s) {
+                           const CUtensorMap& tdo, const BwdArgs& a, int mod, int grid, cudaStream_t s) {
   switch (mod) {
-    case MOD_NONE: return launch_bwd_t<D, MOD_NONE>(tq, tk, tv, tdo, tdq, a, grid, s);
-    case MOD_CAUSAL: return launch_bwd_t<D, MOD_CAUSAL>(tq, tk, tv, tdo, tdq, a, grid, s);
-    case MOD_ALIBI: return launch_bwd_t<D, MOD_ALIBI>(tq, tk, tv, tdo, tdq, a, grid, s);
-    case MOD_SOFTCAP: return launch_bwd_t<D, MOD_SOFTCAP>(tq, tk, tv, tdo, tdq, a, grid, s);
-    case MOD_WINDOW: return launch_bwd_t<D, MOD_WINDOW>(tq, tk, tv, tdo, tdq, a, grid, s);
-    case MOD_BOOST: return launch_bwd_t<D, MOD_BOOST>(tq, tk, tv, tdo, tdq, a, grid, s);
-    case MOD_DOCUMENT: return launch_bwd_t<D, MOD_DOCUMENT>(tq, tk, tv, tdo, tdq, a, grid, s);
+    case MOD_NONE: return launch_bwd_t<D, MOD_NONE>(tq, tk, tv, tdo, a, grid, s);
+    case MOD_CAUSAL: return launch_bwd_t<D, MOD_CAUSAL>(tq, tk, tv, tdo, a, grid, s);
+    case MOD_ALIBI: return launch_bwd_t<D, MOD_ALIBI>(tq, tk, tv, tdo, a, grid, s);
+    case MOD_SOFTCAP: return launch_bwd_t<D, MOD_SOFTCAP>(tq, tk, tv, tdo, a, grid, s);
+    case MOD_WINDOW: return launch_bwd_t<D, MOD_WINDOW>(tq, tk, tv, tdo, a, grid, s);
+    case MOD_BOOST: return launch_bwd_t<D, MOD_BOOST>(tq, tk, tv, tdo, a, grid, s);
+    case MOD_DOCUMENT: return launch_bwd_t<D, MOD_DOCUMENT>(tq, tk, tv, tdo, a, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -943,10 +900,10 @@ cudaError_t launch_bwd_mod(const CUtensorMap& tq, const CUtensorMap& tk, const C
 }  // namespace
 
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int D, int mod,
-                       int grid, cudaStream_t stream) {
-  if (D == 128) return launch_bwd_mod<128>(tq, tk, tv, tdo, tdq, a, mod, grid, stream);
-  if (D == 64) return launch_bwd_mod<64>(tq, tk, tv, tdo, tdq, a, mod, grid, stream);
+                       const CUtensorMap& tdo, const BwdArgs& a, int D, int mod, int grid,
+                       cudaStream_t stream) {
+  if (D == 128) return launch_bwd_mod<128>(tq, tk, tv, tdo, a, mod, grid, stream);
+  if (D == 64) return launch_bwd_mod<64>(tq, tk, tv, tdo, a, mod, grid, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -31,7 +31,7 @@ struct BwdArgs {
   const __nv_bfloat16* out;   // forward output O
   const __nv_bfloat16* dout;  // dO
   const float* lse;           // forward LSE (natural log)
-  float* dq_acc;              // [B*Hq][D][Sq_pad] fp32 (transposed)
+  float* dq_acc;              // [B*Hq][Sq_pad][D] fp32
   float* lse2;                // [B*Hq][Sq_pad]: -LSE * log2(e), -inf where the row keeps nothing
   float* delta;               // [B*Hq][Sq_pad]: -rowsum(dO * O)
   __nv_bfloat16* dq;
@@ -70,8 +70,8 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        const FwdArgs& a, int D, int mod, bool has_lse, int grid,
                        cudaStream_t stream);
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int D, int mod,
-                       int grid, cudaStream_t stream);
+                       const CUtensorMap& tdo, const BwdArgs& a, int D, int mod, int grid,
+                       cudaStream_t stream);
 cudaError_t launch_block_mask(const MaskArgs& a, cudaStream_t stream);
 
 // Register count ptxas gave the forward kernel (for the host's sanity checks).
