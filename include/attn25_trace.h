@@ -3,9 +3,10 @@
  * with -DATTN25_TRACE.  Its kernels time selected barrier waits and phases
  * per warp role with clock64 and add them into a device counter buffer
  * (256 x uint64: forward roles at 0..63, backward roles at 128..255, 16 per
- * role).  After the counters, 512 words hold the clock64 of 16 events in
- * each of 32 consecutive backward steps (steps 96..127 of CTA 0).  The normal
- * library (libattn25.so) does not export these.
+ * role; word 255 holds the first step of the event window).  After the
+ * counters, 512 words hold the clock64 of 16 events in each of 32
+ * consecutive backward steps of CTA 0.  The normal library (libattn25.so)
+ * does not export these.
  */
 #ifndef ATTN25_TRACE_H
 #define ATTN25_TRACE_H
@@ -21,6 +22,9 @@ ATTN25_API int attn_trace_read(unsigned long long* host_out, int n);
 
 /* Synchronise the device, then zero all counters. */
 ATTN25_API int attn_trace_reset(void);
+
+/* Set the first backward step of the event window (after attn_trace_reset). */
+ATTN25_API int attn_trace_window(int first_step);
 
 #ifdef __cplusplus
 }

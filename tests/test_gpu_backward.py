@@ -88,6 +88,17 @@ def test_unequal_lengths(ta, Sq, Skv):
         check_grads(got, c.oracle_bwd(), f"{Sq}x{Skv} mod {mod}")
 
 
+def test_key_tiles_without_queries(ta):
+    # causal with Skv >> Sq: key tiles past the first meet no query, and with
+    # more units than SMs a CTA runs several such units in a row
+    c = Case(34, 1, 32, 32, 128, 2048, 64, oracle.MOD_CAUSAL)
+    for use_mask in (False, True):
+        got = [host_f64(t) for t in run_fwd_bwd(ta, c, use_mask=use_mask)]
+        dk, dv = got[1], got[2]
+        assert not dk[:, :, 128:].any() and not dv[:, :, 128:].any()
+        check_grads(got, c.oracle_bwd(), f"mask={use_mask}")
+
+
 def test_gqa_mqa(ta):
     for Hq, Hkv in ((8, 2), (4, 1)):
         c = Case(32, 2, Hq, Hkv, 384, 384, 128, oracle.MOD_CAUSAL)

@@ -93,6 +93,19 @@ def test_fully_masked_rows_give_zero(ta):
     check_lse(got, L)
 
 
+def test_units_without_key_tiles(ta):
+    # window 16 with Sq >> Skv: every query-tile pair past the first keeps no
+    # key, and with more units than SMs a CTA runs several such units in a row
+    c = Case(13, 1, 32, 8, 2048, 128, 64, oracle.MOD_SLIDING_WINDOW, ModParams(window=16))
+    for use_mask in (False, True):
+        out, lse = run_fwd(ta, c, use_mask=use_mask)
+        O, L = c.oracle_fwd()
+        check_o(host_f64(out), O, f"mask={use_mask}")
+        got = lse.cpu().double().numpy()
+        assert np.isneginf(got[:, :, 143:]).all()
+        check_lse(got, L)
+
+
 def test_gqa_and_mqa(ta):
     for Hq, Hkv in ((8, 2), (4, 1)):
         c = Case(9, 2, Hq, Hkv, 384, 384, 128, oracle.MOD_CAUSAL)

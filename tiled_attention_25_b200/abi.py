@@ -97,6 +97,8 @@ def _load():
         lib.attn_trace_read.restype = I
         lib.attn_trace_reset.argtypes = []
         lib.attn_trace_reset.restype = I
+        lib.attn_trace_window.argtypes = [I]
+        lib.attn_trace_window.restype = I
     return lib
 
 
@@ -287,3 +289,8 @@ def attn_trace_read(n: int = 256) -> list:
 
 def attn_trace_reset():
     _check(LIB.attn_trace_reset(), "attn_trace_reset")
+
+
+def attn_trace_window(first_step: int):
+    """First backward step whose per-role event clocks the profiling build records."""
+    _check(LIB.attn_trace_window(first_step), "attn_trace_window")

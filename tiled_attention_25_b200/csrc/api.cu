@@ -460,6 +460,17 @@ ATTN25_API int attn_trace_reset(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_LAUNCH;
   return cudaMemset(d->trace, 0, kTraceWords * sizeof(unsigned long long)) == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
+
+ATTN25_API int attn_trace_window(int first_step) {
+  DeviceInfo* d = nullptr;
+  int rc = current_device(&d);
+  if (rc != ATTN_OK) return rc;
+  if (d->trace == nullptr || first_step < 0) return ATTN_ERR_ARG;
+  const unsigned long long v = static_cast<unsigned long long>(first_step);
+  return cudaMemcpy(d->trace + kTraceCounters - 1, &v, sizeof(v), cudaMemcpyHostToDevice) == cudaSuccess
+             ? ATTN_OK
+             : ATTN_ERR_LAUNCH;
+}
 #endif
 
 }  // extern "C"

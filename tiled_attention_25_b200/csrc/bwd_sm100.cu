@@ -33,11 +33,11 @@
 // Profiling builds: clock64 of event `id` of step `st` on CTA 0, written by
 // lane 0 of the first warp of each role, for a window of steps.
 #if defined(ATTN25_TRACE)
-#define BWD_EV(st, id)                                                                           \
-  do {                                                                                           \
-    if (blockIdx.x == 0 && lane == 0 && ((warp & 3) == 0 || warp >= 12) && (st) >= kEvStep0 &&  \
-        (st) < kEvStep0 + kEvSteps && a.trace != nullptr)                                        \
-      a.trace[kTraceCounters - 128 + ((st) - kEvStep0) * kEvPerStep + (id)] = clock64();          \
+#define BWD_EV(st, id)                                                                          \
+  do {                                                                                          \
+    if (blockIdx.x == 0 && lane == 0 && ((warp & 3) == 0 || warp >= 12) && (st) >= ev_step0 && \
+        (st) < ev_step0 + kEvSteps && a.trace != nullptr)                                       \
+      a.trace[kTraceCounters - 128 + ((st) - ev_step0) * kEvPerStep + (id)] = clock64();         \
   } while (0)
 #else
 #define BWD_EV(st, id) \
@@ -372,6 +372,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const WaitCtl wc{a.wait_ns, smem_u32(&bars->abort_flag), a.status};
   long long tr[12] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
   (void)tr;
+  // first step of the event window (profiling builds): the host stores it in
+  // the last backward counter word
+  ATTN25_TRACE_ONLY(const int ev_step0 = a.trace != nullptr ? static_cast<int>(a.trace[127]) : 0;)
   ATTN25_TRACE_ONLY(const long long t_start = clock64();)
 
   if (warp >= 12) {
@@ -542,6 +545,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           pred = pred_n;
         }
         if (!ok) break;
+        // a unit without steps still hands the accumulators over in turn: its
+        // (empty) dV/dK may only be announced once the previous unit's
+        // epilogue has read them, or acc_full would run a phase ahead
+        if (n_steps == 0)
+          MMA_WAIT(ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->acc_empty), (unit_iter & 1) ^ 1, wc)));
         mma_commit_w(smem_u32(&bars->kv_empty));
         mma_commit_w(smem_u32(&bars->acc_full));
         if (lane == 0) mbar_arrive(smem_u32(&bars->list_empty[buf]));

@@ -469,8 +469,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (!ok) break;
       mma_commit_w(smem_u32(&bars->q_empty));
-      mma_commit_w(smem_u32(&bars->o_final[0]));
-      mma_commit_w(smem_u32(&bars->o_final[1]));
+      // o_final counts units with at least one step only: the softmax warps
+      // wait for it on those units alone, so that units without key tiles
+      // cannot run its phases ahead of their epilogues
+      if (n_steps > 0) {
+        mma_commit_w(smem_u32(&bars->o_final[0]));
+        mma_commit_w(smem_u32(&bars->o_final[1]));
+      }
       if (lane == 0) mbar_arrive(smem_u32(&bars->list_empty[buf]));
       __syncwarp();
     }
@@ -490,6 +495,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t o_addr = tmem + 256 + t * D + lane_off;
     uint32_t s_cnt = 0, p_cnt = 0;
     int unit_iter = 0;
+    uint32_t o_units = 0;  // units with at least one step seen so far (o_final phases)
     bool ok = true;
     for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
       const UnitCoord uc = decode_unit(a, u);
@@ -570,7 +576,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (!ok) break;
       // ---- epilogue of this unit: O / l -> bf16, LSE
-      if (!ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->o_final[t]), unit_iter & 1, wc))) { ok = false; break; }
+      if (n_steps > 0) {
+        if (!ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->o_final[t]), o_units & 1, wc))) { ok = false; break; }
+        ++o_units;
+      }
       ATTN25_TRACE_ONLY(const long long t_epi = clock64();)
       tc_fence_after();
       const bool row_valid = rc.row < a.Sq;

@@ -31,10 +31,11 @@ constexpr int kErrTimeout = -6;
 #define ATTN25_TRACE_ONLY(x)
 #endif
 
-// Trace buffer of profiling builds: 256 per-role counters, then the event
-// clocks of a window of backward steps on CTA 0 (kEvSteps x kEvPerStep).
+// Trace buffer of profiling builds: 256 per-role counters (word 255 holds the
+// first step of the event window), then the event clocks of a window of
+// backward steps on CTA 0 (kEvSteps x kEvPerStep).
 constexpr int kTraceCounters = 256;
-constexpr int kEvStep0 = 96, kEvSteps = 32, kEvPerStep = 16;
+constexpr int kEvSteps = 32, kEvPerStep = 16;
 constexpr int kTraceWords = kTraceCounters + kEvSteps * kEvPerStep;
 
 // Add one warp's counters into the trace buffer (lane 0 only).
