@@ -52,14 +52,12 @@ namespace {
 constexpr int kBwdThreads = 512;
 constexpr int BM = 64;  // query rows per step
 // Warpgroups: 0 = P^T, 1 = dS^T, 2 = dQ drain, 3 = MMA (warp 12), TMA (warp 13).
-// Register split (setmaxnreg) of the 512 x 128 launch pool, per warpgroup.
-constexpr int kBwdLaunchRegs = 128;
-constexpr int kRegsP = 160;
-constexpr int kRegsDS = 152;
-constexpr int kRegsDrain = 96;
-constexpr int kRegsCtl = 104;
-static_assert(128 * (kRegsP + kRegsDS + kRegsDrain + kRegsCtl) <= kBwdThreads * kBwdLaunchRegs,
-              "register split");
+// No setmaxnreg split: every thread keeps the launch allocation (at most 128
+// registers at 512 threads).  Without the split, ptxas can keep the polling
+// loops of the waits out of line (one copy instead of one per wait site);
+// the smaller code was measured 49% faster on the dense 4x8x4096x128
+// workload (820 vs 550 TFLOP/s), the kernel being bound by instruction
+// fetch with four distinct warp roles.
 
 template <int D>
 struct BwdCfg {
@@ -234,13 +232,11 @@ __device__ __forceinline__ float4 lds128(uint32_t addr) {
   return v;
 }
 
-// One key row of S^T (raw q.k for 64 queries) -> P^T = 2^(x - LSE2) in place.
-// The 64 negated base-2 LSEs come from registers (nl2v, PREFETCHED) or from
-// shared memory at nl2_addr.
-template <int MOD, bool PREFETCHED>
+// One key row of S^T (raw q.k for 64 queries) -> P^T = 2^(x - LSE2) in place;
+// nl2_addr is the shared address of the 64 negated base-2 LSEs.
+template <int MOD>
 __device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h, float dq0, int q0,
-                                        int qlo, int qhi, bool pred, const float4 (&nl2v)[BM / 4],
-                                        uint32_t nl2_addr) {
+                                        int qlo, int qhi, bool pred, uint32_t nl2_addr) {
   float aux = 0.f, aux2 = 0.f;
   if constexpr (MOD == MOD_ALIBI) aux = alibi_slope(a.mod, h, a.Hq) * LOG2E;
   if constexpr (MOD == MOD_SOFTCAP) {
@@ -251,9 +247,7 @@ __device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h,
   const float2 sl2 = make_float2(a.sl2, a.sl2);
 #pragma unroll
   for (int c4 = 0; c4 < BM / 4; ++c4) {
-    float4 l;
-    if constexpr (PREFETCHED) l = nl2v[c4];
-    else l = lds128(nl2_addr + c4 * 16);
+    const float4 l = lds128(nl2_addr + c4 * 16);
 #pragma unroll
     for (int hp = 0; hp < 2; ++hp) {
       const int c = c4 * 4 + hp * 2;
@@ -325,7 +319,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint16_t* lists = reinterpret_cast<uint16_t*>(smem + Cfg::kListOff);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  constexpr bool kSplitRegs = MOD != MOD_SOFTCAP && MOD != MOD_BOOST;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -378,7 +371,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   ATTN25_TRACE_ONLY(const long long t_start = clock64();)
 
   if (warp >= 12) {
-    if constexpr (kSplitRegs) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
     if (warp == 13) {
       // ---------------------------------------------------------- TMA producer
       // all lanes build the query-tile lists; lane 0 issues the copies
@@ -389,13 +381,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const BwdUnit un = decode_bwd_unit(a, u);
         const int buf = unit_iter & 1;
         uint16_t* lst = lists + buf * kMaxSteps;
-        if (!mbar_wait_warp(smem_u32(&bars->list_empty[buf]), ((unit_iter >> 1) & 1) ^ 1, wc)) { ok = false; break; }
+        if (!mbar_wait_warp_ool(smem_u32(&bars->list_empty[buf]), ((unit_iter >> 1) & 1) ^ 1, wc)) { ok = false; break; }
         const int n = build_kv_qtiles(a.tile_class, un.b, un.kt, a.nQ, a.nK, a.Sq, a.Skv, MOD,
                                       a.mod.window, lst);
         if (lane == 0) bars->list_n[buf] = n;
         mbar_arrive(smem_u32(&bars->list_full[buf]));
         if (lane == 0) {
-          if (!ATTN25_TIMED(tr[1], mbar_wait_thread(smem_u32(&bars->kv_empty), (unit_iter & 1) ^ 1, wc))) {
+          if (!ATTN25_TIMED(tr[1], mbar_wait_thread_ool(smem_u32(&bars->kv_empty), (unit_iter & 1) ^ 1, wc))) {
             ok = false;
           } else {
             mbar_arrive_expect_tx(smem_u32(&bars->kv_full), 2 * Cfg::kKVBytes);
@@ -409,7 +401,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             bool pred;
             while (it.next(g, q0, pred)) {
               const int s = step % Cfg::kStages;
-              if (!ATTN25_TIMED(tr[2], mbar_wait_thread(smem_u32(&bars->q_empty[s]), ((step / Cfg::kStages) & 1) ^ 1, wc))) { ok = false; break; }
+              if (!ATTN25_TIMED(tr[2], mbar_wait_thread_ool(smem_u32(&bars->q_empty[s]), ((step / Cfg::kStages) & 1) ^ 1, wc))) { ok = false; break; }
               const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
               const uint32_t bar = smem_u32(&bars->q_full[s]);
               mbar_arrive_expect_tx(bar, 2 * Cfg::kQBytes + 2 * BM * 4);
@@ -429,9 +421,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       if (!ok && lane == 0) {
         const WaitCtl dwc{a.wait_ns, smem_u32(&bars->never_set), a.status};
-        if (kv_loads) mbar_wait_thread(smem_u32(&bars->kv_full), (kv_loads - 1) & 1, dwc);
+        if (kv_loads) mbar_wait_thread_ool(smem_u32(&bars->kv_full), (kv_loads - 1) & 1, dwc);
         for (int s = 0; s < Cfg::kStages; ++s)
-          if (stage_uses[s]) mbar_wait_thread(smem_u32(&bars->q_full[s]), (stage_uses[s] - 1) & 1, dwc);
+          if (stage_uses[s]) mbar_wait_thread_ool(smem_u32(&bars->q_full[s]), (stage_uses[s] - 1) & 1, dwc);
       }
       ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
       trace_flush(a.trace, 48, tr);
@@ -461,8 +453,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
       for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
         const int buf = unit_iter & 1;
-        MMA_WAIT(mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc) &&
-                 ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->kv_full), unit_iter & 1, wc)));
+        MMA_WAIT(mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc) &&
+                 ATTN25_TIMED(tr[1], mbar_wait_warp_ool(smem_u32(&bars->kv_full), unit_iter & 1, wc)));
         StepIter it;
         it.init(lists + buf * kMaxSteps, bars->list_n[buf], a.G, a.Sq);
         int g, q0;
@@ -471,7 +463,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         int n_steps = 0;
         if (has) {  // S^T and dP^T of the unit's first step
           const int s = step % Cfg::kStages, sb = step & 1;
-          MMA_WAIT(ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step / Cfg::kStages) & 1, wc)));
+          MMA_WAIT(ATTN25_TIMED(tr[3], mbar_wait_warp_ool(smem_u32(&bars->q_full[s]), (step / Cfg::kStages) & 1, wc)));
           tc_fence_after();
           const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
           issue_st<D>(tmem + Cfg::kColS + sb * BM, k_smem, st);
@@ -488,7 +480,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const int s_n = (step + 1) % Cfg::kStages, sb_n = (step + 1) & 1;
           const uint32_t st_n = sbase + Cfg::kStageOff + s_n * Cfg::kStageBytes;
           if (has_n) {  // S^T of the next step into the other buffer
-            MMA_WAIT(ATTN25_TIMED(tr[3], mbar_wait_warp(smem_u32(&bars->q_full[s_n]), ((step + 1) / Cfg::kStages) & 1, wc)));
+            MMA_WAIT(ATTN25_TIMED(tr[3], mbar_wait_warp_ool(smem_u32(&bars->q_full[s_n]), ((step + 1) / Cfg::kStages) & 1, wc)));
             tc_fence_after();
             BWD_EV(step + 1, 1);
             issue_st<D>(tmem + Cfg::kColS + sb_n * BM, k_smem, st_n);
@@ -496,9 +488,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           // dV += P^T dO once P^T is in tensor memory (and, on the unit's first
           // step, once the previous unit's epilogue has read the accumulators)
-          MMA_WAIT(ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->p_ready[sb]), (step >> 1) & 1, wc)) &&
+          MMA_WAIT(ATTN25_TIMED(tr[4], mbar_wait_warp_ool(smem_u32(&bars->p_ready[sb]), (step >> 1) & 1, wc)) &&
                    (n_steps > 0 ||
-                    ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->acc_empty), (unit_iter & 1) ^ 1, wc))));
+                    ATTN25_TIMED(tr[2], mbar_wait_warp_ool(smem_u32(&bars->acc_empty), (unit_iter & 1) ^ 1, wc))));
           tc_fence_after();
           BWD_EV(step, 2);
 #pragma unroll
@@ -509,7 +501,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           BWD_EV(step, 3);
           // dP^T of the next step once the dS warps have read this step's
           if (has_n) {
-            MMA_WAIT(ATTN25_TIMED(tr[8], mbar_wait_warp(smem_u32(&bars->dp_empty), step & 1, wc)));
+            MMA_WAIT(ATTN25_TIMED(tr[8], mbar_wait_warp_ool(smem_u32(&bars->dp_empty), step & 1, wc)));
             tc_fence_after();
             BWD_EV(step, 4);
             issue_st<D>(t_dp, v_smem, st_n + Cfg::kQBytes);
@@ -517,7 +509,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           // dK += dS^T Q once dS^T is in shared memory
           const uint32_t ds_smem = sbase + Cfg::kDSOff + sb * Cfg::kDSBytes;
-          MMA_WAIT(ATTN25_TIMED(tr[5], mbar_wait_warp(smem_u32(&bars->ds_ready), step & 1, wc)));
+          MMA_WAIT(ATTN25_TIMED(tr[5], mbar_wait_warp_ool(smem_u32(&bars->ds_ready), step & 1, wc)));
           tc_fence_after();
           BWD_EV(step, 5);
 #pragma unroll
@@ -526,7 +518,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                      smem_desc_sw128(st + kk * 2048, BM * 128, 1024), Cfg::kIdescAcc,
                      (n_steps > 0 || kk > 0) ? 1u : 0u);
           // dQ^T = K^T dS^T once the drain warps have read the previous dQ^T
-          MMA_WAIT(ATTN25_TIMED(tr[6], mbar_wait_warp(smem_u32(&bars->dq_empty), (step & 1) ^ 1, wc)));
+          MMA_WAIT(ATTN25_TIMED(tr[6], mbar_wait_warp_ool(smem_u32(&bars->dq_empty), (step & 1) ^ 1, wc)));
           tc_fence_after();
           BWD_EV(step, 6);
 #pragma unroll
@@ -549,7 +541,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // (empty) dV/dK may only be announced once the previous unit's
         // epilogue has read them, or acc_full would run a phase ahead
         if (n_steps == 0)
-          MMA_WAIT(ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->acc_empty), (unit_iter & 1) ^ 1, wc)));
+          MMA_WAIT(ATTN25_TIMED(tr[2], mbar_wait_warp_ool(smem_u32(&bars->acc_empty), (unit_iter & 1) ^ 1, wc)));
         mma_commit_w(smem_u32(&bars->kv_empty));
         mma_commit_w(smem_u32(&bars->acc_full));
         if (lane == 0) mbar_arrive(smem_u32(&bars->list_empty[buf]));
@@ -557,12 +549,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
 #undef MMA_WAIT
       mma_commit_w(smem_u32(&bars->drain));
-      mbar_wait_warp(smem_u32(&bars->drain), 0, WaitCtl{a.wait_ns, smem_u32(&bars->never_set), a.status});
+      mbar_wait_warp_ool(smem_u32(&bars->drain), 0, WaitCtl{a.wait_ns, smem_u32(&bars->never_set), a.status});
       ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start; tr[7] = step;)
       trace_flush(a.trace, 32, tr);
     }
   } else if (warp < 4) {
-    if constexpr (kSplitRegs) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsP));
     // ------------------------------------------------------------ P^T (thread = key row)
     const int r = threadIdx.x;  // TMEM lane = key row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
@@ -575,7 +566,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int qlo, qhi;
       key_interval<MOD>(a, un.b, kv, qlo, qhi);
       const int buf = unit_iter & 1;
-      if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+      if (!mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
       StepIter it;
       it.init(lists + buf * kMaxSteps, bars->list_n[buf], a.G, a.Sq);
       int g, q0;
@@ -585,16 +576,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int s = step % Cfg::kStages, sb = step & 1;
         const uint32_t nl2_s = sbase + Cfg::kStageOff + s * Cfg::kStageBytes + 2 * Cfg::kQBytes;
         const uint32_t t_s = tmem + Cfg::kColS + sb * BM + lane_off;
-        if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step / Cfg::kStages) & 1, wc))) { ok = false; break; }
-        // the statistics are read before S^T is ready, off the critical path
-        // (without the register split, the mods that need more registers read
-        // them where they are used)
-        float4 nl2v[BM / 4];
-        if constexpr (kSplitRegs) {
-#pragma unroll
-          for (int c4 = 0; c4 < BM / 4; ++c4) nl2v[c4] = lds128(nl2_s + c4 * 16);
-        }
-        if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->s_full[sb]), (step >> 1) & 1, wc))) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[1], mbar_wait_warp_ool(smem_u32(&bars->q_full[s]), (step / Cfg::kStages) & 1, wc))) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[2], mbar_wait_warp_ool(smem_u32(&bars->s_full[sb]), (step >> 1) & 1, wc))) { ok = false; break; }
         tc_fence_after();
         BWD_EV(step, 8);
         ATTN25_TRACE_ONLY(const long long t_p = clock64();)
@@ -604,7 +587,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(t_s + 32, reinterpret_cast<uint32_t(&)[32]>(x[32]));
         tmem_wait_ld();
         ATTN25_TRACE_ONLY(const long long t_p1 = clock64(); tr[4] += t_p1 - t_p;)
-        probs_t<MOD, kSplitRegs>(x, a, h, static_cast<float>(q0 - kv), q0, qlo, qhi, pred, nl2v, nl2_s);
+        probs_t<MOD>(x, a, h, static_cast<float>(q0 - kv), q0, qlo, qhi, pred, nl2_s);
         // P^T (bf16 pairs) over the first 32 columns of this S^T buffer
         uint32_t pk[32];
 #pragma unroll
@@ -622,7 +605,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       if (!ok) break;
       // ---- unit epilogue: dV -> bf16
-      if (!ATTN25_TIMED(tr[7], mbar_wait_warp(smem_u32(&bars->acc_full), unit_iter & 1, wc))) { ok = false; break; }
+      if (!ATTN25_TIMED(tr[7], mbar_wait_warp_ool(smem_u32(&bars->acc_full), unit_iter & 1, wc))) { ok = false; break; }
       tc_fence_after();
       ATTN25_TRACE_ONLY(const long long t_e = clock64();)
       store_acc_rows<D>(a.dv + ((static_cast<size_t>(un.b) * a.Hkv + un.hk) * a.Skv + kv) * D, t_dv, 1.f,
@@ -635,7 +618,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
     trace_flush(a.trace, 0, tr);
   } else if (warp < 8) {
-    if constexpr (kSplitRegs) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsDS));
     // ------------------------------------------------------------ dS^T (thread = key row)
     const int r = threadIdx.x - 128;
     const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
@@ -646,7 +628,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const BwdUnit un = decode_bwd_unit(a, u);
       const int kv = un.kt * TILE + r;
       const int buf = unit_iter & 1;
-      if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+      if (!mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
       StepIter it;
       it.init(lists + buf * kMaxSteps, bars->list_n[buf], a.G, a.Sq);
       int g, q0;
@@ -656,9 +638,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int s = step % Cfg::kStages, sb = step & 1;
         const uint32_t stats = sbase + Cfg::kStageOff + s * Cfg::kStageBytes + 2 * Cfg::kQBytes;
         const uint32_t t_p = tmem + Cfg::kColS + sb * BM + lane_off;
-        if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->q_full[s]), (step / Cfg::kStages) & 1, wc))) { ok = false; break; }
-        if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->p_ready[sb]), (step >> 1) & 1, wc))) { ok = false; break; }
-        if (!ATTN25_TIMED(tr[4], mbar_wait_warp(smem_u32(&bars->dp_full), step & 1, wc))) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[1], mbar_wait_warp_ool(smem_u32(&bars->q_full[s]), (step / Cfg::kStages) & 1, wc))) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[2], mbar_wait_warp_ool(smem_u32(&bars->p_ready[sb]), (step >> 1) & 1, wc))) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[4], mbar_wait_warp_ool(smem_u32(&bars->dp_full), step & 1, wc))) { ok = false; break; }
         tc_fence_after();
         BWD_EV(step, 10);
         ATTN25_TRACE_ONLY(const long long t_ds = clock64();)
@@ -675,7 +657,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_arrive(smem_u32(&bars->dp_empty));
         BWD_EV(step, 11);
         // the dS buffer is free once the drain warps have staged dQ of two steps ago through it
-        if (!ATTN25_TIMED(tr[5], mbar_wait_warp(smem_u32(&bars->ds_empty[sb]), ((step >> 1) & 1) ^ 1, wc))) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[5], mbar_wait_warp_ool(smem_u32(&bars->ds_empty[sb]), ((step >> 1) & 1) ^ 1, wc))) { ok = false; break; }
         uint8_t* ds_row = smem + Cfg::kDSOff + sb * Cfg::kDSBytes + r * 128;
         const float dq0 = static_cast<float>(q0 - kv);
         float cl2_inv = 0.f;
@@ -724,7 +706,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       if (!ok) break;
       // ---- unit epilogue: scale * dK -> bf16
-      if (!ATTN25_TIMED(tr[7], mbar_wait_warp(smem_u32(&bars->acc_full), unit_iter & 1, wc))) { ok = false; break; }
+      if (!ATTN25_TIMED(tr[7], mbar_wait_warp_ool(smem_u32(&bars->acc_full), unit_iter & 1, wc))) { ok = false; break; }
       tc_fence_after();
       ATTN25_TRACE_ONLY(const long long t_e = clock64();)
       store_acc_rows<D>(a.dk + ((static_cast<size_t>(un.b) * a.Hkv + un.hk) * a.Skv + kv) * D, t_dk, a.scale,
@@ -737,7 +719,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
     trace_flush(a.trace, 64, tr);
   } else {
-    if constexpr (kSplitRegs) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsDrain));
     // ------------------------------------------------------------ dQ drain (thread = head-dim lane)
     // dQ^T leaves TMEM row by row (lane = head dim d) and is added into the
     // fp32 accumulator [B*Hq][Sq_pad][D] with reductions performed in L2: one
@@ -755,14 +736,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
       const BwdUnit un = decode_bwd_unit(a, u);
       const int buf = unit_iter & 1;
-      if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+      if (!mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
       StepIter it;
       it.init(lists + buf * kMaxSteps, bars->list_n[buf], a.G, a.Sq);
       int g, q0;
       bool pred;
       while (it.next(g, q0, pred)) {
         const int sb = step & 1;
-        if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->dq_full), step & 1, wc))) { ok = false; break; }
+        if (!ATTN25_TIMED(tr[1], mbar_wait_warp_ool(smem_u32(&bars->dq_full), step & 1, wc))) { ok = false; break; }
         tc_fence_after();
         BWD_EV(step, 13);
         float v[BM];
@@ -868,16 +849,6 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   auto kernel = attn_bwd_kernel<D, MOD>;
-  // The register split assumes the kernel launches with kBwdLaunchRegs per
-  // thread; with fewer, setmaxnreg.inc could wait forever, so refuse.
-  static int launch_regs = -1;
-  if (launch_regs < 0) {
-    cudaFuncAttributes attr;
-    e = cudaFuncGetAttributes(&attr, kernel);
-    if (e != cudaSuccess) return e;
-    launch_regs = attr.numRegs;
-  }
-  if (launch_regs < kBwdLaunchRegs) return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg<D>::kAllocBytes);
   if (e != cudaSuccess) return e;
   kernel<<<grid, kBwdThreads, BwdCfg<D>::kAllocBytes, stream>>>(tq, tk, tv, tdo, a);

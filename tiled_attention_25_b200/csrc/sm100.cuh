@@ -150,6 +150,24 @@ static __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t par
   }
 }
 
+// Forms with the polling loop out of line (one check inline): kernels with
+// many wait sites and several distinct warp roles otherwise spend a large
+// part of their instruction-cache space on polling loops that rarely run.
+// ptxas cannot place these calls inside setmaxnreg register regions, so
+// only kernels without a register split use them.
+static __device__ __noinline__ bool mbar_wait_thread_loop(uint32_t bar, uint32_t parity, WaitCtl w) {
+  return mbar_wait_thread(bar, parity, w);
+}
+static __device__ __noinline__ bool mbar_wait_warp_loop(uint32_t bar, uint32_t parity, WaitCtl w) {
+  return mbar_wait_warp(bar, parity, w);
+}
+static __device__ __forceinline__ bool mbar_wait_thread_ool(uint32_t bar, uint32_t parity, WaitCtl w) {
+  return mbar_try_wait(bar, parity) || mbar_wait_thread_loop(bar, parity, w);
+}
+static __device__ __forceinline__ bool mbar_wait_warp_ool(uint32_t bar, uint32_t parity, WaitCtl w) {
+  return __all_sync(0xffffffffu, mbar_try_wait(bar, parity)) || mbar_wait_warp_loop(bar, parity, w);
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
