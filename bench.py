@@ -123,17 +123,25 @@ def kernel_source_hash(kernel):
 
 
 def measured_traffic(kernel, workload):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the kernel source as it is now (else None: the counters are stale)."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes per launch from the committed ncu summary (the table in
+    profiles/traffic.md), if it was taken on the kernel source as it is now
+    (else None: the counters are stale)."""
+    path = os.path.join(ROOT, "profiles", "traffic.md")
     try:
         with open(path) as f:
-            rec = json.load(f).get(kernel, {})
-    except (OSError, ValueError):
+            lines = f.read().splitlines()
+    except OSError:
         return None
-    if rec.get("workload") != workload or rec.get("source_sha256") != kernel_source_hash(kernel):
-        return None
-    return rec.get("dram_bytes_per_launch")
+    for line in lines:
+        cells = [c.strip().strip("`") for c in line.strip().strip("|").split("|")]
+        if len(cells) >= 4 and cells[0] == kernel and cells[1] == workload:
+            if cells[2] != kernel_source_hash(kernel):
+                return None
+            try:
+                return int(cells[3])
+            except ValueError:
+                return None
+    return None
 
 
 def useful_counts(ta, w, mod_name, params):
@@ -343,17 +351,20 @@ def run_reference(args, rank, world):
         return None
     w, mod_name = parse_workload(args.workload)
     params = mod_params_for(w, mod_name)
-    per_step = []
+    per_step, step_ms = [], []
     cb = None
     for _ in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
         cb = cpu_baseline(w, mod_name, params, heads=1)
+        step_ms.append((time.perf_counter() - t0) * 1e3)
         per_step.append(cb["value"])
     vals = per_step[args.warmup:]
     value = sum(vals) / len(vals)
+    ms = sum(step_ms[args.warmup:]) / args.steps
     cb["value"] = round(value, 6)
     return {
         "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
         "config": {"workload": f"{w.name}:{mod_name}", "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Sq": w.Sq,
                    "Skv": w.Skv, "D": w.D, "mod": mod_name, "seed": w.seed,
