@@ -89,9 +89,9 @@ struct BwdBarriers {
   uint64_t kv_full, kv_empty;
   uint64_t q_full[4], q_empty[4];
   uint64_t s_full[2], p_ready[2];
-  uint64_t dp_full, dp_empty, ds_ready;
+  uint64_t dp_full, dp_empty, ds_ready[2];
   uint64_t ds_empty[2];
-  uint64_t dq_full, dq_empty;
+  uint64_t dq_full;
   uint64_t acc_full, acc_empty;
   uint64_t drain;
   uint32_t tmem_base;
@@ -338,9 +338,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(smem_u32(&bars->dp_full), 1);
     mbar_init(smem_u32(&bars->dp_empty), 128);
-    mbar_init(smem_u32(&bars->ds_ready), 128);
+    // one slot per step parity: 128 dS threads (dS^T(j) stored) and 128 drain
+    // threads (dQ^T(j-1) read)
+    for (int b = 0; b < 2; ++b) mbar_init(smem_u32(&bars->ds_ready[b]), 256);
     mbar_init(smem_u32(&bars->dq_full), 1);
-    mbar_init(smem_u32(&bars->dq_empty), 128);
     mbar_init(smem_u32(&bars->acc_full), 1);
     mbar_init(smem_u32(&bars->acc_empty), 256);
     mbar_init(smem_u32(&bars->drain), 1);
@@ -429,12 +430,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       trace_flush(a.trace, 48, tr);
     } else if (warp == 12) {
       // ---------------------------------------------------------- MMA issuer
-      // Per step j (global step counter; S^T buffer j & 1, stage j % 3):
-      //   S^T(j+1)           once Q(j+1) has landed
-      //   dV  += P^T(j) dO   once P^T(j) is in TMEM
-      //   dP^T(j+1)          once the dS warps have read dP^T(j)
-      //   dK  += dS^T(j) Q   once dS^T(j) is in shared memory
-      //   dQ^T(j) = K^T dS^T once the drain warps have read dQ^T(j-1)
+      // Per step j (global step counter; S^T buffer j & 1, stage j % 3), four
+      // barrier waits:
+      //   q_full(j+1):  Q(j+1) has landed -> S^T(j+1) into the other buffer
+      //   p_ready(j):   P^T(j) is in TMEM -> dV += P^T(j) dO
+      //   dp_empty(j):  the dS warps have read dP^T(j) -> dP^T(j+1)
+      //   ds_ready(j):  dS^T(j) is in shared memory and the drain warps have
+      //                 read dQ^T(j-1) -> dK += dS^T Q, dQ^T(j) = K^T dS^T
       // so that dP^T(j+1) runs while the dS warps still work on step j.
       // S^T(j+1) overwrites the buffer of step j-1, whose P^T the dV MMA of
       // step j-1 (issued earlier by this warp) and the dS warps (before
@@ -507,9 +509,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             issue_st<D>(t_dp, v_smem, st_n + Cfg::kQBytes);
             mma_commit_w(smem_u32(&bars->dp_full));
           }
-          // dK += dS^T Q once dS^T is in shared memory
+          // dK += dS^T Q once dS^T is in shared memory; the same barrier slot also
+          // counts the drain warps' read of dQ^T(step - 1), so dQ^T(step) may follow
           const uint32_t ds_smem = sbase + Cfg::kDSOff + sb * Cfg::kDSBytes;
-          MMA_WAIT(ATTN25_TIMED(tr[5], mbar_wait_warp_ool(smem_u32(&bars->ds_ready), step & 1, wc)));
+          MMA_WAIT(ATTN25_TIMED(tr[5], mbar_wait_warp_ool(smem_u32(&bars->ds_ready[sb]), (step >> 1) & 1, wc)));
           tc_fence_after();
           BWD_EV(step, 5);
 #pragma unroll
@@ -517,9 +520,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mma_ss_w(t_dk, smem_desc_sw128(ds_smem + kk * 32, 16, 1024),
                      smem_desc_sw128(st + kk * 2048, BM * 128, 1024), Cfg::kIdescAcc,
                      (n_steps > 0 || kk > 0) ? 1u : 0u);
-          // dQ^T = K^T dS^T once the drain warps have read the previous dQ^T
-          MMA_WAIT(ATTN25_TIMED(tr[6], mbar_wait_warp_ool(smem_u32(&bars->dq_empty), (step & 1) ^ 1, wc)));
-          tc_fence_after();
           BWD_EV(step, 6);
 #pragma unroll
           for (int kk = 0; kk < TILE / 16; ++kk)
@@ -698,7 +698,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           *reinterpret_cast<uint4*>(ds_row + ((c16 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async_smem();
-        mbar_arrive(smem_u32(&bars->ds_ready));
+        mbar_arrive(smem_u32(&bars->ds_ready[sb]));
         BWD_EV(step, 12);
         ATTN25_TRACE_ONLY(tr[6] += clock64() - t_ds;)
         ++n_steps;
@@ -733,6 +733,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool active = w * 32 < D;
     int unit_iter = 0, step = 0;
     bool ok = true;
+    // ds_ready of step j counts the drain's read of dQ^T(j-1); step 0 has no
+    // predecessor, so its share is given up front
+    mbar_arrive(smem_u32(&bars->ds_ready[0]));
     for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
       const BwdUnit un = decode_bwd_unit(a, u);
       const int buf = unit_iter & 1;
@@ -751,7 +754,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(t_dq + 32, reinterpret_cast<uint32_t(&)[32]>(v[32]));
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(smem_u32(&bars->dq_empty));
+        // dQ^T(step) has been read: its columns may take dQ^T(step + 1), which the
+        // MMA warp issues after waiting for ds_ready of step + 1
+        mbar_arrive(smem_u32(&bars->ds_ready[(step + 1) & 1]));
         BWD_EV(step, 14);
         ATTN25_TRACE_ONLY(const long long t_r = clock64();)
         // the dS buffer is free already (dK and dQ^T of this step completed)
