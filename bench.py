@@ -107,6 +107,13 @@ def parse_workload(spec):
     return w, mod
 
 
+def rank_workload(w, rank):
+    """The replica rank `rank` processes: the same shapes as `w`, its own Q/K/V/dO
+    (seed offset by the rank), so N ranks run N independent problems."""
+    import dataclasses
+    return dataclasses.replace(w, seed=w.seed + rank)
+
+
 KERNEL_SOURCES = {
     "attn_fwd": ["fwd_sm100.cu", "kernel_common.cuh", "mods.cuh", "sm100.cuh", "exp2_poly.h", "launch.h"],
     "attn_bwd": ["bwd_sm100.cu", "kernel_common.cuh", "mods.cuh", "sm100.cuh", "launch.h"],
@@ -144,6 +151,25 @@ def measured_traffic(kernel, workload):
     return None
 
 
+def max_over_ranks(vals, world, device=None):
+    """Element-wise maximum of a list of floats over all ranks of the default
+    process group (identity on one rank).  Time-like quantities are reduced
+    this way: a multi-GPU step is as slow as its slowest rank."""
+    if world <= 1:
+        return list(vals)
+    import torch
+    t = torch.tensor(list(vals), dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(flop_per_rank, world, ms):
+    """Whole-job TFLOP/s: every rank processes its own replica of the workload
+    (weak scaling, no exchange), so the job's work is world x per-rank work,
+    done in the slowest rank's time."""
+    return flop_per_rank * world / (ms * 1e-3) / 1e12
+
+
 def useful_counts(ta, w, mod_name, params):
     mod = MOD_NAMES[mod_name]
     n = ta.useful_elements(mod, w.B, w.Hq, w.Sq, w.Skv, window=params.window, doc_offsets=params.doc_offsets)
@@ -160,8 +186,8 @@ def run_gpu(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     w, mod_name = parse_workload(args.workload)
     mod = MOD_NAMES[mod_name]
-    params = mod_params_for(w, mod_name)
-    bits = draw_workload(w)
+    params = mod_params_for(w, mod_name)   # same structure (and flops) on every rank
+    bits = draw_workload(rank_workload(w, rank))
     to_dev = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
     q, k, v, dout = (to_dev(bits[n]) for n in ("q", "k", "v", "dout"))
     doc_t = None
@@ -229,10 +255,7 @@ def run_gpu(args, rank, world, local_rank):
     ms_fwd = sum(t_fwd) / len(t_fwd)
     ms_bwd = sum(t_bwd) / len(t_bwd)
     ms_mask = sum(t_mask) / len(t_mask)
-    if world > 1:
-        tt = torch.tensor([ms_step, ms_fwd, ms_bwd, ms_mask], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms_step, ms_fwd, ms_bwd, ms_mask = tt.tolist()
+    ms_step, ms_fwd, ms_bwd, ms_mask = max_over_ranks([ms_step, ms_fwd, ms_bwd, ms_mask], world, dev)
 
     # end-to-end through the same API with pinned host buffers: H2D of the
     # step's inputs, the step, D2H of its results (O, dQ, dK, dV)
@@ -256,15 +279,11 @@ def run_gpu(args, rank, world, local_rank):
             e2e_times.append((a0, a1))
     torch.cuda.synchronize()
     ms_e2e = sum(a.elapsed_time(b) for a, b in e2e_times) / max(1, len(e2e_times))
-    if world > 1:
-        tt = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms_e2e = tt.item()
+    ms_e2e = max_over_ranks([ms_e2e], world, dev)[0]
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v, dout))
     d2h = sum(t.numel() * t.element_size() for t in (out, dq, dk, dv))
 
     n_u, f_fwd, f_bwd = useful_counts(ta, w, mod_name, params)
-    total = (f_fwd + f_bwd) * world
     peaks, peak_kind = load_peaks()
     peak = float(peaks["bf16_tflops"])
     fwd_tf = f_fwd / (ms_fwd * 1e-3) / 1e12
@@ -280,7 +299,7 @@ def run_gpu(args, rank, world, local_rank):
     traffic_bwd = measured_traffic("attn_bwd", wl)
     line = {
         "metric": METRIC,
-        "value": round(total / (ms_step * 1e-3) / 1e12, 2),
+        "value": round(job_throughput(f_fwd + f_bwd, world, ms_step), 2),
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
@@ -292,7 +311,7 @@ def run_gpu(args, rank, world, local_rank):
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V/dO, random-free mods)",
         "config": {"workload": f"{w.name}:{mod_name}", "B": B, "Hq": Hq, "Hkv": Hkv, "Sq": Sq, "Skv": Skv,
-                   "D": D, "mod": mod_name, "seed": w.seed, "step": "block mask + forward(O, LSE) + backward",
+                   "D": D, "mod": mod_name, "seed": w.seed, "seed_per_rank": "seed + rank (Q/K/V/dO)", "step": "block mask + forward(O, LSE) + backward",
                    "l2": "flushed before every step (256 MiB write, outside the timed events)",
                    "parallelism": f"independent replicas x{world} (no collective on the data path)"},
         "fwd_tflops": round(fwd_tf, 1),
@@ -307,7 +326,7 @@ def run_gpu(args, rank, world, local_rank):
                          kernel="attn_bwd (prep + main + dQ cast)" if dominant == "backward" else "attn_fwd"),
         "roofline_forward": roof(fwd_tf, traffic_fwd),
         "roofline_backward": roof(bwd_tf, traffic_bwd),
-        "e2e": None if args.no_e2e else {"value": round(total / (ms_e2e * 1e-3) / 1e12, 2), "unit": UNIT,
+        "e2e": None if args.no_e2e else {"value": round(job_throughput(f_fwd + f_bwd, world, ms_e2e), 2), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4)},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
