@@ -12,6 +12,12 @@ from .attention import (  # noqa: F401
     MOD_NONE,
     MOD_SLIDING_WINDOW,
     MOD_SOFTCAP,
+    MASK_CAUSAL,
+    MASK_DOCUMENT,
+    MASK_SLIDING_WINDOW,
+    has_document,
+    has_mask,
+    split_mod,
     alibi_slope,
     attention_backward,
     attention_forward,

@@ -32,7 +32,13 @@ Readings where the pages are silent (each also listed in the design doc):
   * local boost multiplies by ``boost`` where ``|q - kv| < radius``;
   * document mask keeps ``doc(q) == doc(kv) and kv <= q``;
   * GQA: query head ``h`` reads KV head ``h // (Hq // Hkv)``;
-  * a fully masked row has O = 0, LSE = -inf and zero gradient.
+  * a fully masked row has O = 0, LSE = -inf and zero gradient;
+  * composition (FlexAttention composes score and mask mods, "PyTorch
+    FlexAttention, FlashAttention-4 백엔드 …", 핵심 요약 and 섹션별 상세):
+    a mod code is one of the seven kinds, optionally ORed with mask flags
+    (``MASK_CAUSAL``, ``MASK_SLIDING_WINDOW``, ``MASK_DOCUMENT``).  The score
+    transform is the base kind's; an element is kept only where the base kind
+    and every flagged mask keep it (the logical AND of the masks).
 """
 from __future__ import annotations
 
@@ -45,6 +51,32 @@ MOD_SOFTCAP = 3
 MOD_SLIDING_WINDOW = 4
 MOD_LOCAL_BOOST = 5
 MOD_DOCUMENT = 6
+
+# Mask flags ORed onto a base kind to compose mods.
+MASK_CAUSAL = 0x100
+MASK_SLIDING_WINDOW = 0x200
+MASK_DOCUMENT = 0x400
+_FLAG_KIND = ((MASK_CAUSAL, MOD_CAUSAL), (MASK_SLIDING_WINDOW, MOD_SLIDING_WINDOW),
+              (MASK_DOCUMENT, MOD_DOCUMENT))
+
+
+def split_mod(mod):
+    """(base kind, [mask kinds of the flags]) of a mod code; rejects unknown bits."""
+    base, flags = int(mod) & 0xFF, int(mod) & ~0xFF
+    if base > MOD_DOCUMENT or flags & ~(MASK_CAUSAL | MASK_SLIDING_WINDOW | MASK_DOCUMENT):
+        raise ValueError(f"unknown mod {mod:#x}")
+    return base, [kind for flag, kind in _FLAG_KIND if flags & flag]
+
+
+def has_mask(mod) -> bool:
+    """True when the mod masks any element (some kind in it is a mask)."""
+    base, masks = split_mod(mod)
+    return bool(masks) or base in (MOD_CAUSAL, MOD_SLIDING_WINDOW, MOD_DOCUMENT)
+
+
+def has_document(mod) -> bool:
+    base, masks = split_mod(mod)
+    return base == MOD_DOCUMENT or MOD_DOCUMENT in masks
 
 
 def alibi_slope(h: int, Hq: int) -> float:
@@ -65,9 +97,20 @@ def score_mod(s, mod, params, b, h, Hq, qi, kj):
 
     s  : float64 [rows, cols] scaled scores scale * q.k
     qi : int64 [rows, 1] absolute query indices; kj : int64 [1, cols] key indices
+    mod: a kind, optionally ORed with mask flags (composition)
     Returns (s_mod, keep, dmod): the modded score, the keep mask and the
     derivative d s_mod / d s (used by the backward pass).
     """
+    base, masks = split_mod(mod)
+    s_mod, keep, dmod = _single_mod(s, base, params, b, h, Hq, qi, kj)
+    for kind in masks:
+        _, keep_m, _ = _single_mod(s, kind, params, b, h, Hq, qi, kj)
+        keep = keep & keep_m
+    return s_mod, keep, dmod
+
+
+def _single_mod(s, mod, params, b, h, Hq, qi, kj):
+    """One kind of the set: (modded score, keep mask, d s_mod / d s)."""
     keep = np.ones(np.broadcast_shapes(s.shape, qi.shape, kj.shape), dtype=bool)
     dmod = np.ones_like(s)
     s_mod = s
@@ -267,7 +310,7 @@ def useful_elements(mod, params, B, Hq, Sq, Skv) -> int:
     kj = np.arange(Skv, dtype=np.int64)[None, :]
     total = 0
     for b in range(B):
-        if mod in (MOD_CAUSAL, MOD_SLIDING_WINDOW, MOD_DOCUMENT):
+        if has_mask(mod):
             n = 0
             for r0 in range(0, Sq, 2048):
                 r = qi[r0:r0 + 2048]

@@ -26,7 +26,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .attention import MOD_CAUSAL, MOD_DOCUMENT, MOD_SLIDING_WINDOW, score_mod
+from .attention import has_mask, score_mod
 
 TILE = 128
 
@@ -35,7 +35,7 @@ def classify_tiles(mod, params, B, Sq, Skv, tile=TILE):
     nQ = -(-Sq // tile)
     nK = -(-Skv // tile)
     cls = np.full((B, nQ, nK), 2, dtype=np.uint8)
-    if mod not in (MOD_CAUSAL, MOD_SLIDING_WINDOW, MOD_DOCUMENT):
+    if not has_mask(mod):
         return cls
     kj = np.arange(Skv, dtype=np.int64)[None, :]
     for b in range(B):

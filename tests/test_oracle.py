@@ -25,7 +25,7 @@ ALL_MODS = [MOD_NONE, MOD_CAUSAL, MOD_ALIBI, MOD_SOFTCAP, MOD_SLIDING_WINDOW,
 
 def params_for(mod, S, window=5, radius=3, boost=1.1, softcap=2.0, docs=None):
     p = ModParams(softcap=softcap, window=window, boost=boost, boost_radius=radius)
-    if mod == MOD_DOCUMENT:
+    if oracle.has_document(mod):
         p.doc_offsets = docs if docs is not None else [[0, S // 3, S // 2 + 1, S]]
     return p
 

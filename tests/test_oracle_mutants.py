@@ -14,6 +14,7 @@ import oracle.attention as oa
 import oracle.block_sparsity as ob
 import test_oracle as pins
 import test_oracle_block_mask as bm_pins
+import test_oracle_compose as comp_pins
 
 
 def _install(module, func_name, old, new, monkeypatch):
@@ -33,14 +34,14 @@ MUTANTS = [
     # (module, function, original text, planted mistake, pin that must fail)
     (oa, "attention_forward", "s = scale * (q[b, h, r] @ k[b, hk].T)", "s = (q[b, h, r] @ k[b, hk].T)",
      lambda: pins.test_matches_torch_sdpa_float64(False)),
-    (oa, "score_mod", "s_mod = s - alibi_slope(h, Hq) * np.abs(qi - kj)", "s_mod = s + alibi_slope(h, Hq) * np.abs(qi - kj)",
+    (oa, "_single_mod", "s_mod = s - alibi_slope(h, Hq) * np.abs(qi - kj)", "s_mod = s + alibi_slope(h, Hq) * np.abs(qi - kj)",
      pins.test_zero_queries_alibi_geometric_sums),
     (oa, "alibi_slope", "(h + 1)", "h", pins.test_zero_queries_alibi_geometric_sums),
-    (oa, "score_mod", "keep = kj <= qi", "keep = kj < qi", pins.test_causal_first_query_attends_key0),
-    (oa, "score_mod", "keep = kj <= qi", "keep = kj >= qi", pins.test_causal_first_query_attends_key0),
-    (oa, "score_mod", "keep = (diff >= 0) & (diff < params.window)", "keep = (diff >= 0) & (diff <= params.window)",
+    (oa, "_single_mod", "keep = kj <= qi", "keep = kj < qi", pins.test_causal_first_query_attends_key0),
+    (oa, "_single_mod", "keep = kj <= qi", "keep = kj >= qi", pins.test_causal_first_query_attends_key0),
+    (oa, "_single_mod", "keep = (diff >= 0) & (diff < params.window)", "keep = (diff >= 0) & (diff <= params.window)",
      pins.test_window_one_attends_only_self),
-    (oa, "score_mod", "inside = np.abs(qi - kj) < params.boost_radius", "inside = np.abs(qi - kj) <= params.boost_radius",
+    (oa, "_single_mod", "inside = np.abs(qi - kj) < params.boost_radius", "inside = np.abs(qi - kj) <= params.boost_radius",
      lambda: pins.test_single_key_gives_v0(oa.MOD_LOCAL_BOOST)),
     (oa, "_kv_head", "return h // (Hq // Hkv)", "return h % Hkv", pins.test_gqa_equals_mha_with_repeated_kv),
     (oa, "_row_softmax", "e = np.exp(x - m_safe[:, None])", "e = np.exp(x)",
@@ -48,7 +49,7 @@ MUTANTS = [
     (oa, "_row_softmax", "m_safe + np.log(", "m_safe + np.log2(", pins.test_zero_queries_mean_of_values),
     (oa, "attention_backward", "dS = P * (dP - Di[:, None]) * dmod", "dS = P * dP * dmod",
      lambda: pins.test_gradients_match_central_differences(oa.MOD_NONE)),
-    (oa, "score_mod", "dmod = 1.0 - t * t", "dmod = 1.0 - t",
+    (oa, "_single_mod", "dmod = 1.0 - t * t", "dmod = 1.0 - t",
      lambda: pins.test_gradients_match_central_differences(oa.MOD_SOFTCAP)),
     (oa, "attention_backward", "dv_acc += P[:, kv_sel].T @ dout[b, h, r]", "dv_acc += P[:, kv_sel].T @ dout[b, hk, r]",
      pins.test_gqa_equals_mha_with_repeated_kv),
@@ -56,6 +57,12 @@ MUTANTS = [
      lambda: pins.test_gradients_match_central_differences(oa.MOD_NONE)),
     (oa, "online_forward", "l = l * alpha + p.sum(axis=1)", "l = l + p.sum(axis=1)",
      lambda: pins.test_online_softmax_matches_two_pass(oa.MOD_NONE)),
+    (oa, "score_mod", "keep = keep & keep_m", "keep = keep | keep_m",
+     lambda: comp_pins.test_composed_probs_are_restricted_softmax(oa.MOD_ALIBI | oa.MASK_CAUSAL)),
+    (oa, "score_mod", "for kind in masks:", "for kind in masks[:1]:",
+     comp_pins.test_zero_queries_window_and_documents_count_keys),
+    (oa, "score_mod", "_single_mod(s, base, params", "_single_mod(s, masks[0] if masks else base, params",
+     comp_pins.test_zero_queries_causal_alibi_geometric_sums),
     (ob, "classify_tiles", "elif n_keep == blk.size:", "elif n_keep == tile * tile:", bm_pins.test_single_row_tail_tile_is_full),
     (ob, "block_mask", "key=lambda u: (-pair_cost[u], u)", "key=lambda u: (pair_cost[u], u)", bm_pins.test_orders_are_lpt_permutations),
 ]
