@@ -82,21 +82,40 @@ typedef enum attn_mod_kind {
 } attn_mod_kind;
 
 /*
+ * Composition (FlexAttention composes score and mask mods, "PyTorch
+ * FlexAttention, …", 핵심 요약).  A mod_kind argument is one attn_mod_kind,
+ * optionally ORed with any of these flags: the score transform is the kind's
+ * (s' = s for the three mask kinds), and an element is kept only where the
+ * kind and every flagged mask keep it.  Examples:
+ *   ATTN_MOD_ALIBI | ATTN_MASK_CAUSAL          causal ALiBi
+ *   ATTN_MOD_SOFTCAP | ATTN_MASK_SLIDING_WINDOW  softcapped sliding window
+ *   ATTN_MOD_SLIDING_WINDOW | ATTN_MASK_DOCUMENT window inside each document
+ * Each component reads its own fields of attn_mod_params.  Unknown bits or
+ * kinds return ATTN_ERR_ARG.
+ */
+enum {
+  ATTN_MASK_CAUSAL = 0x100,
+  ATTN_MASK_SLIDING_WINDOW = 0x200,
+  ATTN_MASK_DOCUMENT = 0x400
+};
+
+/*
  * Runtime scalars of the mods; a change needs no recompilation (the page
  * notes that its JIT backend recompiles when such a scalar changes).
  * Fields that the chosen mod does not use are ignored.
  */
 typedef struct attn_mod_params {
   float softcap;               /* ATTN_MOD_SOFTCAP: c > 0 (e.g. 50) */
-  int32_t window;              /* ATTN_MOD_SLIDING_WINDOW: W >= 1 (e.g. 1024) */
+  int32_t window;              /* ATTN_MOD_SLIDING_WINDOW / ATTN_MASK_SLIDING_WINDOW: W >= 1 (e.g. 1024) */
   float boost;                 /* ATTN_MOD_LOCAL_BOOST: factor (e.g. 1.1) */
   int32_t boost_radius;        /* ATTN_MOD_LOCAL_BOOST: radius >= 0 (e.g. 128) */
-  const float* alibi_slopes;   /* ATTN_MOD_ALIBI: device fp32 [Hq], or NULL for 2^(-8 (h+1) / Hq) */
-  const int32_t* doc_offsets;  /* ATTN_MOD_DOCUMENT: device int32 [B][num_docs+1]: ascending document
+  const float* alibi_slopes;   /* ATTN_MOD_ALIBI: device fp32 [Hq] (4-byte aligned), or NULL for
+                                  2^(-8 (h+1) / Hq) */
+  const int32_t* doc_offsets;  /* ATTN_MOD_DOCUMENT / ATTN_MASK_DOCUMENT: device int32 (4-byte aligned) [B][num_docs+1]: ascending document
                                   starts, offsets[b][0] = 0, offsets[b][num_docs] = Skv; repeat the last
                                   value to pad rows with fewer documents.  Queries and keys share the
                                   offsets (packed self-attention, Sq == Skv required). */
-  int32_t num_docs;            /* ATTN_MOD_DOCUMENT: 1 <= num_docs <= 4096 */
+  int32_t num_docs;            /* ATTN_MOD_DOCUMENT / ATTN_MASK_DOCUMENT: 1 <= num_docs <= 4096 */
 } attn_mod_params;
 
 /*
@@ -120,7 +139,9 @@ typedef struct attn_block_mask {
   int32_t* fwd_order;
   int32_t* bwd_order;
   int32_t B, Sq, Skv, nq_tiles, nk_tiles;
-  int32_t mod_kind;            /* the mod it was built for; attn_fwd/attn_bwd check it */
+  int32_t mod_kind;            /* the mod it was built for, in canonical form (score kind |
+                                  ATTN_MASK_* flags, so equal for codes that mean the same mod);
+                                  attn_fwd/attn_bwd check it */
 } attn_block_mask;
 
 /*
@@ -131,7 +152,8 @@ typedef struct attn_block_mask {
  * block_mask: NULL for dense iteration (causal and sliding-window tiles are
  * then classified on the fly, document masks test every element), or a mask
  * built by build_block_mask for the same mod and sizes.
- * mod_params may be NULL only for ATTN_MOD_NONE / CAUSAL.
+ * mod_params may be NULL when no component reads it (none, causal, ALiBi with the
+ * default slopes).
  */
 ATTN25_API int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v,
              attn_bf16* out, float* lse,

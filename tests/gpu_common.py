@@ -35,7 +35,7 @@ class Case:
         self.q, self.k, self.v, self.dout = (to_dev(bits[n]) for n in ("q", "k", "v", "dout"))
         self.qf, self.kf, self.vf, self.doutf = (bf16_bits_to_f64(bits[n]) for n in ("q", "k", "v", "dout"))
         doc_t = None
-        if mod == oracle.MOD_DOCUMENT:
+        if oracle.has_document(mod):
             arr, _ = pad_offsets(self.p.doc_offsets)
             doc_t = torch.from_numpy(arr).cuda()
         self.dev_params = ta.ModParams(softcap=self.p.softcap, window=self.p.window, boost=self.p.boost,

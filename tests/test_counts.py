@@ -1,0 +1,31 @@
+"""The library's host-side useful-element counts (used for throughput) against
+the oracle's element-by-element count, for single and composed mods."""
+import pytest
+
+import oracle
+from oracle import (MASK_CAUSAL, MASK_DOCUMENT, MASK_SLIDING_WINDOW, MOD_ALIBI, MOD_CAUSAL,
+                    MOD_DOCUMENT, MOD_LOCAL_BOOST, MOD_NONE, MOD_SLIDING_WINDOW, MOD_SOFTCAP)
+from synth_inputs import ModParams
+
+MODS = [MOD_NONE, MOD_CAUSAL, MOD_ALIBI, MOD_SOFTCAP, MOD_SLIDING_WINDOW, MOD_LOCAL_BOOST,
+        MOD_DOCUMENT, MOD_ALIBI | MASK_CAUSAL, MOD_SOFTCAP | MASK_SLIDING_WINDOW,
+        MOD_LOCAL_BOOST | MASK_DOCUMENT, MOD_SLIDING_WINDOW | MASK_DOCUMENT,
+        MOD_NONE | MASK_CAUSAL | MASK_SLIDING_WINDOW | MASK_DOCUMENT]
+
+
+@pytest.mark.parametrize("mod", MODS)
+def test_counts_match_oracle(mod):
+    from tiled_attention_25_b200.counts import useful_elements
+    S = 700
+    docs = [[0, 130, 300, 301, 555, S], [0, S]]
+    p = ModParams(window=37, doc_offsets=docs)
+    assert useful_elements(mod, 2, 3, S, S, window=37, doc_offsets=docs) == \
+        oracle.useful_elements(mod, p, 2, 3, S, S)
+
+
+@pytest.mark.parametrize("Sq,Skv", [(300, 900), (900, 300)])
+def test_counts_unequal_lengths(Sq, Skv):
+    from tiled_attention_25_b200.counts import useful_elements
+    for mod in (MOD_CAUSAL, MOD_SLIDING_WINDOW, MOD_ALIBI | MASK_SLIDING_WINDOW):
+        assert useful_elements(mod, 1, 2, Sq, Skv, window=100) == \
+            oracle.useful_elements(mod, ModParams(window=100), 1, 2, Sq, Skv)

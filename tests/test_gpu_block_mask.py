@@ -18,7 +18,7 @@ def ta():
 
 def compare(ta, mod, p, B, Sq, Skv):
     doc_t = None
-    if mod == oracle.MOD_DOCUMENT:
+    if oracle.has_document(mod):
         doc_t = torch.from_numpy(pad_offsets(p.doc_offsets)[0]).cuda()
     dp = ta.ModParams(window=p.window, doc_offsets=doc_t)
     mask = ta.new_block_mask(mod, dp, B, Sq, Skv)
@@ -34,7 +34,7 @@ def compare(ta, mod, p, B, Sq, Skv):
 @pytest.mark.parametrize("mod", [oracle.MOD_NONE, oracle.MOD_CAUSAL, oracle.MOD_SLIDING_WINDOW, oracle.MOD_DOCUMENT])
 def test_block_mask_shapes(ta, S, mod):
     p = ModParams(window=max(1, S // 3))
-    if mod == oracle.MOD_DOCUMENT:
+    if oracle.has_document(mod):
         p.doc_offsets = [[0, S], sorted(set([0, S // 4, S // 4 + 1, S // 2, S]))]
     compare(ta, mod, p, 2, S, S)
 
@@ -56,6 +56,6 @@ def test_block_mask_single_token_documents(ta):
 def test_block_mask_workloads(ta, name, mod):
     w = WORKLOADS[name]
     p = ModParams()
-    if mod == oracle.MOD_DOCUMENT:
+    if oracle.has_document(mod):
         p.doc_offsets = doc_offsets_for(w)
     compare(ta, mod, p, w.B, w.Sq, w.Skv)

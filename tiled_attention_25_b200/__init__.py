@@ -13,6 +13,9 @@ from .abi import (  # noqa: F401
     EXPORTED,
     LIB,
     LIB_PATH,
+    MASK_CAUSAL,
+    MASK_DOCUMENT,
+    MASK_SLIDING_WINDOW,
     MOD_ALIBI,
     MOD_CAUSAL,
     MOD_DOCUMENT,

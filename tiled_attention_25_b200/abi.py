@@ -25,6 +25,11 @@ MOD_SOFTCAP = 3
 MOD_SLIDING_WINDOW = 4
 MOD_LOCAL_BOOST = 5
 MOD_DOCUMENT = 6
+# Mask flags ORed onto a kind to compose mods (score transform of the kind,
+# AND of the masks).
+MASK_CAUSAL = 0x100
+MASK_SLIDING_WINDOW = 0x200
+MASK_DOCUMENT = 0x400
 
 ATTN_ERR_TIMEOUT = -6
 

@@ -107,6 +107,40 @@ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 
 uint64_t wait_ns() { return static_cast<uint64_t>(g_wait_ms.load()) * 1000000ull; }
 
+// A mod code split into its score transform and mask bits (composition:
+// one of the seven kinds, optionally ORed with ATTN_MASK_* flags).
+struct ModSpec {
+  int score;      // MOD_NONE, MOD_ALIBI, MOD_SOFTCAP or MOD_BOOST
+  int mask;       // kMask* bits; window and document imply causal
+  int key;        // kernel specialisation key
+  int canonical;  // score | ATTN_MASK_* flags: equal for codes that mean the same mod
+};
+
+bool split_mod(int code, ModSpec& m) {
+  const int base = code & 0xFF, flags = code & ~0xFF;
+  if (base < ATTN_MOD_NONE || base > ATTN_MOD_DOCUMENT) return false;
+  if (flags & ~(ATTN_MASK_CAUSAL | ATTN_MASK_SLIDING_WINDOW | ATTN_MASK_DOCUMENT)) return false;
+  m.score = MOD_NONE;
+  m.mask = 0;
+  switch (base) {
+    case ATTN_MOD_CAUSAL: m.mask |= kMaskCausal; break;
+    case ATTN_MOD_ALIBI: m.score = MOD_ALIBI; break;
+    case ATTN_MOD_SOFTCAP: m.score = MOD_SOFTCAP; break;
+    case ATTN_MOD_SLIDING_WINDOW: m.mask |= kMaskCausal | kMaskWindow; break;
+    case ATTN_MOD_LOCAL_BOOST: m.score = MOD_BOOST; break;
+    case ATTN_MOD_DOCUMENT: m.mask |= kMaskCausal | kMaskDoc; break;
+    default: break;
+  }
+  if (flags & ATTN_MASK_CAUSAL) m.mask |= kMaskCausal;
+  if (flags & ATTN_MASK_SLIDING_WINDOW) m.mask |= kMaskCausal | kMaskWindow;
+  if (flags & ATTN_MASK_DOCUMENT) m.mask |= kMaskCausal | kMaskDoc;
+  m.key = m.score | (m.mask != 0 ? kKeyMasked : 0);
+  m.canonical = m.score | ((m.mask & kMaskCausal) ? ATTN_MASK_CAUSAL : 0) |
+                ((m.mask & kMaskWindow) ? ATTN_MASK_SLIDING_WINDOW : 0) |
+                ((m.mask & kMaskDoc) ? ATTN_MASK_DOCUMENT : 0);
+  return true;
+}
+
 // Shared validation of shapes, mod and mask.
 int check_common(int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale, int mod_kind,
                  const attn_mod_params* mp, const attn_block_mask* bm) {
@@ -119,31 +153,22 @@ int check_common(int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale, in
   if (static_cast<long long>(B) * Hq >= (1ll << 30)) return ATTN_ERR_UNSUPPORTED;
   // per-unit step lists live in shared memory: at most kMaxSteps tiles each way
   if (cdiv(Sq, TILE) > kMaxSteps || cdiv(Skv, TILE) > kMaxSteps) return ATTN_ERR_UNSUPPORTED;
-  if (mod_kind < ATTN_MOD_NONE || mod_kind > ATTN_MOD_DOCUMENT) return ATTN_ERR_ARG;
-  switch (mod_kind) {
-    case ATTN_MOD_SOFTCAP:
-      if (mp == nullptr || !(mp->softcap > 0.f) || !std::isfinite(mp->softcap)) return ATTN_ERR_ARG;
-      break;
-    case ATTN_MOD_SLIDING_WINDOW:
-      if (mp == nullptr || mp->window < 1) return ATTN_ERR_ARG;
-      break;
-    case ATTN_MOD_LOCAL_BOOST:
-      if (mp == nullptr || !std::isfinite(mp->boost) || mp->boost_radius < 0) return ATTN_ERR_ARG;
-      break;
-    case ATTN_MOD_DOCUMENT:
-      if (mp == nullptr || mp->doc_offsets == nullptr || mp->num_docs < 1 || mp->num_docs > 4096)
-        return ATTN_ERR_ARG;
-      if (Sq != Skv) return ATTN_ERR_UNSUPPORTED;
-      if (!aligned16(mp->doc_offsets) && (reinterpret_cast<uintptr_t>(mp->doc_offsets) & 3u))
-        return ATTN_ERR_ALIGN;
-      break;
-    case ATTN_MOD_ALIBI:
-      if (mp != nullptr && mp->alibi_slopes != nullptr &&
-          (reinterpret_cast<uintptr_t>(mp->alibi_slopes) & 3u))
-        return ATTN_ERR_ALIGN;
-      break;
-    default:
-      break;
+  ModSpec ms;
+  if (!split_mod(mod_kind, ms)) return ATTN_ERR_ARG;
+  if (ms.score == MOD_SOFTCAP &&
+      (mp == nullptr || !(mp->softcap > 0.f) || !std::isfinite(mp->softcap)))
+    return ATTN_ERR_ARG;
+  if (ms.score == MOD_BOOST && (mp == nullptr || !std::isfinite(mp->boost) || mp->boost_radius < 0))
+    return ATTN_ERR_ARG;
+  if (ms.score == MOD_ALIBI && mp != nullptr && mp->alibi_slopes != nullptr &&
+      (reinterpret_cast<uintptr_t>(mp->alibi_slopes) & 3u))
+    return ATTN_ERR_ALIGN;
+  if ((ms.mask & kMaskWindow) && (mp == nullptr || mp->window < 1)) return ATTN_ERR_ARG;
+  if (ms.mask & kMaskDoc) {
+    if (mp == nullptr || mp->doc_offsets == nullptr || mp->num_docs < 1 || mp->num_docs > 4096)
+      return ATTN_ERR_ARG;
+    if (Sq != Skv) return ATTN_ERR_UNSUPPORTED;
+    if (reinterpret_cast<uintptr_t>(mp->doc_offsets) & 3u) return ATTN_ERR_ALIGN;
   }
   if (bm != nullptr) {
     if (bm->tile_class == nullptr || bm->kv_count == nullptr || bm->kv_index == nullptr ||
@@ -151,26 +176,38 @@ int check_common(int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale, in
         bm->bwd_order == nullptr)
       return ATTN_ERR_ARG;
     if (bm->B != B || bm->Sq != Sq || bm->Skv != Skv || bm->nq_tiles != cdiv(Sq, TILE) ||
-        bm->nk_tiles != cdiv(Skv, TILE) || bm->mod_kind != mod_kind)
+        bm->nk_tiles != cdiv(Skv, TILE) || bm->mod_kind != ms.canonical)
       return ATTN_ERR_ARG;
   }
   return ATTN_OK;
 }
 
+// Device view of a validated mod code.
 ModDev make_mod(int mod_kind, const attn_mod_params* mp) {
+  ModSpec ms;
+  split_mod(mod_kind, ms);
   ModDev m{};
-  m.kind = mod_kind;
+  m.kind = ms.score;
+  m.mask = ms.mask;
+  m.window = 1 << 30;
   if (mp != nullptr) {
     m.softcap = mp->softcap;
-    m.window = mp->window;
     m.boost = mp->boost;
     m.boost_radius = mp->boost_radius;
     m.alibi_slopes = mp->alibi_slopes;
-    m.doc_offsets = mp->doc_offsets;
-    m.num_docs = mp->num_docs;
+    if (ms.mask & kMaskWindow) m.window = mp->window;
+    if (ms.mask & kMaskDoc) {
+      m.doc_offsets = mp->doc_offsets;
+      m.num_docs = mp->num_docs;
+    }
   }
-  if (mod_kind != ATTN_MOD_SLIDING_WINDOW) m.window = 1 << 30;
   return m;
+}
+
+int mod_key(int mod_kind) {
+  ModSpec ms;
+  split_mod(mod_kind, ms);
+  return ms.key;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -273,11 +310,14 @@ int build_block_mask(int mod_kind, const attn_mod_params* mod_params, int B, int
   DeviceInfo* d = nullptr;
   rc = current_device(&d);
   if (rc != ATTN_OK) return rc;
+  const ModDev md = make_mod(mod_kind, mod_params);
+  ModSpec ms;
+  split_mod(mod_kind, ms);
   MaskArgs a{};
-  a.kind = mod_kind;
-  a.window = (mod_kind == ATTN_MOD_SLIDING_WINDOW) ? mod_params->window : (1 << 30);
-  a.doc_offsets = (mod_kind == ATTN_MOD_DOCUMENT) ? mod_params->doc_offsets : nullptr;
-  a.num_docs = (mod_kind == ATTN_MOD_DOCUMENT) ? mod_params->num_docs : 0;
+  a.mask = md.mask;
+  a.window = md.window;
+  a.doc_offsets = md.doc_offsets;
+  a.num_docs = md.num_docs;
   a.B = B;
   a.Sq = Sq;
   a.Skv = Skv;
@@ -293,7 +333,7 @@ int build_block_mask(int mod_kind, const attn_mod_params* mod_params, int B, int
   a.bwd_order = mask->bwd_order;
   if (launch_block_mask(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_LAUNCH;
-  mask->mod_kind = mod_kind;
+  mask->mod_kind = ms.canonical;
   return ATTN_OK;
 }
 
@@ -342,7 +382,7 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
   a.status = d->status;
   a.trace = d->trace;
   const int grid = a.n_units < d->sms ? a.n_units : d->sms;
-  if (launch_fwd(tq, tk, tv, a, D, mod_kind, lse != nullptr, grid,
+  if (launch_fwd(tq, tk, tv, a, D, mod_key(mod_kind), lse != nullptr, grid,
                  reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_LAUNCH;
   return ATTN_OK;
@@ -414,7 +454,7 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
       !encode_bf16(&tv, v, D, Skv, B * Hkv, TILE) || !encode_bf16(&tdo, dout, D, Sq, B * Hq, 64))
     return ATTN_ERR_ARG;
   const int grid = a.n_units < d->sms ? a.n_units : d->sms;
-  if (launch_bwd(tq, tk, tv, tdo, a, D, mod_kind, grid,
+  if (launch_bwd(tq, tk, tv, tdo, a, D, mod_key(mod_kind), grid,
                  reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_LAUNCH;
   return ATTN_OK;

@@ -5,8 +5,8 @@
 // element predicate only on partial ones ("PyTorch FlexAttention,
 // FlashAttention-4 백엔드 …", 섹션별 상세: block-sparse iteration; "FlashInfer
 // SM120 NVFP4 어텐션 최적화", 코드 분석 4: masking only where the tile needs
-// it).  Every mask of the fixed set keeps an interval of keys [lo(i), hi(i)]
-// per query row, so the kept count of a tile row is a closed-form interval
+// it).  Every mask of the set, and every intersection of them, keeps an
+// interval of keys [lo(i), hi(i)] per query row, so the kept count of a tile row is a closed-form interval
 // length; summing it over the tile's rows counts kept elements exactly, which
 // is the same classification as testing every element.
 //
@@ -25,17 +25,10 @@ namespace {
 
 __device__ __forceinline__ void row_keep_interval(const MaskArgs& a, int b, int i, int& lo,
                                                   int& hi) {
-  lo = 0;
-  hi = a.Skv - 1;
-  if (a.kind == MOD_CAUSAL) {
-    hi = min(hi, i);
-  } else if (a.kind == MOD_WINDOW) {
-    hi = min(hi, i);
-    lo = max(0, i - a.window + 1);
-  } else if (a.kind == MOD_DOCUMENT) {
-    hi = min(hi, i);
-    lo = doc_start(a.doc_offsets + static_cast<size_t>(b) * (a.num_docs + 1), a.num_docs, i);
-  }
+  row_interval(a.mask, a.window,
+               a.doc_offsets == nullptr ? nullptr
+                                        : a.doc_offsets + static_cast<size_t>(b) * (a.num_docs + 1),
+               a.num_docs, i, a.Skv, lo, hi);
 }
 
 // grid (nQ, B): classify one query-tile row of tiles and write its KV list.

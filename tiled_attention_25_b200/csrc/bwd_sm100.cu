@@ -201,27 +201,27 @@ __device__ __forceinline__ void issue_st(uint32_t d_tmem, uint32_t a_smem, uint3
 
 
 // Kept query interval of key row kv (the transposed form of the row
-// intervals): causal [kv, Sq), window [kv, kv + W), document [kv, end of kv's
-// document); key rows past Skv keep nothing.
+// intervals, intersected over the masks): every mask keeps q >= kv; the
+// window keeps q < kv + W; the document keeps q before the end of kv's
+// document; key rows past Skv keep nothing.
 template <int MOD>
 __device__ __forceinline__ void key_interval(const BwdArgs& a, int b, int kv, int& qlo, int& qhi) {
   qlo = 0;
   qhi = a.Sq - 1;
-  if constexpr (MOD == MOD_CAUSAL) {
-    qlo = kv;
-  } else if constexpr (MOD == MOD_WINDOW) {
-    qlo = kv;
-    qhi = min(qhi, kv + a.mod.window - 1);
-  } else if constexpr (MOD == MOD_DOCUMENT) {
-    qlo = kv;
-    const int32_t* offs = a.mod.doc_offsets + static_cast<size_t>(b) * (a.mod.num_docs + 1);
-    const int kvc = min(kv, a.Skv - 1);
-    int lo = 0, hi = a.mod.num_docs;  // the document holding kvc, then its end
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (__ldg(offs + mid) <= kvc) lo = mid; else hi = mid;
+  if constexpr (masked(MOD)) {
+    const int mask = a.mod.mask;
+    if (mask & (kMaskCausal | kMaskWindow | kMaskDoc)) qlo = kv;
+    if (mask & kMaskWindow) qhi = min(qhi, kv + a.mod.window - 1);
+    if (mask & kMaskDoc) {
+      const int32_t* offs = a.mod.doc_offsets + static_cast<size_t>(b) * (a.mod.num_docs + 1);
+      const int kvc = min(kv, a.Skv - 1);
+      int lo = 0, hi = a.mod.num_docs;  // the document holding kvc, then its end
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(offs + mid) <= kvc) lo = mid; else hi = mid;
+      }
+      qhi = min(qhi, __ldg(offs + lo + 1) - 1);
     }
-    qhi = min(qhi, __ldg(offs + lo + 1) - 1);
   }
   if (kv >= a.Skv) qhi = qlo - 1;
 }
@@ -238,12 +238,12 @@ template <int MOD>
 __device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h, float dq0, int q0,
                                         int qlo, int qhi, bool pred, uint32_t nl2_addr) {
   float aux = 0.f, aux2 = 0.f;
-  if constexpr (MOD == MOD_ALIBI) aux = alibi_slope(a.mod, h, a.Hq) * LOG2E;
-  if constexpr (MOD == MOD_SOFTCAP) {
+  if constexpr (score_of(MOD) == MOD_ALIBI) aux = alibi_slope(a.mod, h, a.Hq) * LOG2E;
+  if constexpr (score_of(MOD) == MOD_SOFTCAP) {
     aux = a.scale / a.mod.softcap;
     aux2 = a.mod.softcap * LOG2E;
   }
-  if constexpr (MOD == MOD_BOOST) aux = a.mod.boost * a.sl2;
+  if constexpr (score_of(MOD) == MOD_BOOST) aux = a.mod.boost * a.sl2;
   const float2 sl2 = make_float2(a.sl2, a.sl2);
 #pragma unroll
   for (int c4 = 0; c4 < BM / 4; ++c4) {
@@ -253,13 +253,13 @@ __device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h,
       const int c = c4 * 4 + hp * 2;
       const float2 nl = hp == 0 ? make_float2(l.x, l.y) : make_float2(l.z, l.w);
       float2 v;
-      if constexpr (MOD == MOD_ALIBI) {
+      if constexpr (score_of(MOD) == MOD_ALIBI) {
         v.x = fmaf(x[c], a.sl2, -aux * fabsf(dq0 + static_cast<float>(c))) + nl.x;
         v.y = fmaf(x[c + 1], a.sl2, -aux * fabsf(dq0 + static_cast<float>(c + 1))) + nl.y;
-      } else if constexpr (MOD == MOD_SOFTCAP) {
+      } else if constexpr (score_of(MOD) == MOD_SOFTCAP) {
         v.x = fmaf(aux2, tanhf(x[c] * aux), nl.x);
         v.y = fmaf(aux2, tanhf(x[c + 1] * aux), nl.y);
-      } else if constexpr (MOD == MOD_BOOST) {
+      } else if constexpr (score_of(MOD) == MOD_BOOST) {
         const float r = static_cast<float>(a.mod.boost_radius);
         v.x = fmaf(x[c], fabsf(dq0 + static_cast<float>(c)) < r ? aux : a.sl2, nl.x);
         v.y = fmaf(x[c + 1], fabsf(dq0 + static_cast<float>(c + 1)) < r ? aux : a.sl2, nl.y);
@@ -383,7 +383,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int buf = unit_iter & 1;
         uint16_t* lst = lists + buf * kMaxSteps;
         if (!mbar_wait_warp_ool(smem_u32(&bars->list_empty[buf]), ((unit_iter >> 1) & 1) ^ 1, wc)) { ok = false; break; }
-        const int n = build_kv_qtiles(a.tile_class, un.b, un.kt, a.nQ, a.nK, a.Sq, a.Skv, MOD,
+        const int n = build_kv_qtiles(a.tile_class, un.b, un.kt, a.nQ, a.nK, a.Sq, a.Skv, a.mod.mask,
                                       a.mod.window, lst);
         if (lane == 0) bars->list_n[buf] = n;
         mbar_arrive(smem_u32(&bars->list_full[buf]));
@@ -661,13 +661,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint8_t* ds_row = smem + Cfg::kDSOff + sb * Cfg::kDSBytes + r * 128;
         const float dq0 = static_cast<float>(q0 - kv);
         float cl2_inv = 0.f;
-        if constexpr (MOD == MOD_SOFTCAP) cl2_inv = 1.f / (a.mod.softcap * LOG2E);
+        if constexpr (score_of(MOD) == MOD_SOFTCAP) cl2_inv = 1.f / (a.mod.softcap * LOG2E);
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16) {  // 8 columns (16 bytes) at a time
           const float4 nd0 = lds128(stats + 512 + c16 * 32), nd1 = lds128(stats + 512 + c16 * 32 + 16);
           const float nd[8] = {nd0.x, nd0.y, nd0.z, nd0.w, nd1.x, nd1.y, nd1.z, nd1.w};
           float4 nl0, nl1;
-          if constexpr (MOD == MOD_SOFTCAP) {
+          if constexpr (score_of(MOD) == MOD_SOFTCAP) {
             nl0 = lds128(stats + c16 * 32);
             nl1 = lds128(stats + c16 * 32 + 16);
           }
@@ -679,7 +679,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const float2 pr = make_float2(__uint_as_float(pp << 16), __uint_as_float(pp & 0xffff0000u));
             // dS = P (dP - Delta)
             float2 d = __fmul2_rn(pr, __fadd2_rn(make_float2(dp[c], dp[c + 1]), make_float2(nd[2 * e], nd[2 * e + 1])));
-            if constexpr (MOD == MOD_SOFTCAP) {
+            if constexpr (score_of(MOD) == MOD_SOFTCAP) {
               // d s'/d s = 1 - tanh^2 with tanh = (log2 P + LSE2) / (c log2 e)
               const float nlx = (e < 2) ? (e == 0 ? nl0.x : nl0.z) : (e == 2 ? nl1.x : nl1.z);
               const float nly = (e < 2) ? (e == 0 ? nl0.y : nl0.w) : (e == 2 ? nl1.y : nl1.w);
@@ -687,7 +687,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               const float t1 = (__log2f(pr.y) - nly) * cl2_inv;
               d.x = pr.x > 0.f ? d.x * (1.f - t0 * t0) : 0.f;
               d.y = pr.y > 0.f ? d.y * (1.f - t1 * t1) : 0.f;
-            } else if constexpr (MOD == MOD_BOOST) {
+            } else if constexpr (score_of(MOD) == MOD_BOOST) {
               const float rad = static_cast<float>(a.mod.boost_radius);
               d.x *= fabsf(dq0 + static_cast<float>(c)) < rad ? a.mod.boost : 1.f;
               d.y *= fabsf(dq0 + static_cast<float>(c + 1)) < rad ? a.mod.boost : 1.f;
@@ -868,15 +868,17 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 
 template <int D>
 cudaError_t launch_bwd_mod(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                           const CUtensorMap& tdo, const BwdArgs& a, int mod, int grid, cudaStream_t s) {
-  switch (mod) {
+                           const CUtensorMap& tdo, const BwdArgs& a, int key, int grid, cudaStream_t s) {
+  constexpr int M = kKeyMasked;
+  switch (key) {
     case MOD_NONE: return launch_bwd_t<D, MOD_NONE>(tq, tk, tv, tdo, a, grid, s);
-    case MOD_CAUSAL: return launch_bwd_t<D, MOD_CAUSAL>(tq, tk, tv, tdo, a, grid, s);
     case MOD_ALIBI: return launch_bwd_t<D, MOD_ALIBI>(tq, tk, tv, tdo, a, grid, s);
     case MOD_SOFTCAP: return launch_bwd_t<D, MOD_SOFTCAP>(tq, tk, tv, tdo, a, grid, s);
-    case MOD_WINDOW: return launch_bwd_t<D, MOD_WINDOW>(tq, tk, tv, tdo, a, grid, s);
     case MOD_BOOST: return launch_bwd_t<D, MOD_BOOST>(tq, tk, tv, tdo, a, grid, s);
-    case MOD_DOCUMENT: return launch_bwd_t<D, MOD_DOCUMENT>(tq, tk, tv, tdo, a, grid, s);
+    case M | MOD_NONE: return launch_bwd_t<D, M | MOD_NONE>(tq, tk, tv, tdo, a, grid, s);
+    case M | MOD_ALIBI: return launch_bwd_t<D, M | MOD_ALIBI>(tq, tk, tv, tdo, a, grid, s);
+    case M | MOD_SOFTCAP: return launch_bwd_t<D, M | MOD_SOFTCAP>(tq, tk, tv, tdo, a, grid, s);
+    case M | MOD_BOOST: return launch_bwd_t<D, M | MOD_BOOST>(tq, tk, tv, tdo, a, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -884,10 +886,10 @@ cudaError_t launch_bwd_mod(const CUtensorMap& tq, const CUtensorMap& tk, const C
 }  // namespace
 
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const BwdArgs& a, int D, int mod, int grid,
+                       const CUtensorMap& tdo, const BwdArgs& a, int D, int key, int grid,
                        cudaStream_t stream) {
-  if (D == 128) return launch_bwd_mod<128>(tq, tk, tv, tdo, a, mod, grid, stream);
-  if (D == 64) return launch_bwd_mod<64>(tq, tk, tv, tdo, a, mod, grid, stream);
+  if (D == 128) return launch_bwd_mod<128>(tq, tk, tv, tdo, a, key, grid, stream);
+  if (D == 64) return launch_bwd_mod<64>(tq, tk, tv, tdo, a, key, grid, stream);
   return cudaErrorInvalidValue;
 }
 

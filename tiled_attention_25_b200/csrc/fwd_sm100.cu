@@ -133,11 +133,11 @@ __device__ __forceinline__ void transform32(float (&x)[32], const RowCtx& r, con
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
     float v = x[c];
-    if constexpr (MOD == MOD_ALIBI) {
+    if constexpr (score_of(MOD) == MOD_ALIBI) {
       v = fmaf(v, r.sl2, -r.aux * fabsf(di - static_cast<float>(c)));
-    } else if constexpr (MOD == MOD_SOFTCAP) {
+    } else if constexpr (score_of(MOD) == MOD_SOFTCAP) {
       v = r.aux2 * tanhf(v * r.aux);
-    } else if constexpr (MOD == MOD_BOOST) {
+    } else if constexpr (score_of(MOD) == MOD_BOOST) {
       const bool inside = fabsf(di - static_cast<float>(c)) < static_cast<float>(md.boost_radius);
       v = v * (inside ? r.aux : r.sl2);
     } else {
@@ -152,12 +152,10 @@ __device__ __forceinline__ void transform32(float (&x)[32], const RowCtx& r, con
   }
 }
 
-// Scores whose mod is the plain scale (none and the interval masks) stay raw
-// until the exponent: the row maximum is taken on raw scores and the scale is
-// folded into the exponent's FFMA.
-__host__ __device__ constexpr bool pure_scale(int mod) {
-  return mod == MOD_NONE || mod == MOD_CAUSAL || mod == MOD_WINDOW || mod == MOD_DOCUMENT;
-}
+// Scores whose transform is the plain scale (no score mod, any masks) stay
+// raw until the exponent: the row maximum is taken on raw scores and the
+// scale is folded into the exponent's FFMA.
+__host__ __device__ constexpr bool pure_scale(int key) { return score_of(key) == MOD_NONE; }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
@@ -321,7 +319,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   // softcap and local boost keep the even split: their per-element mods need
   // more registers than any split can give, so they spill either way
-  constexpr bool kSplitRegs = MOD != MOD_SOFTCAP && MOD != MOD_BOOST;
+  constexpr bool kSplitRegs = score_of(MOD) != MOD_SOFTCAP && score_of(MOD) != MOD_BOOST;
   if (warp >= 8) {
   if constexpr (kSplitRegs) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
   if (warp == 9) {
@@ -338,7 +336,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const int buf = unit_iter & 1;
       uint32_t* lst = lists + buf * kMaxSteps;
       if (!mbar_wait_warp(smem_u32(&bars->list_empty[buf]), ((unit_iter >> 1) & 1) ^ 1, wc)) { ok = false; break; }
-      const int n = build_pair_steps(a.tile_class, uc.b, uc.p, a.nQ, a.nK, a.Sq, a.Skv, MOD,
+      const int n = build_pair_steps(a.tile_class, uc.b, uc.p, a.nQ, a.nK, a.Sq, a.Skv, a.mod.mask,
                                      a.mod.window, lst);
       if (lane == 0) bars->list_n[buf] = n;
       mbar_arrive(smem_u32(&bars->list_full[buf]));
@@ -504,15 +502,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       rc.sl2 = a.sl2;
       rc.aux = 0.f;
       rc.aux2 = 0.f;
-      if constexpr (MOD == MOD_ALIBI) rc.aux = alibi_slope(a.mod, uc.h, a.Hq) * LOG2E;
-      if constexpr (MOD == MOD_SOFTCAP) {
+      if constexpr (score_of(MOD) == MOD_ALIBI) rc.aux = alibi_slope(a.mod, uc.h, a.Hq) * LOG2E;
+      if constexpr (score_of(MOD) == MOD_SOFTCAP) {
         rc.aux = a.scale / a.mod.softcap;
         rc.aux2 = a.mod.softcap * LOG2E;
       }
-      if constexpr (MOD == MOD_BOOST) rc.aux = a.mod.boost * a.sl2;
-      row_interval(a.mod, uc.b, min(rc.row, a.Sq - 1), a.Skv, rc.lo, rc.hi);
+      if constexpr (score_of(MOD) == MOD_BOOST) rc.aux = a.mod.boost * a.sl2;
+      if constexpr (masked(MOD)) {
+        row_interval(a.mod, uc.b, min(rc.row, a.Sq - 1), a.Skv, rc.lo, rc.hi);
+      } else {
+        rc.lo = 0;
+        rc.hi = a.Skv - 1;
+      }
       if (rc.row >= a.Sq) rc.hi = rc.lo - 1;  // padding rows keep nothing
-      if constexpr (!is_interval_mask(MOD)) { rc.lo = 0; }
 
       float m_run = -INFINITY, l_run = 0.f;
       int n_act = 0;
@@ -655,15 +657,17 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 
 template <int D, bool LSE>
 cudaError_t launch_fwd_mod(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                           const FwdArgs& a, int mod, int grid, cudaStream_t s) {
-  switch (mod) {
+                           const FwdArgs& a, int key, int grid, cudaStream_t s) {
+  constexpr int M = kKeyMasked;
+  switch (key) {
     case MOD_NONE: return launch_fwd_t<D, MOD_NONE, LSE>(tq, tk, tv, a, grid, s);
-    case MOD_CAUSAL: return launch_fwd_t<D, MOD_CAUSAL, LSE>(tq, tk, tv, a, grid, s);
     case MOD_ALIBI: return launch_fwd_t<D, MOD_ALIBI, LSE>(tq, tk, tv, a, grid, s);
     case MOD_SOFTCAP: return launch_fwd_t<D, MOD_SOFTCAP, LSE>(tq, tk, tv, a, grid, s);
-    case MOD_WINDOW: return launch_fwd_t<D, MOD_WINDOW, LSE>(tq, tk, tv, a, grid, s);
     case MOD_BOOST: return launch_fwd_t<D, MOD_BOOST, LSE>(tq, tk, tv, a, grid, s);
-    case MOD_DOCUMENT: return launch_fwd_t<D, MOD_DOCUMENT, LSE>(tq, tk, tv, a, grid, s);
+    case M | MOD_NONE: return launch_fwd_t<D, M | MOD_NONE, LSE>(tq, tk, tv, a, grid, s);
+    case M | MOD_ALIBI: return launch_fwd_t<D, M | MOD_ALIBI, LSE>(tq, tk, tv, a, grid, s);
+    case M | MOD_SOFTCAP: return launch_fwd_t<D, M | MOD_SOFTCAP, LSE>(tq, tk, tv, a, grid, s);
+    case M | MOD_BOOST: return launch_fwd_t<D, M | MOD_BOOST, LSE>(tq, tk, tv, a, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -671,14 +675,14 @@ cudaError_t launch_fwd_mod(const CUtensorMap& tq, const CUtensorMap& tk, const C
 }  // namespace
 
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const FwdArgs& a, int D, int mod, bool has_lse, int grid,
+                       const FwdArgs& a, int D, int key, bool has_lse, int grid,
                        cudaStream_t stream) {
   if (D == 128)
-    return has_lse ? launch_fwd_mod<128, true>(tq, tk, tv, a, mod, grid, stream)
-                   : launch_fwd_mod<128, false>(tq, tk, tv, a, mod, grid, stream);
+    return has_lse ? launch_fwd_mod<128, true>(tq, tk, tv, a, key, grid, stream)
+                   : launch_fwd_mod<128, false>(tq, tk, tv, a, key, grid, stream);
   if (D == 64)
-    return has_lse ? launch_fwd_mod<64, true>(tq, tk, tv, a, mod, grid, stream)
-                   : launch_fwd_mod<64, false>(tq, tk, tv, a, mod, grid, stream);
+    return has_lse ? launch_fwd_mod<64, true>(tq, tk, tv, a, key, grid, stream)
+                   : launch_fwd_mod<64, false>(tq, tk, tv, a, key, grid, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -51,8 +51,8 @@ struct BwdArgs {
 };
 
 struct MaskArgs {
-  int kind;
-  int window;
+  int mask;      // kMask* bits
+  int window;    // W (1 << 30 without the window mask)
   const int32_t* doc_offsets;
   int num_docs;
   int B, Sq, Skv, nQ, nK, nP;
@@ -67,14 +67,12 @@ struct MaskArgs {
 
 // Each returns cudaSuccess or the launch error.
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const FwdArgs& a, int D, int mod, bool has_lse, int grid,
+                       const FwdArgs& a, int D, int key, bool has_lse, int grid,
                        cudaStream_t stream);
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const BwdArgs& a, int D, int mod, int grid,
+                       const CUtensorMap& tdo, const BwdArgs& a, int D, int key, int grid,
                        cudaStream_t stream);
 cudaError_t launch_block_mask(const MaskArgs& a, cudaStream_t stream);
 
-// Register count ptxas gave the forward kernel (for the host's sanity checks).
-int fwd_kernel_regs(int D, int mod, bool has_lse);
 
 }  // namespace attn25

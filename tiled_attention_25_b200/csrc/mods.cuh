@@ -3,12 +3,14 @@
 // The mods are the FlexAttention-style score_mod / mask_mod set of "PyTorch
 // FlexAttention, FlashAttention-4 백엔드 도입으로 성능 최대 3.2배 향상"
 // (섹션별 상세: local_boost and tanh_softcap take the score and the raw
-// q/kv indices; 핵심 요약: ALiBi, sliding window, document masks).  Every
-// mask of the set keeps, for query row i, an interval of keys
-// [lo(i), hi(i)]:  causal lo = 0, hi = i;  sliding window lo = i - W + 1,
-// hi = i;  document lo = start of the document holding i, hi = i.  Mods
-// without a mask keep [0, Skv).  Scores are handled in the base-2 domain:
-// x = s' * log2(e), so that exp(s' - m) = 2^(x - m2).
+// q/kv indices; 핵심 요약: ALiBi, sliding window, document masks, and their
+// composition).  A mod is one score transform (none, ALiBi, softcap, local
+// boost) and the AND of any of three masks.  Every mask keeps, for query row
+// i, an interval of keys: causal j <= i; sliding window i - W < j <= i;
+// document: j <= i in i's document.  An intersection of intervals is an
+// interval, so every composed mask keeps one interval [lo(i), hi(i)] per row
+// (and, transposed, one interval of queries per key).  Scores are handled in
+// the base-2 domain: x = s' * log2(e), so that exp(s' - m) = 2^(x - m2).
 #pragma once
 
 #include <cstdint>
@@ -27,18 +29,27 @@ constexpr int TILE = 128;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
-__host__ __device__ constexpr bool is_interval_mask(int mod) {
-  return mod == MOD_CAUSAL || mod == MOD_WINDOW || mod == MOD_DOCUMENT;
-}
+// Mask bits of a normalised mod (window and document imply causal).
+constexpr int kMaskCausal = 1;
+constexpr int kMaskWindow = 2;
+constexpr int kMaskDoc = 4;
+
+// Kernel specialisation key: the score transform (MOD_NONE, MOD_ALIBI,
+// MOD_SOFTCAP or MOD_BOOST) plus kKeyMasked when any mask is present; which
+// masks, and their parameters, are runtime values.
+constexpr int kKeyMasked = 16;
+__host__ __device__ constexpr int score_of(int key) { return key & (kKeyMasked - 1); }
+__host__ __device__ constexpr bool masked(int key) { return (key & kKeyMasked) != 0; }
 
 struct ModDev {
-  int kind;
+  int kind;                 // score transform: MOD_NONE, MOD_ALIBI, MOD_SOFTCAP or MOD_BOOST
+  int mask;                 // kMask* bits
   float softcap;            // c
-  int window;               // W
+  int window;               // W (1 << 30 without the window mask)
   float boost;              // local boost factor
   int boost_radius;         // |i - j| < radius gets the boost
   const float* alibi_slopes;  // [Hq] or nullptr (then 2^(-8(h+1)/Hq))
-  const int32_t* doc_offsets; // [B][num_docs + 1]
+  const int32_t* doc_offsets; // [B][num_docs + 1], nullptr without the document mask
   int num_docs;
 };
 
@@ -52,20 +63,23 @@ __device__ __forceinline__ int doc_start(const int32_t* offs, int num_docs, int 
   return __ldg(offs + lo);
 }
 
-// Kept key interval [lo, hi] of query row i (hi already clipped to Skv - 1).
-__device__ __forceinline__ void row_interval(const ModDev& m, int b, int i, int Skv, int& lo,
-                                             int& hi) {
+// Kept key interval [lo, hi] of query row i (hi already clipped to Skv - 1):
+// the intersection of the masks' intervals.
+__device__ __forceinline__ void row_interval(int mask, int window, const int32_t* offs_b,
+                                             int num_docs, int i, int Skv, int& lo, int& hi) {
   lo = 0;
   hi = Skv - 1;
-  if (m.kind == MOD_CAUSAL) {
-    hi = min(hi, i);
-  } else if (m.kind == MOD_WINDOW) {
-    hi = min(hi, i);
-    lo = max(0, i - m.window + 1);
-  } else if (m.kind == MOD_DOCUMENT) {
-    hi = min(hi, i);
-    lo = doc_start(m.doc_offsets + static_cast<size_t>(b) * (m.num_docs + 1), m.num_docs, i);
-  }
+  if (mask & (kMaskCausal | kMaskWindow | kMaskDoc)) hi = min(hi, i);
+  if (mask & kMaskWindow) lo = max(lo, i - window + 1);
+  if (mask & kMaskDoc) lo = max(lo, doc_start(offs_b, num_docs, i));
+}
+
+__device__ __forceinline__ void row_interval(const ModDev& m, int b, int i, int Skv, int& lo,
+                                             int& hi) {
+  row_interval(m.mask, m.window,
+               m.doc_offsets == nullptr ? nullptr
+                                        : m.doc_offsets + static_cast<size_t>(b) * (m.num_docs + 1),
+               m.num_docs, i, Skv, lo, hi);
 }
 
 __device__ __forceinline__ float alibi_slope(const ModDev& m, int h, int Hq) {
@@ -74,21 +88,19 @@ __device__ __forceinline__ float alibi_slope(const ModDev& m, int h, int Hq) {
 }
 
 // Class of the tile rows [q0, q1) x keys [k0, k1) (both already clipped to the
-// sequence lengths) for interval masks, by exact counting of kept elements:
-// 0 EMPTY, 1 PARTIAL, 2 FULL.  Used where the row intervals have closed forms.
-__host__ __device__ inline int interval_tile_class(int kind, int window, int q0, int q1, int k0,
-                                                   int k1) {
-  if (kind == MOD_CAUSAL || kind == MOD_WINDOW) {
-    // kept iff lo(i) <= j <= i with lo(i) = 0 (causal) or i - W + 1
-    const int first_row = q0, last_row = q1 - 1;
-    const bool any = (k0 <= last_row) &&
-                     (kind == MOD_CAUSAL || k1 - 1 >= first_row - window + 1);
-    if (!any) return 0;
-    const bool all = (k1 - 1 <= first_row) &&
-                     (kind == MOD_CAUSAL || k0 >= last_row - window + 1);
-    return all ? 2 : 1;
-  }
-  return 1;
+// sequence lengths) without a block mask: 0 EMPTY, 1 PARTIAL, 2 FULL, exact
+// for the causal and window masks (kept iff i - W < j <= i), and with the
+// document mask never FULL (its intervals need the offsets; PARTIAL tiles take
+// the per-element predicate, which is always exact).
+__host__ __device__ inline int dense_tile_class(int mask, int window, int q0, int q1, int k0,
+                                                int k1) {
+  if (mask == 0) return 2;
+  const int W = (mask & kMaskWindow) ? window : (1 << 30);
+  const int first_row = q0, last_row = q1 - 1;
+  const bool any = (k0 <= last_row) && (k1 - 1 >= first_row - W + 1);
+  if (!any) return 0;
+  const bool all = (k1 - 1 <= first_row) && (k0 >= last_row - W + 1);
+  return (all && !(mask & kMaskDoc)) ? 2 : 1;
 }
 
 }  // namespace attn25
