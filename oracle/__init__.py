@@ -12,9 +12,11 @@ from .attention import (  # noqa: F401
     MOD_NONE,
     MOD_SLIDING_WINDOW,
     MOD_SOFTCAP,
+    MASK_BITMAP,
     MASK_CAUSAL,
     MASK_DOCUMENT,
     MASK_SLIDING_WINDOW,
+    has_bitmap,
     has_document,
     has_mask,
     split_mod,

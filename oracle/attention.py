@@ -38,7 +38,11 @@ Readings where the pages are silent (each also listed in the design doc):
     a mod code is one of the seven kinds, optionally ORed with mask flags
     (``MASK_CAUSAL``, ``MASK_SLIDING_WINDOW``, ``MASK_DOCUMENT``).  The score
     transform is the base kind's; an element is kept only where the base kind
-    and every flagged mask keep it (the logical AND of the masks).
+    and every flagged mask keep it (the logical AND of the masks);
+  * a general mask_mod ("PyTorch FlexAttention, …", 핵심 요약: arbitrary
+    mask functions) is given as its values: ``MASK_BITMAP`` keeps (b, h, i, j)
+    where ``params.bitmap[b', h', i, j]`` is true, with b' = b and h' = h, or 0
+    where the array's batch or head extent is 1 (shared by all).
 """
 from __future__ import annotations
 
@@ -56,14 +60,16 @@ MOD_DOCUMENT = 6
 MASK_CAUSAL = 0x100
 MASK_SLIDING_WINDOW = 0x200
 MASK_DOCUMENT = 0x400
+MASK_BITMAP = 0x800
+_BITMAP = 0x100  # pseudo-kind of the bitmap mask (never a base kind)
 _FLAG_KIND = ((MASK_CAUSAL, MOD_CAUSAL), (MASK_SLIDING_WINDOW, MOD_SLIDING_WINDOW),
-              (MASK_DOCUMENT, MOD_DOCUMENT))
+              (MASK_DOCUMENT, MOD_DOCUMENT), (MASK_BITMAP, _BITMAP))
 
 
 def split_mod(mod):
     """(base kind, [mask kinds of the flags]) of a mod code; rejects unknown bits."""
     base, flags = int(mod) & 0xFF, int(mod) & ~0xFF
-    if base > MOD_DOCUMENT or flags & ~(MASK_CAUSAL | MASK_SLIDING_WINDOW | MASK_DOCUMENT):
+    if base > MOD_DOCUMENT or flags & ~(MASK_CAUSAL | MASK_SLIDING_WINDOW | MASK_DOCUMENT | MASK_BITMAP):
         raise ValueError(f"unknown mod {mod:#x}")
     return base, [kind for flag, kind in _FLAG_KIND if flags & flag]
 
@@ -72,6 +78,10 @@ def has_mask(mod) -> bool:
     """True when the mod masks any element (some kind in it is a mask)."""
     base, masks = split_mod(mod)
     return bool(masks) or base in (MOD_CAUSAL, MOD_SLIDING_WINDOW, MOD_DOCUMENT)
+
+
+def has_bitmap(mod) -> bool:
+    return bool(int(mod) & MASK_BITMAP)
 
 
 def has_document(mod) -> bool:
@@ -132,6 +142,9 @@ def _single_mod(s, mod, params, b, h, Hq, qi, kj):
         inside = np.abs(qi - kj) < params.boost_radius
         s_mod = np.where(inside, s * params.boost, s)
         dmod = np.where(inside, params.boost, 1.0) * np.ones_like(s)
+    elif mod == _BITMAP:
+        bm = np.asarray(params.bitmap, dtype=bool)
+        keep = bm[b if bm.shape[0] > 1 else 0, h if bm.shape[1] > 1 else 0][qi, kj]
     elif mod == MOD_DOCUMENT:
         offs = params.doc_offsets[b]
         S = int(max(qi.max(initial=0), kj.max(initial=0))) + 1
@@ -308,17 +321,20 @@ def useful_elements(mod, params, B, Hq, Sq, Skv) -> int:
     """Number of unmasked (b, h, q, kv) score elements (the useful-work count)."""
     qi = np.arange(Sq, dtype=np.int64)[:, None]
     kj = np.arange(Skv, dtype=np.int64)[None, :]
+    # a per-head bitmap differs between heads; every other mask is shared by them
+    per_head = has_bitmap(mod) and np.asarray(params.bitmap).shape[1] > 1
     total = 0
     for b in range(B):
-        if has_mask(mod):
-            n = 0
-            for r0 in range(0, Sq, 2048):
-                r = qi[r0:r0 + 2048]
-                _, keep, _ = score_mod(np.zeros((len(r), Skv)), mod, params, b, 0, Hq, r, kj)
-                n += int(keep.sum())
-        else:
-            n = Sq * Skv
-        total += n * Hq
+        for h in range(Hq if per_head else 1):
+            if has_mask(mod):
+                n = 0
+                for r0 in range(0, Sq, 2048):
+                    r = qi[r0:r0 + 2048]
+                    _, keep, _ = score_mod(np.zeros((len(r), Skv)), mod, params, b, h, Hq, r, kj)
+                    n += int(keep.sum())
+            else:
+                n = Sq * Skv
+            total += n * (1 if per_head else Hq)
     return total
 
 

@@ -26,28 +26,33 @@ from __future__ import annotations
 
 import numpy as np
 
-from .attention import has_mask, score_mod
+from .attention import has_bitmap, has_mask, score_mod
 
 TILE = 128
 
 
 def classify_tiles(mod, params, B, Sq, Skv, tile=TILE):
+    """Tile classes; with a per-head bitmap the classes hold for every head at
+    once: EMPTY where no head keeps an element, FULL where every head keeps
+    every in-range element, PARTIAL otherwise."""
     nQ = -(-Sq // tile)
     nK = -(-Skv // tile)
     cls = np.full((B, nQ, nK), 2, dtype=np.uint8)
     if not has_mask(mod):
         return cls
+    heads = np.asarray(params.bitmap).shape[1] if has_bitmap(mod) else 1
     kj = np.arange(Skv, dtype=np.int64)[None, :]
     for b in range(B):
         for qi in range(nQ):
             rows = np.arange(qi * tile, min(Sq, (qi + 1) * tile), dtype=np.int64)[:, None]
-            _, keep, _ = score_mod(np.zeros((rows.shape[0], Skv)), mod, params, b, 0, 1, rows, kj)
+            keeps = [score_mod(np.zeros((rows.shape[0], Skv)), mod, params, b, h, heads, rows, kj)[1]
+                     for h in range(heads)]
             for kt in range(nK):
-                blk = keep[:, kt * tile:min(Skv, (kt + 1) * tile)]
-                n_keep = int(blk.sum())
-                if n_keep == 0:
+                blocks = [keep[:, kt * tile:min(Skv, (kt + 1) * tile)] for keep in keeps]
+                counts = [int(blk.sum()) for blk in blocks]
+                if max(counts) == 0:
                     cls[b, qi, kt] = 0
-                elif n_keep == blk.size:
+                elif min(counts) == blocks[0].size:
                     cls[b, qi, kt] = 2
                 else:
                     cls[b, qi, kt] = 1

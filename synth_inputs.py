@@ -52,6 +52,8 @@ class ModParams:
     boost_radius: int = 128
     # per batch row, the ascending document start offsets plus the end (S)
     doc_offsets: list | None = None
+    # general mask values: bool [B or 1][H or 1][Sq][Skv], True = keep
+    bitmap: np.ndarray | None = None
 
 
 @dataclasses.dataclass

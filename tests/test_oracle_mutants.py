@@ -14,6 +14,7 @@ import oracle.attention as oa
 import oracle.block_sparsity as ob
 import test_oracle as pins
 import test_oracle_block_mask as bm_pins
+import test_oracle_bitmap as bitmap_pins
 import test_oracle_compose as comp_pins
 
 
@@ -63,7 +64,13 @@ MUTANTS = [
      comp_pins.test_zero_queries_window_and_documents_count_keys),
     (oa, "score_mod", "_single_mod(s, base, params", "_single_mod(s, masks[0] if masks else base, params",
      comp_pins.test_zero_queries_causal_alibi_geometric_sums),
-    (ob, "classify_tiles", "elif n_keep == blk.size:", "elif n_keep == tile * tile:", bm_pins.test_single_row_tail_tile_is_full),
+    (ob, "classify_tiles", "elif min(counts) == blocks[0].size:", "elif min(counts) == tile * tile:",
+     bm_pins.test_single_row_tail_tile_is_full),
+    (ob, "classify_tiles", "if max(counts) == 0:", "if min(counts) == 0:",
+     bitmap_pins.test_per_head_bitmap_classes_hold_for_every_head),
+    (oa, "_single_mod", "[qi, kj]", "[kj, qi]",
+     lambda: bitmap_pins.test_random_bitmap_is_restricted_softmax(oa.MOD_NONE | oa.MASK_BITMAP)),
+    (oa, "_single_mod", "h if bm.shape[1] > 1 else 0", "0", bitmap_pins.test_per_head_bitmap_equals_separate_heads),
     (ob, "block_mask", "key=lambda u: (-pair_cost[u], u)", "key=lambda u: (pair_cost[u], u)", bm_pins.test_orders_are_lpt_permutations),
 ]
 
