@@ -96,7 +96,9 @@ typedef enum attn_mod_kind {
 enum {
   ATTN_MASK_CAUSAL = 0x100,
   ATTN_MASK_SLIDING_WINDOW = 0x200,
-  ATTN_MASK_DOCUMENT = 0x400
+  ATTN_MASK_DOCUMENT = 0x400,
+  ATTN_MASK_BITMAP = 0x800      /* a general mask given by its values (attn_mod_params.bitmap);
+                                   attn_fwd / attn_bwd then need a block mask built for it */
 };
 
 /*
@@ -116,6 +118,15 @@ typedef struct attn_mod_params {
                                   value to pad rows with fewer documents.  Queries and keys share the
                                   offsets (packed self-attention, Sq == Skv required). */
   int32_t num_docs;            /* ATTN_MOD_DOCUMENT / ATTN_MASK_DOCUMENT: 1 <= num_docs <= 4096 */
+  /* ATTN_MASK_BITMAP: the values of a general mask_mod, one bit per element.
+   * Element (b, h, i, j) is kept when bit (j & 31) of word
+   *   b * bitmap_batch_stride + h * bitmap_head_stride + i * bitmap_row_words + (j >> 5)
+   * is set.  Device memory, 16-byte aligned, read only; bits at j >= Skv are ignored. */
+  const uint32_t* bitmap;
+  int32_t bitmap_row_words;     /* a multiple of 4, >= ceil(Skv / 32) */
+  int32_t bitmap_heads;         /* 1 (one mask for all heads, head stride 0) or Hq */
+  int64_t bitmap_head_stride;   /* words, a multiple of 4; 0 when bitmap_heads == 1 */
+  int64_t bitmap_batch_stride;  /* words, a multiple of 4; 0 = one mask for all batch rows */
 } attn_mod_params;
 
 /*
@@ -218,7 +229,10 @@ ATTN25_API int attn_block_mask_bind(void* buffer, size_t bytes, int B, int Sq, i
 
 /*
  * Classify every 128x128 tile for the mod and fill all arrays of a bound
- * block mask (bit-exact with a per-element classification).
+ * block mask (bit-exact with a per-element classification).  With a per-head
+ * bitmap the classes hold for every head: EMPTY where no head keeps an
+ * element of the tile, FULL where every head keeps all of its in-range
+ * elements, PARTIAL otherwise.
  */
 ATTN25_API int build_block_mask(int mod_kind, const attn_mod_params* mod_params,
                      int B, int Sq, int Skv, attn_block_mask* mask,

@@ -161,3 +161,15 @@ def mod_params_for(w: Workload, mod: str) -> ModParams:
     if mod == "document":
         p.doc_offsets = doc_offsets_for(w)
     return p
+
+
+def pack_bitmap(keep: np.ndarray) -> np.ndarray:
+    """Bool [B'][H'][Sq][Skv] -> int32 words [B'][H'][Sq][4 ceil(Skv / 128)]: bit
+    (j & 31) of word j >> 5 is element j; padding bits are zero."""
+    keep = np.asarray(keep, dtype=bool)
+    nb, nh, sq, skv = keep.shape
+    rw = 4 * (-(-skv // 128))
+    padded = np.zeros((nb, nh, sq, rw * 32), dtype=bool)
+    padded[..., :skv] = keep
+    bits = np.packbits(padded.reshape(nb, nh, sq, rw, 32), axis=-1, bitorder="little")
+    return bits.reshape(nb, nh, sq, rw * 4).view(np.uint32).view(np.int32).copy()

@@ -4,7 +4,7 @@ import numpy as np
 import torch
 
 import oracle
-from synth_inputs import ModParams, bf16_bits_to_f64, draw_qkv, pad_offsets
+from synth_inputs import ModParams, bf16_bits_to_f64, draw_qkv, pack_bitmap, pad_offsets
 
 # Tolerances for bf16 inputs with fp32 accumulation versus the fp64 oracle.
 O_MAX_ABS = 2e-2
@@ -38,8 +38,11 @@ class Case:
         if oracle.has_document(mod):
             arr, _ = pad_offsets(self.p.doc_offsets)
             doc_t = torch.from_numpy(arr).cuda()
+        bm_t = None
+        if oracle.has_bitmap(mod):
+            bm_t = torch.from_numpy(pack_bitmap(self.p.bitmap)).cuda()
         self.dev_params = ta.ModParams(softcap=self.p.softcap, window=self.p.window, boost=self.p.boost,
-                                       boost_radius=self.p.boost_radius, doc_offsets=doc_t)
+                                       boost_radius=self.p.boost_radius, doc_offsets=doc_t, bitmap=bm_t)
 
     def oracle_fwd(self, heads=None, rows=None):
         return oracle.attention_forward(self.qf, self.kf, self.vf, self.scale, self.mod, self.p,

@@ -91,8 +91,9 @@ def test_argument_errors_before_launch(lib):
     assert call(args(mod=3)) == -1   # softcap needs params
     assert call(args(mod=6)) == -1   # document mask needs offsets
     # composed codes: unknown flag bits or kinds, and the components' own parameters
-    assert call(args(mod=0x800)) == -1
+    assert call(args(mod=0x1000)) == -1
     assert call(args(mod=2 | 0x1000)) == -1
+    assert call(args(mod=0x800)) == -1        # bitmap flag needs the bitmap
     assert call(args(mod=7 | 0x100)) == -1
     assert call(args(mod=0x400)) == -1        # document flag needs offsets
     assert call(args(mod=2 | 0x200)) == -1    # window flag needs params

@@ -13,6 +13,7 @@ from .abi import (  # noqa: F401
     EXPORTED,
     LIB,
     LIB_PATH,
+    MASK_BITMAP,
     MASK_CAUSAL,
     MASK_DOCUMENT,
     MASK_SLIDING_WINDOW,

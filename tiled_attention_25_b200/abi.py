@@ -30,6 +30,7 @@ MOD_DOCUMENT = 6
 MASK_CAUSAL = 0x100
 MASK_SLIDING_WINDOW = 0x200
 MASK_DOCUMENT = 0x400
+MASK_BITMAP = 0x800
 
 ATTN_ERR_TIMEOUT = -6
 
@@ -49,6 +50,11 @@ class CModParams(ctypes.Structure):
         ("alibi_slopes", ctypes.c_void_p),
         ("doc_offsets", ctypes.c_void_p),
         ("num_docs", ctypes.c_int32),
+        ("bitmap", ctypes.c_void_p),
+        ("bitmap_row_words", ctypes.c_int32),
+        ("bitmap_heads", ctypes.c_int32),
+        ("bitmap_head_stride", ctypes.c_int64),
+        ("bitmap_batch_stride", ctypes.c_int64),
     ]
 
 
@@ -138,7 +144,7 @@ class ModParams:
     """Mod scalars plus the device tensors they point at (kept alive here)."""
 
     def __init__(self, softcap=50.0, window=1024, boost=1.1, boost_radius=128,
-                 alibi_slopes=None, doc_offsets=None):
+                 alibi_slopes=None, doc_offsets=None, bitmap=None):
         self.softcap = float(softcap)
         self.window = int(window)
         self.boost = float(boost)
@@ -149,12 +155,22 @@ class ModParams:
             assert doc_offsets.dtype == torch.int32 and doc_offsets.is_contiguous() and doc_offsets.dim() == 2
         if alibi_slopes is not None:
             assert alibi_slopes.dtype == torch.float32 and alibi_slopes.is_contiguous()
+        # device int32 [B or 1][Hq or 1][Sq][row_words] keep bits (bit j & 31 of word j >> 5)
+        self.bitmap = bitmap
+        if bitmap is not None:
+            assert bitmap.dtype == torch.int32 and bitmap.is_contiguous() and bitmap.dim() == 4
 
     def c(self) -> CModParams:
+        bm = self.bitmap
+        if bm is None:
+            bm_args = (None, 0, 0, 0, 0)
+        else:
+            nb, nh, sq, rw = bm.shape
+            bm_args = (bm.data_ptr(), rw, nh, 0 if nh == 1 else sq * rw, 0 if nb == 1 else nh * sq * rw)
         return CModParams(self.softcap, self.window, self.boost, self.boost_radius,
                           None if self.alibi_slopes is None else self.alibi_slopes.data_ptr(),
                           None if self.doc_offsets is None else self.doc_offsets.data_ptr(),
-                          0 if self.doc_offsets is None else self.doc_offsets.shape[1] - 1)
+                          0 if self.doc_offsets is None else self.doc_offsets.shape[1] - 1, *bm_args)
 
 
 class BlockMask:
@@ -182,9 +198,16 @@ class BlockMask:
         return self.buffer[off:off + size].view(dtype).view(shape)
 
 
-def _mp(mod_params):
+def _mp(mod_params, mod_kind, B, Hq, Sq):
+    """Marshal the mod params; a bitmap tensor must cover every (b, h, row) the
+    call reads (the C side cannot see its extent)."""
     if mod_params is None:
         return None
+    bm = mod_params.bitmap
+    if int(mod_kind) & MASK_BITMAP and bm is not None:
+        nb, nh, sq, _ = bm.shape
+        if nb not in (1, B) or (Hq is not None and nh not in (1, Hq)) or sq < Sq:
+            raise ValueError(f"bitmap of shape {tuple(bm.shape)} does not cover B={B}, Hq={Hq}, Sq={Sq}")
     cm = mod_params.c()
     return ctypes.byref(cm), cm
 
@@ -206,7 +229,7 @@ def attn_fwd(q, k, v, out, lse=None, scale=None, mod_kind=MOD_NONE, mod_params=N
     if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hq, Sq) or not lse.is_contiguous()):
         raise ValueError("lse must be a contiguous fp32 [B][Hq][Sq] tensor")
     scale = D ** -0.5 if scale is None else float(scale)
-    mp = _mp(mod_params)
+    mp = _mp(mod_params, mod_kind, B, Hq, Sq)
     rc = LIB.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
                       scale, int(mod_kind), None if mp is None else mp[0],
                       None if block_mask is None else ctypes.byref(block_mask.c), _stream(stream))
@@ -227,7 +250,7 @@ def attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, workspace, scale=None, mod_kin
         if t.dtype != torch.bfloat16 or tuple(t.shape) != (B, Hkv, Skv, D) or not t.is_contiguous():
             raise ValueError("dk/dv must be contiguous bf16 like k")
     scale = D ** -0.5 if scale is None else float(scale)
-    mp = _mp(mod_params)
+    mp = _mp(mod_params, mod_kind, B, Hq, Sq)
     rc = LIB.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
                       _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
                       B, Hq, Hkv, Sq, Skv, D, scale, int(mod_kind), None if mp is None else mp[0],
@@ -246,7 +269,7 @@ def attn_bwd_noalloc(q, k, v, out, lse, dout, dq, dk, dv, scale=None, mod_kind=M
         if t.dtype != torch.bfloat16 or tuple(t.shape) != (B, Hkv, Skv, D) or not t.is_contiguous():
             raise ValueError("dk/dv must be contiguous bf16 like k")
     scale = D ** -0.5 if scale is None else float(scale)
-    mp = _mp(mod_params)
+    mp = _mp(mod_params, mod_kind, B, Hq, Sq)
     rc = LIB.attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
                               _ptr(dk), _ptr(dv), B, Hq, Hkv, Sq, Skv, D, scale, int(mod_kind),
                               None if mp is None else mp[0],
@@ -271,7 +294,7 @@ def attn_block_mask_bind(buffer, B, Sq, Skv) -> BlockMask:
 
 
 def build_block_mask(mod_kind, mod_params, B, Sq, Skv, mask: BlockMask, stream=None):
-    mp = _mp(mod_params)
+    mp = _mp(mod_params, mod_kind, B, None, Sq)
     rc = LIB.build_block_mask(int(mod_kind), None if mp is None else mp[0], B, Sq, Skv,
                               ctypes.byref(mask.c), _stream(stream))
     _check(rc, "build_block_mask")

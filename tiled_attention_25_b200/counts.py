@@ -11,7 +11,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .abi import (MASK_CAUSAL, MASK_DOCUMENT, MASK_SLIDING_WINDOW, MOD_CAUSAL, MOD_DOCUMENT,
+from .abi import (MASK_BITMAP, MASK_CAUSAL, MASK_DOCUMENT, MASK_SLIDING_WINDOW, MOD_CAUSAL, MOD_DOCUMENT,
                   MOD_SLIDING_WINDOW)
 
 
@@ -25,7 +25,10 @@ def mask_parts(mod_kind):
 
 
 def useful_elements(mod_kind, B, Hq, Sq, Skv, window=None, doc_offsets=None) -> int:
-    """Unmasked (b, h, q, kv) elements; doc_offsets: per-batch-row offset lists."""
+    """Unmasked (b, h, q, kv) elements; doc_offsets: per-batch-row offset lists.
+    Interval masks only: a bitmap mask's count is the number of its set bits."""
+    if int(mod_kind) & MASK_BITMAP:
+        raise ValueError("count a bitmap mask from its bits")
     causal, win, doc = mask_parts(mod_kind)
     i = np.arange(Sq, dtype=np.int64)
     hi = np.minimum(i, Skv - 1) if causal else np.full(Sq, Skv - 1, dtype=np.int64)

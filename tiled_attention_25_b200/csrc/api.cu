@@ -119,7 +119,8 @@ struct ModSpec {
 bool split_mod(int code, ModSpec& m) {
   const int base = code & 0xFF, flags = code & ~0xFF;
   if (base < ATTN_MOD_NONE || base > ATTN_MOD_DOCUMENT) return false;
-  if (flags & ~(ATTN_MASK_CAUSAL | ATTN_MASK_SLIDING_WINDOW | ATTN_MASK_DOCUMENT)) return false;
+  if (flags & ~(ATTN_MASK_CAUSAL | ATTN_MASK_SLIDING_WINDOW | ATTN_MASK_DOCUMENT | ATTN_MASK_BITMAP))
+    return false;
   m.score = MOD_NONE;
   m.mask = 0;
   switch (base) {
@@ -134,10 +135,12 @@ bool split_mod(int code, ModSpec& m) {
   if (flags & ATTN_MASK_CAUSAL) m.mask |= kMaskCausal;
   if (flags & ATTN_MASK_SLIDING_WINDOW) m.mask |= kMaskCausal | kMaskWindow;
   if (flags & ATTN_MASK_DOCUMENT) m.mask |= kMaskCausal | kMaskDoc;
-  m.key = m.score | (m.mask != 0 ? kKeyMasked : 0);
+  if (flags & ATTN_MASK_BITMAP) m.mask |= kMaskBitmap;
+  m.key = m.score | (m.mask != 0 ? kKeyMasked : 0) | ((m.mask & kMaskBitmap) ? kKeyBitmap : 0);
   m.canonical = m.score | ((m.mask & kMaskCausal) ? ATTN_MASK_CAUSAL : 0) |
                 ((m.mask & kMaskWindow) ? ATTN_MASK_SLIDING_WINDOW : 0) |
-                ((m.mask & kMaskDoc) ? ATTN_MASK_DOCUMENT : 0);
+                ((m.mask & kMaskDoc) ? ATTN_MASK_DOCUMENT : 0) |
+                ((m.mask & kMaskBitmap) ? ATTN_MASK_BITMAP : 0);
   return true;
 }
 
@@ -170,6 +173,15 @@ int check_common(int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale, in
     if (Sq != Skv) return ATTN_ERR_UNSUPPORTED;
     if (reinterpret_cast<uintptr_t>(mp->doc_offsets) & 3u) return ATTN_ERR_ALIGN;
   }
+  if (ms.mask & kMaskBitmap) {
+    if (mp == nullptr || mp->bitmap == nullptr) return ATTN_ERR_ARG;
+    if (!aligned16(mp->bitmap)) return ATTN_ERR_ALIGN;
+    if (mp->bitmap_row_words < cdiv(Skv, 32) || (mp->bitmap_row_words & 3)) return ATTN_ERR_ARG;
+    if (mp->bitmap_heads < 1 || mp->bitmap_head_stride < 0 || mp->bitmap_batch_stride < 0 ||
+        (mp->bitmap_head_stride & 3) || (mp->bitmap_batch_stride & 3))
+      return ATTN_ERR_ARG;
+    if (mp->bitmap_heads == 1 && mp->bitmap_head_stride != 0) return ATTN_ERR_ARG;
+  }
   if (bm != nullptr) {
     if (bm->tile_class == nullptr || bm->kv_count == nullptr || bm->kv_index == nullptr ||
         bm->q_count == nullptr || bm->q_index == nullptr || bm->fwd_order == nullptr ||
@@ -179,6 +191,18 @@ int check_common(int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale, in
         bm->nk_tiles != cdiv(Skv, TILE) || bm->mod_kind != ms.canonical)
       return ATTN_ERR_ARG;
   }
+  return ATTN_OK;
+}
+
+// The bitmap mask's extra rules for attn_fwd / attn_bwd: its heads are the
+// call's query heads (or one shared mask), and a block mask, which is the
+// only place its tile classes come from, is given.
+int check_bitmap_call(int mod_kind, int Hq, const attn_mod_params* mp, const attn_block_mask* bm) {
+  ModSpec ms;
+  split_mod(mod_kind, ms);
+  if (!(ms.mask & kMaskBitmap)) return ATTN_OK;
+  if (bm == nullptr) return ATTN_ERR_ARG;
+  if (mp->bitmap_heads != 1 && mp->bitmap_heads != Hq) return ATTN_ERR_ARG;
   return ATTN_OK;
 }
 
@@ -199,6 +223,12 @@ ModDev make_mod(int mod_kind, const attn_mod_params* mp) {
     if (ms.mask & kMaskDoc) {
       m.doc_offsets = mp->doc_offsets;
       m.num_docs = mp->num_docs;
+    }
+    if (ms.mask & kMaskBitmap) {
+      m.bitmap = mp->bitmap;
+      m.bm_row_words = mp->bitmap_row_words;
+      m.bm_head_stride = mp->bitmap_head_stride;
+      m.bm_batch_stride = mp->bitmap_batch_stride;
     }
   }
   return m;
@@ -318,6 +348,11 @@ int build_block_mask(int mod_kind, const attn_mod_params* mod_params, int B, int
   a.window = md.window;
   a.doc_offsets = md.doc_offsets;
   a.num_docs = md.num_docs;
+  a.bitmap = md.bitmap;
+  a.bm_row_words = md.bm_row_words;
+  a.bm_heads = md.bitmap != nullptr ? mod_params->bitmap_heads : 0;
+  a.bm_head_stride = md.bm_head_stride;
+  a.bm_batch_stride = md.bm_batch_stride;
   a.B = B;
   a.Sq = Sq;
   a.Skv = Skv;
@@ -346,6 +381,7 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
       (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return ATTN_ERR_ALIGN;
   int rc = check_common(B, Hq, Hkv, Sq, Skv, D, scale, mod_kind, mod_params, block_mask);
+  if (rc == ATTN_OK) rc = check_bitmap_call(mod_kind, Hq, mod_params, block_mask);
   if (rc != ATTN_OK) return rc;
   DeviceInfo* d = nullptr;
   rc = current_device(&d);
@@ -407,6 +443,7 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
       (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return ATTN_ERR_ALIGN;
   int rc = check_common(B, Hq, Hkv, Sq, Skv, D, scale, mod_kind, mod_params, block_mask);
+  if (rc == ATTN_OK) rc = check_bitmap_call(mod_kind, Hq, mod_params, block_mask);
   if (rc != ATTN_OK) return rc;
   if (workspace_bytes < attn_bwd_workspace_size(B, Hq, Sq, D)) return ATTN_ERR_WORKSPACE;
   DeviceInfo* d = nullptr;

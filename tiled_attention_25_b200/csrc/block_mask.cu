@@ -47,13 +47,41 @@ __global__ void __launch_bounds__(256) classify_kernel(const MaskArgs a) {
   const size_t row = static_cast<size_t>(b) * a.nQ + qt;
   for (int kt = threadIdx.x; kt < a.nK; kt += blockDim.x) {
     const int k0 = kt * TILE, k1 = min(a.Skv, k0 + TILE);
-    long long kept = 0;
-    for (int r = 0; r < q1 - q0; ++r) {
-      const int lo = max(s_lo[r], k0), hi = min(s_hi[r], k1 - 1);
-      kept += max(0, hi - lo + 1);
-    }
     const long long total = static_cast<long long>(q1 - q0) * (k1 - k0);
-    const uint8_t c = kept == 0 ? 0 : (kept == total ? 2 : 1);
+    long long kept_min, kept_max;  // over the heads the masks distinguish
+    if (a.bitmap == nullptr) {
+      long long kept = 0;
+      for (int r = 0; r < q1 - q0; ++r) {
+        const int lo = max(s_lo[r], k0), hi = min(s_hi[r], k1 - 1);
+        kept += max(0, hi - lo + 1);
+      }
+      kept_min = kept_max = kept;
+    } else {
+      // kept = set bits of the row's 128-key word group inside its interval
+      kept_min = total;
+      kept_max = 0;
+      for (int h = 0; h < a.bm_heads; ++h) {
+        const uint32_t* base = a.bitmap + b * a.bm_batch_stride + h * a.bm_head_stride;
+        long long kept = 0;
+        for (int r = 0; r < q1 - q0; ++r) {
+          const int lo = max(s_lo[r], k0) - k0, hi = min(s_hi[r], k1 - 1) - k0;  // tile columns
+          if (hi < lo) continue;
+          const uint4 w = __ldg(reinterpret_cast<const uint4*>(
+                                    base + static_cast<long long>(q0 + r) * a.bm_row_words) + kt);
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int clo = max(lo - 32 * c, 0), chi = min(hi - 32 * c, 31);
+            if (chi < clo) continue;
+            const uint32_t in = (0xffffffffu >> (31 - chi)) & (0xffffffffu << clo);
+            kept += __popc(ws[c] & in);
+          }
+        }
+        kept_min = min(kept_min, kept);
+        kept_max = max(kept_max, kept);
+      }
+    }
+    const uint8_t c = kept_max == 0 ? 0 : (kept_min == total ? 2 : 1);
     a.tile_class[row * a.nK + kt] = c;
     if (kt < 1024) s_cls[kt] = c;
   }

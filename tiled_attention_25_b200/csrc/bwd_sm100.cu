@@ -51,6 +51,7 @@ namespace {
 
 constexpr int kBwdThreads = 512;
 constexpr int BM = 64;  // query rows per step
+static_assert(BM == 64, "the bitmap mask fetches two 32-query words per lane");
 // Warpgroups: 0 = P^T, 1 = dS^T, 2 = dQ drain, 3 = MMA (warp 12), TMA (warp 13).
 // No setmaxnreg split: every thread keeps the launch allocation (at most 128
 // registers at 512 threads).  Without the split, ptxas can keep the polling
@@ -234,9 +235,12 @@ __device__ __forceinline__ float4 lds128(uint32_t addr) {
 
 // One key row of S^T (raw q.k for 64 queries) -> P^T = 2^(x - LSE2) in place;
 // nl2_addr is the shared address of the 64 negated base-2 LSEs.
+// With the bitmap mask, wa / wb hold (lane l) the keep-bit word of query
+// q0 + l / q0 + 32 + l over this warp's 32 keys; bit (key & 31) keeps.
 template <int MOD>
 __device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h, float dq0, int q0,
-                                        int qlo, int qhi, bool pred, uint32_t nl2_addr) {
+                                        int qlo, int qhi, bool pred, uint32_t nl2_addr, uint32_t wa,
+                                        uint32_t wb) {
   float aux = 0.f, aux2 = 0.f;
   if constexpr (score_of(MOD) == MOD_ALIBI) aux = alibi_slope(a.mod, h, a.Hq) * LOG2E;
   if constexpr (score_of(MOD) == MOD_SOFTCAP) {
@@ -270,6 +274,13 @@ __device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h,
         const int qq = q0 + c;
         v.x = (qq >= qlo && qq <= qhi) ? v.x : -INFINITY;
         v.y = (qq + 1 >= qlo && qq + 1 <= qhi) ? v.y : -INFINITY;
+        if constexpr (has_bitmap(MOD)) {
+          const uint32_t key_bit = 1u << (threadIdx.x & 31);
+          const uint32_t w0 = __shfl_sync(0xffffffffu, c < 32 ? wa : wb, c & 31);
+          const uint32_t w1 = __shfl_sync(0xffffffffu, c + 1 < 32 ? wa : wb, (c + 1) & 31);
+          v.x = (w0 & key_bit) ? v.x : -INFINITY;
+          v.y = (w1 & key_bit) ? v.y : -INFINITY;
+        }
       }
       x[c] = ex2_approx(v.x);  // 0 where masked or on padding rows (-LSE2 = -inf)
       x[c + 1] = ex2_approx(v.y);
@@ -576,6 +587,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int s = step % Cfg::kStages, sb = step & 1;
         const uint32_t nl2_s = sbase + Cfg::kStageOff + s * Cfg::kStageBytes + 2 * Cfg::kQBytes;
         const uint32_t t_s = tmem + Cfg::kColS + sb * BM + lane_off;
+        // bitmap mask on PARTIAL steps: lane l fetches the word of queries q0 + l
+        // and q0 + 32 + l over this warp's 32 keys (issued before the waits)
+        uint32_t wa = 0u, wb = 0u;
+        if constexpr (has_bitmap(MOD)) {
+          if (pred) {
+            const int lane = threadIdx.x & 31;
+            const uint32_t* col = bitmap_row(a.mod, un.b, un.hk * a.G + g, 0) + un.kt * 4 + (r >> 5);
+            const int qa = q0 + lane, qb = q0 + 32 + lane;
+            if (qa < a.Sq) wa = __ldg(col + static_cast<long long>(qa) * a.mod.bm_row_words);
+            if (qb < a.Sq) wb = __ldg(col + static_cast<long long>(qb) * a.mod.bm_row_words);
+          }
+        }
         if (!ATTN25_TIMED(tr[1], mbar_wait_warp_ool(smem_u32(&bars->q_full[s]), (step / Cfg::kStages) & 1, wc))) { ok = false; break; }
         if (!ATTN25_TIMED(tr[2], mbar_wait_warp_ool(smem_u32(&bars->s_full[sb]), (step >> 1) & 1, wc))) { ok = false; break; }
         tc_fence_after();
@@ -587,7 +610,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(t_s + 32, reinterpret_cast<uint32_t(&)[32]>(x[32]));
         tmem_wait_ld();
         ATTN25_TRACE_ONLY(const long long t_p1 = clock64(); tr[4] += t_p1 - t_p;)
-        probs_t<MOD>(x, a, h, static_cast<float>(q0 - kv), q0, qlo, qhi, pred, nl2_s);
+        probs_t<MOD>(x, a, h, static_cast<float>(q0 - kv), q0, qlo, qhi, pred, nl2_s, wa, wb);
         // P^T (bf16 pairs) over the first 32 columns of this S^T buffer
         uint32_t pk[32];
 #pragma unroll
@@ -869,7 +892,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 template <int D>
 cudaError_t launch_bwd_mod(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            const CUtensorMap& tdo, const BwdArgs& a, int key, int grid, cudaStream_t s) {
-  constexpr int M = kKeyMasked;
+  constexpr int M = kKeyMasked, MB = kKeyMasked | kKeyBitmap;
   switch (key) {
     case MOD_NONE: return launch_bwd_t<D, MOD_NONE>(tq, tk, tv, tdo, a, grid, s);
     case MOD_ALIBI: return launch_bwd_t<D, MOD_ALIBI>(tq, tk, tv, tdo, a, grid, s);
@@ -879,6 +902,10 @@ cudaError_t launch_bwd_mod(const CUtensorMap& tq, const CUtensorMap& tk, const C
     case M | MOD_ALIBI: return launch_bwd_t<D, M | MOD_ALIBI>(tq, tk, tv, tdo, a, grid, s);
     case M | MOD_SOFTCAP: return launch_bwd_t<D, M | MOD_SOFTCAP>(tq, tk, tv, tdo, a, grid, s);
     case M | MOD_BOOST: return launch_bwd_t<D, M | MOD_BOOST>(tq, tk, tv, tdo, a, grid, s);
+    case MB | MOD_NONE: return launch_bwd_t<D, MB | MOD_NONE>(tq, tk, tv, tdo, a, grid, s);
+    case MB | MOD_ALIBI: return launch_bwd_t<D, MB | MOD_ALIBI>(tq, tk, tv, tdo, a, grid, s);
+    case MB | MOD_SOFTCAP: return launch_bwd_t<D, MB | MOD_SOFTCAP>(tq, tk, tv, tdo, a, grid, s);
+    case MB | MOD_BOOST: return launch_bwd_t<D, MB | MOD_BOOST>(tq, tk, tv, tdo, a, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }

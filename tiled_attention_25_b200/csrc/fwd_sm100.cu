@@ -123,6 +123,7 @@ struct RowCtx {
   float sl2;    // scale * log2(e)
   float aux;    // ALiBi: slope * log2(e); softcap: scale / c; boost: boost * sl2
   float aux2;   // softcap: c * log2(e)
+  const uint32_t* bits;  // bitmap mask: this row's keep bits (nullptr on padding rows)
 };
 
 // Raw scores of one row (32 columns starting at key k0 + c0) -> base-2 modded scores.
@@ -167,7 +168,7 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // scores; return the row maximum in the base-2 domain.
 template <int MOD, bool PRED>
 __device__ __forceinline__ float row_scores(float (&x)[4][32], const RowCtx& rc, const ModDev& md,
-                                            int k0) {
+                                            int k0, const uint4& bw) {
   float mx = -INFINITY;
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
@@ -179,6 +180,12 @@ __device__ __forceinline__ float row_scores(float (&x)[4][32], const RowCtx& rc,
       }
     } else {
       transform32<MOD>(x[c], rc, md, k0, c * 32, PRED);
+    }
+    if constexpr (PRED && has_bitmap(MOD)) {
+      // the bitmap mask: bit e of word c keeps key k0 + 32 c + e
+      const uint32_t w = c == 0 ? bw.x : (c == 1 ? bw.y : (c == 2 ? bw.z : bw.w));
+#pragma unroll
+      for (int e = 0; e < 32; ++e) x[c][e] = ((w >> e) & 1u) ? x[c][e] : -INFINITY;
     }
     // three-input max: 16 instructions per 32 columns, 4 independent chains
     float m0 = max3(x[c][0], x[c][1], x[c][2]), m1 = max3(x[c][3], x[c][4], x[c][5]);
@@ -515,6 +522,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         rc.hi = a.Skv - 1;
       }
       if (rc.row >= a.Sq) rc.hi = rc.lo - 1;  // padding rows keep nothing
+      rc.bits = nullptr;
+      if constexpr (has_bitmap(MOD)) {
+        if (rc.row < a.Sq) rc.bits = bitmap_row(a.mod, uc.b, uc.h, rc.row);
+      }
 
       float m_run = -INFINITY, l_run = 0.f;
       int n_act = 0;
@@ -529,6 +540,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!(e & act_bit)) continue;
         const int kt = static_cast<int>(e & 0xFFFFFu);
         const bool prt_t = (e & prt_bit) != 0;
+        uint4 bw = make_uint4(0u, 0u, 0u, 0u);  // keep bits of this row's 128 keys (PARTIAL tiles)
+        if constexpr (has_bitmap(MOD)) {
+          if (prt_t && rc.bits != nullptr) bw = __ldg(reinterpret_cast<const uint4*>(rc.bits) + kt);
+        }
         if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->s_full[t]), s_cnt & 1, wc))) { ok = false; break; }
         ++s_cnt;
         ATTN25_TRACE_ONLY(const long long t_tile = clock64(); tr[7] += 1;)
@@ -539,8 +554,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int c = 0; c < 4; ++c)
           tmem_ld32(s_addr + c * 32, reinterpret_cast<uint32_t(&)[32]>(x[c]));
         tmem_wait_ld();
-        const float mx = prt_t ? row_scores<MOD, true>(x, rc, a.mod, k0)
-                               : row_scores<MOD, false>(x, rc, a.mod, k0);
+        const float mx = prt_t ? row_scores<MOD, true>(x, rc, a.mod, k0, bw)
+                               : row_scores<MOD, false>(x, rc, a.mod, k0, bw);
         const float m_new = fmaxf(m_run, mx);
         const bool need = m_new > m_run + kRescaleThreshold;
         if (__any_sync(0xffffffffu, need)) {
@@ -658,7 +673,7 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 template <int D, bool LSE>
 cudaError_t launch_fwd_mod(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            const FwdArgs& a, int key, int grid, cudaStream_t s) {
-  constexpr int M = kKeyMasked;
+  constexpr int M = kKeyMasked, MB = kKeyMasked | kKeyBitmap;
   switch (key) {
     case MOD_NONE: return launch_fwd_t<D, MOD_NONE, LSE>(tq, tk, tv, a, grid, s);
     case MOD_ALIBI: return launch_fwd_t<D, MOD_ALIBI, LSE>(tq, tk, tv, a, grid, s);
@@ -668,6 +683,10 @@ cudaError_t launch_fwd_mod(const CUtensorMap& tq, const CUtensorMap& tk, const C
     case M | MOD_ALIBI: return launch_fwd_t<D, M | MOD_ALIBI, LSE>(tq, tk, tv, a, grid, s);
     case M | MOD_SOFTCAP: return launch_fwd_t<D, M | MOD_SOFTCAP, LSE>(tq, tk, tv, a, grid, s);
     case M | MOD_BOOST: return launch_fwd_t<D, M | MOD_BOOST, LSE>(tq, tk, tv, a, grid, s);
+    case MB | MOD_NONE: return launch_fwd_t<D, MB | MOD_NONE, LSE>(tq, tk, tv, a, grid, s);
+    case MB | MOD_ALIBI: return launch_fwd_t<D, MB | MOD_ALIBI, LSE>(tq, tk, tv, a, grid, s);
+    case MB | MOD_SOFTCAP: return launch_fwd_t<D, MB | MOD_SOFTCAP, LSE>(tq, tk, tv, a, grid, s);
+    case MB | MOD_BOOST: return launch_fwd_t<D, MB | MOD_BOOST, LSE>(tq, tk, tv, a, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -55,6 +55,9 @@ struct MaskArgs {
   int window;    // W (1 << 30 without the window mask)
   const int32_t* doc_offsets;
   int num_docs;
+  const uint32_t* bitmap;  // keep bits (bitmap mask) or nullptr
+  int bm_row_words, bm_heads;
+  long long bm_head_stride, bm_batch_stride;
   int B, Sq, Skv, nQ, nK, nP;
   uint8_t* tile_class;
   int32_t* kv_count;

@@ -33,13 +33,17 @@ constexpr float LN2 = 0.6931471805599453f;
 constexpr int kMaskCausal = 1;
 constexpr int kMaskWindow = 2;
 constexpr int kMaskDoc = 4;
+constexpr int kMaskBitmap = 8;  // a general mask given by its values, one bit per element
 
 // Kernel specialisation key: the score transform (MOD_NONE, MOD_ALIBI,
-// MOD_SOFTCAP or MOD_BOOST) plus kKeyMasked when any mask is present; which
-// masks, and their parameters, are runtime values.
+// MOD_SOFTCAP or MOD_BOOST) plus kKeyMasked when any mask is present, and
+// kKeyBitmap (always with kKeyMasked) when a bitmap mask is; which interval
+// masks, and all parameters, are runtime values.
 constexpr int kKeyMasked = 16;
+constexpr int kKeyBitmap = 32;
 __host__ __device__ constexpr int score_of(int key) { return key & (kKeyMasked - 1); }
 __host__ __device__ constexpr bool masked(int key) { return (key & kKeyMasked) != 0; }
+__host__ __device__ constexpr bool has_bitmap(int key) { return (key & kKeyBitmap) != 0; }
 
 struct ModDev {
   int kind;                 // score transform: MOD_NONE, MOD_ALIBI, MOD_SOFTCAP or MOD_BOOST
@@ -51,7 +55,17 @@ struct ModDev {
   const float* alibi_slopes;  // [Hq] or nullptr (then 2^(-8(h+1)/Hq))
   const int32_t* doc_offsets; // [B][num_docs + 1], nullptr without the document mask
   int num_docs;
+  const uint32_t* bitmap;     // keep bits, nullptr without the bitmap mask
+  int bm_row_words;           // words per query row (a multiple of 4)
+  long long bm_head_stride;   // words between heads (0: shared)
+  long long bm_batch_stride;  // words between batch rows (0: shared)
 };
+
+// First word of query row i of head h, batch row b in the keep bitmap.
+__device__ __forceinline__ const uint32_t* bitmap_row(const ModDev& m, int b, int h, int i) {
+  return m.bitmap + b * m.bm_batch_stride + h * m.bm_head_stride +
+         static_cast<long long>(i) * m.bm_row_words;
+}
 
 // First key of the document that holds position i (offsets ascending, offs[0] = 0).
 __device__ __forceinline__ int doc_start(const int32_t* offs, int num_docs, int i) {
