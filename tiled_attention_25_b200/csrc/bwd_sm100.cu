@@ -389,7 +389,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int unit_iter = 0, step = 0;
       uint32_t kv_loads = 0, stage_uses[4] = {0, 0, 0, 0};
       bool ok = true;
-      for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+      for (int u = snake_unit(0); u < a.n_units && ok; u = snake_unit(++unit_iter)) {
         const BwdUnit un = decode_bwd_unit(a, u);
         const int buf = unit_iter & 1;
         uint16_t* lst = lists + buf * kMaxSteps;
@@ -464,7 +464,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       break;                \
     }                       \
   }
-      for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+      for (int u = snake_unit(0); u < a.n_units && ok; u = snake_unit(++unit_iter)) {
         const int buf = unit_iter & 1;
         MMA_WAIT(mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc) &&
                  ATTN25_TIMED(tr[1], mbar_wait_warp_ool(smem_u32(&bars->kv_full), unit_iter & 1, wc)));
@@ -571,7 +571,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t t_dv = tmem + Cfg::kColDV + lane_off;
     int unit_iter = 0, step = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+    for (int u = snake_unit(0); u < a.n_units && ok; u = snake_unit(++unit_iter)) {
       const BwdUnit un = decode_bwd_unit(a, u);
       const int kv = un.kt * TILE + r;
       int qlo, qhi;
@@ -647,7 +647,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t t_dp = tmem + Cfg::kColDP + lane_off, t_dk = tmem + Cfg::kColDK + lane_off;
     int unit_iter = 0, step = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+    for (int u = snake_unit(0); u < a.n_units && ok; u = snake_unit(++unit_iter)) {
       const BwdUnit un = decode_bwd_unit(a, u);
       const int kv = un.kt * TILE + r;
       const int buf = unit_iter & 1;
@@ -759,7 +759,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ds_ready of step j counts the drain's read of dQ^T(j-1); step 0 has no
     // predecessor, so its share is given up front
     mbar_arrive(smem_u32(&bars->ds_ready[0]));
-    for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+    for (int u = snake_unit(0); u < a.n_units && ok; u = snake_unit(++unit_iter)) {
       const BwdUnit un = decode_bwd_unit(a, u);
       const int buf = unit_iter & 1;
       if (!mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }

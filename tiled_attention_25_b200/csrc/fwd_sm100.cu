@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     int unit_iter = 0;
     uint32_t q_loads = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+    for (int u = snake_unit(0); u < a.n_units && ok; u = snake_unit(++unit_iter)) {
       const UnitCoord uc = decode_unit(a, u);
       const int hk = uc.h / a.G;
       const int buf = unit_iter & 1;
@@ -398,7 +398,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     bool ok = true;
     const uint32_t s_tmem[2] = {tmem, tmem + 128};
     const uint32_t o_tmem[2] = {tmem + 256, tmem + 256 + D};
-    for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+    for (int u = snake_unit(0); u < a.n_units && ok; u = snake_unit(++unit_iter)) {
       const int buf = unit_iter & 1;
       const uint32_t* lst = lists + buf * kMaxSteps;
       if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
@@ -502,7 +502,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     int unit_iter = 0;
     uint32_t o_units = 0;  // units with at least one step seen so far (o_final phases)
     bool ok = true;
-    for (int u = blockIdx.x; u < a.n_units && ok; u += gridDim.x, ++unit_iter) {
+    for (int u = snake_unit(0); u < a.n_units && ok; u = snake_unit(++unit_iter)) {
       const UnitCoord uc = decode_unit(a, u);
       RowCtx rc;
       rc.row = (2 * uc.p + t) * TILE + r;

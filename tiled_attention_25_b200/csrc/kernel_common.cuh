@@ -10,6 +10,21 @@
 
 namespace attn25 {
 
+// ------------------------------------------------------------------ work walk
+//
+// The k-th unit a CTA processes, in the block mask's longest-first order:
+// wave k covers ranks [k G, k G + G) (G = gridDim.x), CTA c takes rank
+// k G + c on even waves and k G + G - 1 - c on odd ones.  Reversing every
+// other wave pairs each CTA's long units with short ones, so per-CTA totals
+// stay level when unit lengths fall steadily (causal, sliding-window and
+// document masks); a plain round-robin gives CTA 0 the longest unit of every
+// wave.  Every role of a CTA computes the same sequence; only the last wave
+// can be partial, so the walk ends at the first rank past the unit count.
+__device__ __forceinline__ int snake_unit(int k) {
+  const int base = k * static_cast<int>(gridDim.x);
+  return (k & 1) ? base + static_cast<int>(gridDim.x - 1 - blockIdx.x) : base + static_cast<int>(blockIdx.x);
+}
+
 // ------------------------------------------------------------------ step lists
 //
 // The TMA warp writes each work unit's list of steps into shared memory once
