@@ -235,8 +235,29 @@ __device__ __forceinline__ float4 lds128(uint32_t addr) {
 
 // One key row of S^T (raw q.k for 64 queries) -> P^T = 2^(x - LSE2) in place;
 // nl2_addr is the shared address of the 64 negated base-2 LSEs.
-// With the bitmap mask, wa / wb hold (lane l) the keep-bit word of query
-// q0 + l / q0 + 32 + l over this warp's 32 keys; bit (key & 31) keeps.
+// Whether query q0 + c is kept for this thread's key on a PARTIAL step: inside
+// the key's query interval and, with the bitmap mask, set in the bitmap.
+// wa / wb hold (lane l) the keep-bit word of query q0 + l / q0 + 32 + l over
+// this warp's 32 keys; bit (key & 31) keeps.  The whole warp must call it.
+template <int MOD>
+__device__ __forceinline__ bool keep_query(int c, int q0, int qlo, int qhi, uint32_t wa, uint32_t wb) {
+  const int qq = q0 + c;
+  bool keep = qq >= qlo && qq <= qhi;
+  if constexpr (has_bitmap(MOD)) {
+    const uint32_t w = __shfl_sync(0xffffffffu, c < 32 ? wa : wb, c & 31);
+    keep = keep && ((w >> (threadIdx.x & 31)) & 1u) != 0u;
+  }
+  return keep;
+}
+
+// The mask runs as a pass of its own after the exponentials (P = 0 where
+// masked, the same as 2^-inf), so that the exponential loop stays one copy
+// for every step and this warp's hot code stays small.  Local boost keeps the
+// mask inside the loop: its per-element radius test leaves no registers for
+// the separate pass.
+template <int MOD>
+constexpr bool kMaskAfterExp = score_of(MOD) != MOD_BOOST;
+
 template <int MOD>
 __device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h, float dq0, int q0,
                                         int qlo, int qhi, bool pred, uint32_t nl2_addr, uint32_t wa,
@@ -270,20 +291,20 @@ __device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h,
       } else {
         v = __ffma2_rn(make_float2(x[c], x[c + 1]), sl2, nl);
       }
-      if (pred) {
-        const int qq = q0 + c;
-        v.x = (qq >= qlo && qq <= qhi) ? v.x : -INFINITY;
-        v.y = (qq + 1 >= qlo && qq + 1 <= qhi) ? v.y : -INFINITY;
-        if constexpr (has_bitmap(MOD)) {
-          const uint32_t key_bit = 1u << (threadIdx.x & 31);
-          const uint32_t w0 = __shfl_sync(0xffffffffu, c < 32 ? wa : wb, c & 31);
-          const uint32_t w1 = __shfl_sync(0xffffffffu, c + 1 < 32 ? wa : wb, (c + 1) & 31);
-          v.x = (w0 & key_bit) ? v.x : -INFINITY;
-          v.y = (w1 & key_bit) ? v.y : -INFINITY;
+      if constexpr (!kMaskAfterExp<MOD>) {
+        if (pred) {
+          v.x = keep_query<MOD>(c, q0, qlo, qhi, wa, wb) ? v.x : -INFINITY;
+          v.y = keep_query<MOD>(c + 1, q0, qlo, qhi, wa, wb) ? v.y : -INFINITY;
         }
       }
-      x[c] = ex2_approx(v.x);  // 0 where masked or on padding rows (-LSE2 = -inf)
+      x[c] = ex2_approx(v.x);  // 0 on padding rows (-LSE2 = -inf)
       x[c + 1] = ex2_approx(v.y);
+    }
+  }
+  if constexpr (kMaskAfterExp<MOD>) {
+    if (pred) {  // PARTIAL steps only
+#pragma unroll
+      for (int c = 0; c < BM; ++c) x[c] = keep_query<MOD>(c, q0, qlo, qhi, wa, wb) ? x[c] : 0.f;
     }
   }
 }
