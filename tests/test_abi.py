@@ -104,3 +104,54 @@ def test_strerror(lib):
     lib.attn_strerror.restype = ctypes.c_char_p
     assert b"timed out" in lib.attn_strerror(-6)
     assert lib.attn_strerror(0) == b"ok"
+
+
+def test_composed_and_bitmap_argument_rules(lib):
+    """Composite mod codes and bitmap fields are validated before any device
+    work: a valid call gets as far as the device lookup (ATTN_ERR_DEVICE here,
+    with no GPU), an invalid one stops at ATTN_ERR_ARG / ATTN_ERR_ALIGN."""
+    import tiled_attention_25_b200.abi as abi
+    P, I = ctypes.c_void_p, ctypes.c_int
+    lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, ctypes.c_float, I, P, P, P]
+    lib.build_block_mask.argtypes = [I, P, I, I, I, P, P]
+    good = ctypes.c_void_p(1 << 32)
+    DEVICE, ARG, ALIGN = -7, -1, -3
+
+    def params(bitmap=1 << 32, row_words=8, heads=1, head_stride=0, batch_stride=0, window=100):
+        return abi.CModParams(50.0, window, 1.1, 128, None, None, 0, ctypes.c_void_p(bitmap), row_words,
+                              heads, head_stride, batch_stride)
+
+    def fwd(mod, mp, Hq=4, Skv=256, bm=None):
+        return lib.attn_fwd(good, good, good, good, None, 1, Hq, 2, 256, Skv, 128, 0.1, mod,
+                            None if mp is None else ctypes.byref(mp), bm, None)
+
+    # composites that need no parameters, or get them
+    assert fwd(0x100 | 2, None) == DEVICE
+    assert fwd(4 | 0x400, params()) == ARG          # document flag without offsets
+    assert fwd(0x200 | 3, params()) == DEVICE       # softcap + window
+    assert fwd(0x200, params(window=0)) == ARG
+    # the bitmap: a block mask is required for attn_fwd
+    assert fwd(0x800, params()) == ARG
+    n = ctypes.c_size_t(1 << 20)
+    m = abi.CBlockMask()
+    assert lib.attn_block_mask_bind(ctypes.c_void_p(1 << 40), n, 1, 256, 256, ctypes.byref(m)) == 0
+    bm = ctypes.byref(m)
+    # build_block_mask checks the bitmap fields
+    build = lambda mod, mp: lib.build_block_mask(mod, ctypes.byref(mp), 1, 256, 256, bm, None)
+    assert build(0x800, params()) == DEVICE
+    assert build(0x800 | 0x100, params(heads=3, head_stride=256 * 8)) == DEVICE
+    assert build(0x800, params(bitmap=(1 << 32) + 4)) == ALIGN
+    assert build(0x800, params(row_words=4)) == ARG           # < ceil(256 / 32)
+    assert build(0x800, params(row_words=10)) == ARG          # not a multiple of 4
+    assert build(0x800, params(heads=0)) == ARG
+    assert build(0x800, params(heads=1, head_stride=64)) == ARG
+    assert build(0x800, params(batch_stride=6)) == ARG
+    assert build(0x800, params(bitmap=0)) == ARG
+    # the mask records the canonical code, which attn_fwd compares with its own
+    m.mod_kind = 0x800 | 0x100       # what building NONE | BITMAP | CAUSAL records
+    assert fwd(1 | 0x800, params(), bm=bm) == DEVICE  # causal kind with the bitmap flag: same mod
+    assert fwd(0x800, params(), bm=bm) == ARG         # another mod
+    # per-head bitmaps must match the call's query heads
+    m.mod_kind = 0x800
+    assert fwd(0x800, params(heads=4, head_stride=256 * 8), bm=bm) == DEVICE
+    assert fwd(0x800, params(heads=3, head_stride=256 * 8), bm=bm) == ARG
