@@ -4,13 +4,16 @@
 // FlexAttention, FlashAttention-4 백엔드 도입으로 성능 최대 3.2배 향상"
 // (섹션별 상세: local_boost and tanh_softcap take the score and the raw
 // q/kv indices; 핵심 요약: ALiBi, sliding window, document masks, and their
-// composition).  A mod is one score transform (none, ALiBi, softcap, local
-// boost) and the AND of any of three masks.  Every mask keeps, for query row
-// i, an interval of keys: causal j <= i; sliding window i - W < j <= i;
-// document: j <= i in i's document.  An intersection of intervals is an
-// interval, so every composed mask keeps one interval [lo(i), hi(i)] per row
-// (and, transposed, one interval of queries per key).  Scores are handled in
-// the base-2 domain: x = s' * log2(e), so that exp(s' - m) = 2^(x - m2).
+// composition, and arbitrary mask functions).  A mod is one score transform
+// (none, ALiBi, softcap, local boost) and the AND of any of four masks.  Three
+// keep, for query row i, an interval of keys: causal j <= i; sliding window
+// i - W < j <= i; document: j <= i in i's document.  An intersection of
+// intervals is an interval, so they keep one interval [lo(i), hi(i)] per row
+// (and, transposed, one interval of queries per key).  The fourth is a bitmap
+// of a general mask's values, read on PARTIAL tiles only.  The kind numbers
+// are those of the C interface; only the score transforms are used here.
+// Scores are handled in the base-2 domain: x = s' * log2(e), so that
+// exp(s' - m) = 2^(x - m2).
 #pragma once
 
 #include <cstdint>
@@ -18,12 +21,9 @@
 namespace attn25 {
 
 constexpr int MOD_NONE = 0;
-constexpr int MOD_CAUSAL = 1;
 constexpr int MOD_ALIBI = 2;
 constexpr int MOD_SOFTCAP = 3;
-constexpr int MOD_WINDOW = 4;
 constexpr int MOD_BOOST = 5;
-constexpr int MOD_DOCUMENT = 6;
 
 constexpr int TILE = 128;
 constexpr float LOG2E = 1.4426950408889634f;
