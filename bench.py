@@ -29,7 +29,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from synth_inputs import (MOD_NAMES, WORKLOADS, bf16_bits_to_f64, draw_workload,  # noqa: E402
-                          mod_params_for, pad_offsets)
+                          mod_params_for, pack_bitmap, pad_offsets)
 
 METRIC = "attention fwd/bwd useful TFLOPS on 1 B200 and % of BF16 tensor peak"
 UNIT = "TFLOP/s"
@@ -172,7 +172,13 @@ def job_throughput(flop_per_rank, world, ms):
 
 def useful_counts(ta, w, mod_name, params):
     mod = MOD_NAMES[mod_name]
-    n = ta.useful_elements(mod, w.B, w.Hq, w.Sq, w.Skv, window=params.window, doc_offsets=params.doc_offsets)
+    if params.bitmap is not None:
+        # a general mask counts its set bits (ANDed with nothing else here),
+        # once per batch row and head that shares it
+        keep = np.asarray(params.bitmap, dtype=bool)
+        n = int(keep.sum()) * (w.B // keep.shape[0]) * (w.Hq // keep.shape[1])
+    else:
+        n = ta.useful_elements(mod, w.B, w.Hq, w.Sq, w.Skv, window=params.window, doc_offsets=params.doc_offsets)
     return n, ta.useful_flops(n, w.D), ta.useful_flops(n, w.D, backward=True)
 
 
@@ -193,8 +199,11 @@ def run_gpu(args, rank, world, local_rank):
     doc_t = None
     if params.doc_offsets is not None:
         doc_t = torch.from_numpy(pad_offsets(params.doc_offsets)[0]).to(dev)
+    bm_t = None
+    if params.bitmap is not None:
+        bm_t = torch.from_numpy(pack_bitmap(params.bitmap)).to(dev)
     dp = ta.ModParams(softcap=params.softcap, window=params.window, boost=params.boost,
-                      boost_radius=params.boost_radius, doc_offsets=doc_t)
+                      boost_radius=params.boost_radius, doc_offsets=doc_t, bitmap=bm_t)
     B, Hq, Hkv, Sq, Skv, D = w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D
     out = torch.empty_like(q)
     lse = torch.empty(B, Hq, Sq, dtype=torch.float32, device=dev)

@@ -12,7 +12,12 @@ Recipe (stated once, used everywhere):
     ``[B][Hq][Sq][D]``, then rounded to bfloat16 (round-to-nearest-even);
   * document lengths for the packed-document workload come from
     ``default_rng(100 + k)``: uniform integers in [512, 4096] until the
-    sequence is filled, the last one truncated to fit.
+    sequence is filled, the last one truncated to fit;
+  * the general (bitmap) mask of workload ``k`` comes from
+    ``default_rng(200 + k)``: each 128 x 128 tile is dropped, kept whole or
+    kept element by element with a density drawn from [0.3, 0.9], with equal
+    odds, and the diagonal is always kept; one mask serves every batch row
+    and head.
 """
 from __future__ import annotations
 
@@ -30,6 +35,11 @@ MOD_SOFTCAP = 3
 MOD_SLIDING_WINDOW = 4
 MOD_LOCAL_BOOST = 5
 MOD_DOCUMENT = 6
+# Mask flags ORed onto a kind to compose mods (the ATTN_MASK_* values).
+MASK_CAUSAL = 0x100
+MASK_SLIDING_WINDOW = 0x200
+MASK_DOCUMENT = 0x400
+MASK_BITMAP = 0x800
 
 MOD_NAMES = {
     "none": MOD_NONE,
@@ -39,6 +49,12 @@ MOD_NAMES = {
     "sliding_window": MOD_SLIDING_WINDOW,
     "local_boost": MOD_LOCAL_BOOST,
     "document": MOD_DOCUMENT,
+    # compositions: a score mod with the AND of masks
+    "alibi+causal": MOD_ALIBI | MASK_CAUSAL,
+    "softcap+sliding_window": MOD_SOFTCAP | MASK_SLIDING_WINDOW,
+    "sliding_window+document": MOD_SLIDING_WINDOW | MASK_DOCUMENT,
+    # a general mask given by its values
+    "bitmap": MOD_NONE | MASK_BITMAP,
 }
 
 
@@ -82,6 +98,9 @@ WORKLOADS = {
     "score_mods": Workload("score_mods", 4, 2, 16, 16, 8192, 8192, 128,
                            ("alibi", "softcap", "sliding_window", "local_boost")),
     "documents": Workload("documents", 5, 1, 16, 16, 32768, 32768, 128, ("document",)),
+    # the composed and general masks on the score-mod shape
+    "composed": Workload("composed", 6, 2, 16, 16, 8192, 8192, 128,
+                         ("alibi+causal", "softcap+sliding_window", "sliding_window+document", "bitmap")),
 }
 
 
@@ -156,10 +175,31 @@ def pad_offsets(offsets_per_b) -> tuple:
     return arr, num_docs
 
 
+def block_bitmap(seed: int, Sq: int, Skv: int) -> np.ndarray:
+    """Bool [1][1][Sq][Skv] general mask: per 128 x 128 tile, dropped, kept, or
+    kept element by element at a random density, with equal odds; the
+    diagonal always kept."""
+    rng = np.random.default_rng(seed)
+    keep = np.zeros((Sq, Skv), dtype=bool)
+    for q0 in range(0, Sq, 128):
+        for k0 in range(0, Skv, 128):
+            kind = int(rng.integers(3))
+            blk = keep[q0:q0 + 128, k0:k0 + 128]
+            if kind == 1:
+                blk[...] = True
+            elif kind == 2:
+                blk[...] = rng.random(blk.shape) < rng.uniform(0.3, 0.9)
+    d = np.arange(min(Sq, Skv))
+    keep[d, d] = True
+    return keep[None, None]
+
+
 def mod_params_for(w: Workload, mod: str) -> ModParams:
     p = ModParams()
-    if mod == "document":
+    if "document" in mod.split("+"):
         p.doc_offsets = doc_offsets_for(w)
+    if mod == "bitmap":
+        p.bitmap = block_bitmap(200 + w.seed, w.Sq, w.Skv)
     return p
 
 
