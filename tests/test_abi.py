@@ -155,3 +155,28 @@ def test_composed_and_bitmap_argument_rules(lib):
     m.mod_kind = 0x800
     assert fwd(0x800, params(heads=4, head_stride=256 * 8), bm=bm) == DEVICE
     assert fwd(0x800, params(heads=3, head_stride=256 * 8), bm=bm) == ARG
+
+
+def test_binding_marshals_bitmap_extents():
+    """The binding turns a bitmap tensor's shape into the C strides, and
+    refuses a tensor that does not cover the call's batch rows, heads and
+    query rows (the C side cannot see its extent)."""
+    import torch
+
+    import tiled_attention_25_b200.abi as abi
+    S, rw = 300, 12
+    for shape, heads, hs, bs in (((1, 1, S, rw), 1, 0, 0), ((2, 1, S, rw), 1, 0, S * rw),
+                                 ((2, 4, S, rw), 4, S * rw, 4 * S * rw)):
+        mp = abi.ModParams(bitmap=torch.zeros(shape, dtype=torch.int32))
+        c = mp.c()
+        assert (c.bitmap_row_words, c.bitmap_heads, c.bitmap_head_stride, c.bitmap_batch_stride) == (rw, heads, hs, bs)
+        assert c.bitmap == mp.bitmap.data_ptr()
+        assert abi._mp(mp, abi.MASK_BITMAP, 2, 4, S) is not None
+    bad = [((3, 1, S, rw), 2, 4, S), ((1, 3, S, rw), 2, 4, S), ((1, 1, S - 1, rw), 2, 4, S)]
+    for shape, B, Hq, Sq in bad:
+        mp = abi.ModParams(bitmap=torch.zeros(shape, dtype=torch.int32))
+        with pytest.raises(ValueError):
+            abi._mp(mp, abi.MASK_BITMAP, B, Hq, Sq)
+    # without the flag the bitmap is not read, so its shape does not matter
+    mp = abi.ModParams(bitmap=torch.zeros((3, 3, 1, rw), dtype=torch.int32))
+    assert abi._mp(mp, abi.MOD_CAUSAL, 2, 4, S) is not None
