@@ -180,3 +180,26 @@ def test_binding_marshals_bitmap_extents():
     # without the flag the bitmap is not read, so its shape does not matter
     mp = abi.ModParams(bitmap=torch.zeros((3, 3, 1, rw), dtype=torch.int32))
     assert abi._mp(mp, abi.MOD_CAUSAL, 2, 4, S) is not None
+
+
+def test_every_mod_code_is_valid_exactly_when_the_oracle_accepts_it(lib):
+    """All 4096 codes below 0x1000: the C boundary and the oracle agree on which
+    are mods.  Parameters are given for every component, so a valid code passes
+    the checks and stops at the device lookup (ATTN_ERR_DEVICE here)."""
+    import oracle
+    import tiled_attention_25_b200.abi as abi
+    P, I = ctypes.c_void_p, ctypes.c_int
+    lib.build_block_mask.argtypes = [I, P, I, I, I, P, P]
+    mp = abi.CModParams(50.0, 100, 1.1, 128, None, ctypes.c_void_p(1 << 32), 2, ctypes.c_void_p(1 << 32),
+                        8, 1, 0, 0)
+    m = abi.CBlockMask()
+    assert lib.attn_block_mask_bind(ctypes.c_void_p(1 << 40), ctypes.c_size_t(1 << 20), 1, 256, 256,
+                                    ctypes.byref(m)) == 0
+    for code in range(0x1000):
+        try:
+            oracle.split_mod(code)
+            valid = True
+        except ValueError:
+            valid = False
+        rc = lib.build_block_mask(code, ctypes.byref(mp), 1, 256, 256, ctypes.byref(m), None)
+        assert rc == (-7 if valid else -1), (hex(code), rc)
