@@ -30,3 +30,10 @@ from .attention import (  # noqa: F401
     useful_flops,
 )
 from .block_sparsity import block_mask, classify_tiles  # noqa: F401
+from .fp8 import (  # noqa: F401
+    attention_forward_fp8,
+    hadamard,
+    quantize_e4m3,
+    quantize_per_head,
+    rotation,
+)

@@ -12,10 +12,12 @@ import pytest
 import oracle
 import oracle.attention as oa
 import oracle.block_sparsity as ob
+import oracle.fp8 as ofp8
 import test_oracle as pins
 import test_oracle_block_mask as bm_pins
 import test_oracle_bitmap as bitmap_pins
 import test_oracle_compose as comp_pins
+import test_oracle_fp8 as fp8_pins
 
 
 def _install(module, func_name, old, new, monkeypatch):
@@ -64,6 +66,13 @@ MUTANTS = [
      comp_pins.test_zero_queries_window_and_documents_count_keys),
     (oa, "score_mod", "_single_mod(s, base, params", "_single_mod(s, masks[0] if masks else base, params",
      comp_pins.test_zero_queries_causal_alibi_geometric_sums),
+    (ofp8, "quantize_e4m3", "q = np.round(a / quantum) * quantum", "q = np.floor(a / quantum + 0.5) * quantum",
+     fp8_pins.test_ties_round_to_even_like_torch),
+    (ofp8, "hadamard", "H = np.block([[H, H], [H, -H]])", "H = np.block([[H, H], [H, H]])",
+     lambda: fp8_pins.test_hadamard_properties(8)),
+    (ofp8, "quantize_per_head", "amax / E4M3_MAX", "amax", fp8_pins.test_on_grid_inputs_give_exact_attention),
+    (ofp8, "attention_forward_fp8", "q, k = q @ R, k @ R", "q, k = q @ R, k",
+     fp8_pins.test_rotation_lowers_the_fp8_error_on_outliers),
     (ob, "classify_tiles", "elif min(counts) == blocks[0].size:", "elif min(counts) == tile * tile:",
      bm_pins.test_single_row_tail_tile_is_full),
     (ob, "classify_tiles", "if max(counts) == 0:", "if min(counts) == 0:",
