@@ -32,7 +32,9 @@ from .attention import (  # noqa: F401
 from .block_sparsity import block_mask, classify_tiles  # noqa: F401
 from .fp8 import (  # noqa: F401
     attention_forward_fp8,
+    fwht,
     hadamard,
+    prep_fp32,
     quantize_e4m3,
     quantize_per_head,
     rotation,

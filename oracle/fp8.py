@@ -75,6 +75,42 @@ def quantize_per_head(x):
     return quantize_e4m3(x / scale[:, :, None, None]), scale
 
 
+def fwht(x):
+    """The fast Walsh-Hadamard transform along the last axis, in the dtype of
+    x: stages h = 1, 2, 4, ..., D/2, each replacing the pair (y[i], y[i + h])
+    of every block of 2h by (y[i] + y[i + h], y[i] - y[i + h]).  Equals
+    x @ hadamard(D) (the Sylvester matrix is symmetric)."""
+    y = np.array(x, copy=True)
+    D = y.shape[-1]
+    if D < 1 or D & (D - 1):
+        raise ValueError("D must be a power of two")
+    h = 1
+    while h < D:
+        y = y.reshape(*y.shape[:-1], D // (2 * h), 2, h)
+        a, b = y[..., 0, :].copy(), y[..., 1, :].copy()
+        y[..., 0, :], y[..., 1, :] = a + b, a - b
+        y = y.reshape(*y.shape[:-3], D)
+        h *= 2
+    return y
+
+
+def prep_fp32(x, signs):
+    """The rotation and per-head quantisation in fp32, one operation at a
+    time, as a kernel computes them: y = fwht(x * signs) * (1 / sqrt(D))
+    (one fp32 product by the fp32 constant), amax per (b, head), scale =
+    amax / 448, codes = e4m3(y / scale) with IEEE fp32 division.  Every
+    step is an exactly rounded fp32 operation, so a kernel that takes the
+    same steps gets the same codes.  Returns (codes as float64, scales)."""
+    x = np.asarray(x, dtype=np.float32)
+    D = x.shape[-1]
+    inv_sqrt_d = np.float32(1.0 / np.sqrt(D))
+    y = fwht(x * np.asarray(signs, dtype=np.float32)) * inv_sqrt_d
+    amax = np.abs(y).max(axis=(2, 3))
+    scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    ratio = (y / scale[:, :, None, None]).astype(np.float32)
+    return quantize_e4m3(ratio.astype(np.float64)), scale.astype(np.float64)
+
+
 def attention_forward_fp8(q, k, v, scale, signs=None, mod=0, params=None, heads=None, rows=None):
     """O and LSE with the scores formed from FP8 Q and K.
 

@@ -143,3 +143,30 @@ def test_outlier_recipe_reproduces_the_printed_gain():
         e_rot = np.sqrt(np.mean((oracle.attention_forward_fp8(q, k, v, scale, signs=signs)[0] - O) ** 2))
         ratios.append(e_plain / e_rot)
     assert 2.0 < np.mean(ratios) < 3.5, ratios
+
+
+@pytest.mark.parametrize("D", [2, 16, 128])
+def test_fwht_is_the_hadamard_product(D):
+    # integer inputs: both sides are exact in fp64
+    x = np.random.default_rng(D).integers(-50, 50, size=(3, D)).astype(np.float64)
+    assert np.array_equal(oracle.fwht(x), x @ oracle.hadamard(D))
+    # and fp32 butterflies stay within rounding of the exact product
+    xf = np.random.default_rng(D + 1).standard_normal((3, D)).astype(np.float32)
+    assert np.allclose(oracle.fwht(xf), xf.astype(np.float64) @ oracle.hadamard(D), rtol=0, atol=1e-5 * D)
+
+
+def test_fp32_prep_agrees_with_the_definition():
+    # the fp32 step sequence quantises to the same codes as the fp64 rotation
+    # except where an fp32 rounding moves a value across a tie
+    q, _, _ = outlier_inputs(20, H=2, S=128)
+    signs = np.where(np.random.default_rng(21).random(128) < 0.5, -1.0, 1.0)
+    codes32, s32 = oracle.prep_fp32(q, signs)
+    codes64, s64 = oracle.quantize_per_head(q @ oracle.rotation(128, signs))
+    assert np.allclose(s32, s64, rtol=1e-6)
+    differ = codes32 != codes64
+    assert differ.mean() < 1e-3
+    # where they differ, they are neighbours on the grid
+    g = e4m3_grid()
+    idx32 = np.searchsorted(g, codes32[differ])
+    idx64 = np.searchsorted(g, codes64[differ])
+    assert np.all(np.abs(idx32 - idx64) == 1)
