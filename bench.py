@@ -288,6 +288,21 @@ def run_gpu(args, rank, world, local_rank):
             e2e_times.append((a0, a1))
     torch.cuda.synchronize()
     ms_e2e = sum(a.elapsed_time(b) for a, b in e2e_times) / max(1, len(e2e_times))
+    e2e_mode = "serial: H2D, step and D2H in one stream, step by step"
+    if args.e2e_pipeline and not args.no_e2e:
+        ms_e2e = e2e_pipelined(args, ta, stream, dev, (q, k, v, dout, out, lse, dq, dk, dv),
+                               (hq, hk, hv, hdo), (ho, hdq, hdk, hdv),
+                               lambda t, s_: (ta.build_block_mask(mod, dp, B, Sq, Skv, mask, s_),
+                                              ta.attn_fwd(t[0], t[1], t[2], t[4], t[5], scale=w.scale, mod_kind=mod,
+                                                          mod_params=dp, block_mask=mask, stream=s_),
+                                              ta.attn_bwd(t[0], t[1], t[2], t[4], t[5], t[3], t[6], t[7], t[8], ws,
+                                                          scale=w.scale, mod_kind=mod, mod_params=dp,
+                                                          block_mask=mask, stream=s_)))
+        e2e_mode = ("pipelined: H2D, step and D2H on three streams with two device buffer sets, so that "
+                    "step i's compute overlaps step i+1's H2D and step i-1's D2H (every copy still timed)")
+        st = ta.attn_get_status(stream)
+        if st != 0:
+            raise RuntimeError(f"kernel status {st} in the pipelined end-to-end pass")
     ms_e2e = max_over_ranks([ms_e2e], world, dev)[0]
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v, dout))
     d2h = sum(t.numel() * t.element_size() for t in (out, dq, dk, dv))
@@ -336,13 +351,60 @@ def run_gpu(args, rank, world, local_rank):
         "roofline_forward": roof(fwd_tf, traffic_fwd),
         "roofline_backward": roof(bwd_tf, traffic_bwd),
         "e2e": None if args.no_e2e else {"value": round(job_throughput(f_fwd + f_bwd, world, ms_e2e), 2), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4)},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4),
+                "mode": e2e_mode},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, mod_name, params, seconds=args.cpu_seconds)
     return line
+
+
+def e2e_pipelined(args, ta, stream, dev, dev_set, host_in, host_out, run_step):
+    """End-to-end time per step with the copies overlapped across steps.
+
+    Two device buffer sets alternate.  Step i uploads its inputs into set
+    i % 2 on an upload stream (after step i-2's compute has read that set),
+    computes on `stream` (after its upload, and after step i-2's outputs in
+    that set were read back), and downloads its outputs on a download stream.
+    Returns the time from the first timed upload to the last timed download,
+    divided by the number of timed steps."""
+    import torch
+    names = ("q", "k", "v", "dout", "out", "lse", "dq", "dk", "dv")
+    sets = [dict(zip(names, dev_set)), {n: torch.empty_like(t) for n, t in zip(names, dev_set)}]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    computed, read_back = [None, None], [None, None]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    for i in range(args.warmup + args.steps):
+        b = sets[i & 1]
+        if computed[i & 1] is not None:
+            s_in.wait_event(computed[i & 1])
+        if i == args.warmup:
+            start.record(s_in)
+        with torch.cuda.stream(s_in):
+            for name, h_ in zip(("q", "k", "v", "dout"), host_in):
+                b[name].copy_(h_, non_blocking=True)
+        uploaded = torch.cuda.Event()
+        uploaded.record(s_in)
+        stream.wait_event(uploaded)
+        if read_back[i & 1] is not None:
+            stream.wait_event(read_back[i & 1])
+        run_step(tuple(b[n] for n in names), stream)
+        done = torch.cuda.Event()
+        done.record(stream)
+        computed[i & 1] = done
+        s_out.wait_event(done)
+        with torch.cuda.stream(s_out):
+            for h_, name in zip(host_out, ("out", "dq", "dk", "dv")):
+                h_.copy_(b[name], non_blocking=True)
+        got = torch.cuda.Event()
+        got.record(s_out)
+        read_back[i & 1] = got
+    end.record(s_out)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / args.steps
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) arm
@@ -412,6 +474,8 @@ def main():
     ap.add_argument("--all", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
+    ap.add_argument("--e2e-pipeline", action="store_true",
+                    help="overlap each step's H2D and D2H with the neighbouring steps' compute")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     if args.warmup < 3:
