@@ -289,7 +289,7 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
     ms_e2e = sum(a.elapsed_time(b) for a, b in e2e_times) / max(1, len(e2e_times))
     e2e_mode = "serial: H2D, step and D2H in one stream, step by step"
-    if args.e2e_pipeline and not args.no_e2e:
+    if getattr(args, "e2e_pipeline", False) and not args.no_e2e:
         ms_e2e = e2e_pipelined(args, ta, stream, dev, (q, k, v, dout, out, lse, dq, dk, dv),
                                (hq, hk, hv, hdo), (ho, hdq, hdk, hdv),
                                lambda t, s_: (ta.build_block_mask(mod, dp, B, Sq, Skv, mask, s_),
