@@ -23,7 +23,7 @@ What it computes (the plain definition, no tiling, no online softmax):
   the plainest reading is the exact gradient of O with respect to Q, K, V,
   written out below.
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
   * mods see ``scale * q.k``; the mask is applied after the mod;
   * causal uses absolute indices, keep ``kv <= q``;
   * sliding window keeps ``0 <= q - kv < W``;

@@ -9,7 +9,7 @@ orthogonal matrix such as a Hadamard matrix; the rotation spreads
 outlier coordinates over all coordinates, so that quantising to FP8 loses
 less; and, the rotation being orthogonal, it cancels in Q K^T.  The pages
 fix neither the FP8 format's details nor the scale granularity nor whether
-V and P are quantised too.  Readings (also listed in the design doc):
+V and P are quantised too.  Readings:
 
 * the rotation is R = diag(sigma) H_D / sqrt(D): H_D the Sylvester Hadamard
   matrix of order D (a power of two), sigma a vector of D random signs
