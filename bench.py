@@ -7,7 +7,7 @@ drawn N(0,1) from a fixed seed.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME[:MOD]]
     python bench.py --impl reference ...   # the fp64 CPU oracle, timed on the host
-    python bench.py --all                  # one line per workload/mod (not the default line)
+    python bench.py --all                  # one line per workload and mod
 
 Prints one JSON line (rank 0).  Throughput counts only unmasked score
 elements: 4 D flop each forward, 10 D backward.
