@@ -16,6 +16,7 @@ from .attention import (  # noqa: F401
     MASK_CAUSAL,
     MASK_DOCUMENT,
     MASK_SLIDING_WINDOW,
+    MASK_VARLEN,
     has_bitmap,
     has_document,
     has_mask,

@@ -42,7 +42,13 @@ Readings where the pages are silent:
   * a general mask_mod ("PyTorch FlexAttention, …", 핵심 요약: arbitrary
     mask functions) is given as its values: ``MASK_BITMAP`` keeps (b, h, i, j)
     where ``params.bitmap[b', h', i, j]`` is true, with b' = b and h' = h, or 0
-    where the array's batch or head extent is 1 (shared by all).
+    where the array's batch or head extent is 1 (shared by all);
+  * packed variable-length sequences with their own query and key lengths
+    (the pages' separate query and key lengths, "FlashInfer SM120 NVFP4 …",
+    코드 분석 1-2): ``MASK_VARLEN`` keeps (i, j) where query i and key j
+    belong to the same sequence d, i.e. q_offsets[b][d] <= i < q_offsets[b][d+1]
+    and k_offsets[b][d] <= j < k_offsets[b][d+1]; it is not causal (a causal
+    packing with equal lengths is the document mask) and takes no other mask.
 """
 from __future__ import annotations
 
@@ -61,17 +67,23 @@ MASK_CAUSAL = 0x100
 MASK_SLIDING_WINDOW = 0x200
 MASK_DOCUMENT = 0x400
 MASK_BITMAP = 0x800
-_BITMAP = 0x100  # pseudo-kind of the bitmap mask (never a base kind)
+MASK_VARLEN = 0x1000
+_BITMAP = 0x100  # pseudo-kinds of the bitmap and varlen masks (never base kinds)
+_VARLEN = 0x101
 _FLAG_KIND = ((MASK_CAUSAL, MOD_CAUSAL), (MASK_SLIDING_WINDOW, MOD_SLIDING_WINDOW),
-              (MASK_DOCUMENT, MOD_DOCUMENT), (MASK_BITMAP, _BITMAP))
+              (MASK_DOCUMENT, MOD_DOCUMENT), (MASK_BITMAP, _BITMAP), (MASK_VARLEN, _VARLEN))
 
 
 def split_mod(mod):
     """(base kind, [mask kinds of the flags]) of a mod code; rejects unknown bits."""
     base, flags = int(mod) & 0xFF, int(mod) & ~0xFF
-    if base > MOD_DOCUMENT or flags & ~(MASK_CAUSAL | MASK_SLIDING_WINDOW | MASK_DOCUMENT | MASK_BITMAP):
+    if base > MOD_DOCUMENT or flags & ~(MASK_CAUSAL | MASK_SLIDING_WINDOW | MASK_DOCUMENT | MASK_BITMAP |
+                                        MASK_VARLEN):
         raise ValueError(f"unknown mod {mod:#x}")
-    return base, [kind for flag, kind in _FLAG_KIND if flags & flag]
+    masks = [kind for flag, kind in _FLAG_KIND if flags & flag]
+    if _VARLEN in masks and (len(masks) > 1 or base in (MOD_CAUSAL, MOD_SLIDING_WINDOW, MOD_DOCUMENT)):
+        raise ValueError(f"the varlen mask takes no other mask: {mod:#x}")
+    return base, masks
 
 
 def has_mask(mod) -> bool:
@@ -142,6 +154,16 @@ def _single_mod(s, mod, params, b, h, Hq, qi, kj):
         inside = np.abs(qi - kj) < params.boost_radius
         s_mod = np.where(inside, s * params.boost, s)
         dmod = np.where(inside, params.boost, 1.0) * np.ones_like(s)
+    elif mod == _VARLEN:
+        qo, ko = params.q_offsets[b], params.k_offsets[b]
+        # sequence index of every query and key; positions past the last
+        # offset belong to no sequence (-1 for queries, -2 for keys)
+        seq_q = np.full(max(int(qi.max(initial=0)) + 1, qo[-1]), -1, dtype=np.int64)
+        seq_k = np.full(max(int(kj.max(initial=0)) + 1, ko[-1]), -2, dtype=np.int64)
+        for d in range(len(qo) - 1):
+            seq_q[qo[d]:qo[d + 1]] = d
+            seq_k[ko[d]:ko[d + 1]] = d
+        keep = seq_q[qi] == seq_k[kj]
     elif mod == _BITMAP:
         bm = np.asarray(params.bitmap, dtype=bool)
         keep = bm[b if bm.shape[0] > 1 else 0, h if bm.shape[1] > 1 else 0][qi, kj]

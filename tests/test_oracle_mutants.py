@@ -18,6 +18,7 @@ import test_oracle_block_mask as bm_pins
 import test_oracle_bitmap as bitmap_pins
 import test_oracle_compose as comp_pins
 import test_oracle_fp8 as fp8_pins
+import test_oracle_varlen as varlen_pins
 
 
 def _install(module, func_name, old, new, monkeypatch):
@@ -73,6 +74,8 @@ MUTANTS = [
     (ofp8, "quantize_per_head", "amax / E4M3_MAX", "amax", fp8_pins.test_on_grid_inputs_give_exact_attention),
     (ofp8, "attention_forward_fp8", "q, k = q @ R, k @ R", "q, k = q @ R, k",
      fp8_pins.test_rotation_lowers_the_fp8_error_on_outliers),
+    (oa, "_single_mod", "seq_k[ko[d]:ko[d + 1]] = d", "seq_k[qo[d]:qo[d + 1]] = d",
+     lambda: varlen_pins.test_sequences_are_independent_problems(oa.MOD_NONE | oa.MASK_VARLEN)),
     (ob, "classify_tiles", "elif min(counts) == blocks[0].size:", "elif min(counts) == tile * tile:",
      bm_pins.test_single_row_tail_tile_is_full),
     (ob, "classify_tiles", "if max(counts) == 0:", "if min(counts) == 0:",
