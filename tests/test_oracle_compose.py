@@ -33,7 +33,7 @@ def params(S, window=4, radius=2, boost=1.3, softcap=1.5, docs=None, B=1):
 def test_split_mod():
     assert oracle.split_mod(MOD_ALIBI | MASK_CAUSAL | MASK_DOCUMENT) == (MOD_ALIBI, [MOD_CAUSAL, MOD_DOCUMENT])
     assert oracle.split_mod(MOD_SLIDING_WINDOW) == (MOD_SLIDING_WINDOW, [])
-    for bad in (7, 0x1000 | MOD_NONE, 0x2000):
+    for bad in (7, 0x2000 | MOD_NONE, 0x4000):
         with pytest.raises(ValueError):
             oracle.split_mod(bad)
     assert oracle.has_mask(MOD_SOFTCAP | MASK_CAUSAL) and not oracle.has_mask(MOD_SOFTCAP)
