@@ -265,6 +265,8 @@ def run_gpu(args, rank, world, local_rank):
     ms_bwd = sum(t_bwd) / len(t_bwd)
     ms_mask = sum(t_mask) / len(t_mask)
     ms_step, ms_fwd, ms_bwd, ms_mask = max_over_ranks([ms_step, ms_fwd, ms_bwd, ms_mask], world, dev)
+    # the spread of the per-step times (each the slowest rank's)
+    ms_step_median, ms_step_min = max_over_ranks([statistics.median(t_step), min(t_step)], world, dev)
 
     # end-to-end through the same API with pinned host buffers: H2D of the
     # step's inputs, the step, D2H of its results (O, dQ, dK, dV)
@@ -329,6 +331,8 @@ def run_gpu(args, rank, world, local_rank):
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(ms_step, 4),
+        "ms_per_step_median": round(ms_step_median, 4),
+        "ms_per_step_min": round(ms_step_min, 4),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
