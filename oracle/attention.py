@@ -28,7 +28,8 @@ Readings where the pages are silent:
   * causal uses absolute indices, keep ``kv <= q``;
   * sliding window keeps ``0 <= q - kv < W``;
   * ALiBi bias ``-slope_h * |q - kv|`` with ``slope_h = 2^(-8 (h+1) / Hq)``,
-    h counted from 0, on both sides of the diagonal;
+    h counted from 0, on both sides of the diagonal, or the caller's slopes
+    (``params.alibi_slopes[h]``) when given;
   * local boost multiplies by ``boost`` where ``|q - kv| < radius``;
   * document mask keeps ``doc(q) == doc(kv) and kv <= q``;
   * GQA: query head ``h`` reads KV head ``h // (Hq // Hkv)``;
@@ -141,7 +142,9 @@ def _single_mod(s, mod, params, b, h, Hq, qi, kj):
     elif mod == MOD_CAUSAL:
         keep = kj <= qi
     elif mod == MOD_ALIBI:
-        s_mod = s - alibi_slope(h, Hq) * np.abs(qi - kj)
+        slopes = getattr(params, "alibi_slopes", None) if params is not None else None
+        slope = alibi_slope(h, Hq) if slopes is None else float(slopes[h])
+        s_mod = s - slope * np.abs(qi - kj)
     elif mod == MOD_SOFTCAP:
         c = params.softcap
         t = np.tanh(s / c)

@@ -70,6 +70,8 @@ class ModParams:
     doc_offsets: list | None = None
     # general mask values: bool [B or 1][H or 1][Sq][Skv], True = keep
     bitmap: np.ndarray | None = None
+    # ALiBi slopes per query head, or None for 2^(-8 (h + 1) / Hq)
+    alibi_slopes: list | None = None
     # packed sequences with their own query and key lengths: per batch row,
     # ascending query and key start offsets plus the ends (Sq, Skv)
     q_offsets: list | None = None

@@ -322,3 +322,24 @@ def test_backward_contributing_rows_under_causal_mask():
     assert np.allclose(part[1][0, 0, kv], full[1][0, 0, kv], atol=1e-13)
     assert np.allclose(part[2][0, 0, kv], full[2][0, 0, kv], atol=1e-13)
     assert np.allclose(part[0][0, :, kv], full[0][0, :, kv], atol=1e-13)
+
+
+def test_alibi_with_given_slopes():
+    # the default slopes given explicitly reproduce the default; a zero slope
+    # removes the bias; Q = 0 gives the geometric sums of each given slope
+    B, H, S, D = 1, 3, 15, 4
+    q, k, v = rand((B, H, S, D), 60), rand((B, H, S, D), 61), rand((B, H, S, D), 62)
+    default = [2.0 ** (-8.0 * (h + 1) / H) for h in range(H)]
+    a = oracle.attention_forward(q, k, v, 0.5, MOD_ALIBI, ModParams())
+    b = oracle.attention_forward(q, k, v, 0.5, MOD_ALIBI, ModParams(alibi_slopes=default))
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    z = oracle.attention_forward(q, k, v, 0.5, MOD_ALIBI, ModParams(alibi_slopes=[0.0] * H))
+    n = oracle.attention_forward(q, k, v, 0.5, MOD_NONE)
+    assert np.allclose(z[0], n[0], atol=1e-14) and np.allclose(z[1], n[1], atol=1e-14)
+    slopes = [0.3, 1.7, 0.05]
+    _, L = oracle.attention_forward(np.zeros_like(q), k, v, 1.0, MOD_ALIBI, ModParams(alibi_slopes=slopes))
+    for h, sl in enumerate(slopes):
+        r = math.exp(-sl)
+        for i in range(S):
+            total = (1 - r ** (i + 1)) / (1 - r) + r * (1 - r ** (S - 1 - i)) / (1 - r)
+            assert abs(L[0, h, i] - math.log(total)) < 1e-12
