@@ -38,7 +38,7 @@ MUTANTS = [
     # (module, function, original text, planted mistake, pin that must fail)
     (oa, "attention_forward", "s = scale * (q[b, h, r] @ k[b, hk].T)", "s = (q[b, h, r] @ k[b, hk].T)",
      lambda: pins.test_matches_torch_sdpa_float64(False)),
-    (oa, "_single_mod", "s_mod = s - alibi_slope(h, Hq) * np.abs(qi - kj)", "s_mod = s + alibi_slope(h, Hq) * np.abs(qi - kj)",
+    (oa, "_single_mod", "s_mod = s - slope * np.abs(qi - kj)", "s_mod = s + slope * np.abs(qi - kj)",
      pins.test_zero_queries_alibi_geometric_sums),
     (oa, "alibi_slope", "(h + 1)", "h", pins.test_zero_queries_alibi_geometric_sums),
     (oa, "_single_mod", "keep = kj <= qi", "keep = kj < qi", pins.test_causal_first_query_attends_key0),
