@@ -282,8 +282,8 @@ __device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h,
         v.x = fmaf(x[c], a.sl2, -aux * fabsf(dq0 + static_cast<float>(c))) + nl.x;
         v.y = fmaf(x[c + 1], a.sl2, -aux * fabsf(dq0 + static_cast<float>(c + 1))) + nl.y;
       } else if constexpr (score_of(MOD) == MOD_SOFTCAP) {
-        v.x = fmaf(aux2, tanhf(x[c] * aux), nl.x);
-        v.y = fmaf(aux2, tanhf(x[c + 1] * aux), nl.y);
+        v.x = fmaf(aux2, tanh_ex2(x[c] * aux), nl.x);
+        v.y = fmaf(aux2, tanh_ex2(x[c + 1] * aux), nl.y);
       } else if constexpr (score_of(MOD) == MOD_BOOST) {
         const float r = static_cast<float>(a.mod.boost_radius);
         v.x = fmaf(x[c], fabsf(dq0 + static_cast<float>(c)) < r ? aux : a.sl2, nl.x);

@@ -137,7 +137,7 @@ __device__ __forceinline__ void transform32(float (&x)[32], const RowCtx& r, con
     if constexpr (score_of(MOD) == MOD_ALIBI) {
       v = fmaf(v, r.sl2, -r.aux * fabsf(di - static_cast<float>(c)));
     } else if constexpr (score_of(MOD) == MOD_SOFTCAP) {
-      v = r.aux2 * tanhf(v * r.aux);
+      v = r.aux2 * tanh_ex2(v * r.aux);
     } else if constexpr (score_of(MOD) == MOD_BOOST) {
       const bool inside = fabsf(di - static_cast<float>(c)) < static_cast<float>(md.boost_radius);
       v = v * (inside ? r.aux : r.sl2);
