@@ -184,69 +184,93 @@ def useful_counts(ta, w, mod_name, params):
 
 # ----------------------------------------------------------------------------- GPU arm
 
-def run_gpu(args, rank, world, local_rank):
+# The parity configurations that get their own entry in the bench line
+# (workload:mod), beside the headline workload.
+CONFIG_ENTRIES = ("dense:causal", "gqa_long:causal", "score_mods:alibi", "score_mods:softcap",
+                  "score_mods:sliding_window", "score_mods:local_boost", "documents:document")
+
+
+class Problem:
+    """One workload's device tensors, mod parameters and block mask."""
+
+    def __init__(self, ta, spec, rank, dev):
+        import torch
+        self.w, self.mod_name = parse_workload(spec)
+        w = self.w
+        self.mod = MOD_NAMES[self.mod_name]
+        self.params = mod_params_for(w, self.mod_name)   # same structure (and flops) on every rank
+        bits = draw_workload(rank_workload(w, rank))
+        to_dev = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
+        self.q, self.k, self.v, self.dout = (to_dev(bits[n]) for n in ("q", "k", "v", "dout"))
+        del bits
+        doc_t = None
+        if self.params.doc_offsets is not None:
+            doc_t = torch.from_numpy(pad_offsets(self.params.doc_offsets)[0]).to(dev)
+        bm_t = None
+        if self.params.bitmap is not None:
+            bm_t = torch.from_numpy(pack_bitmap(self.params.bitmap)).to(dev)
+        p = self.params
+        self.dp = ta.ModParams(softcap=p.softcap, window=p.window, boost=p.boost,
+                               boost_radius=p.boost_radius, doc_offsets=doc_t, bitmap=bm_t)
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty(w.B, w.Hq, w.Sq, dtype=torch.float32, device=dev)
+        self.dq, self.dk, self.dv = torch.empty_like(self.q), torch.empty_like(self.k), torch.empty_like(self.v)
+        self.ws = ta.new_bwd_workspace(w.B, w.Hq, w.Sq, w.D, device=dev)
+        nbytes = ta.attn_block_mask_bytes(w.B, w.Sq, w.Skv)
+        mbuf = torch.empty(nbytes + 256, dtype=torch.uint8, device=dev)
+        off = (-mbuf.data_ptr()) % 256
+        self.mask = ta.attn_block_mask_bind(mbuf[off:off + nbytes], w.B, w.Sq, w.Skv)
+        self.ta = ta
+
+    def block_mask(self, stream):
+        w = self.w
+        self.ta.build_block_mask(self.mod, self.dp, w.B, w.Sq, w.Skv, self.mask, stream)
+
+    def forward(self, stream, with_lse=True):
+        self.ta.attn_fwd(self.q, self.k, self.v, self.out, self.lse if with_lse else None, scale=self.w.scale,
+                         mod_kind=self.mod, mod_params=self.dp, block_mask=self.mask, stream=stream)
+
+    def backward(self, stream):
+        self.ta.attn_bwd(self.q, self.k, self.v, self.out, self.lse, self.dout, self.dq, self.dk, self.dv,
+                         self.ws, scale=self.w.scale, mod_kind=self.mod, mod_params=self.dp,
+                         block_mask=self.mask, stream=stream)
+
+
+def time_steps(ta, pb, stream, flush, steps, warmup, world, dev, fwd_lse=True, with_bwd=True):
+    """Device time of `steps` steps (block mask, forward, backward) after
+    `warmup` untimed ones, L2 flushed before each; CUDA events on the launch
+    stream; per-step times reduced with the maximum over ranks.  Returns the
+    per-phase means and the clock record of the timed region."""
     import torch
-    import tiled_attention_25_b200 as ta
-
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    w, mod_name = parse_workload(args.workload)
-    mod = MOD_NAMES[mod_name]
-    params = mod_params_for(w, mod_name)   # same structure (and flops) on every rank
-    bits = draw_workload(rank_workload(w, rank))
-    to_dev = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
-    q, k, v, dout = (to_dev(bits[n]) for n in ("q", "k", "v", "dout"))
-    doc_t = None
-    if params.doc_offsets is not None:
-        doc_t = torch.from_numpy(pad_offsets(params.doc_offsets)[0]).to(dev)
-    bm_t = None
-    if params.bitmap is not None:
-        bm_t = torch.from_numpy(pack_bitmap(params.bitmap)).to(dev)
-    dp = ta.ModParams(softcap=params.softcap, window=params.window, boost=params.boost,
-                      boost_radius=params.boost_radius, doc_offsets=doc_t, bitmap=bm_t)
-    B, Hq, Hkv, Sq, Skv, D = w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D
-    out = torch.empty_like(q)
-    lse = torch.empty(B, Hq, Sq, dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = ta.new_bwd_workspace(B, Hq, Sq, D, device=dev)
-    nbytes = ta.attn_block_mask_bytes(B, Sq, Skv)
-    mbuf = torch.empty(nbytes + 256, dtype=torch.uint8, device=dev)
-    off = (-mbuf.data_ptr()) % 256
-    mask = ta.attn_block_mask_bind(mbuf[off:off + nbytes], B, Sq, Skv)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    launches_per_step = 3 + 1 + 3  # block mask (3), forward (1), backward (3)
-
     ev = lambda: torch.cuda.Event(enable_timing=True)
 
     def step(times):
         e0, e1, e2, e3 = ev(), ev(), ev(), ev()
         e0.record(stream)
-        ta.build_block_mask(mod, dp, B, Sq, Skv, mask, stream)
+        pb.block_mask(stream)
         e1.record(stream)
-        ta.attn_fwd(q, k, v, out, lse, scale=w.scale, mod_kind=mod, mod_params=dp, block_mask=mask, stream=stream)
+        pb.forward(stream, fwd_lse)
         e2.record(stream)
-        ta.attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, ws, scale=w.scale, mod_kind=mod, mod_params=dp,
-                    block_mask=mask, stream=stream)
+        if with_bwd:
+            pb.backward(stream)
         e3.record(stream)
         times.append((e0, e1, e2, e3))
 
     warm = []
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         flush.fill_(1.0)
         step(warm)
     torch.cuda.synchronize()
     st = ta.attn_get_status(stream)
     if st != 0:
         raise RuntimeError(f"kernel status {st} during warm-up")
-
-    sampler = ClockSampler(local_rank)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
     sampler.start()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     times = []
-    for _ in range(args.steps):
+    for _ in range(steps):
         flush.fill_(1.0)  # L2 flush between steps (outside the timed events)
         step(times)
     torch.cuda.synchronize()
@@ -256,25 +280,78 @@ def run_gpu(args, rank, world, local_rank):
     st = ta.attn_get_status(stream)
     if st != 0:
         raise RuntimeError(f"kernel status {st} in the timed region")
-    t_mask = [a.elapsed_time(b) for a, b, _, _ in times]
-    t_fwd = [b.elapsed_time(c) for _, b, c, _ in times]
-    t_bwd = [c.elapsed_time(d) for _, _, c, d in times]
-    t_step = [a.elapsed_time(d) for a, _, _, d in times]
-    ms_step = sum(t_step) / len(t_step)
-    ms_fwd = sum(t_fwd) / len(t_fwd)
-    ms_bwd = sum(t_bwd) / len(t_bwd)
-    ms_mask = sum(t_mask) / len(t_mask)
-    ms_step, ms_fwd, ms_bwd, ms_mask = max_over_ranks([ms_step, ms_fwd, ms_bwd, ms_mask], world, dev)
-    # the spread of the per-step times (each the slowest rank's)
-    ms_step_median, ms_step_min = max_over_ranks([statistics.median(t_step), min(t_step)], world, dev)
+    # each step's time is the slowest rank's; means, median and minimum follow
+    t_mask = max_over_ranks([a.elapsed_time(b) for a, b, _, _ in times], world, dev)
+    t_fwd = max_over_ranks([b.elapsed_time(c) for _, b, c, _ in times], world, dev)
+    t_bwd = max_over_ranks([c.elapsed_time(d) for _, _, c, d in times], world, dev)
+    t_step = max_over_ranks([a.elapsed_time(d) for a, _, _, d in times], world, dev)
+    mean = lambda x: sum(x) / len(x)
+    return {"ms_step": mean(t_step), "ms_fwd": mean(t_fwd), "ms_bwd": mean(t_bwd), "ms_mask": mean(t_mask),
+            "ms_step_median": statistics.median(t_step), "ms_step_min": min(t_step), "clocks": clocks}
+
+
+def config_entry(ta, spec, rank, world, dev, stream, flush, steps, warmup, peak):
+    """Forward and backward useful TFLOP/s of one parity configuration, timed
+    like the headline (own clock record)."""
+    import torch
+    pb = Problem(ta, spec, rank, dev)
+    t = time_steps(ta, pb, stream, flush, steps, warmup, world, dev)
+    n_u, f_fwd, f_bwd = useful_counts(ta, pb.w, pb.mod_name, pb.params)
+    fwd_tf = f_fwd / (t["ms_fwd"] * 1e-3) / 1e12
+    bwd_tf = f_bwd / (t["ms_bwd"] * 1e-3) / 1e12
+    w = pb.w
+    entry = {"shape": f"B={w.B} Hq={w.Hq} Hkv={w.Hkv} S={w.Sq} D={w.D}", "mod": pb.mod_name,
+             "useful_elements": n_u, "steps": steps, "warmup": warmup,
+             "ms_fwd": round(t["ms_fwd"], 4), "ms_bwd": round(t["ms_bwd"], 4),
+             "ms_block_mask": round(t["ms_mask"], 4),
+             "fwd_tflops": round(fwd_tf, 1), "bwd_tflops": round(bwd_tf, 1),
+             "fwd_frac_of_peak": round(fwd_tf / peak, 4), "bwd_frac_of_peak": round(bwd_tf / peak, 4),
+             "step_tflops": round(job_throughput(f_fwd + f_bwd, world, t["ms_step"]), 1),
+             "clocks": t["clocks"]}
+    del pb
+    torch.cuda.empty_cache()
+    return entry
+
+
+def forward_only_entry(ta, pb, stream, flush, steps, warmup, world, dev, peak, with_lse):
+    """The forward alone (block mask + forward, no backward), with or without
+    the LSE output."""
+    t = time_steps(ta, pb, stream, flush, steps, warmup, world, dev, fwd_lse=with_lse, with_bwd=False)
+    n_u, f_fwd, _ = useful_counts(ta, pb.w, pb.mod_name, pb.params)
+    fwd_tf = f_fwd / (t["ms_fwd"] * 1e-3) / 1e12
+    w = pb.w
+    return {"shape": f"B={w.B} Hq={w.Hq} Hkv={w.Hkv} S={w.Sq} D={w.D}", "mod": pb.mod_name,
+            "lse": with_lse, "useful_elements": n_u, "steps": steps, "warmup": warmup,
+            "ms_fwd": round(t["ms_fwd"], 4), "fwd_tflops": round(fwd_tf, 1),
+            "fwd_frac_of_peak": round(fwd_tf / peak, 4), "clocks": t["clocks"]}
+
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import tiled_attention_25_b200 as ta
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    pb = Problem(ta, args.workload, rank, dev)
+    w, mod_name, params = pb.w, pb.mod_name, pb.params
+    B, Hq, Hkv, Sq, Skv, D = w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 3 + 1 + 3  # block mask (3), forward (1), backward (3)
+
+    t = time_steps(ta, pb, stream, flush, args.steps, args.warmup, world, dev)
+    ms_step, ms_fwd, ms_bwd, ms_mask = t["ms_step"], t["ms_fwd"], t["ms_bwd"], t["ms_mask"]
+    clocks = t["clocks"]
 
     # end-to-end through the same API with pinned host buffers: H2D of the
     # step's inputs, the step, D2H of its results (O, dQ, dK, dV)
+    q, k, v, dout, out, lse, dq, dk, dv = pb.q, pb.k, pb.v, pb.dout, pb.out, pb.lse, pb.dq, pb.dk, pb.dv
+    ev = lambda: torch.cuda.Event(enable_timing=True)
     if args.no_e2e:
         hq = None
     else:
-        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, dout))
-    ho, hdq, hdk, hdv = (torch.empty_like(t, device="cpu").pin_memory() for t in (out, dq, dk, dv))
+        hq, hk, hv, hdo = (t_.cpu().pin_memory() for t_ in (q, k, v, dout))
+    ho, hdq, hdk, hdv = (torch.empty_like(t_, device="cpu").pin_memory() for t_ in (out, dq, dk, dv))
     e2e_times = []
     for i in range(0 if args.no_e2e else args.warmup + args.steps):
         flush.fill_(1.0)
@@ -282,7 +359,9 @@ def run_gpu(args, rank, world, local_rank):
         a0.record(stream)
         for d_, h_ in ((q, hq), (k, hk), (v, hv), (dout, hdo)):
             d_.copy_(h_, non_blocking=True)
-        step([])
+        pb.block_mask(stream)
+        pb.forward(stream)
+        pb.backward(stream)
         for h_, d_ in ((ho, out), (hdq, dq), (hdk, dk), (hdv, dv)):
             h_.copy_(d_, non_blocking=True)
         a1.record(stream)
@@ -292,22 +371,23 @@ def run_gpu(args, rank, world, local_rank):
     ms_e2e = sum(a.elapsed_time(b) for a, b in e2e_times) / max(1, len(e2e_times))
     e2e_mode = "serial: H2D, step and D2H in one stream, step by step"
     if getattr(args, "e2e_pipeline", False) and not args.no_e2e:
+        mod, dp, mask, ws = pb.mod, pb.dp, pb.mask, pb.ws
         ms_e2e = e2e_pipelined(args, ta, stream, dev, (q, k, v, dout, out, lse, dq, dk, dv),
                                (hq, hk, hv, hdo), (ho, hdq, hdk, hdv),
-                               lambda t, s_: (ta.build_block_mask(mod, dp, B, Sq, Skv, mask, s_),
-                                              ta.attn_fwd(t[0], t[1], t[2], t[4], t[5], scale=w.scale, mod_kind=mod,
-                                                          mod_params=dp, block_mask=mask, stream=s_),
-                                              ta.attn_bwd(t[0], t[1], t[2], t[4], t[5], t[3], t[6], t[7], t[8], ws,
-                                                          scale=w.scale, mod_kind=mod, mod_params=dp,
-                                                          block_mask=mask, stream=s_)))
+                               lambda t_, s_: (ta.build_block_mask(mod, dp, B, Sq, Skv, mask, s_),
+                                               ta.attn_fwd(t_[0], t_[1], t_[2], t_[4], t_[5], scale=w.scale, mod_kind=mod,
+                                                           mod_params=dp, block_mask=mask, stream=s_),
+                                               ta.attn_bwd(t_[0], t_[1], t_[2], t_[4], t_[5], t_[3], t_[6], t_[7], t_[8], ws,
+                                                           scale=w.scale, mod_kind=mod, mod_params=dp,
+                                                           block_mask=mask, stream=s_)))
         e2e_mode = ("pipelined: H2D, step and D2H on three streams with two device buffer sets, so that "
                     "step i's compute overlaps step i+1's H2D and step i-1's D2H (every copy still timed)")
         st = ta.attn_get_status(stream)
         if st != 0:
             raise RuntimeError(f"kernel status {st} in the pipelined end-to-end pass")
     ms_e2e = max_over_ranks([ms_e2e], world, dev)[0]
-    h2d = sum(t.numel() * t.element_size() for t in (q, k, v, dout))
-    d2h = sum(t.numel() * t.element_size() for t in (out, dq, dk, dv))
+    h2d = sum(t_.numel() * t_.element_size() for t_ in (q, k, v, dout))
+    d2h = sum(t_.numel() * t_.element_size() for t_ in (out, dq, dk, dv))
 
     n_u, f_fwd, f_bwd = useful_counts(ta, w, mod_name, params)
     peaks, peak_kind = load_peaks()
@@ -331,8 +411,8 @@ def run_gpu(args, rank, world, local_rank):
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(ms_step, 4),
-        "ms_per_step_median": round(ms_step_median, 4),
-        "ms_per_step_min": round(ms_step_min, 4),
+        "ms_per_step_median": round(t["ms_step_median"], 4),
+        "ms_per_step_min": round(t["ms_step_min"], 4),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -351,7 +431,8 @@ def run_gpu(args, rank, world, local_rank):
         "ms_block_mask": round(ms_mask, 4),
         "useful_elements": n_u,
         "roofline": dict(roof(bwd_tf, traffic_bwd) if dominant == "backward" else roof(fwd_tf, traffic_fwd),
-                         kernel="attn_bwd (prep + main + dQ cast)" if dominant == "backward" else "attn_fwd"),
+                         kernel="attn_bwd_kernel (the backward call: prep, main and dQ cast launches)"
+                         if dominant == "backward" else "attn_fwd_kernel"),
         "roofline_forward": roof(fwd_tf, traffic_fwd),
         "roofline_backward": roof(bwd_tf, traffic_bwd),
         "e2e": None if args.no_e2e else {"value": round(job_throughput(f_fwd + f_bwd, world, ms_e2e), 2), "unit": UNIT,
@@ -360,6 +441,18 @@ def run_gpu(args, rank, world, local_rank):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if not args.no_configs and not args.all:
+        # the other parity configurations, each timed on its own
+        configs = {f"{wl}:no_lse_forward": forward_only_entry(ta, pb, stream, flush, args.config_steps, 3,
+                                                              world, dev, peak, with_lse=False),
+                   f"{wl}:lse_forward": forward_only_entry(ta, pb, stream, flush, args.config_steps, 3,
+                                                           world, dev, peak, with_lse=True)}
+        del pb, q, k, v, dout, out, lse, dq, dk, dv
+        torch.cuda.empty_cache()
+        for spec in CONFIG_ENTRIES:
+            if spec != wl:
+                configs[spec] = config_entry(ta, spec, rank, world, dev, stream, flush, args.config_steps, 3, peak)
+        line["configs"] = configs
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, mod_name, params, seconds=args.cpu_seconds)
     return line
@@ -481,6 +574,10 @@ def main():
     ap.add_argument("--e2e-pipeline", action="store_true",
                     help="overlap each step's H2D and D2H with the neighbouring steps' compute")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-configs", action="store_true",
+                    help="time only the headline workload (no per-configuration entries)")
+    ap.add_argument("--config-steps", type=int, default=10,
+                    help="timed steps of each per-configuration entry")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -151,8 +151,13 @@ def test_workload_groups(ta, name, mod_name):
 
 
 def test_gqa_long_sampled(ta):
-    """32K causal GQA: dQ on sampled rows (each needs only its own row), and dK/dV
-    of the last two key tiles, which only the last 256 queries see."""
+    """32K causal GQA: dQ on sampled rows (each needs only its own row); dK/dV
+    of the last two key tiles, which only the last 256 queries see; and dK/dV
+    of a middle key tile [16384, 16512) and an early-middle one [8192, 8320),
+    which accumulate over thousands of query tiles of all four heads of the
+    group.  Causality makes every query before a key's own position
+    contribute exactly zero to it, so the oracle sums only the rows from the
+    earliest requested key on."""
     w, c = _case("gqa_long", "causal")
     dq, dk, dv = run_fwd_bwd(ta, c)
     G = w.Hq // w.Hkv
@@ -160,25 +165,63 @@ def test_gqa_long_sampled(ta):
     tail = np.arange(w.Skv - 256, w.Skv)
     rows = sample_rows(w.Sq, 24, 5)
     ref_q = c.oracle_bwd(groups=[(0, hk)], q_rows=rows, kv_rows=tail[:1], contrib_rows=rows)[0]
-    ref_kv = c.oracle_bwd(groups=[(0, hk)], q_rows=tail, kv_rows=tail, contrib_rows=tail)
+    ref_kv = c.oracle_bwd(groups=[(0, hk)], q_rows=tail[-1:], kv_rows=tail, contrib_rows=tail)
     got_q = np.stack([_gather(dq, 0, h, rows) for h in range(hk * G, hk * G + G)])
     assert rel_l2(got_q, ref_q[0, hk * G:hk * G + G][:, rows]) <= GRAD_REL_L2
     assert rel_l2(_gather(dk, 0, hk, tail), ref_kv[1][0, hk, tail]) <= GRAD_REL_L2
     assert rel_l2(_gather(dv, 0, hk, tail), ref_kv[2][0, hk, tail]) <= GRAD_REL_L2
+    # interior key tiles, in another KV group
+    hk = 2
+    mid = np.concatenate([np.arange(8192, 8320), np.arange(16384, 16512)])
+    ref_mid = c.oracle_bwd(groups=[(0, hk)], q_rows=mid[-1:], kv_rows=mid,
+                           contrib_rows=np.arange(int(mid[0]), w.Sq))
+    for lo in (0, 128):
+        keys = mid[lo:lo + 128]
+        for t, r, nm in ((dk, ref_mid[1], "dk"), (dv, ref_mid[2], "dv")):
+            e = rel_l2(_gather(t, 0, hk, keys), r[0, hk, keys])
+            assert e <= GRAD_REL_L2, f"keys [{keys[0]}, {keys[-1] + 1}) {nm} {e:.3e}"
 
 
-def test_documents_two_docs(ta):
+def test_documents_sampled_docs(ta):
     """Packed documents: each document is an independent causal problem, so the
-    oracle runs on two whole documents cut out of the packed sequence."""
+    oracle runs on whole documents cut out of the packed sequence: the first,
+    a mid-sequence and the last document, in three heads."""
     w, c = _case("documents", "document")
     dq, dk, dv = run_fwd_bwd(ta, c)
     offs = c.p.doc_offsets[0]
-    for d in (0, len(offs) - 2):
+    n_docs = len(offs) - 1
+    for d in (0, n_docs // 2, n_docs - 1):
         a, b = offs[d], offs[d + 1]
         sub = [x[:, :, a:b] for x in (c.qf, c.kf, c.vf, c.doutf)]
-        ref = oracle.attention_backward(*sub, c.scale, oracle.MOD_CAUSAL, groups=[(0, 3)])
+        heads = (3, 8, 15)
+        ref = oracle.attention_backward(*sub, c.scale, oracle.MOD_CAUSAL, groups=[(0, h) for h in heads])
         rows = np.arange(a, b)
-        for t, r, nm in ((dq, ref[0], "dq"), (dk, ref[1], "dk"), (dv, ref[2], "dv")):
-            got = _gather(t, 0, 3, rows)
-            e = rel_l2(got, r[0, 3])
-            assert e <= GRAD_REL_L2, f"doc {d} {nm} {e:.3e}"
+        for h in heads:
+            for t, r, nm in ((dq, ref[0], "dq"), (dk, ref[1], "dk"), (dv, ref[2], "dv")):
+                got = _gather(t, 0, h, rows)
+                e = rel_l2(got, r[0, h])
+                assert e <= GRAD_REL_L2, f"doc {d} head {h} {nm} {e:.3e}"
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_alibi_with_given_slopes(ta, D):
+    """The caller's ALiBi slopes (attn_mod_params.alibi_slopes), distinct per
+    query head, under GQA (query head h reads slope h, KV head h // G) and an
+    odd length."""
+    S, Hq, Hkv = 301, 8, 2
+    slopes = [0.5, 0.05, 0.002, 1.3, 0.25, 0.011, 0.8, 0.0]
+    c = Case(180 + D, 2, Hq, Hkv, S, S, D, oracle.MOD_ALIBI, ModParams(alibi_slopes=slopes))
+    c.dev_params.alibi_slopes = torch.tensor(slopes, dtype=torch.float32, device="cuda")
+    from gpu_common import check_lse, check_o
+    for use_mask in (False, True):
+        mask = ta.new_block_mask(c.mod, c.dev_params, c.B, c.Sq, c.Skv) if use_mask else None
+        out = torch.empty_like(c.q)
+        lse = torch.empty(c.B, c.Hq, c.Sq, dtype=torch.float32, device="cuda")
+        ta.attn_fwd(c.q, c.k, c.v, out, lse, scale=c.scale, mod_kind=c.mod, mod_params=c.dev_params,
+                    block_mask=mask)
+        torch.cuda.synchronize()
+        O, L = c.oracle_fwd()
+        check_o(host_f64(out), O, f"alibi slopes D {D}")
+        check_lse(lse.cpu().double().numpy(), L, f"alibi slopes D {D}")
+        got = [host_f64(t) for t in run_fwd_bwd(ta, c, use_mask)]
+        check_grads(got, c.oracle_bwd(), f"alibi slopes D {D} mask {use_mask}")

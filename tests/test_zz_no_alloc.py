@@ -5,7 +5,8 @@ host that gives its kernels no workspace, or an application whose device
 memory is fixed in advance by its own pool): it runs the backward pass on a
 fixed block the library holds instead of on a caller workspace.  These tests
 call it through the C ABI and check its gradients against attn_bwd on the
-same inputs, on two calls in a row, since every call reuses the same block.
+same inputs and against the fp64 oracle, on two calls in a row, since every
+call reuses the same block.
 This file is collected last so that a failure here leaves every other test
 already run.
 """
@@ -39,8 +40,9 @@ def _call_noalloc(ta, c, out, lse, mask, dq, dk, dv):
 
 
 @pytest.mark.parametrize("mod", [oracle.MOD_NONE, oracle.MOD_CAUSAL])
-def test_noalloc_matches_workspace_backward_twice(ta, mod):
-    c = Case(41, 2, 4, 2, 700, 700, 128, mod)
+@pytest.mark.parametrize("D", [64, 128])
+def test_noalloc_matches_workspace_backward_twice(ta, mod, D):
+    c = Case(41, 2, 4, 2, 700, 700, D, mod)
     assert ta.attn_bwd_workspace_size(c.B, c.Hq, c.Sq, c.D) <= ta.attn_bwd_noalloc_max_workspace()
     mask = ta.new_block_mask(c.mod, c.dev_params, c.B, c.Sq, c.Skv)
     out = torch.empty_like(c.q)
@@ -50,14 +52,17 @@ def test_noalloc_matches_workspace_backward_twice(ta, mod):
     ws = ta.new_bwd_workspace(c.B, c.Hq, c.Sq, c.D)
     ta.attn_bwd(c.q, c.k, c.v, out, lse, c.dout, *ref, ws, scale=c.scale, mod_kind=c.mod,
                 mod_params=c.dev_params, block_mask=mask)
+    exact = c.oracle_bwd()
     for _ in range(2):  # the second call reuses the block the first one left behind
         got = [torch.full_like(c.q, float("nan")), torch.full_like(c.k, float("nan")),
                torch.full_like(c.v, float("nan"))]
         assert _call_noalloc(ta, c, out, lse, mask, *got) == 0
         torch.cuda.synchronize()
         assert ta.attn_get_status() == 0
-        for g, r in zip(got, ref):
+        for g, r, x in zip(got, ref, exact):
             assert rel_l2(host_f64(g), host_f64(r)) <= GRAD_REL_L2
+            # and against the fp64 oracle on the same inputs
+            assert rel_l2(host_f64(g), x) <= GRAD_REL_L2
         # dK and dV have a fixed summation order: identical to the workspace call
         assert torch.equal(got[1].view(torch.int16), ref[1].view(torch.int16))
         assert torch.equal(got[2].view(torch.int16), ref[2].view(torch.int16))

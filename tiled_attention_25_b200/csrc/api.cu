@@ -473,6 +473,7 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
   a.nQ = cdiv(Sq, TILE);
   a.nK = cdiv(Skv, TILE);
   a.n_units = B * Hkv * a.nK;
+  a.num_sms = d->sms;
   a.scale = scale;
   a.sl2 = scale * LOG2E;
   a.mod = make_mod(mod_kind, mod_params);

@@ -893,7 +893,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
                          const CUtensorMap& tdo, const BwdArgs& a, int grid, cudaStream_t stream) {
   const long long rows = static_cast<long long>(a.B) * a.Hq * a.Sq_pad;
   int prep_blocks = static_cast<int>((rows * 32 + 255) / 256);
-  if (prep_blocks > 148 * 16) prep_blocks = 148 * 16;
+  if (prep_blocks > a.num_sms * 16) prep_blocks = a.num_sms * 16;  // two waves of 8 resident blocks per SM
   bwd_prep_kernel<D><<<prep_blocks, 256, 0, stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -905,7 +905,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   if (e != cudaSuccess) return e;
   const long long n8 = static_cast<long long>(a.B) * a.Hq * a.Sq * (D / 8);
   int cast_blocks = static_cast<int>((n8 + 255) / 256);
-  if (cast_blocks > 148 * 16) cast_blocks = 148 * 16;
+  if (cast_blocks > a.num_sms * 16) cast_blocks = a.num_sms * 16;
   bwd_dq_cast_kernel<D><<<cast_blocks, 256, 0, stream>>>(a);
   return cudaGetLastError();
 }

@@ -39,6 +39,7 @@ struct BwdArgs {
   __nv_bfloat16* dv;
   int B, Hq, Hkv, G, Sq, Skv, Sq_pad;
   int nQ, nK, n_units;
+  int num_sms;  // SMs of the device (grid caps of the prep and cast kernels)
   float scale, sl2;
   ModDev mod;
   const uint8_t* tile_class;
