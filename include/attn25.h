@@ -97,8 +97,11 @@ enum {
   ATTN_MASK_CAUSAL = 0x100,
   ATTN_MASK_SLIDING_WINDOW = 0x200,
   ATTN_MASK_DOCUMENT = 0x400,
-  ATTN_MASK_BITMAP = 0x800      /* a general mask given by its values (attn_mod_params.bitmap);
+  ATTN_MASK_BITMAP = 0x800,     /* a general mask given by its values (attn_mod_params.bitmap);
                                    attn_fwd / attn_bwd then need a block mask built for it */
+  ATTN_MASK_VARLEN = 0x1000     /* packed sequences with their own query and key lengths:
+                                   query i and key j interact only within one sequence; not
+                                   causal, and combined with no other mask */
 };
 
 /*
@@ -127,6 +130,11 @@ typedef struct attn_mod_params {
   int32_t bitmap_heads;         /* 1 (one mask for all heads, head stride 0) or Hq */
   int64_t bitmap_head_stride;   /* words, a multiple of 4; 0 when bitmap_heads == 1 */
   int64_t bitmap_batch_stride;  /* words, a multiple of 4; 0 = one mask for all batch rows */
+  /* ATTN_MASK_VARLEN: device int32 [B][num_seqs + 1] ascending starts of each sequence's
+   * queries and keys, plus the ends (Sq and Skv); repeat an offset for an empty sequence. */
+  const int32_t* q_offsets;
+  const int32_t* k_offsets;
+  int32_t num_seqs;             /* 1 <= num_seqs <= 65536 */
 } attn_mod_params;
 
 /*

@@ -38,11 +38,16 @@ class Case:
         if oracle.has_document(mod):
             arr, _ = pad_offsets(self.p.doc_offsets)
             doc_t = torch.from_numpy(arr).cuda()
+        vq_t = vk_t = None
+        if int(mod) & oracle.MASK_VARLEN:
+            vq_t = torch.from_numpy(pad_offsets(self.p.q_offsets)[0]).cuda()
+            vk_t = torch.from_numpy(pad_offsets(self.p.k_offsets)[0]).cuda()
         bm_t = None
         if oracle.has_bitmap(mod):
             bm_t = torch.from_numpy(pack_bitmap(self.p.bitmap)).cuda()
         self.dev_params = ta.ModParams(softcap=self.p.softcap, window=self.p.window, boost=self.p.boost,
-                                       boost_radius=self.p.boost_radius, doc_offsets=doc_t, bitmap=bm_t)
+                                       boost_radius=self.p.boost_radius, doc_offsets=doc_t, bitmap=bm_t,
+                                       q_offsets=vq_t, k_offsets=vk_t)
 
     def oracle_fwd(self, heads=None, rows=None):
         return oracle.attention_forward(self.qf, self.kf, self.vf, self.scale, self.mod, self.p,

@@ -17,6 +17,7 @@ from .abi import (  # noqa: F401
     MASK_CAUSAL,
     MASK_DOCUMENT,
     MASK_SLIDING_WINDOW,
+    MASK_VARLEN,
     MOD_ALIBI,
     MOD_CAUSAL,
     MOD_DOCUMENT,

@@ -31,6 +31,7 @@ MASK_CAUSAL = 0x100
 MASK_SLIDING_WINDOW = 0x200
 MASK_DOCUMENT = 0x400
 MASK_BITMAP = 0x800
+MASK_VARLEN = 0x1000
 
 ATTN_ERR_TIMEOUT = -6
 
@@ -55,6 +56,9 @@ class CModParams(ctypes.Structure):
         ("bitmap_heads", ctypes.c_int32),
         ("bitmap_head_stride", ctypes.c_int64),
         ("bitmap_batch_stride", ctypes.c_int64),
+        ("q_offsets", ctypes.c_void_p),
+        ("k_offsets", ctypes.c_void_p),
+        ("num_seqs", ctypes.c_int32),
     ]
 
 
@@ -144,7 +148,7 @@ class ModParams:
     """Mod scalars plus the device tensors they point at (kept alive here)."""
 
     def __init__(self, softcap=50.0, window=1024, boost=1.1, boost_radius=128,
-                 alibi_slopes=None, doc_offsets=None, bitmap=None):
+                 alibi_slopes=None, doc_offsets=None, bitmap=None, q_offsets=None, k_offsets=None):
         self.softcap = float(softcap)
         self.window = int(window)
         self.boost = float(boost)
@@ -156,6 +160,14 @@ class ModParams:
         if alibi_slopes is not None:
             assert alibi_slopes.dtype == torch.float32 and alibi_slopes.is_contiguous()
         # device int32 [B or 1][Hq or 1][Sq][row_words] keep bits (bit j & 31 of word j >> 5)
+        # device int32 [B][num_seqs + 1] each: the varlen mask's query and key offsets
+        self.q_offsets, self.k_offsets = q_offsets, k_offsets
+        if (q_offsets is None) != (k_offsets is None):
+            raise ValueError("the varlen mask needs both query and key offsets")
+        if q_offsets is not None:
+            for t in (q_offsets, k_offsets):
+                assert t.dtype == torch.int32 and t.is_contiguous() and t.dim() == 2
+            assert q_offsets.shape == k_offsets.shape
         self.bitmap = bitmap
         if bitmap is not None:
             assert bitmap.dtype == torch.int32 and bitmap.is_contiguous() and bitmap.dim() == 4
@@ -170,7 +182,10 @@ class ModParams:
         return CModParams(self.softcap, self.window, self.boost, self.boost_radius,
                           None if self.alibi_slopes is None else self.alibi_slopes.data_ptr(),
                           None if self.doc_offsets is None else self.doc_offsets.data_ptr(),
-                          0 if self.doc_offsets is None else self.doc_offsets.shape[1] - 1, *bm_args)
+                          0 if self.doc_offsets is None else self.doc_offsets.shape[1] - 1, *bm_args,
+                          None if self.q_offsets is None else self.q_offsets.data_ptr(),
+                          None if self.k_offsets is None else self.k_offsets.data_ptr(),
+                          0 if self.q_offsets is None else self.q_offsets.shape[1] - 1)
 
 
 class BlockMask:

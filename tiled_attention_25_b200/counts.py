@@ -29,6 +29,8 @@ def useful_elements(mod_kind, B, Hq, Sq, Skv, window=None, doc_offsets=None) -> 
     Interval masks only: a bitmap mask's count is the number of its set bits."""
     if int(mod_kind) & MASK_BITMAP:
         raise ValueError("count a bitmap mask from its bits")
+    if int(mod_kind) & 0x1000:
+        raise ValueError("count a varlen mask as the sum over sequences of query length x key length")
     causal, win, doc = mask_parts(mod_kind)
     i = np.arange(Sq, dtype=np.int64)
     hi = np.minimum(i, Skv - 1) if causal else np.full(Sq, Skv - 1, dtype=np.int64)

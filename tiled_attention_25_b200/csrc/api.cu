@@ -119,7 +119,13 @@ struct ModSpec {
 bool split_mod(int code, ModSpec& m) {
   const int base = code & 0xFF, flags = code & ~0xFF;
   if (base < ATTN_MOD_NONE || base > ATTN_MOD_DOCUMENT) return false;
-  if (flags & ~(ATTN_MASK_CAUSAL | ATTN_MASK_SLIDING_WINDOW | ATTN_MASK_DOCUMENT | ATTN_MASK_BITMAP))
+  if (flags & ~(ATTN_MASK_CAUSAL | ATTN_MASK_SLIDING_WINDOW | ATTN_MASK_DOCUMENT | ATTN_MASK_BITMAP |
+                ATTN_MASK_VARLEN))
+    return false;
+  // the varlen mask takes no other mask (a causal packing of equal lengths is the document mask)
+  if ((flags & ATTN_MASK_VARLEN) &&
+      ((flags & ~ATTN_MASK_VARLEN) || base == ATTN_MOD_CAUSAL || base == ATTN_MOD_SLIDING_WINDOW ||
+       base == ATTN_MOD_DOCUMENT))
     return false;
   m.score = MOD_NONE;
   m.mask = 0;
@@ -136,11 +142,13 @@ bool split_mod(int code, ModSpec& m) {
   if (flags & ATTN_MASK_SLIDING_WINDOW) m.mask |= kMaskCausal | kMaskWindow;
   if (flags & ATTN_MASK_DOCUMENT) m.mask |= kMaskCausal | kMaskDoc;
   if (flags & ATTN_MASK_BITMAP) m.mask |= kMaskBitmap;
+  if (flags & ATTN_MASK_VARLEN) m.mask |= kMaskVarlen;
   m.key = m.score | (m.mask != 0 ? kKeyMasked : 0) | ((m.mask & kMaskBitmap) ? kKeyBitmap : 0);
   m.canonical = m.score | ((m.mask & kMaskCausal) ? ATTN_MASK_CAUSAL : 0) |
                 ((m.mask & kMaskWindow) ? ATTN_MASK_SLIDING_WINDOW : 0) |
                 ((m.mask & kMaskDoc) ? ATTN_MASK_DOCUMENT : 0) |
-                ((m.mask & kMaskBitmap) ? ATTN_MASK_BITMAP : 0);
+                ((m.mask & kMaskBitmap) ? ATTN_MASK_BITMAP : 0) |
+                ((m.mask & kMaskVarlen) ? ATTN_MASK_VARLEN : 0);
   return true;
 }
 
@@ -172,6 +180,13 @@ int check_common(int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale, in
       return ATTN_ERR_ARG;
     if (Sq != Skv) return ATTN_ERR_UNSUPPORTED;
     if (reinterpret_cast<uintptr_t>(mp->doc_offsets) & 3u) return ATTN_ERR_ALIGN;
+  }
+  if (ms.mask & kMaskVarlen) {
+    if (mp == nullptr || mp->q_offsets == nullptr || mp->k_offsets == nullptr || mp->num_seqs < 1 ||
+        mp->num_seqs > 65536)
+      return ATTN_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(mp->q_offsets) & 3u) || (reinterpret_cast<uintptr_t>(mp->k_offsets) & 3u))
+      return ATTN_ERR_ALIGN;
   }
   if (ms.mask & kMaskBitmap) {
     if (mp == nullptr || mp->bitmap == nullptr) return ATTN_ERR_ARG;
@@ -223,6 +238,11 @@ ModDev make_mod(int mod_kind, const attn_mod_params* mp) {
     if (ms.mask & kMaskDoc) {
       m.doc_offsets = mp->doc_offsets;
       m.num_docs = mp->num_docs;
+    }
+    if (ms.mask & kMaskVarlen) {
+      m.vq_offsets = mp->q_offsets;
+      m.vk_offsets = mp->k_offsets;
+      m.n_seqs = mp->num_seqs;
     }
     if (ms.mask & kMaskBitmap) {
       m.bitmap = mp->bitmap;
@@ -353,6 +373,9 @@ int build_block_mask(int mod_kind, const attn_mod_params* mod_params, int B, int
   a.bm_heads = md.bitmap != nullptr ? mod_params->bitmap_heads : 0;
   a.bm_head_stride = md.bm_head_stride;
   a.bm_batch_stride = md.bm_batch_stride;
+  a.vq_offsets = md.vq_offsets;
+  a.vk_offsets = md.vk_offsets;
+  a.n_seqs = md.n_seqs;
   a.B = B;
   a.Sq = Sq;
   a.Skv = Skv;

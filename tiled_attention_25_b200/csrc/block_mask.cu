@@ -25,10 +25,12 @@ namespace {
 
 __device__ __forceinline__ void row_keep_interval(const MaskArgs& a, int b, int i, int& lo,
                                                   int& hi) {
+  const size_t vb = static_cast<size_t>(b) * (a.n_seqs + 1);
   row_interval(a.mask, a.window,
                a.doc_offsets == nullptr ? nullptr
                                         : a.doc_offsets + static_cast<size_t>(b) * (a.num_docs + 1),
-               a.num_docs, i, a.Skv, lo, hi);
+               a.num_docs, a.vq_offsets == nullptr ? nullptr : a.vq_offsets + vb,
+               a.vk_offsets == nullptr ? nullptr : a.vk_offsets + vb, a.n_seqs, i, a.Skv, lo, hi);
 }
 
 // grid (nQ, B): classify one query-tile row of tiles and write its KV list.

@@ -211,7 +211,7 @@ __device__ __forceinline__ void key_interval(const BwdArgs& a, int b, int kv, in
   qhi = a.Sq - 1;
   if constexpr (masked(MOD)) {
     const int mask = a.mod.mask;
-    if (mask & (kMaskCausal | kMaskWindow | kMaskDoc)) qlo = kv;
+    if (mask & kMaskCausalBits) qlo = kv;
     if (mask & kMaskWindow) qhi = min(qhi, kv + a.mod.window - 1);
     if (mask & kMaskDoc) {
       const int32_t* offs = a.mod.doc_offsets + static_cast<size_t>(b) * (a.mod.num_docs + 1);
@@ -222,6 +222,12 @@ __device__ __forceinline__ void key_interval(const BwdArgs& a, int b, int kv, in
         if (__ldg(offs + mid) <= kvc) lo = mid; else hi = mid;
       }
       qhi = min(qhi, __ldg(offs + lo + 1) - 1);
+    }
+    if (mask & kMaskVarlen) {  // the query range of the sequence that holds the key
+      const size_t vb = static_cast<size_t>(b) * (a.mod.n_seqs + 1);
+      const int d = segment_of(a.mod.vk_offsets + vb, a.mod.n_seqs, min(kv, a.Skv - 1));
+      qlo = max(qlo, __ldg(a.mod.vq_offsets + vb + d));
+      qhi = min(qhi, __ldg(a.mod.vq_offsets + vb + d + 1) - 1);
     }
   }
   if (kv >= a.Skv) qhi = qlo - 1;

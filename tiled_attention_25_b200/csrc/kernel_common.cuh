@@ -54,7 +54,7 @@ __device__ __forceinline__ int build_pair_steps(const uint8_t* tile_class, int b
   const int q0a = qt0 * TILE, q1a = min(Sq, q0a + TILE);
   const int q0b = qt1 * TILE, q1b = has1 ? min(Sq, q0b + TILE) : q0b;
   int k_begin = 0, k_end = nK;
-  if (tile_class == nullptr && mask != 0) {
+  if (tile_class == nullptr && (mask & kMaskCausalBits)) {
     k_end = min(nK, (max(q1a, q1b) - 1) / TILE + 1);
     if (mask & kMaskWindow) k_begin = max(0, (q0a - window + 1) / TILE);
   }
@@ -102,7 +102,7 @@ __device__ __forceinline__ int build_kv_qtiles(const uint8_t* tile_class, int b,
                                                uint16_t* list) {
   const int lane = threadIdx.x & 31;
   int q_begin = 0;
-  if (tile_class == nullptr && mask != 0) q_begin = kt;  // every mask keeps q >= kv
+  if (tile_class == nullptr && (mask & kMaskCausalBits)) q_begin = kt;  // these masks keep q >= kv
   const bool tail_kv = (Skv % TILE) != 0 && kt == nK - 1;
   const int k0 = kt * TILE, k1 = min(Skv, k0 + TILE);
   int n = 0;

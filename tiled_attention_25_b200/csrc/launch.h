@@ -59,6 +59,9 @@ struct MaskArgs {
   const uint32_t* bitmap;  // keep bits (bitmap mask) or nullptr
   int bm_row_words, bm_heads;
   long long bm_head_stride, bm_batch_stride;
+  const int32_t* vq_offsets;  // varlen mask or nullptr
+  const int32_t* vk_offsets;
+  int n_seqs;
   int B, Sq, Skv, nQ, nK, nP;
   uint8_t* tile_class;
   int32_t* kv_count;

@@ -34,6 +34,9 @@ constexpr int kMaskCausal = 1;
 constexpr int kMaskWindow = 2;
 constexpr int kMaskDoc = 4;
 constexpr int kMaskBitmap = 8;  // a general mask given by its values, one bit per element
+constexpr int kMaskVarlen = 16; // packed sequences with their own query and key lengths
+// the masks that keep only keys at or before the query (kv <= q)
+constexpr int kMaskCausalBits = kMaskCausal | kMaskWindow | kMaskDoc;
 
 // Kernel specialisation key: the score transform (MOD_NONE, MOD_ALIBI,
 // MOD_SOFTCAP or MOD_BOOST) plus kKeyMasked when any mask is present, and
@@ -59,6 +62,9 @@ struct ModDev {
   int bm_row_words;           // words per query row (a multiple of 4)
   long long bm_head_stride;   // words between heads (0: shared)
   long long bm_batch_stride;  // words between batch rows (0: shared)
+  const int32_t* vq_offsets;  // varlen mask: [B][n_seqs + 1] query and key starts plus ends
+  const int32_t* vk_offsets;
+  int n_seqs;
 };
 
 // First word of query row i of head h, batch row b in the keep bitmap.
@@ -77,23 +83,43 @@ __device__ __forceinline__ int doc_start(const int32_t* offs, int num_docs, int 
   return __ldg(offs + lo);
 }
 
+// Index of the segment [offs[d], offs[d+1]) that holds position i (offsets
+// ascending; empty segments repeat an offset and never hold a position).
+__device__ __forceinline__ int segment_of(const int32_t* offs, int n, int i) {
+  int lo = 0, hi = n;  // invariant: offs[lo] <= i, answer in [lo, hi)
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(offs + mid) <= i) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
 // Kept key interval [lo, hi] of query row i (hi already clipped to Skv - 1):
-// the intersection of the masks' intervals.
+// the intersection of the masks' intervals.  The varlen mask keeps the key
+// range of the sequence that holds i.
 __device__ __forceinline__ void row_interval(int mask, int window, const int32_t* offs_b,
-                                             int num_docs, int i, int Skv, int& lo, int& hi) {
+                                             int num_docs, const int32_t* vq_b, const int32_t* vk_b,
+                                             int n_seqs, int i, int Skv, int& lo, int& hi) {
   lo = 0;
   hi = Skv - 1;
-  if (mask & (kMaskCausal | kMaskWindow | kMaskDoc)) hi = min(hi, i);
+  if (mask & kMaskCausalBits) hi = min(hi, i);
   if (mask & kMaskWindow) lo = max(lo, i - window + 1);
   if (mask & kMaskDoc) lo = max(lo, doc_start(offs_b, num_docs, i));
+  if (mask & kMaskVarlen) {
+    const int d = segment_of(vq_b, n_seqs, i);
+    lo = max(lo, __ldg(vk_b + d));
+    hi = min(hi, __ldg(vk_b + d + 1) - 1);
+  }
 }
 
 __device__ __forceinline__ void row_interval(const ModDev& m, int b, int i, int Skv, int& lo,
                                              int& hi) {
+  const size_t vb = static_cast<size_t>(b) * (m.n_seqs + 1);
   row_interval(m.mask, m.window,
                m.doc_offsets == nullptr ? nullptr
                                         : m.doc_offsets + static_cast<size_t>(b) * (m.num_docs + 1),
-               m.num_docs, i, Skv, lo, hi);
+               m.num_docs, m.vq_offsets == nullptr ? nullptr : m.vq_offsets + vb,
+               m.vk_offsets == nullptr ? nullptr : m.vk_offsets + vb, m.n_seqs, i, Skv, lo, hi);
 }
 
 __device__ __forceinline__ float alibi_slope(const ModDev& m, int h, int Hq) {
@@ -109,6 +135,7 @@ __device__ __forceinline__ float alibi_slope(const ModDev& m, int h, int Hq) {
 __host__ __device__ inline int dense_tile_class(int mask, int window, int q0, int q1, int k0,
                                                 int k1) {
   if (mask == 0) return 2;
+  if (mask & kMaskVarlen) return 1;  // the sequences' rectangles need the offsets
   const int W = (mask & kMaskWindow) ? window : (1 << 30);
   const int first_row = q0, last_row = q1 - 1;
   const bool any = (k0 <= last_row) && (k1 - 1 >= first_row - W + 1);
