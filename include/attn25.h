@@ -246,6 +246,38 @@ ATTN25_API int build_block_mask(int mod_kind, const attn_mod_params* mod_params,
                      int B, int Sq, int Skv, attn_block_mask* mask,
                      attn_stream_t stream);
 
+/*
+ * Strided tensors.  Each bf16 tensor is a [B][H][S][D] view whose D elements
+ * are contiguous; these are its element strides between batch rows, heads
+ * and sequence positions (each a positive multiple of 8, so that a row
+ * starts on 16 bytes).  Contiguous [B][H][S][D] has {H*S*D, S*D, D}; the
+ * common [B][S][H][D] storage has {S*H*D, D, H*D}.
+ */
+typedef struct attn_strides {
+  int64_t b, h, s;
+} attn_strides;
+
+typedef struct attn_layouts {
+  attn_strides q, k, v, out, dout, dq, dk, dv;  /* attn_fwd_strided reads q, k, v, out */
+} attn_layouts;
+
+/* attn_fwd and attn_bwd on strided tensors (layouts NULL: contiguous);
+ * bad strides return ATTN_ERR_ALIGN.  LSE stays contiguous [B][Hq][Sq]. */
+ATTN25_API int attn_fwd_strided(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v,
+                                attn_bf16* out, float* lse,
+                                int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+                                int mod_kind, const attn_mod_params* mod_params,
+                                const attn_block_mask* block_mask, const attn_layouts* layouts,
+                                attn_stream_t stream);
+ATTN25_API int attn_bwd_strided(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v,
+                                const attn_bf16* out, const float* lse, const attn_bf16* dout,
+                                attn_bf16* dq, attn_bf16* dk, attn_bf16* dv,
+                                void* workspace, size_t workspace_bytes,
+                                int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+                                int mod_kind, const attn_mod_params* mod_params,
+                                const attn_block_mask* block_mask, const attn_layouts* layouts,
+                                attn_stream_t stream);
+
 /* Synchronise the stream, then return and clear the device status word. */
 ATTN25_API int attn_get_status(attn_stream_t stream);
 

@@ -31,10 +31,12 @@ from .abi import (  # noqa: F401
     attn_block_mask_bind,
     attn_block_mask_bytes,
     attn_bwd,
+    attn_bwd_strided,
     attn_bwd_noalloc,
     attn_bwd_noalloc_max_workspace,
     attn_bwd_workspace_size,
     attn_fwd,
+    attn_fwd_strided,
     attn_get_status,
     attn_set_wait_limit_ms,
     attn_strerror,

@@ -62,6 +62,14 @@ class CModParams(ctypes.Structure):
     ]
 
 
+class CStrides(ctypes.Structure):
+    _fields_ = [("b", ctypes.c_int64), ("h", ctypes.c_int64), ("s", ctypes.c_int64)]
+
+
+class CLayouts(ctypes.Structure):
+    _fields_ = [(n, CStrides) for n in ("q", "k", "v", "out", "dout", "dq", "dk", "dv")]
+
+
 class CBlockMask(ctypes.Structure):
     _fields_ = [
         ("tile_class", ctypes.c_void_p),
@@ -101,6 +109,10 @@ def _load():
     lib.attn_block_mask_bind.restype = I
     lib.build_block_mask.argtypes = [I, P, I, I, I, ctypes.POINTER(CBlockMask), P]
     lib.build_block_mask.restype = I
+    lib.attn_fwd_strided.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, P, P, P, P]
+    lib.attn_fwd_strided.restype = I
+    lib.attn_bwd_strided.argtypes = [P, P, P, P, P, P, P, P, P, P, S, I, I, I, I, I, I, F, I, P, P, P, P]
+    lib.attn_bwd_strided.restype = I
     lib.attn_get_status.argtypes = [P]
     lib.attn_get_status.restype = I
     lib.attn_set_wait_limit_ms.argtypes = [ctypes.c_uint32]
@@ -122,7 +134,7 @@ LIB = _load()
 EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_bwd_noalloc",
             "attn_bwd_noalloc_max_workspace", "attn_block_mask_bytes",
             "attn_block_mask_bind", "build_block_mask", "attn_get_status",
-            "attn_set_wait_limit_ms", "attn_strerror")
+            "attn_set_wait_limit_ms", "attn_strerror", "attn_fwd_strided", "attn_bwd_strided")
 
 
 def attn_strerror(code: int) -> str:
@@ -249,6 +261,58 @@ def attn_fwd(q, k, v, out, lse=None, scale=None, mod_kind=MOD_NONE, mod_params=N
                       scale, int(mod_kind), None if mp is None else mp[0],
                       None if block_mask is None else ctypes.byref(block_mask.c), _stream(stream))
     _check(rc, "attn_fwd")
+
+
+def _strides(t, shape, what):
+    """Element strides (b, h, s) of a [B][H][S][D] CUDA bf16 view with D contiguous."""
+    if t.dtype != torch.bfloat16 or not t.is_cuda or t.dim() != 4 or tuple(t.shape) != tuple(shape) \
+            or t.stride(3) != 1:
+        raise ValueError(f"{what} must be a CUDA bf16 {tuple(shape)} view with its last dimension contiguous")
+    return CStrides(t.stride(0), t.stride(1), t.stride(2))
+
+
+def _layouts(**views):
+    lay = CLayouts()
+    for name, (t, shape) in views.items():
+        setattr(lay, name, _strides(t, shape, name))
+    return lay
+
+
+def attn_fwd_strided(q, k, v, out, lse=None, scale=None, mod_kind=MOD_NONE, mod_params=None, block_mask=None,
+                     stream=None):
+    """attn_fwd on [B][H][S][D] views of any strides whose last dimension is
+    contiguous (e.g. x.permute(0, 2, 1, 3) of a [B][S][H][D] tensor)."""
+    B, Hq, Sq, D = q.shape
+    _, Hkv, Skv, _ = k.shape
+    lay = _layouts(q=(q, (B, Hq, Sq, D)), k=(k, (B, Hkv, Skv, D)), v=(v, (B, Hkv, Skv, D)),
+                   out=(out, (B, Hq, Sq, D)))
+    if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hq, Sq) or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous fp32 [B][Hq][Sq] tensor")
+    scale = D ** -0.5 if scale is None else float(scale)
+    mp = _mp(mod_params, mod_kind, B, Hq, Sq)
+    rc = LIB.attn_fwd_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D, scale,
+                              int(mod_kind), None if mp is None else mp[0],
+                              None if block_mask is None else ctypes.byref(block_mask.c), ctypes.byref(lay),
+                              _stream(stream))
+    _check(rc, "attn_fwd_strided")
+
+
+def attn_bwd_strided(q, k, v, out, lse, dout, dq, dk, dv, workspace, scale=None, mod_kind=MOD_NONE,
+                     mod_params=None, block_mask=None, stream=None):
+    """attn_bwd on strided views (see attn_fwd_strided)."""
+    B, Hq, Sq, D = q.shape
+    _, Hkv, Skv, _ = k.shape
+    qs, ks = (B, Hq, Sq, D), (B, Hkv, Skv, D)
+    lay = _layouts(q=(q, qs), k=(k, ks), v=(v, ks), out=(out, qs), dout=(dout, qs), dq=(dq, qs), dk=(dk, ks),
+                   dv=(dv, ks))
+    scale = D ** -0.5 if scale is None else float(scale)
+    mp = _mp(mod_params, mod_kind, B, Hq, Sq)
+    rc = LIB.attn_bwd_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                              _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(), B, Hq, Hkv,
+                              Sq, Skv, D, scale, int(mod_kind), None if mp is None else mp[0],
+                              None if block_mask is None else ctypes.byref(block_mask.c), ctypes.byref(lay),
+                              _stream(stream))
+    _check(rc, "attn_bwd_strided")
 
 
 def attn_bwd_workspace_size(B, Hq, Sq, D) -> int:

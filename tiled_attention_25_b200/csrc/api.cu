@@ -88,17 +88,30 @@ int current_device(DeviceInfo** out) {
 }
 
 // bf16 tensor [outer][rows][inner] with rows x 64-column boxes, 128-byte swizzle.
-bool encode_bf16(CUtensorMap* m, const void* base, int inner, int rows, int outer, int box_rows) {
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
-                        static_cast<cuuint64_t>(outer)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * 2,
-                           static_cast<cuuint64_t>(inner) * rows * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+// A [B][H][S][D] bf16 tensor whose D elements are contiguous, as the 4-D map
+// (D, S, H, B) with the tensor's own strides; boxes of 64 x box_rows x 1 x 1.
+bool encode_bf16_4d(CUtensorMap* m, const void* base, int D, int S, int H, int B, const Strides& st,
+                    int box_rows) {
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(st.s) * 2, static_cast<cuuint64_t>(st.h) * 2,
+                           static_cast<cuuint64_t>(st.b) * 2};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The strides of a tensor: the caller's, or those of contiguous [B][H][S][D].
+bool layout_of(const attn_strides* given, int H, int S, int D, Strides& st) {
+  if (given == nullptr) {
+    st = Strides{static_cast<long long>(H) * S * D, static_cast<long long>(S) * D, D};
+    return true;
+  }
+  st = Strides{given->b, given->h, given->s};
+  // the tensor maps take strides of whole 16-byte units
+  return st.b >= 8 && st.h >= 8 && st.s >= 8 && st.b % 8 == 0 && st.h % 8 == 0 && st.s % 8 == 0;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -395,10 +408,10 @@ int build_block_mask(int mod_kind, const attn_mod_params* mod_params, int B, int
   return ATTN_OK;
 }
 
-int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* out,
-             float* lse, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
-             int mod_kind, const attn_mod_params* mod_params, const attn_block_mask* block_mask,
-             attn_stream_t stream) {
+int attn_fwd_strided(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* out,
+                     float* lse, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+                     int mod_kind, const attn_mod_params* mod_params, const attn_block_mask* block_mask,
+                     const attn_layouts* layouts, attn_stream_t stream) {
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ATTN_ERR_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
       (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
@@ -410,13 +423,20 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
   rc = current_device(&d);
   if (rc != ATTN_OK) return rc;
 
+  Strides sq, sk, sv, so;
+  if (!layout_of(layouts ? &layouts->q : nullptr, Hq, Sq, D, sq) ||
+      !layout_of(layouts ? &layouts->k : nullptr, Hkv, Skv, D, sk) ||
+      !layout_of(layouts ? &layouts->v : nullptr, Hkv, Skv, D, sv) ||
+      !layout_of(layouts ? &layouts->out : nullptr, Hq, Sq, D, so))
+    return ATTN_ERR_ALIGN;
   CUtensorMap tq, tk, tv;
-  if (!encode_bf16(&tq, q, D, Sq, B * Hq, TILE) || !encode_bf16(&tk, k, D, Skv, B * Hkv, TILE) ||
-      !encode_bf16(&tv, v, D, Skv, B * Hkv, TILE))
+  if (!encode_bf16_4d(&tq, q, D, Sq, Hq, B, sq, TILE) || !encode_bf16_4d(&tk, k, D, Skv, Hkv, B, sk, TILE) ||
+      !encode_bf16_4d(&tv, v, D, Skv, Hkv, B, sv, TILE))
     return ATTN_ERR_ARG;
 
   FwdArgs a{};
   a.out = reinterpret_cast<__nv_bfloat16*>(out);
+  a.o_st = so;
   a.lse = lse;
   a.B = B;
   a.Hq = Hq;
@@ -447,17 +467,25 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
   return ATTN_OK;
 }
 
+int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* out,
+             float* lse, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+             int mod_kind, const attn_mod_params* mod_params, const attn_block_mask* block_mask,
+             attn_stream_t stream) {
+  return attn_fwd_strided(q, k, v, out, lse, B, Hq, Hkv, Sq, Skv, D, scale, mod_kind, mod_params, block_mask,
+                          nullptr, stream);
+}
+
 size_t attn_bwd_workspace_size(int B, int Hq, int Sq, int D) {
   if (B < 1 || Hq < 1 || Sq < 1 || (D != 64 && D != 128)) return 0;
   const size_t rows = static_cast<size_t>(B) * Hq * (cdiv(Sq, TILE) * TILE);
   return align256(rows * D * 4) + 2 * align256(rows * 4);
 }
 
-int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* out,
-             const float* lse, const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk, attn_bf16* dv,
-             void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int Sq, int Skv,
-             int D, float scale, int mod_kind, const attn_mod_params* mod_params,
-             const attn_block_mask* block_mask, attn_stream_t stream) {
+int attn_bwd_strided(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* out,
+                     const float* lse, const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk, attn_bf16* dv,
+                     void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int Sq, int Skv,
+                     int D, float scale, int mod_kind, const attn_mod_params* mod_params,
+                     const attn_block_mask* block_mask, const attn_layouts* layouts, attn_stream_t stream) {
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr ||
       dout == nullptr || dq == nullptr || dk == nullptr || dv == nullptr || workspace == nullptr)
     return ATTN_ERR_ARG;
@@ -510,15 +538,34 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
   a.status = d->status;
   a.trace = d->trace == nullptr ? nullptr : d->trace + 128;
 
+  Strides sq, sk, sv;
+  if (!layout_of(layouts ? &layouts->q : nullptr, Hq, Sq, D, sq) ||
+      !layout_of(layouts ? &layouts->k : nullptr, Hkv, Skv, D, sk) ||
+      !layout_of(layouts ? &layouts->v : nullptr, Hkv, Skv, D, sv) ||
+      !layout_of(layouts ? &layouts->out : nullptr, Hq, Sq, D, a.o_st) ||
+      !layout_of(layouts ? &layouts->dout : nullptr, Hq, Sq, D, a.do_st) ||
+      !layout_of(layouts ? &layouts->dq : nullptr, Hq, Sq, D, a.dq_st) ||
+      !layout_of(layouts ? &layouts->dk : nullptr, Hkv, Skv, D, a.dk_st) ||
+      !layout_of(layouts ? &layouts->dv : nullptr, Hkv, Skv, D, a.dv_st))
+    return ATTN_ERR_ALIGN;
   CUtensorMap tq, tk, tv, tdo;
-  if (!encode_bf16(&tq, q, D, Sq, B * Hq, 64) || !encode_bf16(&tk, k, D, Skv, B * Hkv, TILE) ||
-      !encode_bf16(&tv, v, D, Skv, B * Hkv, TILE) || !encode_bf16(&tdo, dout, D, Sq, B * Hq, 64))
+  if (!encode_bf16_4d(&tq, q, D, Sq, Hq, B, sq, 64) || !encode_bf16_4d(&tk, k, D, Skv, Hkv, B, sk, TILE) ||
+      !encode_bf16_4d(&tv, v, D, Skv, Hkv, B, sv, TILE) || !encode_bf16_4d(&tdo, dout, D, Sq, Hq, B, a.do_st, 64))
     return ATTN_ERR_ARG;
   const int grid = a.n_units < d->sms ? a.n_units : d->sms;
   if (launch_bwd(tq, tk, tv, tdo, a, D, mod_key(mod_kind), grid,
                  reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_LAUNCH;
   return ATTN_OK;
+}
+
+int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* out,
+             const float* lse, const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk, attn_bf16* dv,
+             void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int Sq, int Skv,
+             int D, float scale, int mod_kind, const attn_mod_params* mod_params,
+             const attn_block_mask* block_mask, attn_stream_t stream) {
+  return attn_bwd_strided(q, k, v, out, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, Sq, Skv,
+                          D, scale, mod_kind, mod_params, block_mask, nullptr, stream);
 }
 
 size_t attn_bwd_noalloc_max_workspace(void) { return kNoAllocScratchBytes; }

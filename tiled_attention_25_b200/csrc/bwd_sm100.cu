@@ -164,18 +164,19 @@ struct StepIter {
   }
 };
 
+// Tiles of head h of batch row b through 4-D tensor maps (D, S, H, B).
 template <int D>
 __device__ __forceinline__ void load_kv_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                             int row0, int bh) {
+                                             int row0, int h, int b) {
 #pragma unroll
-  for (int c = 0; c < D / 64; ++c) tma_load_3d(dst + c * (TILE * 128), map, bar, c * 64, row0, bh);
+  for (int c = 0; c < D / 64; ++c) tma_load_4d(dst + c * (TILE * 128), map, bar, c * 64, row0, h, b);
 }
 
 template <int D>
 __device__ __forceinline__ void load_q_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int row0, int bh) {
+                                            int row0, int h, int b) {
 #pragma unroll
-  for (int c = 0; c < D / 64; ++c) tma_load_3d(dst + c * (BM * 128), map, bar, c * 64, row0, bh);
+  for (int c = 0; c < D / 64; ++c) tma_load_4d(dst + c * (BM * 128), map, bar, c * 64, row0, h, b);
 }
 
 __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes,
@@ -431,9 +432,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           } else {
             mbar_arrive_expect_tx(smem_u32(&bars->kv_full), 2 * Cfg::kKVBytes);
             ++kv_loads;
-            const int bh_kv = un.b * a.Hkv + un.hk;
-            load_kv_tile<D>(k_smem, &tm_k, smem_u32(&bars->kv_full), un.kt * TILE, bh_kv);
-            load_kv_tile<D>(v_smem, &tm_v, smem_u32(&bars->kv_full), un.kt * TILE, bh_kv);
+            load_kv_tile<D>(k_smem, &tm_k, smem_u32(&bars->kv_full), un.kt * TILE, un.hk, un.b);
+            load_kv_tile<D>(v_smem, &tm_v, smem_u32(&bars->kv_full), un.kt * TILE, un.hk, un.b);
             StepIter it;
             it.init(lst, n, a.G, a.Sq);
             int g, q0;
@@ -447,8 +447,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               ++stage_uses[s];
               const int bh = un.b * a.Hq + un.hk * a.G + g;
               BWD_EV(step, 0);
-              load_q_tile<D>(st, &tm_q, bar, q0, bh);
-              load_q_tile<D>(st + Cfg::kQBytes, &tm_do, bar, q0, bh);
+              load_q_tile<D>(st, &tm_q, bar, q0, un.hk * a.G + g, un.b);
+              load_q_tile<D>(st + Cfg::kQBytes, &tm_do, bar, q0, un.hk * a.G + g, un.b);
               const size_t row = static_cast<size_t>(bh) * a.Sq_pad + q0;
               bulk_load_1d(st + 2 * Cfg::kQBytes, a.lse2 + row, BM * 4, bar);
               bulk_load_1d(st + 2 * Cfg::kQBytes + 512, a.delta + row, BM * 4, bar);
@@ -658,7 +658,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ATTN25_TIMED(tr[7], mbar_wait_warp_ool(smem_u32(&bars->acc_full), unit_iter & 1, wc))) { ok = false; break; }
       tc_fence_after();
       ATTN25_TRACE_ONLY(const long long t_e = clock64();)
-      store_acc_rows<D>(a.dv + ((static_cast<size_t>(un.b) * a.Hkv + un.hk) * a.Skv + kv) * D, t_dv, 1.f,
+      store_acc_rows<D>(a.dv + un.b * a.dv_st.b + un.hk * a.dv_st.h + static_cast<long long>(kv) * a.dv_st.s, t_dv, 1.f,
                         n_steps > 0, kv < a.Skv);
       tc_fence_before();
       mbar_arrive(smem_u32(&bars->acc_empty));
@@ -759,7 +759,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ATTN25_TIMED(tr[7], mbar_wait_warp_ool(smem_u32(&bars->acc_full), unit_iter & 1, wc))) { ok = false; break; }
       tc_fence_after();
       ATTN25_TRACE_ONLY(const long long t_e = clock64();)
-      store_acc_rows<D>(a.dk + ((static_cast<size_t>(un.b) * a.Hkv + un.hk) * a.Skv + kv) * D, t_dk, a.scale,
+      store_acc_rows<D>(a.dk + un.b * a.dk_st.b + un.hk * a.dk_st.h + static_cast<long long>(kv) * a.dk_st.s, t_dk, a.scale,
                         n_steps > 0, kv < a.Skv);
       tc_fence_before();
       mbar_arrive(smem_u32(&bars->acc_empty));
@@ -846,10 +846,12 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
     const int q = static_cast<int>(row - bh * a.Sq_pad);
     float acc = 0.f;
     if (q < a.Sq) {
-      const size_t base = (static_cast<size_t>(bh) * a.Sq + q) * D;
+      const long long b = bh / a.Hq, h = bh - b * a.Hq;
+      const __nv_bfloat16* orow = a.out + b * a.o_st.b + h * a.o_st.h + q * a.o_st.s;
+      const __nv_bfloat16* grow = a.dout + b * a.do_st.b + h * a.do_st.h + q * a.do_st.s;
       for (int d = lane * 2; d < D; d += 64) {
-        const __nv_bfloat162 o2 = *reinterpret_cast<const __nv_bfloat162*>(a.out + base + d);
-        const __nv_bfloat162 g2 = *reinterpret_cast<const __nv_bfloat162*>(a.dout + base + d);
+        const __nv_bfloat162 o2 = *reinterpret_cast<const __nv_bfloat162*>(orow + d);
+        const __nv_bfloat162 g2 = *reinterpret_cast<const __nv_bfloat162*>(grow + d);
         acc = fmaf(__bfloat162float(o2.x), __bfloat162float(g2.x), acc);
         acc = fmaf(__bfloat162float(o2.y), __bfloat162float(g2.y), acc);
       }
@@ -890,7 +892,8 @@ __global__ void __launch_bounds__(256) bwd_dq_cast_kernel(const BwdArgs a) {
     o.y = pack_bf16x2(x0.z * a.scale, x0.w * a.scale);
     o.z = pack_bf16x2(x1.x * a.scale, x1.y * a.scale);
     o.w = pack_bf16x2(x1.z * a.scale, x1.w * a.scale);
-    *reinterpret_cast<uint4*>(a.dq + e) = o;
+    const long long b = bh / a.Hq, h = bh - b * a.Hq;
+    *reinterpret_cast<uint4*>(a.dq + b * a.dq_st.b + h * a.dq_st.h + q * a.dq_st.s + d) = o;
   }
 }
 

@@ -87,13 +87,14 @@ __device__ __forceinline__ UnitCoord decode_unit(const FwdArgs& a, int u) {
   return c;
 }
 
-// Load the tile rows [row0, row0+128) of head `bh` (all D columns) as
-// D/64 boxes of 64 columns, each 128 rows x 128 bytes with 128-byte swizzle.
+// Load the tile rows [row0, row0+128) of head h of batch row b (all D
+// columns) as D/64 boxes of 64 columns, each 128 rows x 128 bytes with
+// 128-byte swizzle; the tensor map is 4-D (D, S, H, B) with the tensor's strides.
 template <int D>
 __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                          int row0, int bh) {
+                                          int row0, int h, int b) {
 #pragma unroll
-  for (int c = 0; c < D / 64; ++c) tma_load_3d(dst + c * (TILE * 128), map, bar, c * 64, row0, bh);
+  for (int c = 0; c < D / 64; ++c) tma_load_4d(dst + c * (TILE * 128), map, bar, c * 64, row0, h, b);
 }
 
 template <int D>
@@ -354,10 +355,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         } else {
           mbar_arrive_expect_tx(smem_u32(&bars->q_full), 2 * Cfg::kTileBytes);
           ++q_loads;
-          const int bh_q = uc.b * a.Hq + uc.h;
-          load_tile<D>(q_smem[0], &tm_q, smem_u32(&bars->q_full), (2 * uc.p) * TILE, bh_q);
-          load_tile<D>(q_smem[1], &tm_q, smem_u32(&bars->q_full), (2 * uc.p + 1) * TILE, bh_q);
-          const int bh_kv = uc.b * a.Hkv + hk;
+          load_tile<D>(q_smem[0], &tm_q, smem_u32(&bars->q_full), (2 * uc.p) * TILE, uc.h, uc.b);
+          load_tile<D>(q_smem[1], &tm_q, smem_u32(&bars->q_full), (2 * uc.p + 1) * TILE, uc.h, uc.b);
           for (int j2 = 0; j2 < n && ok; ++j2) {
             const int kt = static_cast<int>(lst[j2] & 0xFFFFFu);
 #pragma unroll
@@ -368,7 +367,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               const uint32_t bar = smem_u32(&bars->kv_full[slot]);
               mbar_arrive_expect_tx(bar, Cfg::kTileBytes);
               load_tile<D>(ring + slot * Cfg::kTileBytes, which == 0 ? &tm_k : &tm_v, bar, kt * TILE,
-                           bh_kv);
+                           hk, uc.b);
               ++slot_uses[slot];
               ++ring_pos;
             }
@@ -601,7 +600,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tc_fence_after();
       const bool row_valid = rc.row < a.Sq;
       const size_t row_idx = (static_cast<size_t>(uc.b) * a.Hq + uc.h) * a.Sq + rc.row;
-      __nv_bfloat16* orow = a.out + row_idx * D;
+      __nv_bfloat16* orow = a.out + uc.b * a.o_st.b + uc.h * a.o_st.h + static_cast<long long>(rc.row) * a.o_st.s;
       const float inv_l = (l_run > 0.f) ? 1.0f / l_run : 0.f;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {

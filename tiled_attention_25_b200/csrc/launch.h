@@ -10,8 +10,14 @@
 
 namespace attn25 {
 
+// Element strides of a [B][H][S][D] tensor whose D elements are contiguous.
+struct Strides {
+  long long b, h, s;
+};
+
 struct FwdArgs {
   __nv_bfloat16* out;
+  Strides o_st;  // of out
   float* lse;
   int B, Hq, Hkv, G, Sq, Skv;
   int nQ, nK, nP, n_units;
@@ -37,6 +43,7 @@ struct BwdArgs {
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
+  Strides o_st, do_st, dq_st, dk_st, dv_st;  // of out, dout, dq, dk, dv
   int B, Hq, Hkv, G, Sq, Skv, Sq_pad;
   int nQ, nK, n_units;
   int num_sms;  // SMs of the device (grid caps of the prep and cast kernels)
