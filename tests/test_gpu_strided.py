@@ -6,8 +6,8 @@ import pytest
 import torch
 
 import oracle
-from gpu_common import Case
-from test_gpu_backward import small_params
+from gpu_common import Case, check_lse, check_o, host_f64
+from test_gpu_backward import check_grads, small_params
 
 pytestmark = pytest.mark.gpu
 
@@ -51,6 +51,11 @@ def test_bshd_views_match_contiguous_bitwise(ta, mod, D):
         assert torch.equal(a.view(torch.int16), b.contiguous().view(torch.int16))
     # dQ goes through L2 reductions in any order: close, not bitwise
     assert torch.allclose(dq.float(), dq2.float(), atol=2e-3, rtol=2e-2)
+    # and the strided results against the fp64 oracle
+    O, L = c.oracle_fwd()
+    check_o(host_f64(out2), O, f"strided mod {mod} D {D}")
+    check_lse(lse2.cpu().double().numpy(), L, f"strided mod {mod} D {D}")
+    check_grads([host_f64(t) for t in (dq2, dk2, dv2)], c.oracle_bwd(), f"strided mod {mod} D {D}")
 
 
 def test_bad_strides_are_refused(ta):
