@@ -278,6 +278,35 @@ ATTN25_API int attn_bwd_strided(const attn_bf16* q, const attn_bf16* k, const at
                                 const attn_block_mask* block_mask, const attn_layouts* layouts,
                                 attn_stream_t stream);
 
+/*
+ * The backward pass with a bitwise reproducible dQ.  dQ of a query row is a
+ * sum over the key tiles that meet it ("FlashAttention-2 — GPU attention의
+ * 사실상 표준", §4 Backward: the gradient of each query block collects one
+ * term per key block); attn_bwd adds those terms into its fp32 accumulator
+ * in whatever order the key tiles finish, so dQ's last bits vary from run to
+ * run.  Here every key tile waits for its turn before adding, and the terms
+ * enter each row's sum in ascending key-tile order, so dQ (like dK and dV)
+ * is the same bit for bit on every run, with or without a block mask.
+ *
+ * Arguments as attn_bwd (contiguous tensors).  workspace: device memory of
+ * attn_bwd_deterministic_workspace_size bytes, 256-byte aligned: the
+ * attn_bwd workspace plus four 32-bit counters per block of 64 query rows;
+ * its contents on entry do not matter.  The key tiles run in ascending order
+ * (not longest first), and a key tile may wait for the tiles before it: the
+ * kernel relies on all its CTAs being resident at once (one per SM), which
+ * holds unless other work shares the GPU's SMs at the same time (then a
+ * wait runs out and the call reports ATTN_ERR_TIMEOUT through
+ * attn_get_status instead of hanging).
+ */
+ATTN25_API size_t attn_bwd_deterministic_workspace_size(int B, int Hq, int Sq, int D);
+ATTN25_API int attn_bwd_deterministic(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v,
+                                      const attn_bf16* out, const float* lse, const attn_bf16* dout,
+                                      attn_bf16* dq, attn_bf16* dk, attn_bf16* dv,
+                                      void* workspace, size_t workspace_bytes,
+                                      int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+                                      int mod_kind, const attn_mod_params* mod_params,
+                                      const attn_block_mask* block_mask, attn_stream_t stream);
+
 /* Synchronise the stream, then return and clear the device status word. */
 ATTN25_API int attn_get_status(attn_stream_t stream);
 

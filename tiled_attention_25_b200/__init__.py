@@ -31,6 +31,8 @@ from .abi import (  # noqa: F401
     attn_block_mask_bind,
     attn_block_mask_bytes,
     attn_bwd,
+    attn_bwd_deterministic,
+    attn_bwd_deterministic_workspace_size,
     attn_bwd_strided,
     attn_bwd_noalloc,
     attn_bwd_noalloc_max_workspace,
@@ -56,9 +58,10 @@ def new_block_mask(mod_kind, mod_params, B, Sq, Skv, device="cuda", stream=None)
     return mask
 
 
-def new_bwd_workspace(B, Hq, Sq, D, device="cuda") -> torch.Tensor:
-    """A 256-byte-aligned workspace of attn_bwd_workspace_size bytes."""
-    nbytes = attn_bwd_workspace_size(B, Hq, Sq, D)
+def new_bwd_workspace(B, Hq, Sq, D, device="cuda", deterministic=False) -> torch.Tensor:
+    """A 256-byte-aligned workspace of attn_bwd_workspace_size bytes (or, with
+    deterministic=True, attn_bwd_deterministic_workspace_size bytes)."""
+    nbytes = (attn_bwd_deterministic_workspace_size if deterministic else attn_bwd_workspace_size)(B, Hq, Sq, D)
     buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
     off = (-buf.data_ptr()) % 256
     return buf[off:off + nbytes]

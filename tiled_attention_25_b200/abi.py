@@ -113,6 +113,10 @@ def _load():
     lib.attn_fwd_strided.restype = I
     lib.attn_bwd_strided.argtypes = [P, P, P, P, P, P, P, P, P, P, S, I, I, I, I, I, I, F, I, P, P, P, P]
     lib.attn_bwd_strided.restype = I
+    lib.attn_bwd_deterministic.argtypes = [P, P, P, P, P, P, P, P, P, P, S, I, I, I, I, I, I, F, I, P, P, P]
+    lib.attn_bwd_deterministic.restype = I
+    lib.attn_bwd_deterministic_workspace_size.argtypes = [I, I, I, I]
+    lib.attn_bwd_deterministic_workspace_size.restype = S
     lib.attn_get_status.argtypes = [P]
     lib.attn_get_status.restype = I
     lib.attn_set_wait_limit_ms.argtypes = [ctypes.c_uint32]
@@ -134,7 +138,8 @@ LIB = _load()
 EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_bwd_noalloc",
             "attn_bwd_noalloc_max_workspace", "attn_block_mask_bytes",
             "attn_block_mask_bind", "build_block_mask", "attn_get_status",
-            "attn_set_wait_limit_ms", "attn_strerror", "attn_fwd_strided", "attn_bwd_strided")
+            "attn_set_wait_limit_ms", "attn_strerror", "attn_fwd_strided", "attn_bwd_strided",
+            "attn_bwd_deterministic", "attn_bwd_deterministic_workspace_size")
 
 
 def attn_strerror(code: int) -> str:
@@ -313,6 +318,30 @@ def attn_bwd_strided(q, k, v, out, lse, dout, dq, dk, dv, workspace, scale=None,
                               None if block_mask is None else ctypes.byref(block_mask.c), ctypes.byref(lay),
                               _stream(stream))
     _check(rc, "attn_bwd_strided")
+
+
+def attn_bwd_deterministic_workspace_size(B, Hq, Sq, D) -> int:
+    return int(LIB.attn_bwd_deterministic_workspace_size(B, Hq, Sq, D))
+
+
+def attn_bwd_deterministic(q, k, v, out, lse, dout, dq, dk, dv, workspace, scale=None, mod_kind=MOD_NONE,
+                           mod_params=None, block_mask=None, stream=None):
+    """attn_bwd with a bitwise reproducible dQ (see include/attn25.h)."""
+    B, Hq, Hkv, Sq, Skv, D = _dims(q, k, v, out)
+    for t in (dout, dq):
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != (B, Hq, Sq, D) or not t.is_contiguous():
+            raise ValueError("dout/dq must be contiguous bf16 like q")
+    for t in (dk, dv):
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != (B, Hkv, Skv, D) or not t.is_contiguous():
+            raise ValueError("dk/dv must be contiguous bf16 like k")
+    scale = D ** -0.5 if scale is None else float(scale)
+    mp = _mp(mod_params, mod_kind, B, Hq, Sq)
+    rc = LIB.attn_bwd_deterministic(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+                                    _ptr(dk), _ptr(dv), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), B, Hq, Hkv, Sq, Skv, D,
+                                    scale, int(mod_kind), None if mp is None else mp[0],
+                                    None if block_mask is None else ctypes.byref(block_mask.c), _stream(stream))
+    _check(rc, "attn_bwd_deterministic")
 
 
 def attn_bwd_workspace_size(B, Hq, Sq, D) -> int:

@@ -481,11 +481,21 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Sq, int D) {
   return align256(rows * D * 4) + 2 * align256(rows * 4);
 }
 
-int attn_bwd_strided(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* out,
-                     const float* lse, const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk, attn_bf16* dv,
-                     void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int Sq, int Skv,
-                     int D, float scale, int mod_kind, const attn_mod_params* mod_params,
-                     const attn_block_mask* block_mask, const attn_layouts* layouts, attn_stream_t stream) {
+size_t attn_bwd_deterministic_workspace_size(int B, int Hq, int Sq, int D) {
+  const size_t base = attn_bwd_workspace_size(B, Hq, Sq, D);
+  if (base == 0) return 0;
+  // four counters per block of 64 query rows (one per 32-column slice of dQ)
+  const size_t blocks = static_cast<size_t>(B) * Hq * (cdiv(Sq, TILE) * TILE / 64);
+  return base + align256(blocks * 4 * sizeof(unsigned));
+}
+
+// The backward pass: det selects the ordered (bitwise reproducible) dQ sum.
+static int bwd_impl(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* out,
+                    const float* lse, const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk, attn_bf16* dv,
+                    void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int Sq, int Skv,
+                    int D, float scale, int mod_kind, const attn_mod_params* mod_params,
+                    const attn_block_mask* block_mask, const attn_layouts* layouts, bool det,
+                    attn_stream_t stream) {
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr ||
       dout == nullptr || dq == nullptr || dk == nullptr || dv == nullptr || workspace == nullptr)
     return ATTN_ERR_ARG;
@@ -496,7 +506,9 @@ int attn_bwd_strided(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v,
   int rc = check_common(B, Hq, Hkv, Sq, Skv, D, scale, mod_kind, mod_params, block_mask);
   if (rc == ATTN_OK) rc = check_bitmap_call(mod_kind, Hq, mod_params, block_mask);
   if (rc != ATTN_OK) return rc;
-  if (workspace_bytes < attn_bwd_workspace_size(B, Hq, Sq, D)) return ATTN_ERR_WORKSPACE;
+  const size_t need = det ? attn_bwd_deterministic_workspace_size(B, Hq, Sq, D)
+                         : attn_bwd_workspace_size(B, Hq, Sq, D);
+  if (workspace_bytes < need) return ATTN_ERR_WORKSPACE;
   DeviceInfo* d = nullptr;
   rc = current_device(&d);
   if (rc != ATTN_OK) return rc;
@@ -534,6 +546,13 @@ int attn_bwd_strided(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v,
     a.q_index = block_mask->q_index;
     a.bwd_order = block_mask->bwd_order;
   }
+  if (det) {
+    a.dq_sem = reinterpret_cast<unsigned*>(ws + attn_bwd_workspace_size(B, Hq, Sq, D));
+    if (block_mask != nullptr) {
+      a.kv_count = block_mask->kv_count;
+      a.kv_index = block_mask->kv_index;
+    }
+  }
   a.wait_ns = wait_ns();
   a.status = d->status;
   a.trace = d->trace == nullptr ? nullptr : d->trace + 128;
@@ -557,6 +576,25 @@ int attn_bwd_strided(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v,
                  reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_LAUNCH;
   return ATTN_OK;
+}
+
+int attn_bwd_strided(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* out,
+                     const float* lse, const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk, attn_bf16* dv,
+                     void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int Sq, int Skv,
+                     int D, float scale, int mod_kind, const attn_mod_params* mod_params,
+                     const attn_block_mask* block_mask, const attn_layouts* layouts, attn_stream_t stream) {
+  return bwd_impl(q, k, v, out, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, Sq, Skv, D,
+                  scale, mod_kind, mod_params, block_mask, layouts, false, stream);
+}
+
+int attn_bwd_deterministic(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* out,
+                           const float* lse, const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk,
+                           attn_bf16* dv, void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
+                           int Sq, int Skv, int D, float scale, int mod_kind,
+                           const attn_mod_params* mod_params, const attn_block_mask* block_mask,
+                           attn_stream_t stream) {
+  return bwd_impl(q, k, v, out, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, Sq, Skv, D,
+                  scale, mod_kind, mod_params, block_mask, nullptr, true, stream);
 }
 
 int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* out,

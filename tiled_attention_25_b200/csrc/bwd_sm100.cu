@@ -73,7 +73,10 @@ struct BwdCfg {
   static constexpr int kDSBytes = TILE * BM * 2;
   static constexpr int kBarOff = kDSOff + 2 * kDSBytes;
   static constexpr int kListOff = kBarOff + 1024;  // two query-tile lists (16-bit entries)
-  static constexpr int kSmemBytes = kListOff + 2 * kMaxSteps * 2;
+  // deterministic dQ: for each list entry, how many key tiles before this
+  // unit's add into that query tile (16-bit entries, two lists)
+  static constexpr int kPosOff = kListOff + 2 * kMaxSteps * 2;
+  static constexpr int kSmemBytes = kPosOff + 2 * kMaxSteps * 2;
   static constexpr int kAllocBytes = kSmemBytes + 1024;
   static_assert(kAllocBytes <= 232448, "shared memory");
   // TMEM columns: two S^T buffers (P^T overwrites their first 32 columns), dP^T,
@@ -112,12 +115,18 @@ struct BwdUnit {
 
 __device__ __forceinline__ BwdUnit decode_bwd_unit(const BwdArgs& a, int u) {
   const int pair_idx = u / a.Hkv;
-  const int hk = u - pair_idx * a.Hkv;
-  const int pair = (a.bwd_order != nullptr) ? __ldg(a.bwd_order + pair_idx) : pair_idx;
   BwdUnit r;
+  r.hk = u - pair_idx * a.Hkv;
+  if (a.dq_sem != nullptr) {
+    // deterministic dQ: ascending key tiles (across batch rows and KV heads),
+    // so that every unit waits only on units of lower rank
+    r.kt = pair_idx / a.B;
+    r.b = pair_idx - r.kt * a.B;
+    return r;
+  }
+  const int pair = (a.bwd_order != nullptr) ? __ldg(a.bwd_order + pair_idx) : pair_idx;
   r.b = pair / a.nK;
   r.kt = pair - r.b * a.nK;
-  r.hk = hk;
   return r;
 }
 
@@ -162,7 +171,90 @@ struct StepIter {
       return true;
     }
   }
+
+  // List index of the entry of the last step next() returned.
+  __device__ __forceinline__ int entry() const { return j - 1; }
 };
+
+// ------------------------------------------------------------------ deterministic dQ
+//
+// Every key tile that meets a query tile adds its dQ part into the fp32
+// accumulator; to make the sum's order fixed, the adds into each block of 64
+// query rows (and each 32-column slice, one per drain warp) are ordered by
+// key tile: a counter per (row block, slice) holds how many key tiles have
+// added, and the unit of key tile kt waits until it equals the number of
+// key tiles before kt that meet the query tile (its position).  Units are
+// walked in ascending key-tile order and each CTA takes them in ascending
+// rank, so a unit only ever waits on units of lower rank, which are running
+// or done on other CTAs (all CTAs are resident: one per SM).
+
+// Positions of the list entries of key tile kt (whole warp): the lower bound
+// of kt in the block mask's ascending key-tile list of each query tile, or,
+// without a block mask, the count of earlier key tiles with a non-empty dense
+// class (the same classes the units' step lists come from).
+__device__ __forceinline__ void build_positions(const BwdArgs& a, int b, int kt, const uint16_t* lst,
+                                                int n, uint16_t* pos) {
+  __syncwarp();  // the list entries were written by other lanes
+  for (int j = threadIdx.x & 31; j < n; j += 32) {
+    const int qt = static_cast<int>(lst[j] & kQtIndexMask);
+    int p = 0;
+    if (a.kv_index != nullptr) {
+      const size_t r = static_cast<size_t>(b) * a.nQ + qt;
+      const int32_t* row = a.kv_index + r * a.nK;
+      int hi = __ldg(a.kv_count + r);
+      while (p < hi) {
+        const int mid = (p + hi) >> 1;
+        if (__ldg(row + mid) < kt) p = mid + 1; else hi = mid;
+      }
+    } else {
+      const int q0 = qt * TILE, q1 = min(a.Sq, q0 + TILE);
+      for (int k2 = 0; k2 < kt; ++k2)
+        p += dense_tile_class(a.mod.mask, a.mod.window, q0, q1, k2 * TILE, min(a.Skv, k2 * TILE + TILE)) != 0;
+    }
+    pos[j] = static_cast<uint16_t>(p);
+  }
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Warp-collective: wait (bounded) until the counter equals `want`; every lane
+// then holds an acquire of it, so its reductions follow the earlier adds.
+static __device__ __noinline__ bool sem_wait_eq(const unsigned* sem, unsigned want, WaitCtl w) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) {
+    uint64_t t0 = 0;
+    bool timed = false;
+    while (ld_acquire_gpu(sem) != want) {
+      if (aborted(w)) {
+        ok = false;
+        break;
+      }
+      const uint64_t t = globaltimer();
+      if (!timed) {
+        t0 = t;
+        timed = true;
+      } else if (t - t0 > w.limit_ns) {
+        record_error(kErrTimeout, w);
+        ok = false;
+        break;
+      }
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  if (ok) (void)ld_acquire_gpu(sem);
+  return ok;
+}
+
+// Warp-collective: publish this warp's adds (each lane fences its own), then count them.
+__device__ __forceinline__ void sem_release(unsigned* sem) {
+  __threadfence();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) atomicAdd(sem, 1u);
+}
 
 // Tiles of head h of batch row b through 4-D tensor maps (D, S, H, B).
 template <int D>
@@ -356,6 +448,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t k_smem = sbase + Cfg::kKOff;
   const uint32_t v_smem = sbase + Cfg::kVOff;
   uint16_t* lists = reinterpret_cast<uint16_t*>(smem + Cfg::kListOff);
+  uint16_t* positions = reinterpret_cast<uint16_t*>(smem + Cfg::kPosOff);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -424,6 +517,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!mbar_wait_warp_ool(smem_u32(&bars->list_empty[buf]), ((unit_iter >> 1) & 1) ^ 1, wc)) { ok = false; break; }
         const int n = build_kv_qtiles(a.tile_class, un.b, un.kt, a.nQ, a.nK, a.Sq, a.Skv, a.mod.mask,
                                       a.mod.window, lst);
+        if (a.dq_sem != nullptr) build_positions(a, un.b, un.kt, lst, n, positions + buf * kMaxSteps);
         if (lane == 0) bars->list_n[buf] = n;
         mbar_arrive(smem_u32(&bars->list_full[buf]));
         if (lane == 0) {
@@ -814,8 +908,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (active) {
           const int bh = un.b * a.Hq + un.hk * a.G + g;
           float* dst = a.dq_acc + (static_cast<size_t>(bh) * a.Sq_pad + q0) * D + w * 32 + lane;
+          unsigned* sem = nullptr;
+          if (a.dq_sem != nullptr) {  // deterministic dQ: wait for this unit's turn
+            sem = a.dq_sem + (static_cast<size_t>(bh) * (a.Sq_pad / BM) + q0 / BM) * 4 + w;
+            if (!sem_wait_eq(sem, positions[buf * kMaxSteps + it.entry()], wc)) {
+              ok = false;
+              break;
+            }
+          }
 #pragma unroll
           for (int c = 0; c < BM; ++c) atomicAdd(dst + static_cast<size_t>(c) * D, v[c]);
+          if (sem != nullptr) sem_release(sem);
         }
         ATTN25_TRACE_ONLY(tr[2] += clock64() - t_r;)
         BWD_EV(step, 15);
@@ -860,6 +963,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     float4* z = reinterpret_cast<float4*>(a.dq_acc + static_cast<size_t>(row) * D);
     for (int i = lane; i < D / 4; i += 32) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    // deterministic dQ: the counters of this 64-row block start at zero
+    if (a.dq_sem != nullptr && (q % BM) == 0 && lane < 4) a.dq_sem[(row / BM) * 4 + lane] = 0u;
     if (lane == 0) {
       // stored negated, so that the main kernel's exponent is one FFMA:
       // -LSE log2(e), or -inf where the row keeps nothing or lies past Sq (P = 0)

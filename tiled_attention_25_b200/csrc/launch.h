@@ -53,6 +53,15 @@ struct BwdArgs {
   const int32_t* q_count;
   const int32_t* q_index;
   const int32_t* bwd_order;
+  // Deterministic dQ: per (row block of 64 queries, 32-column slice of dQ)
+  // counters [B*Hq][Sq_pad/64][4] of the key tiles that have added their
+  // part, so that the parts enter the fp32 sum in ascending key-tile order
+  // (nullptr: reductions in any order).  The positions come from the block
+  // mask's key-tile lists (kv_count / kv_index) or, without one, from the
+  // dense tile classes.
+  unsigned int* dq_sem;
+  const int32_t* kv_count;
+  const int32_t* kv_index;
   uint64_t wait_ns;
   int* status;
   unsigned long long* trace;  // profiling builds only (else nullptr)
