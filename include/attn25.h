@@ -313,6 +313,17 @@ ATTN25_API int attn_get_status(attn_stream_t stream);
 /* Set the per-wait time limit of the kernels in milliseconds (default 4000). */
 ATTN25_API void attn_set_wait_limit_ms(uint32_t ms);
 
+/*
+ * Self-check of the timeout path (the pages have no counterpart: it exists
+ * so that a caller can see the error path work on its own GPU).  Launches on
+ * the stream a kernel whose one wait is on a barrier that nothing arrives at;
+ * after the current wait limit it gives up, records ATTN_ERR_TIMEOUT in the
+ * device status word and returns, as an attention kernel does when one of
+ * its waits runs out.  attn_get_status then returns ATTN_ERR_TIMEOUT (and
+ * clears it); the context stays usable.  Returns ATTN_OK once launched.
+ */
+ATTN25_API int attn_check_wait_timeout(attn_stream_t stream);
+
 /* A static description of an attn_status value. */
 ATTN25_API const char* attn_strerror(int status);
 

@@ -37,6 +37,7 @@ from .abi import (  # noqa: F401
     attn_bwd_noalloc,
     attn_bwd_noalloc_max_workspace,
     attn_bwd_workspace_size,
+    attn_check_wait_timeout,
     attn_fwd,
     attn_fwd_strided,
     attn_get_status,

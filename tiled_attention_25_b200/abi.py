@@ -121,6 +121,8 @@ def _load():
     lib.attn_get_status.restype = I
     lib.attn_set_wait_limit_ms.argtypes = [ctypes.c_uint32]
     lib.attn_set_wait_limit_ms.restype = None
+    lib.attn_check_wait_timeout.argtypes = [P]
+    lib.attn_check_wait_timeout.restype = I
     lib.attn_strerror.argtypes = [I]
     lib.attn_strerror.restype = ctypes.c_char_p
     if hasattr(lib, "attn_trace_read"):  # profiling build only
@@ -139,7 +141,7 @@ EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_bwd_noalloc
             "attn_bwd_noalloc_max_workspace", "attn_block_mask_bytes",
             "attn_block_mask_bind", "build_block_mask", "attn_get_status",
             "attn_set_wait_limit_ms", "attn_strerror", "attn_fwd_strided", "attn_bwd_strided",
-            "attn_bwd_deterministic", "attn_bwd_deterministic_workspace_size")
+            "attn_bwd_deterministic", "attn_bwd_deterministic_workspace_size", "attn_check_wait_timeout")
 
 
 def attn_strerror(code: int) -> str:
@@ -414,6 +416,12 @@ def attn_get_status(stream=None) -> int:
 
 def attn_set_wait_limit_ms(ms: int):
     LIB.attn_set_wait_limit_ms(int(ms))
+
+
+def attn_check_wait_timeout(stream=None):
+    """Launch the timeout self-check (see include/attn25.h); read the outcome
+    with attn_get_status."""
+    _check(LIB.attn_check_wait_timeout(_stream(stream)), "attn_check_wait_timeout")
 
 
 def attn_trace_read(n: int = 256) -> list:

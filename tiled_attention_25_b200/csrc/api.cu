@@ -120,6 +120,22 @@ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 
 uint64_t wait_ns() { return static_cast<uint64_t>(g_wait_ms.load()) * 1000000ull; }
 
+// One warp waits, with the kernels' bounded wait, on a barrier that nothing
+// arrives at: after the wait limit it records ATTN_ERR_TIMEOUT in the status
+// word and returns, the same path a kernel takes when one of its waits runs out.
+__global__ void wait_check_kernel(uint64_t limit_ns, int* status) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t abort_word;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_word = 0;
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const WaitCtl wc{limit_ns, smem_u32(&abort_word), status};
+  (void)mbar_wait_warp(smem_u32(&bar), 0, wc);
+}
+
 // A mod code split into its score transform and mask bits (composition:
 // one of the seven kinds, optionally ORed with ATTN_MASK_* flags).
 struct ModSpec {
@@ -317,6 +333,14 @@ const char* attn_strerror(int status) {
 }
 
 void attn_set_wait_limit_ms(uint32_t ms) { g_wait_ms.store(ms < 1 ? 1 : ms); }
+
+int attn_check_wait_timeout(attn_stream_t stream) {
+  DeviceInfo* d = nullptr;
+  const int rc = current_device(&d);
+  if (rc != ATTN_OK) return rc;
+  wait_check_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(wait_ns(), d->status);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
 
 int attn_get_status(attn_stream_t stream) {
   DeviceInfo* d = nullptr;

@@ -552,8 +552,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       }
-      if (!ok && lane == 0) {
-        const WaitCtl dwc{a.wait_ns, smem_u32(&bars->never_set), a.status};
+      if (lane == 0) {
+        // let the copies in flight land before the CTA exits (also after a
+        // normal end: a consumer that gave up may have left them unconsumed)
+        const WaitCtl dwc{drain_limit(a.wait_ns), smem_u32(&bars->never_set), a.status};
         if (kv_loads) mbar_wait_thread_ool(smem_u32(&bars->kv_full), (kv_loads - 1) & 1, dwc);
         for (int s = 0; s < Cfg::kStages; ++s)
           if (stage_uses[s]) mbar_wait_thread_ool(smem_u32(&bars->q_full[s]), (stage_uses[s] - 1) & 1, dwc);
@@ -681,7 +683,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
 #undef MMA_WAIT
       mma_commit_w(smem_u32(&bars->drain));
-      mbar_wait_warp_ool(smem_u32(&bars->drain), 0, WaitCtl{a.wait_ns, smem_u32(&bars->never_set), a.status});
+      mbar_wait_warp_ool(smem_u32(&bars->drain), 0, WaitCtl{drain_limit(a.wait_ns), smem_u32(&bars->never_set), a.status});
       ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start; tr[7] = step;)
       trace_flush(a.trace, 32, tr);
     }

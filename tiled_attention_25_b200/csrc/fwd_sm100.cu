@@ -376,9 +376,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     }
-    if (!ok && lane == 0) {
-      // let copies already in flight land before the CTA exits
-      const WaitCtl drain_wc{a.wait_ns, smem_u32(&bars->never_set), a.status};
+    if (lane == 0) {
+      // let the copies in flight land before the CTA exits: after a failed wait
+      // of this warp, and also after a normal end, since a consumer that gave
+      // up may have left the last copies unconsumed (instant otherwise)
+      const WaitCtl drain_wc{drain_limit(a.wait_ns), smem_u32(&bars->never_set), a.status};
       for (int s2 = 0; s2 < Cfg::kStages; ++s2) {
         if (slot_uses[s2] == 0) continue;
         mbar_wait_thread(smem_u32(&bars->kv_full[s2]), (slot_uses[s2] - 1) & 1, drain_wc);
@@ -485,7 +487,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     // drain: wait until every MMA this warp issued has completed
     mma_commit_w(smem_u32(&bars->drain));
-    mbar_wait_warp(smem_u32(&bars->drain), 0, WaitCtl{a.wait_ns, smem_u32(&bars->never_set), a.status});
+    mbar_wait_warp(smem_u32(&bars->drain), 0, WaitCtl{drain_limit(a.wait_ns), smem_u32(&bars->never_set), a.status});
     ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
     trace_flush(a.trace, 32, tr);
   }

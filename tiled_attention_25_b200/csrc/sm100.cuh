@@ -59,6 +59,14 @@ struct WaitCtl {
   int* status;           // device status word (0, or the first error recorded)
 };
 
+// Limit of the waits by which a role lets its own copies and MMAs land before
+// the CTA exits: those complete on their own within microseconds, so they get
+// at least a second whatever limit the caller set for the other waits.
+constexpr uint64_t kDrainFloorNs = 1000000000ull;
+__device__ __forceinline__ uint64_t drain_limit(uint64_t limit_ns) {
+  return limit_ns > kDrainFloorNs ? limit_ns : kDrainFloorNs;
+}
+
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
