@@ -44,7 +44,10 @@ def same_bits(a, b):
 @pytest.mark.parametrize("use_mask", [False, True])
 def test_deterministic_repeats_and_matches_oracle(ta, mod, D, use_mask):
     S = 700  # six key tiles, a ragged tail
-    c = Case(90 + mod + D, 2, 4, 2, S, S, D, mod, small_params(mod, S))
+    p = small_params(mod, S)
+    if p.doc_offsets is not None:  # one list of documents per batch row
+        p.doc_offsets = [p.doc_offsets[0], [0, 100, 555, S]]
+    c = Case(90 + mod + D, 2, 4, 2, S, S, D, mod, p)
     a = run_det(ta, c, use_mask, fill=0x7F)
     b = run_det(ta, c, use_mask, fill=0x00)
     assert same_bits(a, b)

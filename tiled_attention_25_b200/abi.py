@@ -237,6 +237,16 @@ def _mp(mod_params, mod_kind, B, Hq, Sq):
     call reads (the C side cannot see its extent)."""
     if mod_params is None:
         return None
+    code = int(mod_kind)
+    # offsets arrays: one row per batch row (the C side cannot see their extent)
+    if (code & 0xFF) == MOD_DOCUMENT or code & MASK_DOCUMENT:
+        t = mod_params.doc_offsets
+        if t is None or t.shape[0] < B:
+            raise ValueError(f"the document mask needs doc_offsets with {B} rows")
+    if code & MASK_VARLEN:
+        t = mod_params.q_offsets
+        if t is None or t.shape[0] < B:
+            raise ValueError(f"the varlen mask needs q_offsets and k_offsets with {B} rows")
     bm = mod_params.bitmap
     if int(mod_kind) & MASK_BITMAP and bm is not None:
         nb, nh, sq, _ = bm.shape
