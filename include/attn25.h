@@ -307,6 +307,41 @@ ATTN25_API int attn_bwd_deterministic(const attn_bf16* q, const attn_bf16* k, co
                                       int mod_kind, const attn_mod_params* mod_params,
                                       const attn_block_mask* block_mask, attn_stream_t stream);
 
+/*
+ * FP8 incoherent processing of queries or keys ("FlashAttention-3 …",
+ * FlashAttention-3의 기술적 혁신, item 3).  Each row of x (device bf16
+ * [B][H][S][D], D = 64 or 128, 16-byte aligned) is rotated by
+ * diag(signs) H_D / sqrt(D), H_D the Sylvester Hadamard matrix and signs
+ * (device int8 [D]) a vector of +-1 that the caller draws once; then every
+ * (b, h) is quantised to OCP e4m3 (round to nearest even, saturating at 448)
+ * with one scale, its absolute maximum / 448.
+ *   codes:  device uint8 [B][H][S][D] (16-byte aligned): the e4m3 values;
+ *   scales: device fp32 [B][H]: x rotated ~= codes * scales.
+ * The steps are exactly rounded fp32 operations in a fixed order (sign flip,
+ * Walsh-Hadamard butterflies h = 1, 2, ..., D/2, one product by fp32
+ * 1/sqrt(D), IEEE division by the scale), so the codes are reproducible.
+ * B * H must not exceed 65535.
+ */
+ATTN25_API int attn_fp8_rotate_quantize(const attn_bf16* x, const int8_t* signs, uint8_t* codes,
+                                        float* scales, int B, int H, int S, int D,
+                                        attn_stream_t stream);
+
+/*
+ * The forward pass with FP8 scores: q8 and k8 are the e4m3 codes that
+ * attn_fp8_rotate_quantize made of Q and K (device uint8 [B][Hq][Sq][D] and
+ * [B][Hkv][Skv][D], 16-byte aligned, rotated by the same signs), and
+ * q_scales [B][Hq], k_scales [B][Hkv] their fp32 scales.  S = Q8 K8^T is
+ * formed by tcgen05 MMAs of kind f8f6f4 and dequantised in the softmax's
+ * scale; v, out, lse, the masks and the block mask are as in attn_fwd.
+ * D must be 128; mod_kind may hold masks but no score transform
+ * (ATTN_ERR_UNSUPPORTED otherwise).
+ */
+ATTN25_API int attn_fwd_fp8(const uint8_t* q8, const uint8_t* k8, const float* q_scales,
+                            const float* k_scales, const attn_bf16* v, attn_bf16* out, float* lse,
+                            int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+                            int mod_kind, const attn_mod_params* mod_params,
+                            const attn_block_mask* block_mask, attn_stream_t stream);
+
 /* Synchronise the stream, then return and clear the device status word. */
 ATTN25_API int attn_get_status(attn_stream_t stream);
 

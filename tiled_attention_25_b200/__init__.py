@@ -38,7 +38,9 @@ from .abi import (  # noqa: F401
     attn_bwd_noalloc_max_workspace,
     attn_bwd_workspace_size,
     attn_check_wait_timeout,
+    attn_fp8_rotate_quantize,
     attn_fwd,
+    attn_fwd_fp8,
     attn_fwd_strided,
     attn_get_status,
     attn_set_wait_limit_ms,

@@ -117,6 +117,10 @@ def _load():
     lib.attn_bwd_deterministic.restype = I
     lib.attn_bwd_deterministic_workspace_size.argtypes = [I, I, I, I]
     lib.attn_bwd_deterministic_workspace_size.restype = S
+    lib.attn_fwd_fp8.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P, P, P]
+    lib.attn_fwd_fp8.restype = I
+    lib.attn_fp8_rotate_quantize.argtypes = [P, P, P, P, I, I, I, I, P]
+    lib.attn_fp8_rotate_quantize.restype = I
     lib.attn_get_status.argtypes = [P]
     lib.attn_get_status.restype = I
     lib.attn_set_wait_limit_ms.argtypes = [ctypes.c_uint32]
@@ -141,7 +145,8 @@ EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_bwd_noalloc
             "attn_bwd_noalloc_max_workspace", "attn_block_mask_bytes",
             "attn_block_mask_bind", "build_block_mask", "attn_get_status",
             "attn_set_wait_limit_ms", "attn_strerror", "attn_fwd_strided", "attn_bwd_strided",
-            "attn_bwd_deterministic", "attn_bwd_deterministic_workspace_size", "attn_check_wait_timeout")
+            "attn_bwd_deterministic", "attn_bwd_deterministic_workspace_size", "attn_check_wait_timeout",
+            "attn_fp8_rotate_quantize", "attn_fwd_fp8")
 
 
 def attn_strerror(code: int) -> str:
@@ -330,6 +335,47 @@ def attn_bwd_strided(q, k, v, out, lse, dout, dq, dk, dv, workspace, scale=None,
                               None if block_mask is None else ctypes.byref(block_mask.c), ctypes.byref(lay),
                               _stream(stream))
     _check(rc, "attn_bwd_strided")
+
+
+def attn_fp8_rotate_quantize(x, signs, codes, scales, stream=None):
+    """x: CUDA bf16 [B][H][S][D]; signs: CUDA int8 [D] of +-1; codes: CUDA uint8
+    like x; scales: CUDA fp32 [B][H]."""
+    if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous() or x.dim() != 4:
+        raise ValueError("x must be a contiguous CUDA bf16 [B][H][S][D] tensor")
+    B, H, S, D = x.shape
+    if signs.dtype != torch.int8 or tuple(signs.shape) != (D,) or not signs.is_contiguous():
+        raise ValueError("signs must be a contiguous int8 [D] tensor")
+    if codes.dtype != torch.uint8 or tuple(codes.shape) != (B, H, S, D) or not codes.is_contiguous():
+        raise ValueError("codes must be a contiguous uint8 tensor shaped like x")
+    if scales.dtype != torch.float32 or tuple(scales.shape) != (B, H) or not scales.is_contiguous():
+        raise ValueError("scales must be a contiguous fp32 [B][H] tensor")
+    _check(LIB.attn_fp8_rotate_quantize(_ptr(x), _ptr(signs), _ptr(codes), _ptr(scales), B, H, S, D,
+                                        _stream(stream)), "attn_fp8_rotate_quantize")
+
+
+def attn_fwd_fp8(q8, k8, q_scales, k_scales, v, out, lse=None, scale=None, mod_kind=MOD_NONE, mod_params=None,
+                 block_mask=None, stream=None):
+    """The forward with e4m3 Q and K (codes from attn_fp8_rotate_quantize)."""
+    for t, name in ((q8, "q8"), (k8, "k8")):
+        if t.dtype != torch.uint8 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous CUDA uint8 [B][H][S][D] tensor")
+    B, Hq, Sq, D = q8.shape
+    Bk, Hkv, Skv, Dk = k8.shape
+    if (Bk, Dk) != (B, D) or tuple(v.shape) != (B, Hkv, Skv, D) or tuple(out.shape) != (B, Hq, Sq, D):
+        raise ValueError("inconsistent q8/k8/v/out shapes")
+    for t in (v, out):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("v and out must be contiguous CUDA bf16 tensors")
+    if tuple(q_scales.shape) != (B, Hq) or tuple(k_scales.shape) != (B, Hkv):
+        raise ValueError("q_scales must be [B][Hq] and k_scales [B][Hkv]")
+    if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hq, Sq) or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous fp32 [B][Hq][Sq] tensor")
+    scale = D ** -0.5 if scale is None else float(scale)
+    mp = _mp(mod_params, mod_kind, B, Hq, Sq)
+    rc = LIB.attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(q_scales), _ptr(k_scales), _ptr(v), _ptr(out), _ptr(lse),
+                          B, Hq, Hkv, Sq, Skv, D, scale, int(mod_kind), None if mp is None else mp[0],
+                          None if block_mask is None else ctypes.byref(block_mask.c), _stream(stream))
+    _check(rc, "attn_fwd_fp8")
 
 
 def attn_bwd_deterministic_workspace_size(B, Hq, Sq, D) -> int:

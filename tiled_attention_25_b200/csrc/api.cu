@@ -103,6 +103,20 @@ bool encode_bf16_4d(CUtensorMap* m, const void* base, int D, int S, int H, int B
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Contiguous [B][H][S][D = 128] e4m3 codes as the 4-D map (D, S, H, B): one
+// box of 128 bytes x box_rows rows, 128-byte swizzle.
+bool encode_u8_4d(CUtensorMap* m, const void* base, int D, int S, int H, int B, int box_rows) {
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S) * D,
+                           static_cast<cuuint64_t>(H) * S * D};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(D), static_cast<cuuint32_t>(box_rows), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // The strides of a tensor: the caller's, or those of contiguous [B][H][S][D].
 bool layout_of(const attn_strides* given, int H, int S, int D, Strides& st) {
   if (given == nullptr) {
@@ -432,10 +446,12 @@ int build_block_mask(int mod_kind, const attn_mod_params* mod_params, int B, int
   return ATTN_OK;
 }
 
-int attn_fwd_strided(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* out,
-                     float* lse, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
-                     int mod_kind, const attn_mod_params* mod_params, const attn_block_mask* block_mask,
-                     const attn_layouts* layouts, attn_stream_t stream) {
+// The forward: bf16 Q and K (strided), or (fp8) contiguous e4m3 codes of Q
+// and K with their per-head scales.
+static int fwd_impl(const void* q, const void* k, const attn_bf16* v, attn_bf16* out, float* lse,
+                    const float* q_scales, const float* k_scales, bool fp8, int B, int Hq, int Hkv, int Sq,
+                    int Skv, int D, float scale, int mod_kind, const attn_mod_params* mod_params,
+                    const attn_block_mask* block_mask, const attn_layouts* layouts, attn_stream_t stream) {
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ATTN_ERR_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
       (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
@@ -454,14 +470,17 @@ int attn_fwd_strided(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v,
       !layout_of(layouts ? &layouts->out : nullptr, Hq, Sq, D, so))
     return ATTN_ERR_ALIGN;
   CUtensorMap tq, tk, tv;
-  if (!encode_bf16_4d(&tq, q, D, Sq, Hq, B, sq, TILE) || !encode_bf16_4d(&tk, k, D, Skv, Hkv, B, sk, TILE) ||
-      !encode_bf16_4d(&tv, v, D, Skv, Hkv, B, sv, TILE))
-    return ATTN_ERR_ARG;
+  const bool qk_ok = fp8 ? encode_u8_4d(&tq, q, D, Sq, Hq, B, TILE) && encode_u8_4d(&tk, k, D, Skv, Hkv, B, TILE)
+                         : encode_bf16_4d(&tq, q, D, Sq, Hq, B, sq, TILE) &&
+                               encode_bf16_4d(&tk, k, D, Skv, Hkv, B, sk, TILE);
+  if (!qk_ok || !encode_bf16_4d(&tv, v, D, Skv, Hkv, B, sv, TILE)) return ATTN_ERR_ARG;
 
   FwdArgs a{};
   a.out = reinterpret_cast<__nv_bfloat16*>(out);
   a.o_st = so;
   a.lse = lse;
+  a.q_scales = q_scales;
+  a.k_scales = k_scales;
   a.B = B;
   a.Hq = Hq;
   a.Hkv = Hkv;
@@ -485,10 +504,48 @@ int attn_fwd_strided(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v,
   a.status = d->status;
   a.trace = d->trace;
   const int grid = a.n_units < d->sms ? a.n_units : d->sms;
-  if (launch_fwd(tq, tk, tv, a, D, mod_key(mod_kind), lse != nullptr, grid,
-                 reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return ATTN_ERR_LAUNCH;
-  return ATTN_OK;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const cudaError_t e = fp8 ? launch_fwd_fp8(tq, tk, tv, a, mod_key(mod_kind), lse != nullptr, grid, st)
+                            : launch_fwd(tq, tk, tv, a, D, mod_key(mod_kind), lse != nullptr, grid, st);
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+int attn_fwd_strided(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* out,
+                     float* lse, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+                     int mod_kind, const attn_mod_params* mod_params, const attn_block_mask* block_mask,
+                     const attn_layouts* layouts, attn_stream_t stream) {
+  return fwd_impl(q, k, v, out, lse, nullptr, nullptr, false, B, Hq, Hkv, Sq, Skv, D, scale, mod_kind,
+                  mod_params, block_mask, layouts, stream);
+}
+
+int attn_fwd_fp8(const uint8_t* q8, const uint8_t* k8, const float* q_scales, const float* k_scales,
+                 const attn_bf16* v, attn_bf16* out, float* lse, int B, int Hq, int Hkv, int Sq, int Skv,
+                 int D, float scale, int mod_kind, const attn_mod_params* mod_params,
+                 const attn_block_mask* block_mask, attn_stream_t stream) {
+  if (q_scales == nullptr || k_scales == nullptr) return ATTN_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(q_scales) & 3u) || (reinterpret_cast<uintptr_t>(k_scales) & 3u))
+    return ATTN_ERR_ALIGN;
+  if (D != 128) return ATTN_ERR_UNSUPPORTED;
+  ModSpec ms;
+  if (split_mod(mod_kind, ms) && ms.score != MOD_NONE) return ATTN_ERR_UNSUPPORTED;  // masks only
+  return fwd_impl(q8, k8, v, out, lse, q_scales, k_scales, true, B, Hq, Hkv, Sq, Skv, D, scale, mod_kind,
+                  mod_params, block_mask, nullptr, stream);
+}
+
+int attn_fp8_rotate_quantize(const attn_bf16* x, const int8_t* signs, uint8_t* codes, float* scales, int B,
+                             int H, int S, int D, attn_stream_t stream) {
+  if (x == nullptr || signs == nullptr || codes == nullptr || scales == nullptr) return ATTN_ERR_ARG;
+  if (B < 1 || H < 1 || S < 1) return ATTN_ERR_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > 65535) return ATTN_ERR_UNSUPPORTED;  // one grid row per head
+  if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u)) return ATTN_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  const int rc = current_device(&d);
+  if (rc != ATTN_OK) return rc;
+  return launch_fp8_prep(x, signs, codes, scales, B * H, S, D, d->sms, reinterpret_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? ATTN_OK
+             : ATTN_ERR_LAUNCH;
 }
 
 int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* out,

@@ -54,6 +54,8 @@ struct FwdCfg {
   static constexpr int kSmemBytes = kListOff + 2 * kMaxSteps * 4;
   static constexpr int kAllocBytes = kSmemBytes + 1024;     // + alignment slack
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
+  static constexpr uint32_t kIdescQK8 = idesc_e4m3_f32(128, 128, false, false);
+  static constexpr int kTileBytes8 = TILE * D;             // one 128 x D e4m3 tile
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);
 };
 
@@ -97,13 +99,36 @@ __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* map, 
   for (int c = 0; c < D / 64; ++c) tma_load_4d(dst + c * (TILE * 128), map, bar, c * 64, row0, h, b);
 }
 
-template <int D>
+template <int D, bool FP8 = false>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+  if constexpr (FP8) {
+    // e4m3 rows of D = 128 bytes fill one 128-byte swizzle row: 4 MMAs of K = 32
+    static_assert(D == 128, "FP8 scores need D = 128");
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * (TILE * 128) + (kk & 3) * 32;
-    mma_ss_w(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024), smem_desc_sw128(k_smem + off, 16, 1024),
-             FwdCfg<D>::kIdescQK, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < D / 32; ++kk) {
+      const uint32_t off = kk * 32;
+      mma_ss_f8_w(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024), smem_desc_sw128(k_smem + off, 16, 1024),
+                  FwdCfg<D>::kIdescQK8, kk > 0 ? 1u : 0u);
+    }
+  } else {
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t off = (kk >> 2) * (TILE * 128) + (kk & 3) * 32;
+      mma_ss_w(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024), smem_desc_sw128(k_smem + off, 16, 1024),
+               FwdCfg<D>::kIdescQK, kk > 0 ? 1u : 0u);
+    }
+  }
+}
+
+// Q or K tile: bf16 (D/64 boxes of 64 columns) or e4m3 (one box of D = 128
+// bytes per row), through 4-D tensor maps (D, S, H, B).
+template <int D, bool FP8>
+__device__ __forceinline__ void load_qk_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar, int row0,
+                                             int h, int b) {
+  if constexpr (FP8) {
+    tma_load_4d(dst, map, bar, 0, row0, h, b);
+  } else {
+    load_tile<D>(dst, map, bar, row0, h, b);
   }
 }
 
@@ -267,7 +292,7 @@ __device__ __forceinline__ float row_probs(float (&x)[4][32], const RowCtx& rc, 
   return acc.x + acc.y;
 }
 
-template <int D, int MOD, bool HAS_LSE>
+template <int D, int MOD, bool HAS_LSE, bool FP8 = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
@@ -353,10 +378,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!ATTN25_TIMED(tr[1], mbar_wait_thread(smem_u32(&bars->q_empty), (unit_iter & 1) ^ 1, wc))) {
           ok = false;
         } else {
-          mbar_arrive_expect_tx(smem_u32(&bars->q_full), 2 * Cfg::kTileBytes);
+          constexpr int kQKBytes = FP8 ? Cfg::kTileBytes8 : Cfg::kTileBytes;
+          mbar_arrive_expect_tx(smem_u32(&bars->q_full), 2 * kQKBytes);
           ++q_loads;
-          load_tile<D>(q_smem[0], &tm_q, smem_u32(&bars->q_full), (2 * uc.p) * TILE, uc.h, uc.b);
-          load_tile<D>(q_smem[1], &tm_q, smem_u32(&bars->q_full), (2 * uc.p + 1) * TILE, uc.h, uc.b);
+          load_qk_tile<D, FP8>(q_smem[0], &tm_q, smem_u32(&bars->q_full), (2 * uc.p) * TILE, uc.h, uc.b);
+          load_qk_tile<D, FP8>(q_smem[1], &tm_q, smem_u32(&bars->q_full), (2 * uc.p + 1) * TILE, uc.h, uc.b);
           for (int j2 = 0; j2 < n && ok; ++j2) {
             const int kt = static_cast<int>(lst[j2] & 0xFFFFFu);
 #pragma unroll
@@ -365,9 +391,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               const uint32_t phase = (ring_pos / Cfg::kStages) & 1;
               if (!ATTN25_TIMED(tr[2], mbar_wait_thread(smem_u32(&bars->kv_empty[slot]), phase ^ 1, wc))) { ok = false; break; }
               const uint32_t bar = smem_u32(&bars->kv_full[slot]);
-              mbar_arrive_expect_tx(bar, Cfg::kTileBytes);
-              load_tile<D>(ring + slot * Cfg::kTileBytes, which == 0 ? &tm_k : &tm_v, bar, kt * TILE,
-                           hk, uc.b);
+              if (which == 0) {  // K: e4m3 or bf16
+                mbar_arrive_expect_tx(bar, kQKBytes);
+                load_qk_tile<D, FP8>(ring + slot * Cfg::kTileBytes, &tm_k, bar, kt * TILE, hk, uc.b);
+              } else {           // V: bf16
+                mbar_arrive_expect_tx(bar, Cfg::kTileBytes);
+                load_tile<D>(ring + slot * Cfg::kTileBytes, &tm_v, bar, kt * TILE, hk, uc.b);
+              }
               ++slot_uses[slot];
               ++ring_pos;
             }
@@ -422,7 +452,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int t = 0; t < 2; ++t)
           if (act[t]) {
-            issue_qk<D>(s_tmem[t], q_smem[t], ring + slot_k * Cfg::kTileBytes);
+            issue_qk<D, FP8>(s_tmem[t], q_smem[t], ring + slot_k * Cfg::kTileBytes);
             mma_commit_w(smem_u32(&bars->s_full[t]));
           }
         mma_commit_w(smem_u32(&bars->kv_empty[slot_k]));
@@ -459,7 +489,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               tc_fence_after();
             }
             if (act_n[t]) {
-              issue_qk<D>(s_tmem[t], q_smem[t], ring + slot_kn * Cfg::kTileBytes);
+              issue_qk<D, FP8>(s_tmem[t], q_smem[t], ring + slot_kn * Cfg::kTileBytes);
               mma_commit_w(smem_u32(&bars->s_full[t]));
             }
           }
@@ -508,6 +538,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       RowCtx rc;
       rc.row = (2 * uc.p + t) * TILE + r;
       rc.sl2 = a.sl2;
+      if constexpr (FP8) {  // the scores come out of the MMA in code units: dequantise in the exponent's scale
+        static_assert(score_of(MOD) == MOD_NONE, "FP8 scores take masks only");
+        rc.sl2 *= __ldg(a.q_scales + uc.b * a.Hq + uc.h) * __ldg(a.k_scales + uc.b * a.Hkv + uc.h / a.G);
+      }
       rc.aux = 0.f;
       rc.aux2 = 0.f;
       if constexpr (score_of(MOD) == MOD_ALIBI) rc.aux = alibi_slope(a.mod, uc.h, a.Hq) * LOG2E;
@@ -650,10 +684,10 @@ namespace attn25 {
 
 namespace {
 
-template <int D, int MOD, bool LSE>
+template <int D, int MOD, bool LSE, bool FP8 = false>
 cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const FwdArgs& a, int grid, cudaStream_t stream) {
-  auto kernel = attn_fwd_kernel<D, MOD, LSE>;
+  auto kernel = attn_fwd_kernel<D, MOD, LSE, FP8>;
   // The register split assumes the kernel launches with kLaunchRegs per
   // thread; with fewer, setmaxnreg.inc could wait forever, so refuse.
   static int launch_regs = -1;
@@ -693,6 +727,23 @@ cudaError_t launch_fwd_mod(const CUtensorMap& tq, const CUtensorMap& tk, const C
 }
 
 }  // namespace
+
+cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const FwdArgs& a, int key, bool has_lse, int grid, cudaStream_t s) {
+  constexpr int M = kKeyMasked, MB = kKeyMasked | kKeyBitmap;
+  switch (key) {
+    case MOD_NONE:
+      return has_lse ? launch_fwd_t<128, MOD_NONE, true, true>(tq, tk, tv, a, grid, s)
+                     : launch_fwd_t<128, MOD_NONE, false, true>(tq, tk, tv, a, grid, s);
+    case M | MOD_NONE:
+      return has_lse ? launch_fwd_t<128, M | MOD_NONE, true, true>(tq, tk, tv, a, grid, s)
+                     : launch_fwd_t<128, M | MOD_NONE, false, true>(tq, tk, tv, a, grid, s);
+    case MB | MOD_NONE:
+      return has_lse ? launch_fwd_t<128, MB | MOD_NONE, true, true>(tq, tk, tv, a, grid, s)
+                     : launch_fwd_t<128, MB | MOD_NONE, false, true>(tq, tk, tv, a, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
 
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdArgs& a, int D, int key, bool has_lse, int grid,

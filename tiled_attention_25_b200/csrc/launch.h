@@ -17,6 +17,8 @@ struct Strides {
 
 struct FwdArgs {
   __nv_bfloat16* out;
+  const float* q_scales;  // FP8 scores: per (b, query head) and per (b, KV head) scales of the
+  const float* k_scales;  // e4m3 Q and K codes (nullptr for bf16 Q and K)
   Strides o_st;  // of out
   float* lse;
   int B, Hq, Hkv, G, Sq, Skv;
@@ -92,6 +94,12 @@ struct MaskArgs {
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdArgs& a, int D, int key, bool has_lse, int grid,
                        cudaStream_t stream);
+// The forward with e4m3 Q and K (D = 128; masks, no score transform).
+cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const FwdArgs& a, int key, bool has_lse, int grid, cudaStream_t stream);
+// FP8 incoherent processing of x [BH][S][D] bf16 -> e4m3 codes and one scale per row of BH.
+cudaError_t launch_fp8_prep(const void* x, const int8_t* signs, uint8_t* codes, float* scales, int BH, int S,
+                            int D, int sms, cudaStream_t stream);
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const BwdArgs& a, int D, int key, int grid,
                        cudaStream_t stream);
