@@ -369,6 +369,24 @@ __device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h,
   }
   if constexpr (score_of(MOD) == MOD_BOOST) aux = a.mod.boost * a.sl2;
   const float2 sl2 = make_float2(a.sl2, a.sl2);
+  // softcap: scores well below the cap across the warp's step take tanh from
+  // its series on the FMA pipe, the others from its exponential form (MUFU)
+  bool series = false;
+  if constexpr (score_of(MOD) == MOD_SOFTCAP) {
+    float mx = 0.f;
+#pragma unroll
+    for (int c = 0; c < BM; ++c) mx = fmaxf(mx, fabsf(x[c]));
+    series = __all_sync(0xffffffffu, mx <= kTanhSeriesLimit * a.mod.softcap / a.scale);
+  }
+  // local boost: the band |q - kv| < radius covers the warp's step wholly,
+  // or misses it wholly, except near its edges
+  int band = 0;  // 1: all inside, 2: all outside, 0: per element
+  if constexpr (score_of(MOD) == MOD_BOOST) {
+    const float rad = static_cast<float>(a.mod.boost_radius);
+    const float lo = dq0, hi = dq0 + static_cast<float>(BM - 1);
+    if (__all_sync(0xffffffffu, fabsf(lo) < rad && fabsf(hi) < rad)) band = 1;
+    else if (__all_sync(0xffffffffu, lo >= rad || hi <= -rad)) band = 2;
+  }
 #pragma unroll
   for (int c4 = 0; c4 < BM / 4; ++c4) {
     const float4 l = lds128(nl2_addr + c4 * 16);
@@ -381,12 +399,22 @@ __device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h,
         v.x = fmaf(x[c], a.sl2, -aux * fabsf(dq0 + static_cast<float>(c))) + nl.x;
         v.y = fmaf(x[c + 1], a.sl2, -aux * fabsf(dq0 + static_cast<float>(c + 1))) + nl.y;
       } else if constexpr (score_of(MOD) == MOD_SOFTCAP) {
-        v.x = fmaf(aux2, tanh_ex2(x[c] * aux), nl.x);
-        v.y = fmaf(aux2, tanh_ex2(x[c + 1] * aux), nl.y);
+        if (series) {
+          v.x = fmaf(aux2, tanh_series(x[c] * aux), nl.x);
+          v.y = fmaf(aux2, tanh_series(x[c + 1] * aux), nl.y);
+        } else {
+          v.x = fmaf(aux2, tanh_ex2(x[c] * aux), nl.x);
+          v.y = fmaf(aux2, tanh_ex2(x[c + 1] * aux), nl.y);
+        }
       } else if constexpr (score_of(MOD) == MOD_BOOST) {
-        const float r = static_cast<float>(a.mod.boost_radius);
-        v.x = fmaf(x[c], fabsf(dq0 + static_cast<float>(c)) < r ? aux : a.sl2, nl.x);
-        v.y = fmaf(x[c + 1], fabsf(dq0 + static_cast<float>(c + 1)) < r ? aux : a.sl2, nl.y);
+        if (band != 0) {
+          const float f = band == 1 ? aux : a.sl2;
+          v = __ffma2_rn(make_float2(x[c], x[c + 1]), make_float2(f, f), nl);
+        } else {
+          const float r = static_cast<float>(a.mod.boost_radius);
+          v.x = fmaf(x[c], fabsf(dq0 + static_cast<float>(c)) < r ? aux : a.sl2, nl.x);
+          v.y = fmaf(x[c + 1], fabsf(dq0 + static_cast<float>(c + 1)) < r ? aux : a.sl2, nl.y);
+        }
       } else {
         v = __ffma2_rn(make_float2(x[c], x[c + 1]), sl2, nl);
       }
@@ -808,6 +836,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float dq0 = static_cast<float>(q0 - kv);
         float cl2_inv = 0.f;
         if constexpr (score_of(MOD) == MOD_SOFTCAP) cl2_inv = 1.f / (a.mod.softcap * LOG2E);
+        // local boost: the band covers the warp's step wholly (1), misses it (2), or neither (0)
+        int band = 0;
+        if constexpr (score_of(MOD) == MOD_BOOST) {
+          const float rad = static_cast<float>(a.mod.boost_radius);
+          const float lo = dq0, hi = dq0 + static_cast<float>(BM - 1);
+          if (__all_sync(0xffffffffu, fabsf(lo) < rad && fabsf(hi) < rad)) band = 1;
+          else if (__all_sync(0xffffffffu, lo >= rad || hi <= -rad)) band = 2;
+        }
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16) {  // 8 columns (16 bytes) at a time
           const float4 nd0 = lds128(stats + 512 + c16 * 32), nd1 = lds128(stats + 512 + c16 * 32 + 16);
@@ -834,9 +870,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               d.x = pr.x > 0.f ? d.x * (1.f - t0 * t0) : 0.f;
               d.y = pr.y > 0.f ? d.y * (1.f - t1 * t1) : 0.f;
             } else if constexpr (score_of(MOD) == MOD_BOOST) {
-              const float rad = static_cast<float>(a.mod.boost_radius);
-              d.x *= fabsf(dq0 + static_cast<float>(c)) < rad ? a.mod.boost : 1.f;
-              d.y *= fabsf(dq0 + static_cast<float>(c + 1)) < rad ? a.mod.boost : 1.f;
+              if (band == 1) {
+                d = __fmul2_rn(d, make_float2(a.mod.boost, a.mod.boost));
+              } else if (band == 0) {
+                const float rad = static_cast<float>(a.mod.boost_radius);
+                d.x *= fabsf(dq0 + static_cast<float>(c)) < rad ? a.mod.boost : 1.f;
+                d.y *= fabsf(dq0 + static_cast<float>(c + 1)) < rad ? a.mod.boost : 1.f;
+              }
             }
             w[e] = pack_bf16x2(d.x, d.y);
           }

@@ -149,6 +149,7 @@ struct RowCtx {
   float sl2;    // scale * log2(e)
   float aux;    // ALiBi: slope * log2(e); softcap: scale / c; boost: boost * sl2
   float aux2;   // softcap: c * log2(e)
+  float lim;    // softcap: raw scores up to this size take tanh's series (|s / c| <= 0.4)
   const uint32_t* bits;  // bitmap mask: this row's keep bits (nullptr on padding rows)
 };
 
@@ -157,20 +158,49 @@ template <int MOD>
 __device__ __forceinline__ void transform32(float (&x)[32], const RowCtx& r, const ModDev& md,
                                             int k0, int c0, bool pred) {
   const float di = static_cast<float>(r.row - k0 - c0);
+  if constexpr (score_of(MOD) == MOD_SOFTCAP) {
+    // scores well below the cap everywhere in the warp's chunk take tanh from
+    // its series on the FMA pipe, the others from its exponential form (MUFU)
+    float mx = 0.f;
 #pragma unroll
-  for (int c = 0; c < 32; ++c) {
-    float v = x[c];
-    if constexpr (score_of(MOD) == MOD_ALIBI) {
-      v = fmaf(v, r.sl2, -r.aux * fabsf(di - static_cast<float>(c)));
-    } else if constexpr (score_of(MOD) == MOD_SOFTCAP) {
-      v = r.aux2 * tanh_ex2(v * r.aux);
-    } else if constexpr (score_of(MOD) == MOD_BOOST) {
-      const bool inside = fabsf(di - static_cast<float>(c)) < static_cast<float>(md.boost_radius);
-      v = v * (inside ? r.aux : r.sl2);
+    for (int c = 0; c < 32; ++c) mx = fmaxf(mx, fabsf(x[c]));
+    if (__all_sync(0xffffffffu, mx <= r.lim)) {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) x[c] = r.aux2 * tanh_series(x[c] * r.aux);
     } else {
-      v = v * r.sl2;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) x[c] = r.aux2 * tanh_ex2(x[c] * r.aux);
     }
-    x[c] = v;
+  } else if constexpr (score_of(MOD) == MOD_BOOST) {
+    // the boost band |i - j| < radius covers the warp's chunk wholly, or
+    // misses it wholly, except near its edges
+    const float rad = static_cast<float>(md.boost_radius);
+    const bool all_in = fabsf(di) < rad && fabsf(di - 31.f) < rad;
+    const bool all_out = di - 31.f >= rad || di <= -rad;
+    if (__all_sync(0xffffffffu, all_in)) {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) x[c] *= r.aux;
+    } else if (__all_sync(0xffffffffu, all_out)) {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) x[c] *= r.sl2;
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const bool inside = fabsf(di - static_cast<float>(c)) < rad;
+        x[c] *= inside ? r.aux : r.sl2;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      float v = x[c];
+      if constexpr (score_of(MOD) == MOD_ALIBI) {
+        v = fmaf(v, r.sl2, -r.aux * fabsf(di - static_cast<float>(c)));
+      } else {
+        v = v * r.sl2;
+      }
+      x[c] = v;
+    }
   }
   if (pred) {
     const int jlo = r.lo - k0 - c0, jhi = r.hi - k0 - c0;
@@ -350,9 +380,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   (void)tr;
   ATTN25_TRACE_ONLY(const long long t_start = clock64();)
 
-  // softcap and local boost keep the even split: their per-element mods need
-  // more registers than any split can give, so they spill either way
-  constexpr bool kSplitRegs = score_of(MOD) != MOD_SOFTCAP && score_of(MOD) != MOD_BOOST;
+  // every kernel takes the register split (the softcap and boost transforms
+  // have warp-uniform fast paths that fit in the softmax warps' registers)
+  constexpr bool kSplitRegs = true;
   if (warp >= 8) {
   if constexpr (kSplitRegs) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
   if (warp == 9) {
@@ -544,10 +574,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       rc.aux = 0.f;
       rc.aux2 = 0.f;
+      rc.lim = 0.f;
       if constexpr (score_of(MOD) == MOD_ALIBI) rc.aux = alibi_slope(a.mod, uc.h, a.Hq) * LOG2E;
       if constexpr (score_of(MOD) == MOD_SOFTCAP) {
         rc.aux = a.scale / a.mod.softcap;
         rc.aux2 = a.mod.softcap * LOG2E;
+        rc.lim = kTanhSeriesLimit * a.mod.softcap / a.scale;
       }
       if constexpr (score_of(MOD) == MOD_BOOST) rc.aux = a.mod.boost * a.sl2;
       if constexpr (masked(MOD)) {
