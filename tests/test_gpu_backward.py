@@ -225,3 +225,26 @@ def test_alibi_with_given_slopes(ta, D):
         check_lse(lse.cpu().double().numpy(), L, f"alibi slopes D {D}")
         got = [host_f64(t) for t in run_fwd_bwd(ta, c, use_mask)]
         check_grads(got, c.oracle_bwd(), f"alibi slopes D {D} mask {use_mask}")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_softcap_near_and_far_from_the_cap(ta, D):
+    """Softcap with scores on both sides of the kernels' series limit (a warp
+    whose raw scores all satisfy |s| <= 0.4 c takes tanh's series, the others
+    its exponential form): scale 1 makes the scores N(0, D); with c = 70 (D 64)
+    or 100 (D 128) about half the forward chunks and a third to a half of the
+    backward steps take the series.  Forward and backward against the oracle."""
+    from gpu_common import check_lse, check_o
+    S = 300
+    c = Case(190 + D, 1, 4, 2, S, S, D, oracle.MOD_SOFTCAP, ModParams(softcap=70.0 if D == 64 else 100.0),
+             scale=1.0)
+    mask = ta.new_block_mask(c.mod, c.dev_params, c.B, c.Sq, c.Skv)
+    out = torch.empty_like(c.q)
+    lse = torch.empty(c.B, c.Hq, c.Sq, dtype=torch.float32, device="cuda")
+    ta.attn_fwd(c.q, c.k, c.v, out, lse, scale=c.scale, mod_kind=c.mod, mod_params=c.dev_params, block_mask=mask)
+    torch.cuda.synchronize()
+    O, L = c.oracle_fwd()
+    check_o(host_f64(out), O, f"softcap far D {D}")
+    check_lse(lse.cpu().double().numpy(), L, f"softcap far D {D}")
+    got = [host_f64(t) for t in run_fwd_bwd(ta, c)]
+    check_grads(got, c.oracle_bwd(), f"softcap far D {D}")
