@@ -349,6 +349,25 @@ ATTN25_API int attn_get_status(attn_stream_t stream);
 ATTN25_API void attn_set_wait_limit_ms(uint32_t ms);
 
 /*
+ * How the persistent forward and backward kernels take their work units
+ * (query-tile pairs forward, key tiles backward), which they always take in
+ * the block mask's longest-first order (ascending key tiles for
+ * attn_bwd_deterministic):
+ *   ATTN_WALK_STATIC (default): one CTA per SM; wave k of the order goes to
+ *     the CTAs in turn, every other wave reversed (a snake), fixed in advance;
+ *   ATTN_WALK_CLUSTER_LAUNCH_CONTROL: one CTA per unit is launched; a CTA that
+ *     finishes its unit asks the hardware (Blackwell's cluster launch control)
+ *     to cancel the next CTA that has not started and does that CTA's unit, so
+ *     the walk adapts to data-dependent unit lengths as it runs ("PyTorch
+ *     FlexAttention, FlashAttention-4 백엔드 …", 섹션별 상세 and 실무
+ *     Takeaway: dynamic scheduling through CLC balances the SMs under
+ *     data-dependent masks).
+ * Applies to calls made after it; returns ATTN_ERR_ARG for another value.
+ */
+enum { ATTN_WALK_STATIC = 0, ATTN_WALK_CLUSTER_LAUNCH_CONTROL = 1 };
+ATTN25_API int attn_set_work_walk(int walk);
+
+/*
  * Self-check of the timeout path (the pages have no counterpart: it exists
  * so that a caller can see the error path work on its own GPU).  Launches on
  * the stream a kernel whose one wait is on a barrier that nothing arrives at;

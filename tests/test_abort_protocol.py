@@ -31,14 +31,15 @@ from protocol_sim import Sim
 STAGES_BWD = 3
 
 
-def forward(units, seed, give_up, stages=4, drain_kv=True, drain_always=True):
+def forward(units, seed, give_up, stages=4, drain_kv=True, drain_always=True, clc=False):
     sim = Sim(seed)
     full, empty, drain = sim.full, sim.empty, sim.drain
     for b in range(2):
         sim.bar(f"list_full{b}", 1)
         sim.bar(f"list_empty{b}", 3)
-    for name in ("q_full", "q_empty", "drain"):
+    for name in ("q_full", "q_empty", "drain", "clc_bar"):
         sim.bar(name, 1)
+    walk = list(units) + [None]  # None: the published end of the walk
     for t in range(2):
         for name in ("s_full", "p_full", "o_full", "o_final"):
             sim.bar(f"{name}{t}", 1)
@@ -48,13 +49,19 @@ def forward(units, seed, give_up, stages=4, drain_kv=True, drain_always=True):
 
     def tma():
         ring, q_loads, uses = 0, 0, [0] * stages
+        asked = answered = 0
         ok = True
-        for u, steps in enumerate(units):
+        for u, steps in enumerate(walk):
             b = u & 1
             ok = yield empty(f"list_empty{b}", u >> 1)
             if not ok:
                 break
             sim.arrive(f"list_full{b}")
+            if steps is None:
+                break
+            if clc:
+                sim.load("clc_bar")
+                asked += 1
             ok = yield empty("q_empty", u)
             if not ok:
                 break
@@ -73,7 +80,14 @@ def forward(units, seed, give_up, stages=4, drain_kv=True, drain_always=True):
                     break
             if not ok:
                 break
+            if clc:
+                ok = yield full("clc_bar", u)
+                if not ok:
+                    break
+                answered += 1
         if drain_always or not ok:  # let the copies in flight land
+            if asked > answered:
+                yield drain("clc_bar", asked - 1)
             for s in range(stages):
                 if uses[s] and drain_kv:
                     yield drain(f"kv_full{s}", uses[s] - 1)
@@ -83,9 +97,13 @@ def forward(units, seed, give_up, stages=4, drain_kv=True, drain_always=True):
     def mma():
         ring, pv = 0, [0, 0]
         ok = True
-        for u, steps in enumerate(units):
-            b, n = u & 1, len(steps)
-            ok = (yield full(f"list_full{b}", u >> 1)) and (yield full("q_full", u))
+        for u, steps in enumerate(walk):
+            b = u & 1
+            ok = yield full(f"list_full{b}", u >> 1)
+            if not ok or steps is None:
+                break
+            n = len(steps)
+            ok = yield full("q_full", u)
             if not ok:
                 break
             if n > 0:
@@ -139,9 +157,9 @@ def forward(units, seed, give_up, stages=4, drain_kv=True, drain_always=True):
 
     def softmax(t):
         s_cnt = p_cnt = o_units = 0
-        for u, steps in enumerate(units):
+        for u, steps in enumerate(walk):
             b = u & 1
-            if not (yield full(f"list_full{b}", u >> 1)):
+            if not (yield full(f"list_full{b}", u >> 1)) or steps is None:
                 return
             n_act = 0
             for step in steps:
@@ -167,7 +185,7 @@ def forward(units, seed, give_up, stages=4, drain_kv=True, drain_always=True):
     return stuck, sim.in_flight_at_exit
 
 
-def backward(units, seed, give_up, drain_stages=True, drain_always=True):
+def backward(units, seed, give_up, drain_stages=True, drain_always=True, clc=False):
     sim = Sim(seed)
     full, empty, drain = sim.full, sim.empty, sim.drain
     S = STAGES_BWD
@@ -178,8 +196,9 @@ def backward(units, seed, give_up, drain_stages=True, drain_always=True):
         sim.bar(f"p_ready{b}", 1)
         sim.bar(f"ds_ready{b}", 2)
         sim.bar(f"ds_empty{b}", 1)
-    for name in ("kv_full", "kv_empty", "dp_full", "dp_empty", "dq_full", "acc_full", "drain"):
+    for name in ("kv_full", "kv_empty", "dp_full", "dp_empty", "dq_full", "acc_full", "drain", "clc_bar"):
         sim.bar(name, 1)
+    walk = list(units) + [None]  # None: the published end of the walk
     sim.bar("acc_empty", 2)
     for s in range(S):
         sim.bar(f"q_full{s}", 1)
@@ -187,13 +206,19 @@ def backward(units, seed, give_up, drain_stages=True, drain_always=True):
 
     def tma():
         step, kv_loads, uses = 0, 0, [0] * S
+        asked = answered = 0
         ok = True
-        for u, n in enumerate(units):
+        for u, n in enumerate(walk):
             b = u & 1
             ok = yield empty(f"list_empty{b}", u >> 1)
             if not ok:
                 break
             sim.arrive(f"list_full{b}")
+            if n is None:
+                break
+            if clc:
+                sim.load("clc_bar")
+                asked += 1
             ok = yield empty("kv_empty", u)
             if not ok:
                 break
@@ -209,7 +234,14 @@ def backward(units, seed, give_up, drain_stages=True, drain_always=True):
                 step += 1
             if not ok:
                 break
+            if clc:
+                ok = yield full("clc_bar", u)
+                if not ok:
+                    break
+                answered += 1
         if drain_always or not ok:
+            if asked > answered:
+                yield drain("clc_bar", asked - 1)
             if kv_loads:
                 yield drain("kv_full", kv_loads - 1)
             for s in range(S):
@@ -219,9 +251,12 @@ def backward(units, seed, give_up, drain_stages=True, drain_always=True):
     def mma():
         step = 0
         ok = True
-        for u, n in enumerate(units):
+        for u, n in enumerate(walk):
             b = u & 1
-            ok = (yield full(f"list_full{b}", u >> 1)) and (yield full("kv_full", u))
+            ok = yield full(f"list_full{b}", u >> 1)
+            if not ok or n is None:
+                break
+            ok = yield full("kv_full", u)
             if not ok:
                 break
             if n > 0:
@@ -268,9 +303,9 @@ def backward(units, seed, give_up, drain_stages=True, drain_always=True):
 
     def p_warps():
         step = 0
-        for u, n in enumerate(units):
+        for u, n in enumerate(walk):
             b = u & 1
-            if not (yield full(f"list_full{b}", u >> 1)):
+            if not (yield full(f"list_full{b}", u >> 1)) or n is None:
                 return
             for _ in range(n):
                 s, sb = step % S, step & 1
@@ -285,9 +320,9 @@ def backward(units, seed, give_up, drain_stages=True, drain_always=True):
 
     def ds_warps():
         step = 0
-        for u, n in enumerate(units):
+        for u, n in enumerate(walk):
             b = u & 1
-            if not (yield full(f"list_full{b}", u >> 1)):
+            if not (yield full(f"list_full{b}", u >> 1)) or n is None:
                 return
             for _ in range(n):
                 s, sb = step % S, step & 1
@@ -308,9 +343,9 @@ def backward(units, seed, give_up, drain_stages=True, drain_always=True):
     def dq_drain():
         step = 0
         sim.arrive("ds_ready0")
-        for u, n in enumerate(units):
+        for u, n in enumerate(walk):
             b = u & 1
-            if not (yield full(f"list_full{b}", u >> 1)):
+            if not (yield full(f"list_full{b}", u >> 1)) or n is None:
                 return
             for _ in range(n):
                 if not (yield full("dq_full", step)):
@@ -330,28 +365,31 @@ FWD_UNITS = [[BOTH] * 5, [BOTH, FIRST], [], [BOTH] * 3]
 BWD_UNITS = [4, 0, 3, 1]
 
 
+@pytest.mark.parametrize("clc", [False, True], ids=["static", "clc"])
 @pytest.mark.parametrize("role", ["tma", "mma", "softmax0", "softmax1"])
-def test_forward_timeout_at_any_wait_ends_clean(role):
+def test_forward_timeout_at_any_wait_ends_clean(role, clc):
     for n in range(0, 40, 3):
         for seed in range(12):
-            stuck, left = forward(FWD_UNITS, seed, (role, n))
+            stuck, left = forward(FWD_UNITS, seed, (role, n), clc=clc)
             assert stuck is None, f"{role} wait {n} seed {seed}: stuck {stuck}"
             assert left == 0, f"{role} wait {n} seed {seed}: {left} copies/MMAs in flight at exit"
 
 
+@pytest.mark.parametrize("clc", [False, True], ids=["static", "clc"])
 @pytest.mark.parametrize("role", ["tma", "mma", "p", "ds", "drain"])
-def test_backward_timeout_at_any_wait_ends_clean(role):
+def test_backward_timeout_at_any_wait_ends_clean(role, clc):
     for n in range(0, 40, 3):
         for seed in range(12):
-            stuck, left = backward(BWD_UNITS, seed, (role, n))
+            stuck, left = backward(BWD_UNITS, seed, (role, n), clc=clc)
             assert stuck is None, f"{role} wait {n} seed {seed}: stuck {stuck}"
             assert left == 0, f"{role} wait {n} seed {seed}: {left} copies/MMAs in flight at exit"
 
 
 def test_without_timeouts_the_models_run_as_before():
     for seed in range(20):
-        assert forward(FWD_UNITS, seed, None) == (None, 0)
-        assert backward(BWD_UNITS, seed, None) == (None, 0)
+        for clc in (False, True):
+            assert forward(FWD_UNITS, seed, None, clc=clc) == (None, 0)
+            assert backward(BWD_UNITS, seed, None, clc=clc) == (None, 0)
 
 
 def test_the_check_notices_copies_left_in_flight():

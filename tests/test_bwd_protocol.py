@@ -19,7 +19,7 @@ from protocol_sim import Sim
 STAGES = 3  # Q / dO stages
 
 
-def simulate(units, seed, drain_share=True, empty_unit_waits=True):
+def simulate(units, seed, drain_share=True, empty_unit_waits=True, clc=False):
     """Run the roles to completion; return None, or the stuck roles' waits.
     The two switches remove a step of the protocol, to show the model notices."""
     sim = Sim(seed)
@@ -41,13 +41,19 @@ def simulate(units, seed, drain_share=True, empty_unit_waits=True):
     sim.bar("dq_full", 1)
     sim.bar("acc_full", 1)
     sim.bar("acc_empty", 2)              # P warps + dS warps after the epilogue
+    sim.bar("clc_bar", 1)                # the cancel request's response (cluster launch control)
+    walk = list(units) + [None]          # None: the published end of the walk
 
     def tma():
         step = 0
-        for u, n in enumerate(units):
+        for u, n in enumerate(walk):
             b = u & 1
             yield empty(f"list_empty{b}", u >> 1)
             sim.arrive(f"list_full{b}")
+            if n is None:
+                break
+            if clc:
+                sim.load("clc_bar")       # ask for the next unit; answered later
             yield empty("kv_empty", u)
             sim.load("kv_full")           # K and V, one expected byte count
             for _ in range(n):
@@ -55,12 +61,16 @@ def simulate(units, seed, drain_share=True, empty_unit_waits=True):
                 yield empty(f"q_empty{s}", step // STAGES)
                 sim.load(f"q_full{s}")    # Q, dO and the row statistics
                 step += 1
+            if clc:
+                yield full("clc_bar", u)  # the answer: the next unit, or the end
 
     def mma():
         step = 0
-        for u, n in enumerate(units):
+        for u, n in enumerate(walk):
             b = u & 1
             yield full(f"list_full{b}", u >> 1)
+            if n is None:
+                break
             yield full("kv_full", u)
             if n > 0:  # S^T(0) and dP^T(0) of the unit
                 yield full(f"q_full{step % STAGES}", step // STAGES)
@@ -90,9 +100,11 @@ def simulate(units, seed, drain_share=True, empty_unit_waits=True):
 
     def p_warps():
         step = 0
-        for u, n in enumerate(units):
+        for u, n in enumerate(walk):
             b = u & 1
             yield full(f"list_full{b}", u >> 1)
+            if n is None:
+                break
             for _ in range(n):
                 s, sb = step % STAGES, step & 1
                 yield full(f"q_full{s}", step // STAGES)
@@ -105,9 +117,11 @@ def simulate(units, seed, drain_share=True, empty_unit_waits=True):
 
     def ds_warps():
         step = 0
-        for u, n in enumerate(units):
+        for u, n in enumerate(walk):
             b = u & 1
             yield full(f"list_full{b}", u >> 1)
+            if n is None:
+                break
             for _ in range(n):
                 s, sb = step % STAGES, step & 1
                 yield full(f"q_full{s}", step // STAGES)
@@ -125,9 +139,11 @@ def simulate(units, seed, drain_share=True, empty_unit_waits=True):
         step = 0
         if drain_share:
             sim.arrive("ds_ready0")  # its share of step 0, given up front
-        for u, n in enumerate(units):
+        for u, n in enumerate(walk):
             b = u & 1
             yield full(f"list_full{b}", u >> 1)
+            if n is None:
+                break
             for _ in range(n):
                 yield full("dq_full", step)
                 # dQ^T(j) read: the share of step j+1, then the dS buffer of step j
@@ -143,10 +159,11 @@ UNIT_PATTERNS = [[10], [4], [1], [2], [3], [10, 10], [3, 5, 1, 2], [0, 4], [7, 0
                  [1, 1, 1, 1], [5, 0, 0, 5], [0], [0, 0], [2, 0, 1, 0, 3, 0]]
 
 
+@pytest.mark.parametrize("clc", [False, True], ids=["static", "clc"])
 @pytest.mark.parametrize("units", UNIT_PATTERNS, ids=lambda u: "-".join(map(str, u)))
-def test_backward_protocol_never_deadlocks_or_aliases(units):
+def test_backward_protocol_never_deadlocks_or_aliases(units, clc):
     for seed in range(200):
-        stuck = simulate(units, seed)
+        stuck = simulate(units, seed, clc=clc)
         assert stuck is None, f"deadlock with units {units}, seed {seed}: {stuck}"
 
 

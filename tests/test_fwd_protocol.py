@@ -24,7 +24,7 @@ import pytest
 from protocol_sim import Sim
 
 
-def simulate(units, seed, stages=4, final_on_empty_units=False):
+def simulate(units, seed, stages=4, final_on_empty_units=False, clc=False):
     """units: per unit, a list of steps (act0, act1).  Returns None, or the
     stuck roles' waits.  final_on_empty_units commits o_final for units
     without steps too, as the kernel once did, to show the model notices."""
@@ -35,6 +35,8 @@ def simulate(units, seed, stages=4, final_on_empty_units=False):
         sim.bar(f"list_empty{b}", 3)      # MMA warp + the two softmax warpgroups
     sim.bar("q_full", 1)
     sim.bar("q_empty", 1)
+    sim.bar("clc_bar", 1)                 # the cancel request's response (cluster launch control)
+    walk = list(units) + [None]           # None: the published end of the walk
     for t in range(2):
         sim.bar(f"s_full{t}", 1)
         sim.bar(f"p_full{t}", 1)
@@ -46,10 +48,14 @@ def simulate(units, seed, stages=4, final_on_empty_units=False):
 
     def tma():
         ring = 0
-        for u, steps in enumerate(units):
+        for u, steps in enumerate(walk):
             b = u & 1
             yield empty(f"list_empty{b}", u >> 1)
             sim.arrive(f"list_full{b}")
+            if steps is None:
+                break
+            if clc:
+                sim.load("clc_bar")             # ask for the next unit; answered later
             yield empty("q_empty", u)
             sim.load("q_full")                  # both query tiles, one byte count
             for _ in steps:
@@ -58,14 +64,18 @@ def simulate(units, seed, stages=4, final_on_empty_units=False):
                     yield empty(f"kv_empty{slot}", ring // stages)
                     sim.load(f"kv_full{slot}")
                     ring += 1
+            if clc:
+                yield full("clc_bar", u)        # the answer: the next unit, or the end
 
     def mma():
         ring = 0
         pv = [0, 0]                             # PV products issued per query tile
-        for u, steps in enumerate(units):
+        for u, steps in enumerate(walk):
             b = u & 1
-            n = len(steps)
             yield full(f"list_full{b}", u >> 1)
+            if steps is None:
+                break
+            n = len(steps)
             yield full("q_full", u)
             if n > 0:                           # S_t(0)
                 slot_k = ring % stages
@@ -104,9 +114,11 @@ def simulate(units, seed, stages=4, final_on_empty_units=False):
 
     def softmax(t):
         s_cnt = p_cnt = o_units = 0
-        for u, steps in enumerate(units):
+        for u, steps in enumerate(walk):
             b = u & 1
             yield full(f"list_full{b}", u >> 1)
+            if steps is None:
+                break
             n_act = 0
             for step in steps:
                 if not step[t]:
@@ -138,11 +150,12 @@ UNIT_PATTERNS = {
 }
 
 
+@pytest.mark.parametrize("clc", [False, True], ids=["static", "clc"])
 @pytest.mark.parametrize("stages", [4, 6])
 @pytest.mark.parametrize("name", sorted(UNIT_PATTERNS))
-def test_forward_protocol_never_deadlocks_or_aliases(name, stages):
+def test_forward_protocol_never_deadlocks_or_aliases(name, stages, clc):
     for seed in range(150):
-        stuck = simulate(UNIT_PATTERNS[name], seed, stages=stages)
+        stuck = simulate(UNIT_PATTERNS[name], seed, stages=stages, clc=clc)
         assert stuck is None, f"deadlock in {name}, seed {seed}: {stuck}"
 
 

@@ -25,6 +25,8 @@ from .abi import (  # noqa: F401
     MOD_NONE,
     MOD_SLIDING_WINDOW,
     MOD_SOFTCAP,
+    WALK_CLUSTER_LAUNCH_CONTROL,
+    WALK_STATIC,
     AttnError,
     BlockMask,
     ModParams,
@@ -44,6 +46,7 @@ from .abi import (  # noqa: F401
     attn_fwd_strided,
     attn_get_status,
     attn_set_wait_limit_ms,
+    attn_set_work_walk,
     attn_strerror,
     build_block_mask,
 )

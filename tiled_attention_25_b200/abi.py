@@ -125,6 +125,8 @@ def _load():
     lib.attn_get_status.restype = I
     lib.attn_set_wait_limit_ms.argtypes = [ctypes.c_uint32]
     lib.attn_set_wait_limit_ms.restype = None
+    lib.attn_set_work_walk.argtypes = [I]
+    lib.attn_set_work_walk.restype = I
     lib.attn_check_wait_timeout.argtypes = [P]
     lib.attn_check_wait_timeout.restype = I
     lib.attn_strerror.argtypes = [I]
@@ -146,7 +148,7 @@ EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_bwd_noalloc
             "attn_block_mask_bind", "build_block_mask", "attn_get_status",
             "attn_set_wait_limit_ms", "attn_strerror", "attn_fwd_strided", "attn_bwd_strided",
             "attn_bwd_deterministic", "attn_bwd_deterministic_workspace_size", "attn_check_wait_timeout",
-            "attn_fp8_rotate_quantize", "attn_fwd_fp8")
+            "attn_fp8_rotate_quantize", "attn_fwd_fp8", "attn_set_work_walk")
 
 
 def attn_strerror(code: int) -> str:
@@ -472,6 +474,15 @@ def attn_get_status(stream=None) -> int:
 
 def attn_set_wait_limit_ms(ms: int):
     LIB.attn_set_wait_limit_ms(int(ms))
+
+
+WALK_STATIC = 0
+WALK_CLUSTER_LAUNCH_CONTROL = 1
+
+
+def attn_set_work_walk(walk: int):
+    """How the persistent kernels take their work units (see include/attn25.h)."""
+    _check(LIB.attn_set_work_walk(int(walk)), "attn_set_work_walk")
 
 
 def attn_check_wait_timeout(stream=None):

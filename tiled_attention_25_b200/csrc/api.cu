@@ -34,6 +34,7 @@ static __device__ __align__(256) unsigned char g_bwd_scratch[kNoAllocScratchByte
 namespace {
 
 std::atomic<uint32_t> g_wait_ms{4000};
+std::atomic<int> g_work_walk{0};  // ATTN_WALK_STATIC or ATTN_WALK_CLUSTER_LAUNCH_CONTROL
 
 constexpr int kMaxDevices = 64;
 
@@ -348,6 +349,12 @@ const char* attn_strerror(int status) {
 
 void attn_set_wait_limit_ms(uint32_t ms) { g_wait_ms.store(ms < 1 ? 1 : ms); }
 
+int attn_set_work_walk(int walk) {
+  if (walk != ATTN_WALK_STATIC && walk != ATTN_WALK_CLUSTER_LAUNCH_CONTROL) return ATTN_ERR_ARG;
+  g_work_walk.store(walk);
+  return ATTN_OK;
+}
+
 int attn_check_wait_timeout(attn_stream_t stream) {
   DeviceInfo* d = nullptr;
   const int rc = current_device(&d);
@@ -503,7 +510,9 @@ static int fwd_impl(const void* q, const void* k, const attn_bf16* v, attn_bf16*
   a.wait_ns = wait_ns();
   a.status = d->status;
   a.trace = d->trace;
-  const int grid = a.n_units < d->sms ? a.n_units : d->sms;
+  // cluster launch control launches one CTA per unit; the static walk one per SM
+  a.clc = g_work_walk.load() == ATTN_WALK_CLUSTER_LAUNCH_CONTROL ? 1 : 0;
+  const int grid = a.clc ? a.n_units : (a.n_units < d->sms ? a.n_units : d->sms);
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const cudaError_t e = fp8 ? launch_fwd_fp8(tq, tk, tv, a, mod_key(mod_kind), lse != nullptr, grid, st)
                             : launch_fwd(tq, tk, tv, a, D, mod_key(mod_kind), lse != nullptr, grid, st);
@@ -652,7 +661,8 @@ static int bwd_impl(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, 
   if (!encode_bf16_4d(&tq, q, D, Sq, Hq, B, sq, 64) || !encode_bf16_4d(&tk, k, D, Skv, Hkv, B, sk, TILE) ||
       !encode_bf16_4d(&tv, v, D, Skv, Hkv, B, sv, TILE) || !encode_bf16_4d(&tdo, dout, D, Sq, Hq, B, a.do_st, 64))
     return ATTN_ERR_ARG;
-  const int grid = a.n_units < d->sms ? a.n_units : d->sms;
+  a.clc = g_work_walk.load() == ATTN_WALK_CLUSTER_LAUNCH_CONTROL ? 1 : 0;
+  const int grid = a.clc ? a.n_units : (a.n_units < d->sms ? a.n_units : d->sms);
   if (launch_bwd(tq, tk, tv, tdo, a, D, mod_key(mod_kind), grid,
                  reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_LAUNCH;

@@ -89,6 +89,8 @@ struct BwdCfg {
 };
 
 struct BwdBarriers {
+  alignas(16) uint32_t clc_resp[4];  // cluster launch control response (the next unit)
+  uint64_t clc_bar;
   uint64_t list_full[2], list_empty[2];
   uint64_t kv_full, kv_empty;
   uint64_t q_full[4], q_empty[4];
@@ -102,6 +104,7 @@ struct BwdBarriers {
   uint32_t abort_flag;
   uint32_t never_set;  // abort word for drain waits that must not stop early
   int32_t list_n[2];   // lengths of the two query-tile lists
+  int32_t list_unit[2];  // the unit of each list (rank in the work order); -1 ends the walk
 };
 
 // Consumers of a query-tile list: the MMA warp and the P, dS and drain warps
@@ -487,6 +490,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(smem_u32(&bars->kv_full), 1);
     mbar_init(smem_u32(&bars->kv_empty), 1);
+    mbar_init(smem_u32(&bars->clc_bar), 1);
     for (int b = 0; b < Cfg::kStages; ++b) {
       mbar_init(smem_u32(&bars->q_full[b]), 1);
       mbar_init(smem_u32(&bars->q_empty[b]), 1);
@@ -536,18 +540,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // ---------------------------------------------------------- TMA producer
       // all lanes build the query-tile lists; lane 0 issues the copies
       int unit_iter = 0, step = 0;
-      uint32_t kv_loads = 0, stage_uses[4] = {0, 0, 0, 0};
+      uint32_t kv_loads = 0, stage_uses[4] = {0, 0, 0, 0}, clc_asked = 0, clc_read = 0;
+      const uint32_t clc_resp = smem_u32(bars->clc_resp), clc_bar = smem_u32(&bars->clc_bar);
       bool ok = true;
-      for (int u = snake_unit(0); u < a.n_units && ok; u = snake_unit(++unit_iter)) {
-        const BwdUnit un = decode_bwd_unit(a, u);
+      // The first unit: with cluster launch control (one CTA launched per
+      // unit) this CTA's own, then the unit of each not-yet-started CTA the
+      // hardware cancels for it; otherwise the static snake walk.  Each list
+      // is published with its unit's rank, and rank -1 ends every role's walk.
+      int u = a.clc ? static_cast<int>(blockIdx.x) : snake_unit(0);
+      for (;; ++unit_iter) {
         const int buf = unit_iter & 1;
         uint16_t* lst = lists + buf * kMaxSteps;
         if (!mbar_wait_warp_ool(smem_u32(&bars->list_empty[buf]), ((unit_iter >> 1) & 1) ^ 1, wc)) { ok = false; break; }
-        const int n = build_kv_qtiles(a.tile_class, un.b, un.kt, a.nQ, a.nK, a.Sq, a.Skv, a.mod.mask,
-                                      a.mod.window, lst);
-        if (a.dq_sem != nullptr) build_positions(a, un.b, un.kt, lst, n, positions + buf * kMaxSteps);
-        if (lane == 0) bars->list_n[buf] = n;
+        if (u >= a.n_units) u = -1;
+        BwdUnit un{};
+        int n = 0;
+        if (u >= 0) {
+          un = decode_bwd_unit(a, u);
+          n = build_kv_qtiles(a.tile_class, un.b, un.kt, a.nQ, a.nK, a.Sq, a.Skv, a.mod.mask, a.mod.window, lst);
+          if (a.dq_sem != nullptr) build_positions(a, un.b, un.kt, lst, n, positions + buf * kMaxSteps);
+        }
+        if (lane == 0) {
+          bars->list_n[buf] = n;
+          bars->list_unit[buf] = u;
+        }
         mbar_arrive(smem_u32(&bars->list_full[buf]));
+        if (u < 0) break;
+        if (lane == 0 && a.clc) {  // ask for the next unit now; the answer lands while this one streams
+          mbar_arrive_expect_tx(clc_bar, 16);
+          clc_try_cancel(clc_resp, clc_bar);
+          ++clc_asked;
+        }
         if (lane == 0) {
           if (!ATTN25_TIMED(tr[1], mbar_wait_thread_ool(smem_u32(&bars->kv_empty), (unit_iter & 1) ^ 1, wc))) {
             ok = false;
@@ -579,11 +602,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        if (a.clc) {  // the next unit: the rank of the cancelled CTA, or -1
+          if (!mbar_wait_warp_ool(clc_bar, clc_read & 1, wc)) { ok = false; break; }
+          ++clc_read;
+          u = clc_cancelled_x(clc_resp);
+        } else {
+          u = snake_unit(unit_iter + 1);
+        }
       }
       if (lane == 0) {
         // let the copies in flight land before the CTA exits (also after a
         // normal end: a consumer that gave up may have left them unconsumed)
         const WaitCtl dwc{drain_limit(a.wait_ns), smem_u32(&bars->never_set), a.status};
+        if (clc_asked > clc_read) mbar_wait_thread_ool(clc_bar, (clc_asked - 1) & 1, dwc);
         if (kv_loads) mbar_wait_thread_ool(smem_u32(&bars->kv_full), (kv_loads - 1) & 1, dwc);
         for (int s = 0; s < Cfg::kStages; ++s)
           if (stage_uses[s]) mbar_wait_thread_ool(smem_u32(&bars->q_full[s]), (stage_uses[s] - 1) & 1, dwc);
@@ -615,10 +647,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       break;                \
     }                       \
   }
-      for (int u = snake_unit(0); u < a.n_units && ok; u = snake_unit(++unit_iter)) {
+      for (;; ++unit_iter) {
         const int buf = unit_iter & 1;
-        MMA_WAIT(mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc) &&
-                 ATTN25_TIMED(tr[1], mbar_wait_warp_ool(smem_u32(&bars->kv_full), unit_iter & 1, wc)));
+        MMA_WAIT(mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc));
+        if (bars->list_unit[buf] < 0) break;
+        MMA_WAIT(ATTN25_TIMED(tr[1], mbar_wait_warp_ool(smem_u32(&bars->kv_full), unit_iter & 1, wc)));
         StepIter it;
         it.init(lists + buf * kMaxSteps, bars->list_n[buf], a.G, a.Sq);
         int g, q0;
@@ -722,13 +755,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t t_dv = tmem + Cfg::kColDV + lane_off;
     int unit_iter = 0, step = 0;
     bool ok = true;
-    for (int u = snake_unit(0); u < a.n_units && ok; u = snake_unit(++unit_iter)) {
+    for (;; ++unit_iter) {
+      const int buf = unit_iter & 1;
+      if (!mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+      const int u = bars->list_unit[buf];
+      if (u < 0) break;
       const BwdUnit un = decode_bwd_unit(a, u);
       const int kv = un.kt * TILE + r;
       int qlo, qhi;
       key_interval<MOD>(a, un.b, kv, qlo, qhi);
-      const int buf = unit_iter & 1;
-      if (!mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
       StepIter it;
       it.init(lists + buf * kMaxSteps, bars->list_n[buf], a.G, a.Sq);
       int g, q0;
@@ -798,11 +833,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t t_dp = tmem + Cfg::kColDP + lane_off, t_dk = tmem + Cfg::kColDK + lane_off;
     int unit_iter = 0, step = 0;
     bool ok = true;
-    for (int u = snake_unit(0); u < a.n_units && ok; u = snake_unit(++unit_iter)) {
-      const BwdUnit un = decode_bwd_unit(a, u);
-      const int kv = un.kt * TILE + r;
+    for (;; ++unit_iter) {
       const int buf = unit_iter & 1;
       if (!mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+      const int u = bars->list_unit[buf];
+      if (u < 0) break;
+      const BwdUnit un = decode_bwd_unit(a, u);
+      const int kv = un.kt * TILE + r;
       StepIter it;
       it.init(lists + buf * kMaxSteps, bars->list_n[buf], a.G, a.Sq);
       int g, q0;
@@ -922,10 +959,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ds_ready of step j counts the drain's read of dQ^T(j-1); step 0 has no
     // predecessor, so its share is given up front
     mbar_arrive(smem_u32(&bars->ds_ready[0]));
-    for (int u = snake_unit(0); u < a.n_units && ok; u = snake_unit(++unit_iter)) {
-      const BwdUnit un = decode_bwd_unit(a, u);
+    for (;; ++unit_iter) {
       const int buf = unit_iter & 1;
       if (!mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+      const int u = bars->list_unit[buf];
+      if (u < 0) break;
+      const BwdUnit un = decode_bwd_unit(a, u);
       StepIter it;
       it.init(lists + buf * kMaxSteps, bars->list_n[buf], a.G, a.Sq);
       int g, q0;

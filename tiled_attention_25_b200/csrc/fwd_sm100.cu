@@ -60,6 +60,8 @@ struct FwdCfg {
 };
 
 struct FwdBarriers {
+  alignas(16) uint32_t clc_resp[4];  // cluster launch control response (the next unit)
+  uint64_t clc_bar;
   uint64_t list_full[2], list_empty[2];
   uint64_t q_full, q_empty;
   uint64_t s_full[2], p_full[2], o_full[2], o_final[2];
@@ -69,6 +71,7 @@ struct FwdBarriers {
   uint32_t abort_flag;
   uint32_t never_set;  // abort word for drain waits that must not stop early
   int32_t list_n[2];   // step counts of the two step lists
+  int32_t list_unit[2];  // the unit of each list (rank in the work order); -1 ends the walk
 };
 
 // Consumers of a step list: the MMA warp and the 8 softmax warps (lane 0 each).
@@ -347,6 +350,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     mbar_init(smem_u32(&bars->q_full), 1);
     mbar_init(smem_u32(&bars->q_empty), 1);
+    mbar_init(smem_u32(&bars->clc_bar), 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(smem_u32(&bars->s_full[t]), 1);
       mbar_init(smem_u32(&bars->p_full[t]), 128);
@@ -391,18 +395,37 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint32_t slot_uses[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     int ring_pos = 0;
     int unit_iter = 0;
-    uint32_t q_loads = 0;
+    uint32_t q_loads = 0, clc_asked = 0, clc_read = 0;
+    const uint32_t clc_resp = smem_u32(bars->clc_resp), clc_bar = smem_u32(&bars->clc_bar);
     bool ok = true;
-    for (int u = snake_unit(0); u < a.n_units && ok; u = snake_unit(++unit_iter)) {
-      const UnitCoord uc = decode_unit(a, u);
-      const int hk = uc.h / a.G;
+    // The first unit: with cluster launch control (one CTA launched per unit)
+    // this CTA's own, then the unit of each not-yet-started CTA the hardware
+    // cancels for it; otherwise the static snake walk.  Either way each unit's
+    // list is published with its rank, and rank -1 ends every role's walk.
+    int u = a.clc ? static_cast<int>(blockIdx.x) : snake_unit(0);
+    for (;; ++unit_iter) {
       const int buf = unit_iter & 1;
       uint32_t* lst = lists + buf * kMaxSteps;
       if (!mbar_wait_warp(smem_u32(&bars->list_empty[buf]), ((unit_iter >> 1) & 1) ^ 1, wc)) { ok = false; break; }
-      const int n = build_pair_steps(a.tile_class, uc.b, uc.p, a.nQ, a.nK, a.Sq, a.Skv, a.mod.mask,
-                                     a.mod.window, lst);
-      if (lane == 0) bars->list_n[buf] = n;
+      if (u >= a.n_units) u = -1;
+      UnitCoord uc{};
+      int n = 0;
+      if (u >= 0) {
+        uc = decode_unit(a, u);
+        n = build_pair_steps(a.tile_class, uc.b, uc.p, a.nQ, a.nK, a.Sq, a.Skv, a.mod.mask, a.mod.window, lst);
+      }
+      if (lane == 0) {
+        bars->list_n[buf] = n;
+        bars->list_unit[buf] = u;
+      }
       mbar_arrive(smem_u32(&bars->list_full[buf]));
+      if (u < 0) break;
+      const int hk = uc.h / a.G;
+      if (lane == 0 && a.clc) {  // ask for the next unit now; the answer lands while this one streams
+        mbar_arrive_expect_tx(clc_bar, 16);
+        clc_try_cancel(clc_resp, clc_bar);
+        ++clc_asked;
+      }
       if (lane == 0) {
         // Q buffers are free once the previous unit's QK^T products finished
         if (!ATTN25_TIMED(tr[1], mbar_wait_thread(smem_u32(&bars->q_empty), (unit_iter & 1) ^ 1, wc))) {
@@ -435,12 +458,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      if (a.clc) {  // the next unit: the rank of the cancelled CTA, or -1
+        if (!mbar_wait_warp(clc_bar, clc_read & 1, wc)) { ok = false; break; }
+        ++clc_read;
+        u = clc_cancelled_x(clc_resp);
+      } else {
+        u = snake_unit(unit_iter + 1);
+      }
     }
     if (lane == 0) {
       // let the copies in flight land before the CTA exits: after a failed wait
       // of this warp, and also after a normal end, since a consumer that gave
       // up may have left the last copies unconsumed (instant otherwise)
       const WaitCtl drain_wc{drain_limit(a.wait_ns), smem_u32(&bars->never_set), a.status};
+      if (clc_asked > clc_read) mbar_wait_thread(clc_bar, (clc_asked - 1) & 1, drain_wc);
       for (int s2 = 0; s2 < Cfg::kStages; ++s2) {
         if (slot_uses[s2] == 0) continue;
         mbar_wait_thread(smem_u32(&bars->kv_full[s2]), (slot_uses[s2] - 1) & 1, drain_wc);
@@ -459,10 +491,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     bool ok = true;
     const uint32_t s_tmem[2] = {tmem, tmem + 128};
     const uint32_t o_tmem[2] = {tmem + 256, tmem + 256 + D};
-    for (int u = snake_unit(0); u < a.n_units && ok; u = snake_unit(++unit_iter)) {
+    for (;; ++unit_iter) {
       const int buf = unit_iter & 1;
       const uint32_t* lst = lists + buf * kMaxSteps;
       if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+      if (bars->list_unit[buf] < 0) break;
       const int n_steps = bars->list_n[buf];
       if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->q_full), unit_iter & 1, wc))) { ok = false; break; }
       tc_fence_after();
@@ -563,7 +596,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     int unit_iter = 0;
     uint32_t o_units = 0;  // units with at least one step seen so far (o_final phases)
     bool ok = true;
-    for (int u = snake_unit(0); u < a.n_units && ok; u = snake_unit(++unit_iter)) {
+    for (;; ++unit_iter) {
+      const int buf = unit_iter & 1;
+      if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+      const int u = bars->list_unit[buf];
+      if (u < 0) break;
       const UnitCoord uc = decode_unit(a, u);
       RowCtx rc;
       rc.row = (2 * uc.p + t) * TILE + r;
@@ -596,9 +633,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
       float m_run = -INFINITY, l_run = 0.f;
       int n_act = 0;
-      const int buf = unit_iter & 1;
       const uint32_t* lst = lists + buf * kMaxSteps;
-      if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
       const int n_steps = bars->list_n[buf];
       const uint32_t act_bit = t == 0 ? kStepAct0 : kStepAct1;
       const uint32_t prt_bit = t == 0 ? kStepPrt0 : kStepPrt1;

@@ -30,6 +30,7 @@ struct FwdArgs {
   const int32_t* kv_count;
   const int32_t* kv_index;
   const int32_t* fwd_order;
+  int clc;                    // work walk: 0 static snake over the order, 1 cluster launch control
   uint64_t wait_ns;
   int* status;
   unsigned long long* trace;  // profiling builds only (else nullptr)
@@ -64,6 +65,7 @@ struct BwdArgs {
   unsigned int* dq_sem;
   const int32_t* kv_count;
   const int32_t* kv_index;
+  int clc;                    // work walk: 0 static snake over the order, 1 cluster launch control
   uint64_t wait_ns;
   int* status;
   unsigned long long* trace;  // profiling builds only (else nullptr)

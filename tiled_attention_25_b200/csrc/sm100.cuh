@@ -465,4 +465,33 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// ------------------------------------------------------------------ cluster launch control
+//
+// Ask the hardware to cancel a CTA of this grid that has not started yet, so
+// that the asking CTA takes over its work.  The 16-byte response lands in
+// shared memory and completes `bar` (armed by the caller with expect_tx of
+// 16 bytes).  Once a response reports that nothing was cancelled, no further
+// request may be made.
+__device__ __forceinline__ void clc_try_cancel(uint32_t resp, uint32_t bar) {
+  asm volatile(
+      "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];" ::"r"(resp),
+      "r"(bar)
+      : "memory");
+}
+
+// The x index of the CTA a completed response cancelled, or -1 if it cancelled none.
+__device__ __forceinline__ int clc_cancelled_x(uint32_t resp) {
+  uint32_t ok, x = 0;
+  asm volatile(
+      "{\n\t.reg .b128 r;\n\t.reg .pred p;\n\t"
+      "ld.shared.b128 r, [%2];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "@p clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, r;\n\t}"
+      : "=r"(ok), "+r"(x)
+      : "r"(resp)
+      : "memory");
+  return ok ? static_cast<int>(x) : -1;
+}
+
 }  // namespace attn25
