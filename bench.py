@@ -190,11 +190,22 @@ CONFIG_ENTRIES = ("dense:causal", "gqa_long:causal", "score_mods:alibi", "score_
                   "score_mods:sliding_window", "score_mods:local_boost", "documents:document")
 
 
+# Variants of the path, each on the same workload (bench.py --variant):
+#   det   the backward with the bitwise reproducible dQ (attn_bwd_deterministic)
+#   bshd  Q, K, V, O, dO and the gradients stored [B][S][H][D], passed as
+#         strided [B][H][S][D] views (attn_fwd_strided / attn_bwd_strided)
+#   fp8   the forward with FP8 scores: Q and K rotated and quantised to e4m3
+#         (attn_fp8_rotate_quantize, inside the timed forward) and
+#         attn_fwd_fp8; forward only (its LSE belongs to the FP8 scores)
+VARIANTS = ("det", "bshd", "fp8")
+
+
 class Problem:
     """One workload's device tensors, mod parameters and block mask."""
 
-    def __init__(self, ta, spec, rank, dev):
+    def __init__(self, ta, spec, rank, dev, variant=None):
         import torch
+        self.variant = variant
         self.w, self.mod_name = parse_workload(spec)
         w = self.w
         self.mod = MOD_NAMES[self.mod_name]
@@ -215,7 +226,18 @@ class Problem:
         self.out = torch.empty_like(self.q)
         self.lse = torch.empty(w.B, w.Hq, w.Sq, dtype=torch.float32, device=dev)
         self.dq, self.dk, self.dv = torch.empty_like(self.q), torch.empty_like(self.k), torch.empty_like(self.v)
-        self.ws = ta.new_bwd_workspace(w.B, w.Hq, w.Sq, w.D, device=dev)
+        self.ws = ta.new_bwd_workspace(w.B, w.Hq, w.Sq, w.D, device=dev, deterministic=variant == "det")
+        if variant == "bshd":  # the same values in [B][S][H][D] storage, seen as [B][H][S][D] views
+            bshd = lambda t: t.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+            self.q, self.k, self.v, self.dout = (bshd(t) for t in (self.q, self.k, self.v, self.dout))
+            self.out, self.dq, self.dk, self.dv = (bshd(t) for t in (self.out, self.dq, self.dk, self.dv))
+        if variant == "fp8":
+            g = torch.Generator().manual_seed(1000 + w.seed)
+            self.signs = (torch.randint(0, 2, (w.D,), generator=g, dtype=torch.int8) * 2 - 1).to(dev)
+            self.q8 = torch.empty(w.B, w.Hq, w.Sq, w.D, dtype=torch.uint8, device=dev)
+            self.k8 = torch.empty(w.B, w.Hkv, w.Skv, w.D, dtype=torch.uint8, device=dev)
+            self.qs = torch.empty(w.B, w.Hq, dtype=torch.float32, device=dev)
+            self.ks = torch.empty(w.B, w.Hkv, dtype=torch.float32, device=dev)
         nbytes = ta.attn_block_mask_bytes(w.B, w.Sq, w.Skv)
         mbuf = torch.empty(nbytes + 256, dtype=torch.uint8, device=dev)
         off = (-mbuf.data_ptr()) % 256
@@ -227,13 +249,26 @@ class Problem:
         self.ta.build_block_mask(self.mod, self.dp, w.B, w.Sq, w.Skv, self.mask, stream)
 
     def forward(self, stream, with_lse=True):
-        self.ta.attn_fwd(self.q, self.k, self.v, self.out, self.lse if with_lse else None, scale=self.w.scale,
-                         mod_kind=self.mod, mod_params=self.dp, block_mask=self.mask, stream=stream)
+        lse = self.lse if with_lse else None
+        kw = dict(scale=self.w.scale, mod_kind=self.mod, mod_params=self.dp, block_mask=self.mask, stream=stream)
+        if self.variant == "fp8":
+            self.ta.attn_fp8_rotate_quantize(self.q, self.signs, self.q8, self.qs, stream=stream)
+            self.ta.attn_fp8_rotate_quantize(self.k, self.signs, self.k8, self.ks, stream=stream)
+            self.ta.attn_fwd_fp8(self.q8, self.k8, self.qs, self.ks, self.v, self.out, lse, **kw)
+        elif self.variant == "bshd":
+            self.ta.attn_fwd_strided(self.q, self.k, self.v, self.out, lse, **kw)
+        else:
+            self.ta.attn_fwd(self.q, self.k, self.v, self.out, lse, **kw)
 
     def backward(self, stream):
-        self.ta.attn_bwd(self.q, self.k, self.v, self.out, self.lse, self.dout, self.dq, self.dk, self.dv,
-                         self.ws, scale=self.w.scale, mod_kind=self.mod, mod_params=self.dp,
-                         block_mask=self.mask, stream=stream)
+        args = (self.q, self.k, self.v, self.out, self.lse, self.dout, self.dq, self.dk, self.dv, self.ws)
+        kw = dict(scale=self.w.scale, mod_kind=self.mod, mod_params=self.dp, block_mask=self.mask, stream=stream)
+        if self.variant == "det":
+            self.ta.attn_bwd_deterministic(*args, **kw)
+        elif self.variant == "bshd":
+            self.ta.attn_bwd_strided(*args, **kw)
+        else:
+            self.ta.attn_bwd(*args, **kw)
 
 
 def time_steps(ta, pb, stream, flush, steps, warmup, world, dev, fwd_lse=True, with_bwd=True):
@@ -290,24 +325,40 @@ def time_steps(ta, pb, stream, flush, steps, warmup, world, dev, fwd_lse=True, w
             "ms_step_median": statistics.median(t_step), "ms_step_min": min(t_step), "clocks": clocks}
 
 
-def config_entry(ta, spec, rank, world, dev, stream, flush, steps, warmup, peak):
+# Entries of the other paths the library offers, on parity workloads:
+# (workload:mod, variant, work walk)
+EXTENSION_ENTRIES = (("dense:none", "det", None), ("dense:none", "bshd", None), ("dense:none", "fp8", None),
+                     ("dense:causal", None, "clc"), ("documents:document", None, "clc"))
+
+
+def config_entry(ta, spec, rank, world, dev, stream, flush, steps, warmup, peak, variant=None, walk=None):
     """Forward and backward useful TFLOP/s of one parity configuration, timed
-    like the headline (own clock record)."""
+    like the headline (own clock record); optionally a variant of the path
+    (VARIANTS) or the cluster-launch-control work walk."""
     import torch
-    pb = Problem(ta, spec, rank, dev)
-    t = time_steps(ta, pb, stream, flush, steps, warmup, world, dev)
+    pb = Problem(ta, spec, rank, dev, variant=variant)
+    fwd_only = variant == "fp8"
+    if walk == "clc":
+        ta.attn_set_work_walk(ta.WALK_CLUSTER_LAUNCH_CONTROL)
+    try:
+        t = time_steps(ta, pb, stream, flush, steps, warmup, world, dev, with_bwd=not fwd_only)
+    finally:
+        ta.attn_set_work_walk(ta.WALK_STATIC)
     n_u, f_fwd, f_bwd = useful_counts(ta, pb.w, pb.mod_name, pb.params)
     fwd_tf = f_fwd / (t["ms_fwd"] * 1e-3) / 1e12
-    bwd_tf = f_bwd / (t["ms_bwd"] * 1e-3) / 1e12
+    bwd_tf = 0.0 if fwd_only else f_bwd / (t["ms_bwd"] * 1e-3) / 1e12
     w = pb.w
     entry = {"shape": f"B={w.B} Hq={w.Hq} Hkv={w.Hkv} S={w.Sq} D={w.D}", "mod": pb.mod_name,
+             "variant": variant, "walk": walk or "static",
              "useful_elements": n_u, "steps": steps, "warmup": warmup,
-             "ms_fwd": round(t["ms_fwd"], 4), "ms_bwd": round(t["ms_bwd"], 4),
-             "ms_block_mask": round(t["ms_mask"], 4),
-             "fwd_tflops": round(fwd_tf, 1), "bwd_tflops": round(bwd_tf, 1),
-             "fwd_frac_of_peak": round(fwd_tf / peak, 4), "bwd_frac_of_peak": round(bwd_tf / peak, 4),
-             "step_tflops": round(job_throughput(f_fwd + f_bwd, world, t["ms_step"]), 1),
-             "clocks": t["clocks"]}
+             "ms_fwd": round(t["ms_fwd"], 4), "ms_block_mask": round(t["ms_mask"], 4),
+             "fwd_tflops": round(fwd_tf, 1), "fwd_frac_of_peak": round(fwd_tf / peak, 4), "clocks": t["clocks"]}
+    if fwd_only:
+        entry["note"] = "forward only: the rotation and e4m3 quantisation of Q and K are inside the timed forward"
+    else:
+        entry.update({"ms_bwd": round(t["ms_bwd"], 4), "bwd_tflops": round(bwd_tf, 1),
+                      "bwd_frac_of_peak": round(bwd_tf / peak, 4),
+                      "step_tflops": round(job_throughput(f_fwd + f_bwd, world, t["ms_step"]), 1)})
     del pb
     torch.cuda.empty_cache()
     return entry
@@ -452,6 +503,10 @@ def run_gpu(args, rank, world, local_rank):
         for spec in CONFIG_ENTRIES:
             if spec != wl:
                 configs[spec] = config_entry(ta, spec, rank, world, dev, stream, flush, args.config_steps, 3, peak)
+        for spec, variant, walk in EXTENSION_ENTRIES:
+            name = f"{spec}:{variant or walk}"
+            configs[name] = config_entry(ta, spec, rank, world, dev, stream, flush, args.config_steps, 3, peak,
+                                         variant=variant, walk=walk)
         line["configs"] = configs
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, mod_name, params, seconds=args.cpu_seconds)
