@@ -104,7 +104,7 @@ struct BwdBarriers {
   uint32_t abort_flag;
   uint32_t never_set;  // abort word for drain waits that must not stop early
   int32_t list_n[2];   // lengths of the two query-tile lists
-  int32_t list_unit[2];  // the unit of each list (rank in the work order); -1 ends the walk
+  int32_t list_unit[2];  // cluster launch control: the unit of each list; -1 ends the walk
 };
 
 // Consumers of a query-tile list: the MMA warp and the P, dS and drain warps
@@ -402,22 +402,12 @@ __device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h,
         v.x = fmaf(x[c], a.sl2, -aux * fabsf(dq0 + static_cast<float>(c))) + nl.x;
         v.y = fmaf(x[c + 1], a.sl2, -aux * fabsf(dq0 + static_cast<float>(c + 1))) + nl.y;
       } else if constexpr (score_of(MOD) == MOD_SOFTCAP) {
-        if (series) {
-          v.x = fmaf(aux2, tanh_series(x[c] * aux), nl.x);
-          v.y = fmaf(aux2, tanh_series(x[c + 1] * aux), nl.y);
-        } else {
-          v.x = fmaf(aux2, tanh_ex2(x[c] * aux), nl.x);
-          v.y = fmaf(aux2, tanh_ex2(x[c + 1] * aux), nl.y);
-        }
+        v.x = fmaf(aux2, tanh_ex2(x[c] * aux), nl.x);
+        v.y = fmaf(aux2, tanh_ex2(x[c + 1] * aux), nl.y);
       } else if constexpr (score_of(MOD) == MOD_BOOST) {
-        if (band != 0) {
-          const float f = band == 1 ? aux : a.sl2;
-          v = __ffma2_rn(make_float2(x[c], x[c + 1]), make_float2(f, f), nl);
-        } else {
-          const float r = static_cast<float>(a.mod.boost_radius);
-          v.x = fmaf(x[c], fabsf(dq0 + static_cast<float>(c)) < r ? aux : a.sl2, nl.x);
-          v.y = fmaf(x[c + 1], fabsf(dq0 + static_cast<float>(c + 1)) < r ? aux : a.sl2, nl.y);
-        }
+        const float r = static_cast<float>(a.mod.boost_radius);
+        v.x = fmaf(x[c], fabsf(dq0 + static_cast<float>(c)) < r ? aux : a.sl2, nl.x);
+        v.y = fmaf(x[c + 1], fabsf(dq0 + static_cast<float>(c + 1)) < r ? aux : a.sl2, nl.y);
       } else {
         v = __ffma2_rn(make_float2(x[c], x[c + 1]), sl2, nl);
       }
@@ -465,7 +455,7 @@ __device__ __forceinline__ void store_acc_rows(__nv_bfloat16* dst, uint32_t src,
   }
 }
 
-template <int D, int MOD>
+template <int D, int MOD, bool CLC>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -543,33 +533,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       uint32_t kv_loads = 0, stage_uses[4] = {0, 0, 0, 0}, clc_asked = 0, clc_read = 0;
       const uint32_t clc_resp = smem_u32(bars->clc_resp), clc_bar = smem_u32(&bars->clc_bar);
       bool ok = true;
-      // The first unit: with cluster launch control (one CTA launched per
-      // unit) this CTA's own, then the unit of each not-yet-started CTA the
-      // hardware cancels for it; otherwise the static snake walk.  Each list
-      // is published with its unit's rank, and rank -1 ends every role's walk.
-      int u = a.clc ? static_cast<int>(blockIdx.x) : snake_unit(0);
-      for (;; ++unit_iter) {
+      // The static walk: the snake over the order.  Cluster launch control (one
+      // CTA launched per unit): this CTA's own unit, then the unit of each
+      // not-yet-started CTA the hardware cancels for it; each list is published
+      // with its unit's rank, and rank -1 ends every role's walk.
+      for (int u = CLC ? static_cast<int>(blockIdx.x) : snake_unit(0); ok; ++unit_iter) {
+        if constexpr (!CLC) {
+          if (u >= a.n_units) break;
+        }
         const int buf = unit_iter & 1;
         uint16_t* lst = lists + buf * kMaxSteps;
-        if (!mbar_wait_warp_ool(smem_u32(&bars->list_empty[buf]), ((unit_iter >> 1) & 1) ^ 1, wc)) { ok = false; break; }
-        if (u >= a.n_units) u = -1;
         BwdUnit un{};
+        if constexpr (!CLC) un = decode_bwd_unit(a, u);
+        if (!mbar_wait_warp_ool(smem_u32(&bars->list_empty[buf]), ((unit_iter >> 1) & 1) ^ 1, wc)) { ok = false; break; }
         int n = 0;
+        if constexpr (CLC) {
+          if (u >= a.n_units) u = -1;
+          if (u >= 0) un = decode_bwd_unit(a, u);
+          if (lane == 0) bars->list_unit[buf] = u;
+        }
         if (u >= 0) {
-          un = decode_bwd_unit(a, u);
           n = build_kv_qtiles(a.tile_class, un.b, un.kt, a.nQ, a.nK, a.Sq, a.Skv, a.mod.mask, a.mod.window, lst);
           if (a.dq_sem != nullptr) build_positions(a, un.b, un.kt, lst, n, positions + buf * kMaxSteps);
         }
-        if (lane == 0) {
-          bars->list_n[buf] = n;
-          bars->list_unit[buf] = u;
-        }
+        if (lane == 0) bars->list_n[buf] = n;
         mbar_arrive(smem_u32(&bars->list_full[buf]));
-        if (u < 0) break;
-        if (lane == 0 && a.clc) {  // ask for the next unit now; the answer lands while this one streams
-          mbar_arrive_expect_tx(clc_bar, 16);
-          clc_try_cancel(clc_resp, clc_bar);
-          ++clc_asked;
+        if constexpr (CLC) {
+          if (u < 0) break;
+          if (lane == 0) {  // ask for the next unit now; the answer lands while this one streams
+            mbar_arrive_expect_tx(clc_bar, 16);
+            clc_try_cancel(clc_resp, clc_bar);
+            ++clc_asked;
+          }
         }
         if (lane == 0) {
           if (!ATTN25_TIMED(tr[1], mbar_wait_thread_ool(smem_u32(&bars->kv_empty), (unit_iter & 1) ^ 1, wc))) {
@@ -603,7 +598,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
-        if (a.clc) {  // the next unit: the rank of the cancelled CTA, or -1
+        if constexpr (CLC) {  // the next unit: the rank of the cancelled CTA, or -1
           if (!mbar_wait_warp_ool(clc_bar, clc_read & 1, wc)) { ok = false; break; }
           ++clc_read;
           u = clc_cancelled_x(clc_resp);
@@ -649,9 +644,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
       for (;; ++unit_iter) {
         const int buf = unit_iter & 1;
-        MMA_WAIT(mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc));
-        if (bars->list_unit[buf] < 0) break;
-        MMA_WAIT(ATTN25_TIMED(tr[1], mbar_wait_warp_ool(smem_u32(&bars->kv_full), unit_iter & 1, wc)));
+        if constexpr (CLC) {
+          MMA_WAIT(mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc));
+          if (bars->list_unit[buf] < 0) break;
+          MMA_WAIT(ATTN25_TIMED(tr[1], mbar_wait_warp_ool(smem_u32(&bars->kv_full), unit_iter & 1, wc)));
+        } else {
+          if (snake_unit(unit_iter) >= a.n_units) break;
+          MMA_WAIT(mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc) &&
+                   ATTN25_TIMED(tr[1], mbar_wait_warp_ool(smem_u32(&bars->kv_full), unit_iter & 1, wc)));
+        }
         StepIter it;
         it.init(lists + buf * kMaxSteps, bars->list_n[buf], a.G, a.Sq);
         int g, q0;
@@ -757,13 +758,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
     for (;; ++unit_iter) {
       const int buf = unit_iter & 1;
-      if (!mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
-      const int u = bars->list_unit[buf];
-      if (u < 0) break;
+      int u;
+      if constexpr (CLC) {
+        if (!mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+        u = bars->list_unit[buf];
+        if (u < 0) break;
+      } else {
+        u = snake_unit(unit_iter);
+        if (u >= a.n_units) break;
+      }
       const BwdUnit un = decode_bwd_unit(a, u);
       const int kv = un.kt * TILE + r;
       int qlo, qhi;
       key_interval<MOD>(a, un.b, kv, qlo, qhi);
+      if constexpr (!CLC) {
+        if (!mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+      }
       StepIter it;
       it.init(lists + buf * kMaxSteps, bars->list_n[buf], a.G, a.Sq);
       int g, q0;
@@ -835,11 +845,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
     for (;; ++unit_iter) {
       const int buf = unit_iter & 1;
-      if (!mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
-      const int u = bars->list_unit[buf];
-      if (u < 0) break;
+      int u;
+      if constexpr (CLC) {
+        if (!mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+        u = bars->list_unit[buf];
+        if (u < 0) break;
+      } else {
+        u = snake_unit(unit_iter);
+        if (u >= a.n_units) break;
+      }
       const BwdUnit un = decode_bwd_unit(a, u);
       const int kv = un.kt * TILE + r;
+      if constexpr (!CLC) {
+        if (!mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+      }
       StepIter it;
       it.init(lists + buf * kMaxSteps, bars->list_n[buf], a.G, a.Sq);
       int g, q0;
@@ -907,13 +926,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               d.x = pr.x > 0.f ? d.x * (1.f - t0 * t0) : 0.f;
               d.y = pr.y > 0.f ? d.y * (1.f - t1 * t1) : 0.f;
             } else if constexpr (score_of(MOD) == MOD_BOOST) {
-              if (band == 1) {
-                d = __fmul2_rn(d, make_float2(a.mod.boost, a.mod.boost));
-              } else if (band == 0) {
-                const float rad = static_cast<float>(a.mod.boost_radius);
-                d.x *= fabsf(dq0 + static_cast<float>(c)) < rad ? a.mod.boost : 1.f;
-                d.y *= fabsf(dq0 + static_cast<float>(c + 1)) < rad ? a.mod.boost : 1.f;
-              }
+              const float rad = static_cast<float>(a.mod.boost_radius);
+              d.x *= fabsf(dq0 + static_cast<float>(c)) < rad ? a.mod.boost : 1.f;
+              d.y *= fabsf(dq0 + static_cast<float>(c + 1)) < rad ? a.mod.boost : 1.f;
             }
             w[e] = pack_bf16x2(d.x, d.y);
           }
@@ -961,10 +976,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_arrive(smem_u32(&bars->ds_ready[0]));
     for (;; ++unit_iter) {
       const int buf = unit_iter & 1;
-      if (!mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
-      const int u = bars->list_unit[buf];
-      if (u < 0) break;
+      int u;
+      if constexpr (CLC) {
+        if (!mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+        u = bars->list_unit[buf];
+        if (u < 0) break;
+      } else {
+        u = snake_unit(unit_iter);
+        if (u >= a.n_units) break;
+      }
       const BwdUnit un = decode_bwd_unit(a, u);
+      if constexpr (!CLC) {
+        if (!mbar_wait_warp_ool(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+      }
       StepIter it;
       it.init(lists + buf * kMaxSteps, bars->list_n[buf], a.G, a.Sq);
       int g, q0;
@@ -1092,7 +1116,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   bwd_prep_kernel<D><<<prep_blocks, 256, 0, stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  auto kernel = attn_bwd_kernel<D, MOD>;
+  auto kernel = a.clc ? attn_bwd_kernel<D, MOD, true> : attn_bwd_kernel<D, MOD, false>;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg<D>::kAllocBytes);
   if (e != cudaSuccess) return e;
   kernel<<<grid, kBwdThreads, BwdCfg<D>::kAllocBytes, stream>>>(tq, tk, tv, tdo, a);

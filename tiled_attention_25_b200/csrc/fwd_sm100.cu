@@ -71,7 +71,7 @@ struct FwdBarriers {
   uint32_t abort_flag;
   uint32_t never_set;  // abort word for drain waits that must not stop early
   int32_t list_n[2];   // step counts of the two step lists
-  int32_t list_unit[2];  // the unit of each list (rank in the work order); -1 ends the walk
+  int32_t list_unit[2];  // cluster launch control: the unit of each list; -1 ends the walk
 };
 
 // Consumers of a step list: the MMA warp and the 8 softmax warps (lane 0 each).
@@ -325,7 +325,7 @@ __device__ __forceinline__ float row_probs(float (&x)[4][32], const RowCtx& rc, 
   return acc.x + acc.y;
 }
 
-template <int D, int MOD, bool HAS_LSE, bool FP8 = false>
+template <int D, int MOD, bool HAS_LSE, bool FP8, bool CLC>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
@@ -398,34 +398,38 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint32_t q_loads = 0, clc_asked = 0, clc_read = 0;
     const uint32_t clc_resp = smem_u32(bars->clc_resp), clc_bar = smem_u32(&bars->clc_bar);
     bool ok = true;
-    // The first unit: with cluster launch control (one CTA launched per unit)
-    // this CTA's own, then the unit of each not-yet-started CTA the hardware
-    // cancels for it; otherwise the static snake walk.  Either way each unit's
-    // list is published with its rank, and rank -1 ends every role's walk.
-    int u = a.clc ? static_cast<int>(blockIdx.x) : snake_unit(0);
-    for (;; ++unit_iter) {
+    // The static walk: the snake over the order.  Cluster launch control (one
+    // CTA launched per unit): this CTA's own unit, then the unit of each
+    // not-yet-started CTA the hardware cancels for it; each list is published
+    // with its unit's rank, and rank -1 ends every role's walk.
+    for (int u = CLC ? static_cast<int>(blockIdx.x) : snake_unit(0); ok; ++unit_iter) {
+      if constexpr (!CLC) {
+        if (u >= a.n_units) break;
+      }
+      UnitCoord uc{};
+      if constexpr (!CLC) uc = decode_unit(a, u);
       const int buf = unit_iter & 1;
       uint32_t* lst = lists + buf * kMaxSteps;
       if (!mbar_wait_warp(smem_u32(&bars->list_empty[buf]), ((unit_iter >> 1) & 1) ^ 1, wc)) { ok = false; break; }
-      if (u >= a.n_units) u = -1;
-      UnitCoord uc{};
       int n = 0;
-      if (u >= 0) {
-        uc = decode_unit(a, u);
+      if constexpr (CLC) {
+        if (u >= a.n_units) u = -1;
+        if (u >= 0) uc = decode_unit(a, u);
+        if (lane == 0) bars->list_unit[buf] = u;
+      }
+      if (u >= 0)
         n = build_pair_steps(a.tile_class, uc.b, uc.p, a.nQ, a.nK, a.Sq, a.Skv, a.mod.mask, a.mod.window, lst);
-      }
-      if (lane == 0) {
-        bars->list_n[buf] = n;
-        bars->list_unit[buf] = u;
-      }
+      if (lane == 0) bars->list_n[buf] = n;
       mbar_arrive(smem_u32(&bars->list_full[buf]));
-      if (u < 0) break;
-      const int hk = uc.h / a.G;
-      if (lane == 0 && a.clc) {  // ask for the next unit now; the answer lands while this one streams
-        mbar_arrive_expect_tx(clc_bar, 16);
-        clc_try_cancel(clc_resp, clc_bar);
-        ++clc_asked;
+      if constexpr (CLC) {
+        if (u < 0) break;
+        if (lane == 0) {  // ask for the next unit now; the answer lands while this one streams
+          mbar_arrive_expect_tx(clc_bar, 16);
+          clc_try_cancel(clc_resp, clc_bar);
+          ++clc_asked;
+        }
       }
+      const int hk = uc.h / a.G;
       if (lane == 0) {
         // Q buffers are free once the previous unit's QK^T products finished
         if (!ATTN25_TIMED(tr[1], mbar_wait_thread(smem_u32(&bars->q_empty), (unit_iter & 1) ^ 1, wc))) {
@@ -459,7 +463,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
-      if (a.clc) {  // the next unit: the rank of the cancelled CTA, or -1
+      if constexpr (CLC) {  // the next unit: the rank of the cancelled CTA, or -1
         if (!mbar_wait_warp(clc_bar, clc_read & 1, wc)) { ok = false; break; }
         ++clc_read;
         u = clc_cancelled_x(clc_resp);
@@ -492,10 +496,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t s_tmem[2] = {tmem, tmem + 128};
     const uint32_t o_tmem[2] = {tmem + 256, tmem + 256 + D};
     for (;; ++unit_iter) {
+      if constexpr (!CLC) {
+        if (snake_unit(unit_iter) >= a.n_units) break;
+      }
       const int buf = unit_iter & 1;
       const uint32_t* lst = lists + buf * kMaxSteps;
       if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
-      if (bars->list_unit[buf] < 0) break;
+      if constexpr (CLC) {
+        if (bars->list_unit[buf] < 0) break;
+      }
       const int n_steps = bars->list_n[buf];
       if (!ATTN25_TIMED(tr[1], mbar_wait_warp(smem_u32(&bars->q_full), unit_iter & 1, wc))) { ok = false; break; }
       tc_fence_after();
@@ -598,9 +607,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     bool ok = true;
     for (;; ++unit_iter) {
       const int buf = unit_iter & 1;
-      if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
-      const int u = bars->list_unit[buf];
-      if (u < 0) break;
+      int u;
+      if constexpr (CLC) {
+        if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+        u = bars->list_unit[buf];
+        if (u < 0) break;
+      } else {
+        u = snake_unit(unit_iter);
+        if (u >= a.n_units) break;
+      }
       const UnitCoord uc = decode_unit(a, u);
       RowCtx rc;
       rc.row = (2 * uc.p + t) * TILE + r;
@@ -634,6 +649,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       float m_run = -INFINITY, l_run = 0.f;
       int n_act = 0;
       const uint32_t* lst = lists + buf * kMaxSteps;
+      if constexpr (!CLC) {
+        if (!mbar_wait_warp(smem_u32(&bars->list_full[buf]), (unit_iter >> 1) & 1, wc)) { ok = false; break; }
+      }
       const int n_steps = bars->list_n[buf];
       const uint32_t act_bit = t == 0 ? kStepAct0 : kStepAct1;
       const uint32_t prt_bit = t == 0 ? kStepPrt0 : kStepPrt1;
@@ -751,10 +769,10 @@ namespace attn25 {
 
 namespace {
 
-template <int D, int MOD, bool LSE, bool FP8 = false>
-cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+template <int D, int MOD, bool LSE, bool FP8, bool CLC>
+cudaError_t launch_fwd_k(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const FwdArgs& a, int grid, cudaStream_t stream) {
-  auto kernel = attn_fwd_kernel<D, MOD, LSE, FP8>;
+  auto kernel = attn_fwd_kernel<D, MOD, LSE, FP8, CLC>;
   // The register split assumes the kernel launches with kLaunchRegs per
   // thread; with fewer, setmaxnreg.inc could wait forever, so refuse.
   static int launch_regs = -1;
@@ -770,6 +788,13 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   if (e != cudaSuccess) return e;
   kernel<<<grid, kFwdThreads, FwdCfg<D>::kAllocBytes, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
+}
+
+template <int D, int MOD, bool LSE, bool FP8 = false>
+cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const FwdArgs& a, int grid, cudaStream_t stream) {
+  return a.clc ? launch_fwd_k<D, MOD, LSE, FP8, true>(tq, tk, tv, a, grid, stream)
+               : launch_fwd_k<D, MOD, LSE, FP8, false>(tq, tk, tv, a, grid, stream);
 }
 
 template <int D, bool LSE>
