@@ -262,7 +262,10 @@ typedef struct attn_layouts {
 } attn_layouts;
 
 /* attn_fwd and attn_bwd on strided tensors (layouts NULL: contiguous);
- * bad strides return ATTN_ERR_ALIGN.  LSE stays contiguous [B][Hq][Sq]. */
+ * bad strides return ATTN_ERR_ALIGN.  LSE stays contiguous [B][Hq][Sq], the
+ * shape the FlashInfer page allocates for it ("FlashInfer SM120 NVFP4 어텐션
+ * 최적화", 코드 분석 1); the pages fix no layout for Q, K, V and O, so the
+ * library takes the two common ones and any strides between. */
 ATTN25_API int attn_fwd_strided(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v,
                                 attn_bf16* out, float* lse,
                                 int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
@@ -279,11 +282,12 @@ ATTN25_API int attn_bwd_strided(const attn_bf16* q, const attn_bf16* k, const at
                                 attn_stream_t stream);
 
 /*
- * The backward pass with a bitwise reproducible dQ.  dQ of a query row is a
- * sum over the key tiles that meet it ("FlashAttention-2 — GPU attention의
- * 사실상 표준", §4 Backward: the gradient of each query block collects one
- * term per key block); attn_bwd adds those terms into its fp32 accumulator
- * in whatever order the key tiles finish, so dQ's last bits vary from run to
+ * The backward pass with a bitwise reproducible dQ.  With Q, K and V split
+ * into blocks ("FlashAttention-2 — GPU attention의 사실상 표준", §3 item 1,
+ * Tiling) and the backward recomputing the scores block by block (§3 item 2
+ * and §4, the Backward item), dQ of a query row is a sum of one term per key
+ * tile that meets it; attn_bwd adds those terms into its fp32 accumulator in
+ * whatever order the key tiles finish, so dQ's last bits vary from run to
  * run.  Here every key tile waits for its turn before adding, and the terms
  * enter each row's sum in ascending key-tile order, so dQ (like dK and dV)
  * is the same bit for bit on every run, with or without a block mask.

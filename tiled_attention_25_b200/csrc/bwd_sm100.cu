@@ -1,8 +1,8 @@
 // Backward attention kernels for sm_100a.
 //
 // The scores are recomputed from Q, K and the saved logsumexp instead of
-// being stored ("FlashAttention-2 — GPU attention의 사실상 표준", §3
-// Recomputation and §4 Backward).  With s' = mod(scale q.k) and
+// being stored ("FlashAttention-2 — GPU attention의 사실상 표준", §3 item 2
+// Recomputation, and §4 Architecture, its Backward item).  With s' = mod(scale q.k) and
 // P = exp(s' - LSE), the exact gradient of O = P V is
 //     dV = P^T dO,  dP = dO V^T,  Delta_i = rowsum(dO_i * O_i),
 //     dS = P * (dP - Delta) * ds'/ds,  dQ = scale dS K,  dK = scale dS^T Q.
