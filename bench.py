@@ -328,7 +328,7 @@ def time_steps(ta, pb, stream, flush, steps, warmup, world, dev, fwd_lse=True, w
 # Entries of the other paths the library offers, on parity workloads:
 # (workload:mod, variant, work walk)
 EXTENSION_ENTRIES = (("dense:none", "det", None), ("dense:none", "bshd", None), ("dense:none", "fp8", None),
-                     ("dense:causal", None, "clc"), ("documents:document", None, "clc"))
+                     ("dense:causal", None, "static"), ("documents:document", None, "static"))
 
 
 def config_entry(ta, spec, rank, world, dev, stream, flush, steps, warmup, peak, variant=None, walk=None):
@@ -338,18 +338,18 @@ def config_entry(ta, spec, rank, world, dev, stream, flush, steps, warmup, peak,
     import torch
     pb = Problem(ta, spec, rank, dev, variant=variant)
     fwd_only = variant == "fp8"
-    if walk == "clc":
-        ta.attn_set_work_walk(ta.WALK_CLUSTER_LAUNCH_CONTROL)
+    if walk == "static":
+        ta.attn_set_work_walk(ta.WALK_STATIC)
     try:
         t = time_steps(ta, pb, stream, flush, steps, warmup, world, dev, with_bwd=not fwd_only)
     finally:
-        ta.attn_set_work_walk(ta.WALK_STATIC)
+        ta.attn_set_work_walk(ta.WALK_DEFAULT)
     n_u, f_fwd, f_bwd = useful_counts(ta, pb.w, pb.mod_name, pb.params)
     fwd_tf = f_fwd / (t["ms_fwd"] * 1e-3) / 1e12
     bwd_tf = 0.0 if fwd_only else f_bwd / (t["ms_bwd"] * 1e-3) / 1e12
     w = pb.w
     entry = {"shape": f"B={w.B} Hq={w.Hq} Hkv={w.Hkv} S={w.Sq} D={w.D}", "mod": pb.mod_name,
-             "variant": variant, "walk": walk or "static",
+             "variant": variant, "walk": walk or "cluster launch control",
              "useful_elements": n_u, "steps": steps, "warmup": warmup,
              "ms_fwd": round(t["ms_fwd"], 4), "ms_block_mask": round(t["ms_mask"], 4),
              "fwd_tflops": round(fwd_tf, 1), "fwd_frac_of_peak": round(fwd_tf / peak, 4), "clocks": t["clocks"]}

@@ -357,9 +357,9 @@ ATTN25_API void attn_set_wait_limit_ms(uint32_t ms);
  * (query-tile pairs forward, key tiles backward), which they always take in
  * the block mask's longest-first order (ascending key tiles for
  * attn_bwd_deterministic):
- *   ATTN_WALK_STATIC (default): one CTA per SM; wave k of the order goes to
- *     the CTAs in turn, every other wave reversed (a snake), fixed in advance;
- *   ATTN_WALK_CLUSTER_LAUNCH_CONTROL: one CTA per unit is launched; a CTA that
+ *   ATTN_WALK_STATIC: one CTA per SM; wave k of the order goes to the CTAs
+ *     in turn, every other wave reversed (a snake), fixed in advance;
+ *   ATTN_WALK_CLUSTER_LAUNCH_CONTROL (default): one CTA per unit is launched; a CTA that
  *     finishes its unit asks the hardware (Blackwell's cluster launch control)
  *     to cancel the next CTA that has not started and does that CTA's unit, so
  *     the walk adapts to data-dependent unit lengths as it runs ("PyTorch

@@ -20,7 +20,7 @@ pytestmark = pytest.mark.gpu
 def ta():
     import tiled_attention_25_b200 as m
     yield m
-    m.attn_set_work_walk(m.WALK_STATIC)
+    m.attn_set_work_walk(m.WALK_DEFAULT)
 
 
 def run_both(ta, c, use_mask=True):
@@ -35,7 +35,7 @@ def run_both(ta, c, use_mask=True):
         torch.cuda.synchronize()
         assert ta.attn_get_status() == 0
         res[walk] = (out, lse, run_fwd_bwd(ta, c, use_mask))
-    ta.attn_set_work_walk(ta.WALK_STATIC)
+    ta.attn_set_work_walk(ta.WALK_DEFAULT)
     return res[ta.WALK_STATIC], res[ta.WALK_CLUSTER_LAUNCH_CONTROL]
 
 
@@ -76,11 +76,12 @@ def test_deterministic_dq_under_cluster_launch_control(ta):
     so dQ is still bitwise the same on every run (and equal to the static walk's)."""
     from test_gpu_deterministic import run_det, same_bits
     c = Case(73, 4, 8, 4, 2048, 2048, 128, oracle.MOD_CAUSAL)
-    a = run_det(ta, c)
-    ta.attn_set_work_walk(ta.WALK_CLUSTER_LAUNCH_CONTROL)
+    ta.attn_set_work_walk(ta.WALK_STATIC)
     try:
+        a = run_det(ta, c)
+        ta.attn_set_work_walk(ta.WALK_CLUSTER_LAUNCH_CONTROL)
         b = run_det(ta, c)
         d = run_det(ta, c)
     finally:
-        ta.attn_set_work_walk(ta.WALK_STATIC)
+        ta.attn_set_work_walk(ta.WALK_DEFAULT)
     assert same_bits(a, b) and same_bits(b, d)

@@ -26,6 +26,7 @@ from .abi import (  # noqa: F401
     MOD_SLIDING_WINDOW,
     MOD_SOFTCAP,
     WALK_CLUSTER_LAUNCH_CONTROL,
+    WALK_DEFAULT,
     WALK_STATIC,
     AttnError,
     BlockMask,

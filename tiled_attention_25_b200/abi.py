@@ -478,6 +478,7 @@ def attn_set_wait_limit_ms(ms: int):
 
 WALK_STATIC = 0
 WALK_CLUSTER_LAUNCH_CONTROL = 1
+WALK_DEFAULT = WALK_CLUSTER_LAUNCH_CONTROL
 
 
 def attn_set_work_walk(walk: int):

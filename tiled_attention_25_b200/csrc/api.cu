@@ -34,7 +34,7 @@ static __device__ __align__(256) unsigned char g_bwd_scratch[kNoAllocScratchByte
 namespace {
 
 std::atomic<uint32_t> g_wait_ms{4000};
-std::atomic<int> g_work_walk{0};  // ATTN_WALK_STATIC or ATTN_WALK_CLUSTER_LAUNCH_CONTROL
+std::atomic<int> g_work_walk{1};  // ATTN_WALK_CLUSTER_LAUNCH_CONTROL (default) or ATTN_WALK_STATIC
 
 constexpr int kMaxDevices = 64;
 
