@@ -335,8 +335,6 @@ __device__ __forceinline__ float4 lds128(uint32_t addr) {
   return v;
 }
 
-// One key row of S^T (raw q.k for 64 queries) -> P^T = 2^(x - LSE2) in place;
-// nl2_addr is the shared address of the 64 negated base-2 LSEs.
 // Whether query q0 + c is kept for this thread's key on a PARTIAL step: inside
 // the key's query interval and, with the bitmap mask, set in the bitmap.
 // wa / wb hold (lane l) the keep-bit word of query q0 + l / q0 + 32 + l over
@@ -352,44 +350,33 @@ __device__ __forceinline__ bool keep_query(int c, int q0, int qlo, int qhi, uint
   return keep;
 }
 
-// The mask runs as a pass of its own after the exponentials (P = 0 where
-// masked, the same as 2^-inf), so that the exponential loop stays one copy
-// for every step and this warp's hot code stays small.  Local boost keeps the
-// mask inside the loop: its per-element radius test leaves no registers for
-// the separate pass.
-template <int MOD>
-constexpr bool kMaskAfterExp = score_of(MOD) != MOD_BOOST;
+// Whether the local boost band |q - kv| < radius meets any of this warp's
+// steps (dq0 = q0 - kv of the thread's key); warp-uniform.
+__device__ __forceinline__ bool boost_band_meets(const BwdArgs& a, float dq0) {
+  const float rad = static_cast<float>(a.mod.boost_radius);
+  return !__all_sync(0xffffffffu, dq0 >= rad || dq0 + static_cast<float>(BM - 1) <= -rad);
+}
 
+// One key row of S^T (raw q.k for 64 queries) -> P^T = 2^(x - LSE2) in place;
+// nl2_addr is the shared address of the 64 negated base-2 LSEs.  Every mod
+// shares one exponential loop: the boost multiplies the raw scores in a pass
+// of its own that runs only where the band meets the warp's step, and the
+// mask runs after the exponentials (P = 0 where masked, the same as 2^-inf).
 template <int MOD>
-__device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h, float dq0, int q0,
-                                        int qlo, int qhi, bool pred, uint32_t nl2_addr, uint32_t wa,
-                                        uint32_t wb) {
-  float aux = 0.f, aux2 = 0.f;
+__device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h, float dq0, int q0, int qlo,
+                                        int qhi, bool pred, uint32_t nl2_addr, uint32_t wa, uint32_t wb) {
+  float aux = 0.f;
   if constexpr (score_of(MOD) == MOD_ALIBI) aux = alibi_slope(a.mod, h, a.Hq) * LOG2E;
-  if constexpr (score_of(MOD) == MOD_SOFTCAP) {
-    aux = a.scale / a.mod.softcap;
-    aux2 = a.mod.softcap * LOG2E;
-  }
-  if constexpr (score_of(MOD) == MOD_BOOST) aux = a.mod.boost * a.sl2;
-  const float2 sl2 = make_float2(a.sl2, a.sl2);
-  // softcap: scores well below the cap across the warp's step take tanh from
-  // its series on the FMA pipe, the others from its exponential form (MUFU)
-  bool series = false;
-  if constexpr (score_of(MOD) == MOD_SOFTCAP) {
-    float mx = 0.f;
-#pragma unroll
-    for (int c = 0; c < BM; ++c) mx = fmaxf(mx, fabsf(x[c]));
-    series = __all_sync(0xffffffffu, mx <= kTanhSeriesLimit * a.mod.softcap / a.scale);
-  }
-  // local boost: the band |q - kv| < radius covers the warp's step wholly,
-  // or misses it wholly, except near its edges
-  int band = 0;  // 1: all inside, 2: all outside, 0: per element
   if constexpr (score_of(MOD) == MOD_BOOST) {
-    const float rad = static_cast<float>(a.mod.boost_radius);
-    const float lo = dq0, hi = dq0 + static_cast<float>(BM - 1);
-    if (__all_sync(0xffffffffu, fabsf(lo) < rad && fabsf(hi) < rad)) band = 1;
-    else if (__all_sync(0xffffffffu, lo >= rad || hi <= -rad)) band = 2;
+    if (boost_band_meets(a, dq0)) {
+      // columns c with |dq0 + c| < radius: c_lo <= c <= c_hi
+      const int d = static_cast<int>(dq0), rad = a.mod.boost_radius;
+      const int c_lo = -rad - d + 1, c_hi = rad - d - 1;
+#pragma unroll
+      for (int c = 0; c < BM; ++c) x[c] *= (c >= c_lo && c <= c_hi) ? a.mod.boost : 1.f;
+    }
   }
+  const float2 sl2 = make_float2(a.sl2, a.sl2);
 #pragma unroll
   for (int c4 = 0; c4 < BM / 4; ++c4) {
     const float4 l = lds128(nl2_addr + c4 * 16);
@@ -401,32 +388,67 @@ __device__ __forceinline__ void probs_t(float (&x)[BM], const BwdArgs& a, int h,
       if constexpr (score_of(MOD) == MOD_ALIBI) {
         v.x = fmaf(x[c], a.sl2, -aux * fabsf(dq0 + static_cast<float>(c))) + nl.x;
         v.y = fmaf(x[c + 1], a.sl2, -aux * fabsf(dq0 + static_cast<float>(c + 1))) + nl.y;
-      } else if constexpr (score_of(MOD) == MOD_SOFTCAP) {
-        v.x = fmaf(aux2, tanh_ex2(x[c] * aux), nl.x);
-        v.y = fmaf(aux2, tanh_ex2(x[c + 1] * aux), nl.y);
-      } else if constexpr (score_of(MOD) == MOD_BOOST) {
-        const float r = static_cast<float>(a.mod.boost_radius);
-        v.x = fmaf(x[c], fabsf(dq0 + static_cast<float>(c)) < r ? aux : a.sl2, nl.x);
-        v.y = fmaf(x[c + 1], fabsf(dq0 + static_cast<float>(c + 1)) < r ? aux : a.sl2, nl.y);
       } else {
         v = __ffma2_rn(make_float2(x[c], x[c + 1]), sl2, nl);
-      }
-      if constexpr (!kMaskAfterExp<MOD>) {
-        if (pred) {
-          v.x = keep_query<MOD>(c, q0, qlo, qhi, wa, wb) ? v.x : -INFINITY;
-          v.y = keep_query<MOD>(c + 1, q0, qlo, qhi, wa, wb) ? v.y : -INFINITY;
-        }
       }
       x[c] = ex2_approx(v.x);  // 0 on padding rows (-LSE2 = -inf)
       x[c + 1] = ex2_approx(v.y);
     }
   }
-  if constexpr (kMaskAfterExp<MOD>) {
-    if (pred) {  // PARTIAL steps only
+  if (pred) {  // PARTIAL steps only
 #pragma unroll
-      for (int c = 0; c < BM; ++c) x[c] = keep_query<MOD>(c, q0, qlo, qhi, wa, wb) ? x[c] : 0.f;
+    for (int c = 0; c < BM; ++c) x[c] = keep_query<MOD>(c, q0, qlo, qhi, wa, wb) ? x[c] : 0.f;
+  }
+}
+
+// Softcap keeps each 32-query half of an S^T buffer as [P^T | P ds'/ds]: 16
+// columns of P^T bf16 pairs (the A operand of dV += P^T dO) and 16 of
+// P (1 - tanh^2), the factor the dS warps take (the derivative of
+// c tanh(s / c)); the other mods keep P^T in the buffer's first 32 columns.
+template <int MOD>
+constexpr bool kSoftcapHalves = score_of(MOD) == MOD_SOFTCAP;
+// TMEM column, within an S^T buffer, of P^T's 16-query K-chunk kk
+template <int MOD>
+__device__ __forceinline__ constexpr uint32_t p_col(int kk) {
+  return kSoftcapHalves<MOD> ? static_cast<uint32_t>((kk >> 1) * 32 + (kk & 1) * 8) : static_cast<uint32_t>(kk * 8);
+}
+
+// Softcap, one 32-query half (columns t_half ...) of a key row of S^T:
+// P = 2^(c log2(e) tanh(scale x / c) - LSE2) and P (1 - tanh^2), masked on
+// PARTIAL steps, stored as bf16 pairs over the half's columns.  One loop body
+// serves both halves (the warp's hot code stays small).
+template <int MOD>
+__device__ __forceinline__ void softcap_half(uint32_t t_half, int hf, const BwdArgs& a, int q0, int qlo,
+                                             int qhi, bool pred, uint32_t nl2_addr, uint32_t wa, uint32_t wb) {
+  float x[32];
+  tmem_ld32(t_half, reinterpret_cast<uint32_t(&)[32]>(x[0]));
+  tmem_wait_ld();
+  const float aux = a.scale / a.mod.softcap, aux2 = a.mod.softcap * LOG2E;
+  uint32_t pk[16], pd[16];
+#pragma unroll
+  for (int c4 = 0; c4 < 8; ++c4) {
+    const float4 l = lds128(nl2_addr + (hf * 8 + c4) * 16);
+#pragma unroll
+    for (int hp = 0; hp < 2; ++hp) {
+      const int c = c4 * 4 + hp * 2;
+      const float2 nl = hp == 0 ? make_float2(l.x, l.y) : make_float2(l.z, l.w);
+      const float t0 = tanh_ex2(x[c] * aux), t1 = tanh_ex2(x[c + 1] * aux);
+      const float p0 = ex2_approx(fmaf(aux2, t0, nl.x)), p1 = ex2_approx(fmaf(aux2, t1, nl.y));  // 0 on padding rows
+      pk[c >> 1] = pack_bf16x2(p0, p1);
+      pd[c >> 1] = pack_bf16x2(p0 * fmaf(-t0, t0, 1.f), p1 * fmaf(-t1, t1, 1.f));
     }
   }
+  if (pred) {  // PARTIAL steps only
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint32_t keep = (keep_query<MOD>(hf * 32 + 2 * e, q0, qlo, qhi, wa, wb) ? 0x0000ffffu : 0u) |
+                            (keep_query<MOD>(hf * 32 + 2 * e + 1, q0, qlo, qhi, wa, wb) ? 0xffff0000u : 0u);
+      pk[e] &= keep;
+      pd[e] &= keep;
+    }
+  }
+  tmem_st16(t_half, pk);
+  tmem_st16(t_half + 16, pd);
 }
 
 // One accumulator row (dV or dK) of this thread's key: TMEM fp32 -> mul -> bf16 -> global.
@@ -530,7 +552,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // ---------------------------------------------------------- TMA producer
       // all lanes build the query-tile lists; lane 0 issues the copies
       int unit_iter = 0, step = 0;
-      uint32_t kv_loads = 0, stage_uses[4] = {0, 0, 0, 0}, clc_asked = 0, clc_read = 0;
+      uint32_t kv_loads = 0, clc_asked = 0, clc_read = 0;
       const uint32_t clc_resp = smem_u32(bars->clc_resp), clc_bar = smem_u32(&bars->clc_bar);
       bool ok = true;
       // The static walk: the snake over the order.  Cluster launch control (one
@@ -584,7 +606,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               const uint32_t st = sbase + Cfg::kStageOff + s * Cfg::kStageBytes;
               const uint32_t bar = smem_u32(&bars->q_full[s]);
               mbar_arrive_expect_tx(bar, 2 * Cfg::kQBytes + 2 * BM * 4);
-              ++stage_uses[s];
               const int bh = un.b * a.Hq + un.hk * a.G + g;
               BWD_EV(step, 0);
               load_q_tile<D>(st, &tm_q, bar, q0, un.hk * a.G + g, un.b);
@@ -612,8 +633,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const WaitCtl dwc{drain_limit(a.wait_ns), smem_u32(&bars->never_set), a.status};
         if (clc_asked > clc_read) mbar_wait_thread_ool(clc_bar, (clc_asked - 1) & 1, dwc);
         if (kv_loads) mbar_wait_thread_ool(smem_u32(&bars->kv_full), (kv_loads - 1) & 1, dwc);
-        for (int s = 0; s < Cfg::kStages; ++s)
-          if (stage_uses[s]) mbar_wait_thread_ool(smem_u32(&bars->q_full[s]), (stage_uses[s] - 1) & 1, dwc);
+        // stage s took the loads of steps s, s + kStages, ... below `step`
+        for (int s = 0; s < Cfg::kStages && s < step; ++s)
+          mbar_wait_thread_ool(smem_u32(&bars->q_full[s]), ((step - 1 - s) / Cfg::kStages) & 1, dwc);
       }
       ATTN25_TRACE_ONLY(tr[0] = clock64() - t_start;)
       trace_flush(a.trace, 48, tr);
@@ -693,7 +715,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           BWD_EV(step, 2);
 #pragma unroll
           for (int kk = 0; kk < BM / 16; ++kk)
-            mma_ts_w(t_dv, tmem + Cfg::kColS + sb * BM + kk * 8,
+            mma_ts_w(t_dv, tmem + Cfg::kColS + sb * BM + p_col<MOD>(kk),
                      smem_desc_sw128(st + Cfg::kQBytes + kk * 2048, BM * 128, 1024), Cfg::kIdescAcc,
                      (n_steps > 0 || kk > 0) ? 1u : 0u);
           BWD_EV(step, 3);
@@ -801,20 +823,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         BWD_EV(step, 8);
         ATTN25_TRACE_ONLY(const long long t_p = clock64();)
         const int h = un.hk * a.G + g;
-        float x[BM];
-        tmem_ld32(t_s, reinterpret_cast<uint32_t(&)[32]>(x[0]));
-        tmem_ld32(t_s + 32, reinterpret_cast<uint32_t(&)[32]>(x[32]));
-        tmem_wait_ld();
-        ATTN25_TRACE_ONLY(const long long t_p1 = clock64(); tr[4] += t_p1 - t_p;)
-        probs_t<MOD>(x, a, h, static_cast<float>(q0 - kv), q0, qlo, qhi, pred, nl2_s, wa, wb);
-        // P^T (bf16 pairs) over the first 32 columns of this S^T buffer
-        uint32_t pk[32];
+        if constexpr (kSoftcapHalves<MOD>) {
+          (void)h;
+#pragma unroll 1
+          for (int hf = 0; hf < 2; ++hf) softcap_half<MOD>(t_s + hf * 32, hf, a, q0, qlo, qhi, pred, nl2_s, wa, wb);
+          ATTN25_TRACE_ONLY(const long long t_p2 = clock64(); tr[5] += t_p2 - t_p;)
+          tmem_wait_st();
+          ATTN25_TRACE_ONLY(tr[6] += clock64() - t_p2;)
+        } else {
+          float x[BM];
+          tmem_ld32(t_s, reinterpret_cast<uint32_t(&)[32]>(x[0]));
+          tmem_ld32(t_s + 32, reinterpret_cast<uint32_t(&)[32]>(x[32]));
+          tmem_wait_ld();
+          ATTN25_TRACE_ONLY(const long long t_p1 = clock64(); tr[4] += t_p1 - t_p;)
+          probs_t<MOD>(x, a, h, static_cast<float>(q0 - kv), q0, qlo, qhi, pred, nl2_s, wa, wb);
+          // P^T (bf16 pairs) over the first 32 columns of this S^T buffer
+          uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
-        ATTN25_TRACE_ONLY(const long long t_p2 = clock64(); tr[5] += t_p2 - t_p1;)
-        tmem_st32(t_s, pk);
-        tmem_wait_st();
-        ATTN25_TRACE_ONLY(tr[6] += clock64() - t_p2;)
+          for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+          ATTN25_TRACE_ONLY(const long long t_p2 = clock64(); tr[5] += t_p2 - t_p1;)
+          tmem_st32(t_s, pk);
+          tmem_wait_st();
+          ATTN25_TRACE_ONLY(tr[6] += clock64() - t_p2;)
+        }
         tc_fence_before();
         mbar_arrive(smem_u32(&bars->p_ready[sb]));
         BWD_EV(step, 9);
@@ -878,7 +909,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint32_t pb[32];
         tmem_ld32(t_dp, reinterpret_cast<uint32_t(&)[32]>(dp[0]));
         tmem_ld32(t_dp + 32, reinterpret_cast<uint32_t(&)[32]>(dp[32]));
-        tmem_ld32(t_p, pb);
+        if constexpr (kSoftcapHalves<MOD>) {  // the factor P (1 - tanh^2) the P warps stored beside P^T
+          tmem_ld16(t_p + 16, reinterpret_cast<uint32_t(&)[16]>(pb[0]));
+          tmem_ld16(t_p + 48, reinterpret_cast<uint32_t(&)[16]>(pb[16]));
+        } else {
+          tmem_ld32(t_p, pb);
+        }
         tmem_wait_ld();
         ATTN25_TRACE_ONLY(tr[3] += clock64() - t_ds;)
         // dP^T has been read: the next step's dP^T may overwrite it.  (P^T of
@@ -889,47 +925,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // the dS buffer is free once the drain warps have staged dQ of two steps ago through it
         if (!ATTN25_TIMED(tr[5], mbar_wait_warp_ool(smem_u32(&bars->ds_empty[sb]), ((step >> 1) & 1) ^ 1, wc))) { ok = false; break; }
         uint8_t* ds_row = smem + Cfg::kDSOff + sb * Cfg::kDSBytes + r * 128;
-        const float dq0 = static_cast<float>(q0 - kv);
-        float cl2_inv = 0.f;
-        if constexpr (score_of(MOD) == MOD_SOFTCAP) cl2_inv = 1.f / (a.mod.softcap * LOG2E);
-        // local boost: the band covers the warp's step wholly (1), misses it (2), or neither (0)
-        int band = 0;
+        // local boost: dS carries the boost inside the band, folded into dP
+        // there, (dP' - Delta) = boost (dP - Delta) with dP' = boost dP + (boost - 1)(-Delta)
         if constexpr (score_of(MOD) == MOD_BOOST) {
-          const float rad = static_cast<float>(a.mod.boost_radius);
-          const float lo = dq0, hi = dq0 + static_cast<float>(BM - 1);
-          if (__all_sync(0xffffffffu, fabsf(lo) < rad && fabsf(hi) < rad)) band = 1;
-          else if (__all_sync(0xffffffffu, lo >= rad || hi <= -rad)) band = 2;
+          const float dq0 = static_cast<float>(q0 - kv);
+          if (boost_band_meets(a, dq0)) {
+            const float rad = static_cast<float>(a.mod.boost_radius), bst = a.mod.boost;
+#pragma unroll
+            for (int c4 = 0; c4 < BM / 4; ++c4) {
+              const float4 n4 = lds128(stats + 512 + c4 * 16);
+              const float nd4[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int c = c4 * 4 + e;
+                if (fabsf(dq0 + static_cast<float>(c)) < rad) dp[c] = fmaf(dp[c], bst, (bst - 1.f) * nd4[e]);
+              }
+            }
+          }
         }
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16) {  // 8 columns (16 bytes) at a time
           const float4 nd0 = lds128(stats + 512 + c16 * 32), nd1 = lds128(stats + 512 + c16 * 32 + 16);
           const float nd[8] = {nd0.x, nd0.y, nd0.z, nd0.w, nd1.x, nd1.y, nd1.z, nd1.w};
-          float4 nl0, nl1;
-          if constexpr (score_of(MOD) == MOD_SOFTCAP) {
-            nl0 = lds128(stats + c16 * 32);
-            nl1 = lds128(stats + c16 * 32 + 16);
-          }
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = c16 * 8 + 2 * e;
             const uint32_t pp = pb[c >> 1];
             const float2 pr = make_float2(__uint_as_float(pp << 16), __uint_as_float(pp & 0xffff0000u));
-            // dS = P (dP - Delta)
-            float2 d = __fmul2_rn(pr, __fadd2_rn(make_float2(dp[c], dp[c + 1]), make_float2(nd[2 * e], nd[2 * e + 1])));
-            if constexpr (score_of(MOD) == MOD_SOFTCAP) {
-              // d s'/d s = 1 - tanh^2 with tanh = (log2 P + LSE2) / (c log2 e)
-              const float nlx = (e < 2) ? (e == 0 ? nl0.x : nl0.z) : (e == 2 ? nl1.x : nl1.z);
-              const float nly = (e < 2) ? (e == 0 ? nl0.y : nl0.w) : (e == 2 ? nl1.y : nl1.w);
-              const float t0 = (__log2f(pr.x) - nlx) * cl2_inv;
-              const float t1 = (__log2f(pr.y) - nly) * cl2_inv;
-              d.x = pr.x > 0.f ? d.x * (1.f - t0 * t0) : 0.f;
-              d.y = pr.y > 0.f ? d.y * (1.f - t1 * t1) : 0.f;
-            } else if constexpr (score_of(MOD) == MOD_BOOST) {
-              const float rad = static_cast<float>(a.mod.boost_radius);
-              d.x *= fabsf(dq0 + static_cast<float>(c)) < rad ? a.mod.boost : 1.f;
-              d.y *= fabsf(dq0 + static_cast<float>(c + 1)) < rad ? a.mod.boost : 1.f;
-            }
+            // dS = P (dP - Delta) (softcap: P (1 - tanh^2) (dP - Delta))
+            const float2 d = __fmul2_rn(pr, __fadd2_rn(make_float2(dp[c], dp[c + 1]), make_float2(nd[2 * e], nd[2 * e + 1])));
             w[e] = pack_bf16x2(d.x, d.y);
           }
           // 128-byte swizzle: 16-byte chunk c16 of row r lands at chunk c16 ^ (r % 8)
