@@ -156,6 +156,13 @@ struct RowCtx {
   const uint32_t* bits;  // bitmap mask: this row's keep bits (nullptr on padding rows)
 };
 
+// Three-input maximum (one instruction).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Raw scores of one row (32 columns starting at key k0 + c0) -> base-2 modded scores.
 template <int MOD>
 __device__ __forceinline__ void transform32(float (&x)[32], const RowCtx& r, const ModDev& md,
@@ -164,12 +171,25 @@ __device__ __forceinline__ void transform32(float (&x)[32], const RowCtx& r, con
   if constexpr (score_of(MOD) == MOD_SOFTCAP) {
     // scores well below the cap everywhere in the warp's chunk take tanh from
     // its series on the FMA pipe, the others from its exponential form (MUFU)
-    float mx = 0.f;
+    // (largest |x| of the chunk: four chains of three-input maxima)
+    float m0 = max3(fabsf(x[0]), fabsf(x[1]), fabsf(x[2])), m1 = max3(fabsf(x[3]), fabsf(x[4]), fabsf(x[5]));
+    float m2 = max3(fabsf(x[6]), fabsf(x[7]), fabsf(x[8])), m3 = max3(fabsf(x[9]), fabsf(x[10]), fabsf(x[11]));
 #pragma unroll
-    for (int c = 0; c < 32; ++c) mx = fmaxf(mx, fabsf(x[c]));
-    if (__all_sync(0xffffffffu, mx <= r.lim)) {
+    for (int e = 12; e < 28; e += 8) {
+      m0 = max3(m0, fabsf(x[e]), fabsf(x[e + 1]));
+      m1 = max3(m1, fabsf(x[e + 2]), fabsf(x[e + 3]));
+      m2 = max3(m2, fabsf(x[e + 4]), fabsf(x[e + 5]));
+      m3 = max3(m3, fabsf(x[e + 6]), fabsf(x[e + 7]));
+    }
+    m0 = max3(m0, fabsf(x[28]), fabsf(x[29]));
+    m1 = max3(m1, fabsf(x[30]), fabsf(x[31]));
+    if (__all_sync(0xffffffffu, fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) <= r.lim)) {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) x[c] = r.aux2 * tanh_series(x[c] * r.aux);
+      for (int c = 0; c < 32; c += 2) {
+        const float2 t = tanh_series2(make_float2(x[c], x[c + 1]), r.aux, r.aux2);
+        x[c] = t.x;
+        x[c + 1] = t.y;
+      }
     } else {
 #pragma unroll
       for (int c = 0; c < 32; ++c) x[c] = r.aux2 * tanh_ex2(x[c] * r.aux);
@@ -217,11 +237,6 @@ __device__ __forceinline__ void transform32(float (&x)[32], const RowCtx& r, con
 // scale is folded into the exponent's FFMA.
 __host__ __device__ constexpr bool pure_scale(int key) { return score_of(key) == MOD_NONE; }
 
-__device__ __forceinline__ float max3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
 
 // Apply mask (and, for the other mods, the mod itself) to one row of raw
 // scores; return the row maximum in the base-2 domain.
@@ -700,9 +715,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
         ATTN25_TRACE_ONLY(const long long t_mid = clock64(); tr[2] += t_mid - t_tile;)
-        // full tiles hold no -inf, so part of their exponentials can run on the FMA pipe
-        const float lsum = prt_t ? row_probs<MOD, false>(x, rc, m_use, s_addr)
-                                 : row_probs<MOD, true>(x, rc, m_use, s_addr);
+        // full tiles hold no -inf, so part of their exponentials can run on the FMA
+        // pipe (not with softcap, whose tanh series already loads that pipe)
+        float lsum;
+        if constexpr (score_of(MOD) == MOD_SOFTCAP) lsum = row_probs<MOD, false>(x, rc, m_use, s_addr);
+        else lsum = prt_t ? row_probs<MOD, false>(x, rc, m_use, s_addr) : row_probs<MOD, true>(x, rc, m_use, s_addr);
         l_run += lsum;
         ATTN25_TRACE_ONLY(tr[3] += clock64() - t_mid;)
         tmem_wait_st();

@@ -432,13 +432,19 @@ __device__ __forceinline__ float tanh_ex2(float y) {
 // through the u^9 term: u (1 - u^2/3 + 2u^4/15 - 17u^6/315 + 62u^8/2835).
 // The first omitted term, 1382 u^11 / 155925, is below 4e-7 at |u| = 0.4.
 constexpr float kTanhSeriesLimit = 0.4f;
-__device__ __forceinline__ float tanh_series(float u) {
-  const float w = u * u;
-  float p = fmaf(w, 0.021869488f, -0.053968254f);
-  p = fmaf(p, w, 0.13333334f);
-  p = fmaf(p, w, -0.33333334f);
-  p = fmaf(p, w, 1.0f);
-  return u * p;
+constexpr float kTanhS4 = 0.021869488f, kTanhS3 = -0.053968254f, kTanhS2 = 0.13333334f, kTanhS1 = -0.33333334f;
+
+// k tanh(aux x) for a pair of scores x with |aux x| <= 0.4, on the FMA pipe in
+// packed fp32 pairs: u = aux x, w = u^2, and the series' factor with every
+// coefficient multiplied by k, so that k tanh(u) = u (k + k c1 w + ... + k c4 w^4).
+__device__ __forceinline__ float2 tanh_series2(float2 x, float aux, float k) {
+  const float2 u = __fmul2_rn(x, make_float2(aux, aux));
+  const float2 w = __fmul2_rn(u, u);
+  float2 p = __ffma2_rn(w, make_float2(k * kTanhS4, k * kTanhS4), make_float2(k * kTanhS3, k * kTanhS3));
+  p = __ffma2_rn(p, w, make_float2(k * kTanhS2, k * kTanhS2));
+  p = __ffma2_rn(p, w, make_float2(k * kTanhS1, k * kTanhS1));
+  p = __ffma2_rn(p, w, make_float2(k, k));
+  return __fmul2_rn(u, p);
 }
 
 // 2^x on the FMA pipe (finite x only): x = n + f with n = round(x) taken from
