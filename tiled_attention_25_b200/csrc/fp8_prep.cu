@@ -27,16 +27,47 @@ namespace attn25 {
 namespace {
 
 constexpr int kPrepThreads = 256;
+constexpr int kPrepRows = 4;  // rows a warp has in flight
+
+// Lane l of a warp holds elements l V .. l V + V - 1 (V = D / 32) of a row.
+template <int D>
+struct RowBits {
+  uint32_t w[D / 64];  // V bf16, two per word
+};
 
 template <int D>
-__device__ __forceinline__ void rotate_row(const __nv_bfloat16* row, const int8_t* signs, float inv_sqrt_d,
+__device__ __forceinline__ RowBits<D> load_row(const __nv_bfloat16* row) {
+  const int lane = threadIdx.x & 31;
+  RowBits<D> r;
+  if constexpr (D == 128) {  // 8 bytes per lane
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(row) + lane);
+    r.w[0] = v.x;
+    r.w[1] = v.y;
+  } else {  // 4 bytes per lane
+    r.w[0] = __ldg(reinterpret_cast<const uint32_t*>(row) + lane);
+  }
+  return r;
+}
+
+// The lane's signs of the sign flip, as floats.
+template <int D>
+__device__ __forceinline__ void load_signs(const int8_t* signs, float (&sg)[D / 32]) {
+  constexpr int V = D / 32;
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < V; ++j) sg[j] = static_cast<float>(__ldg(signs + lane * V + j));
+}
+
+// The sign flip, the butterflies and the 1/sqrt(D) product of one row.
+template <int D>
+__device__ __forceinline__ void rotate_row(const RowBits<D>& bits, const float (&sg)[D / 32], float inv_sqrt_d,
                                            float (&y)[D / 32]) {
   constexpr int V = D / 32;
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int j = 0; j < V; ++j) {
-    const int e = lane * V + j;
-    y[j] = __bfloat162float(row[e]) * static_cast<float>(__ldg(signs + e));
+    const uint32_t wd = bits.w[j >> 1];
+    y[j] = __uint_as_float((j & 1) ? (wd & 0xffff0000u) : (wd << 16)) * sg[j];
   }
 #pragma unroll
   for (int h = 1; h < V; h *= 2) {  // pairs inside the lane
@@ -64,18 +95,30 @@ __device__ __forceinline__ void rotate_row(const __nv_bfloat16* row, const int8_
 }
 
 // grid (row blocks, B*H): the absolute maximum of each (b, head) after the
-// rotation, as float bits (non-negative floats order like unsigned ints)
+// rotation, as float bits (non-negative floats order like unsigned ints).
+// Each warp takes kPrepRows rows at a time, their loads issued together.
 template <int D>
 __global__ void __launch_bounds__(kPrepThreads) fp8_amax_kernel(const __nv_bfloat16* x, const int8_t* signs,
                                                                  uint32_t* amax, int S, float inv_sqrt_d) {
   const int bh = blockIdx.y, warp = threadIdx.x >> 5;
   constexpr int kWarps = kPrepThreads / 32;
+  float sg[D / 32];
+  load_signs<D>(signs, sg);
   float m = 0.f;
-  for (int r = blockIdx.x * kWarps + warp; r < S; r += gridDim.x * kWarps) {
-    float y[D / 32];
-    rotate_row<D>(x + (static_cast<size_t>(bh) * S + r) * D, signs, inv_sqrt_d, y);
+  for (int r0 = (blockIdx.x * kWarps + warp) * kPrepRows; r0 < S; r0 += gridDim.x * kWarps * kPrepRows) {
+    RowBits<D> bits[kPrepRows];
 #pragma unroll
-    for (int j = 0; j < D / 32; ++j) m = fmaxf(m, fabsf(y[j]));
+    for (int i = 0; i < kPrepRows; ++i)
+      if (r0 + i < S) bits[i] = load_row<D>(x + (static_cast<size_t>(bh) * S + r0 + i) * D);
+#pragma unroll
+    for (int i = 0; i < kPrepRows; ++i) {
+      if (r0 + i < S) {
+        float y[D / 32];
+        rotate_row<D>(bits[i], sg, inv_sqrt_d, y);
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) m = fmaxf(m, fabsf(y[j]));
+      }
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -110,16 +153,27 @@ __global__ void __launch_bounds__(kPrepThreads) fp8_quantize_kernel(const __nv_b
   const int bh = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int kWarps = kPrepThreads / 32;
   const float scale = head_scale(__ldg(amax + bh));
-  for (int r = blockIdx.x * kWarps + warp; r < S; r += gridDim.x * kWarps) {
-    const size_t row = static_cast<size_t>(bh) * S + r;
-    float y[V];
-    rotate_row<D>(x + row * D, signs, inv_sqrt_d, y);
-    uint8_t* out = codes + row * D + lane * V;
-    if constexpr (V == 4) {
-      const uint32_t lo = e4m3x2(y[0] / scale, y[1] / scale), hi = e4m3x2(y[2] / scale, y[3] / scale);
-      *reinterpret_cast<uint32_t*>(out) = lo | (hi << 16);
-    } else {
-      *reinterpret_cast<uint16_t*>(out) = e4m3x2(y[0] / scale, y[1] / scale);
+  float sg[V];
+  load_signs<D>(signs, sg);
+  for (int r0 = (blockIdx.x * kWarps + warp) * kPrepRows; r0 < S; r0 += gridDim.x * kWarps * kPrepRows) {
+    RowBits<D> bits[kPrepRows];
+#pragma unroll
+    for (int i = 0; i < kPrepRows; ++i)
+      if (r0 + i < S) bits[i] = load_row<D>(x + (static_cast<size_t>(bh) * S + r0 + i) * D);
+#pragma unroll
+    for (int i = 0; i < kPrepRows; ++i) {
+      if (r0 + i < S) {
+        const size_t row = static_cast<size_t>(bh) * S + r0 + i;
+        float y[V];
+        rotate_row<D>(bits[i], sg, inv_sqrt_d, y);
+        uint8_t* out = codes + row * D + lane * V;
+        if constexpr (V == 4) {
+          const uint32_t lo = e4m3x2(y[0] / scale, y[1] / scale), hi = e4m3x2(y[2] / scale, y[3] / scale);
+          *reinterpret_cast<uint32_t*>(out) = lo | (hi << 16);
+        } else {
+          *reinterpret_cast<uint16_t*>(out) = e4m3x2(y[0] / scale, y[1] / scale);
+        }
+      }
     }
   }
 }
@@ -152,9 +206,9 @@ cudaError_t launch_fp8_prep_t(const __nv_bfloat16* x, const int8_t* signs, uint8
 
 cudaError_t launch_fp8_prep(const void* x, const int8_t* signs, uint8_t* codes, float* scales, int BH, int S,
                             int D, int sms, cudaStream_t stream) {
-  // about four blocks per SM over all heads, each block taking whole rows
-  const int rows_per_block = kPrepThreads / 32;
-  long long want = (4LL * sms + BH - 1) / BH;
+  // about eight blocks per SM over all heads, each block taking whole rows
+  const int rows_per_block = kPrepThreads / 32 * kPrepRows;
+  long long want = (8LL * sms + BH - 1) / BH;
   const long long most = (S + rows_per_block - 1) / rows_per_block;
   const int row_blocks = static_cast<int>(want < 1 ? 1 : (want > most ? most : want));
   const float inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));

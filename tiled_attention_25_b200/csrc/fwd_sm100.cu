@@ -689,8 +689,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int c = 0; c < 4; ++c)
           tmem_ld32(s_addr + c * 32, reinterpret_cast<uint32_t(&)[32]>(x[c]));
         tmem_wait_ld();
-        const float mx = prt_t ? row_scores<MOD, true>(x, rc, a.mod, k0, bw)
-                               : row_scores<MOD, false>(x, rc, a.mod, k0, bw);
+        // local boost: a tile whose keys lie outside every row's band (the warp's
+        // rows, warp-uniform) takes the plain-scale path of the masks-only key
+        constexpr int kPlain = MOD & ~(kKeyMasked - 1);
+        bool plain = false;
+        if constexpr (score_of(MOD) == MOD_BOOST) {
+          const float rad = static_cast<float>(a.mod.boost_radius), di = static_cast<float>(rc.row - k0);
+          plain = __all_sync(0xffffffffu, di - static_cast<float>(TILE - 1) >= rad || di <= -rad);
+        }
+        float mx;
+        if (plain) {
+          mx = prt_t ? row_scores<kPlain, true>(x, rc, a.mod, k0, bw) : row_scores<kPlain, false>(x, rc, a.mod, k0, bw);
+        } else {
+          mx = prt_t ? row_scores<MOD, true>(x, rc, a.mod, k0, bw) : row_scores<MOD, false>(x, rc, a.mod, k0, bw);
+        }
         const float m_new = fmaxf(m_run, mx);
         const bool need = m_new > m_run + kRescaleThreshold;
         if (__any_sync(0xffffffffu, need)) {
@@ -719,6 +731,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // pipe (not with softcap, whose tanh series already loads that pipe)
         float lsum;
         if constexpr (score_of(MOD) == MOD_SOFTCAP) lsum = row_probs<MOD, false>(x, rc, m_use, s_addr);
+        else if (plain) lsum = prt_t ? row_probs<kPlain, false>(x, rc, m_use, s_addr) : row_probs<kPlain, true>(x, rc, m_use, s_addr);
         else lsum = prt_t ? row_probs<MOD, false>(x, rc, m_use, s_addr) : row_probs<MOD, true>(x, rc, m_use, s_addr);
         l_run += lsum;
         ATTN25_TRACE_ONLY(tr[3] += clock64() - t_mid;)
