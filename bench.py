@@ -349,7 +349,9 @@ def config_entry(ta, spec, rank, world, dev, stream, flush, steps, warmup, peak,
     bwd_tf = 0.0 if fwd_only else f_bwd / (t["ms_bwd"] * 1e-3) / 1e12
     w = pb.w
     entry = {"shape": f"B={w.B} Hq={w.Hq} Hkv={w.Hkv} S={w.Sq} D={w.D}", "mod": pb.mod_name,
-             "variant": variant, "walk": walk or "cluster launch control",
+             "variant": variant,
+             "walk": walk or ("static backward (always, for the ordered dQ adds)" if variant == "det"
+                              else "cluster launch control"),
              "useful_elements": n_u, "steps": steps, "warmup": warmup,
              "ms_fwd": round(t["ms_fwd"], 4), "ms_block_mask": round(t["ms_mask"], 4),
              "fwd_tflops": round(fwd_tf, 1), "fwd_frac_of_peak": round(fwd_tf / peak, 4), "clocks": t["clocks"]}

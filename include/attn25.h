@@ -356,7 +356,9 @@ ATTN25_API void attn_set_wait_limit_ms(uint32_t ms);
  * How the persistent forward and backward kernels take their work units
  * (query-tile pairs forward, key tiles backward), which they always take in
  * the block mask's longest-first order (ascending key tiles for
- * attn_bwd_deterministic):
+ * attn_bwd_deterministic, which always takes the static walk: its ordered dQ
+ * adds need every unit of lower rank started, which the static walk's
+ * resident CTAs guarantee):
  *   ATTN_WALK_STATIC: one CTA per SM; wave k of the order goes to the CTAs
  *     in turn, every other wave reversed (a snake), fixed in advance;
  *   ATTN_WALK_CLUSTER_LAUNCH_CONTROL (default): one CTA per unit is launched; a CTA that

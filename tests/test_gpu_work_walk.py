@@ -71,9 +71,10 @@ def test_many_units_per_sm_and_units_without_work(ta):
 
 
 def test_deterministic_dq_under_cluster_launch_control(ta):
-    """The deterministic backward takes units in ascending key tiles; with
-    cluster launch control the CTAs start, and are cancelled, in that order,
-    so dQ is still bitwise the same on every run (and equal to the static walk's)."""
+    """The deterministic backward takes the static walk whatever walk is set
+    (its ordered adds need every lower-ranked unit started), so with cluster
+    launch control selected dQ is still bitwise the same on every run, and
+    equal to the static walk's."""
     from test_gpu_deterministic import run_det, same_bits
     c = Case(73, 4, 8, 4, 2048, 2048, 128, oracle.MOD_CAUSAL)
     ta.attn_set_work_walk(ta.WALK_STATIC)

@@ -661,7 +661,10 @@ static int bwd_impl(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, 
   if (!encode_bf16_4d(&tq, q, D, Sq, Hq, B, sq, 64) || !encode_bf16_4d(&tk, k, D, Skv, Hkv, B, sk, TILE) ||
       !encode_bf16_4d(&tv, v, D, Skv, Hkv, B, sv, TILE) || !encode_bf16_4d(&tdo, dout, D, Sq, Hq, B, a.do_st, 64))
     return ATTN_ERR_ARG;
-  a.clc = g_work_walk.load() == ATTN_WALK_CLUSTER_LAUNCH_CONTROL ? 1 : 0;
+  // The ordered adds need every unit of lower rank started before a unit waits
+  // on it: only the static walk's resident CTAs (one per SM, ascending ranks)
+  // guarantee that, so the deterministic backward always takes it.
+  a.clc = !det && g_work_walk.load() == ATTN_WALK_CLUSTER_LAUNCH_CONTROL ? 1 : 0;
   const int grid = a.clc ? a.n_units : (a.n_units < d->sms ? a.n_units : d->sms);
   if (launch_bwd(tq, tk, tv, tdo, a, D, mod_key(mod_kind), grid,
                  reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
