@@ -452,27 +452,42 @@ __device__ __forceinline__ void softcap_half(uint32_t t_half, int hf, const BwdA
 }
 
 // One accumulator row (dV or dK) of this thread's key: TMEM fp32 -> mul -> bf16 -> global.
-template <int D>
+// N 32-column chunks per TMEM round trip (two, except where the kernel's
+// registers allow only one); 32-byte stores where the row allows them.
+template <int D, int N>
 __device__ __forceinline__ void store_acc_rows(__nv_bfloat16* dst, uint32_t src, float mul, bool have,
                                                bool row_ok) {
+  const bool wide = (reinterpret_cast<uintptr_t>(dst) & 31u) == 0;
 #pragma unroll
-  for (int c = 0; c < D / 32; ++c) {
-    uint32_t o[32];
-    if (have) {
-      tmem_ld32(src + c * 32, o);
-      tmem_wait_ld();
-    } else {
+  for (int c2 = 0; c2 < D / (32 * N); ++c2) {
+    uint32_t o[N][32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) o[e] = 0u;
+    for (int h = 0; h < N; ++h) {
+      if (have) {
+        tmem_ld32(src + (N * c2 + h) * 32, o[h]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[h][e] = 0u;
+      }
     }
-    uint32_t pk[16];
+    if (have) tmem_wait_ld();
 #pragma unroll
-    for (int e = 0; e < 16; ++e)
-      pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * mul, __uint_as_float(o[2 * e + 1]) * mul);
-    if (row_ok) {
-      uint4* p = reinterpret_cast<uint4*>(dst + c * 32);
+    for (int h = 0; h < N; ++h) {
+      const int c = N * c2 + h;
+      uint32_t pk[16];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) p[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+      for (int e = 0; e < 16; ++e)
+        pk[e] = pack_bf16x2(__uint_as_float(o[h][2 * e]) * mul, __uint_as_float(o[h][2 * e + 1]) * mul);
+      if (row_ok) {
+        if (wide) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) st_global_v8(dst + c * 32 + e * 16, &pk[8 * e]);
+        } else {
+          uint4* p = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) p[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+      }
     }
   }
 }
@@ -858,7 +873,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ATTN25_TIMED(tr[7], mbar_wait_warp_ool(smem_u32(&bars->acc_full), unit_iter & 1, wc))) { ok = false; break; }
       tc_fence_after();
       ATTN25_TRACE_ONLY(const long long t_e = clock64();)
-      store_acc_rows<D>(a.dv + un.b * a.dv_st.b + un.hk * a.dv_st.h + static_cast<long long>(kv) * a.dv_st.s, t_dv, 1.f,
+      store_acc_rows<D, kSoftcapHalves<MOD> ? 1 : 2>(a.dv + un.b * a.dv_st.b + un.hk * a.dv_st.h + static_cast<long long>(kv) * a.dv_st.s, t_dv, 1.f,
                         n_steps > 0, kv < a.Skv);
       tc_fence_before();
       mbar_arrive(smem_u32(&bars->acc_empty));
@@ -972,7 +987,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ATTN25_TIMED(tr[7], mbar_wait_warp_ool(smem_u32(&bars->acc_full), unit_iter & 1, wc))) { ok = false; break; }
       tc_fence_after();
       ATTN25_TRACE_ONLY(const long long t_e = clock64();)
-      store_acc_rows<D>(a.dk + un.b * a.dk_st.b + un.hk * a.dk_st.h + static_cast<long long>(kv) * a.dk_st.s, t_dk, a.scale,
+      store_acc_rows<D, kSoftcapHalves<MOD> ? 1 : 2>(a.dk + un.b * a.dk_st.b + un.hk * a.dk_st.h + static_cast<long long>(kv) * a.dk_st.s, t_dk, a.scale,
                         n_steps > 0, kv < a.Skv);
       tc_fence_before();
       mbar_arrive(smem_u32(&bars->acc_empty));

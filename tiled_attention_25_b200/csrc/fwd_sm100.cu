@@ -753,24 +753,38 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const size_t row_idx = (static_cast<size_t>(uc.b) * a.Hq + uc.h) * a.Sq + rc.row;
       __nv_bfloat16* orow = a.out + uc.b * a.o_st.b + uc.h * a.o_st.h + static_cast<long long>(rc.row) * a.o_st.s;
       const float inv_l = (l_run > 0.f) ? 1.0f / l_run : 0.f;
+      // 32-byte stores where the row allows them (a full L2 sector per lane)
+      const bool wide = (reinterpret_cast<uintptr_t>(orow) & 31u) == 0;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        if (n_act > 0) {
-          tmem_ld32(o_addr + c * 32, o);
-          tmem_wait_ld();
-        } else {
+      for (int c2 = 0; c2 < D / 64; ++c2) {  // two 32-column chunks per TMEM round trip
+        uint32_t o[2][32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        for (int h = 0; h < 2; ++h) {
+          if (n_act > 0) {
+            tmem_ld32(o_addr + (2 * c2 + h) * 32, o[h]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[h][e] = 0u;
+          }
         }
-        uint32_t pk[16];
+        if (n_act > 0) tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-        if (row_valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        for (int h = 0; h < 2; ++h) {
+          const int c = 2 * c2 + h;
+          uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(o[h][2 * e]) * inv_l, __uint_as_float(o[h][2 * e + 1]) * inv_l);
+          if (row_valid) {
+            if (wide) {
+#pragma unroll
+              for (int e = 0; e < 2; ++e) st_global_v8(orow + c * 32 + e * 16, &pk[8 * e]);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            }
+          }
         }
       }
       if constexpr (HAS_LSE) {
