@@ -288,8 +288,7 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   const float2 t = __fadd2_rn(x, magic);
   const float2 n = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
   const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
-  float2 p = __ffma2_rn(make_float2(kExp2C4, kExp2C4), f, make_float2(kExp2C3, kExp2C3));
-  p = __ffma2_rn(p, f, make_float2(kExp2C2, kExp2C2));
+  float2 p = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
   p = __ffma2_rn(p, f, make_float2(kExp2C1, kExp2C1));
   p = __ffma2_rn(p, f, make_float2(kExp2C0, kExp2C0));
   return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),

@@ -457,8 +457,7 @@ __device__ __forceinline__ float exp2_poly(float x) {
   const float t = x + 12582912.0f;
   const float n = t - 12582912.0f;
   const float f = x - n;
-  float p = fmaf(kExp2C4, f, kExp2C3);
-  p = fmaf(p, f, kExp2C2);
+  float p = fmaf(kExp2C3, f, kExp2C2);
   p = fmaf(p, f, kExp2C1);
   p = fmaf(p, f, kExp2C0);
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
