@@ -131,6 +131,8 @@ def forward(units, seed, give_up, stages=4, drain_kv=True, drain_always=True, cl
                             break
                         pv[t] += 1
                         sim.commit(f"o_full{t}")
+                    if not nxt:
+                        sim.commit(f"o_final{t}")
                     if nxt:
                         if t == 0:
                             ok = yield full(f"kv_full{slot_kn}", ph_kn)
@@ -148,9 +150,6 @@ def forward(units, seed, give_up, stages=4, drain_kv=True, drain_always=True, cl
             if not ok:
                 break
             sim.commit("q_empty")
-            if n > 0:
-                sim.commit("o_final0")
-                sim.commit("o_final1")
             sim.arrive(f"list_empty{b}")
         sim.commit("drain")  # every MMA issued so far completes before this arrival
         yield drain("drain", 0)

@@ -9,7 +9,8 @@ arrival here):
   tiles and streams K and V through a ring of slots;
 * the MMA warp issues S_t = Q_t K^T and O_t += P_t V for the two query tiles
   t of the unit, in the ping-pong order, committing s_full, o_full, the ring's
-  empty slots, q_empty and, on units with steps, o_final;
+  empty slots, q_empty and, on units with steps, o_final (each tile's right
+  after its last PV);
 * two softmax warpgroups, one per query tile, turn S_t into P_t (p_full) and
   sometimes rescale O_t, which first waits for the previous PV (o_full);
   the rescale decision depends on the data, so the model draws it.
@@ -96,6 +97,8 @@ def simulate(units, seed, stages=4, final_on_empty_units=False, clc=False):
                         yield full(f"p_full{t}", pv[t])
                         pv[t] += 1
                         sim.commit(f"o_full{t}")
+                    if not nxt:                 # tile t's O is final after its last PV
+                        sim.commit(f"o_final{t}")
                     if nxt:                     # S_t(j+1)
                         if t == 0:
                             yield full(f"kv_full{slot_kn}", ph_kn)
@@ -107,7 +110,7 @@ def simulate(units, seed, stages=4, final_on_empty_units=False, clc=False):
                 if nxt:
                     ring += 1
             sim.commit("q_empty")
-            if n > 0 or final_on_empty_units:
+            if n == 0 and final_on_empty_units:
                 sim.commit("o_final0")
                 sim.commit("o_final1")
             sim.arrive(f"list_empty{b}")

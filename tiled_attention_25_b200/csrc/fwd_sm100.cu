@@ -569,6 +569,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mma_commit_w(smem_u32(&bars->o_full[t]));
             o_started[t] = true;
           }
+          // the unit's last step: tile t's O is final once this PV completes, so its
+          // epilogue need not wait for the other tile's last softmax.  (o_final
+          // counts units with at least one step only, so that units without key
+          // tiles cannot run its phases ahead of the epilogues.)
+          if (!has_n) mma_commit_w(smem_u32(&bars->o_final[t]));
           if (has_n) {
             if (t == 0) {
               if (!ATTN25_TIMED(tr[2], mbar_wait_warp(smem_u32(&bars->kv_full[slot_kn]), ph_kn, wc))) { ok = false; break; }
@@ -591,13 +596,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (!ok) break;
       mma_commit_w(smem_u32(&bars->q_empty));
-      // o_final counts units with at least one step only: the softmax warps
-      // wait for it on those units alone, so that units without key tiles
-      // cannot run its phases ahead of their epilogues
-      if (n_steps > 0) {
-        mma_commit_w(smem_u32(&bars->o_final[0]));
-        mma_commit_w(smem_u32(&bars->o_final[1]));
-      }
       if (lane == 0) mbar_arrive(smem_u32(&bars->list_empty[buf]));
       __syncwarp();
     }
