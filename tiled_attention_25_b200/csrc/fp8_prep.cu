@@ -83,11 +83,14 @@ __device__ __forceinline__ void rotate_row(const RowBits<D>& bits, const float (
 #pragma unroll
   for (int h = V; h < D; h *= 2) {  // pairs across lanes
     const int d = h / V;
-    const bool upper = (lane & d) != 0;  // this lane holds the y[i + h] half
+    // this lane holds the y[i + h] half (p - y) or the y[i] half (y + p): one
+    // fused multiply-add by -1 or +1, exact product and one rounding, the same
+    // value as the subtraction or the addition
+    const float sg = (lane & d) != 0 ? -1.f : 1.f;
 #pragma unroll
     for (int j = 0; j < V; ++j) {
       const float p = __shfl_xor_sync(0xffffffffu, y[j], d);
-      y[j] = upper ? p - y[j] : y[j] + p;
+      y[j] = fmaf(sg, y[j], p);
     }
   }
 #pragma unroll
